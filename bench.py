@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Benchmark of the streaming hot path of RTR-DiT's rerenderer on B200.
+
+One step = one pass of the hot path for one DiT layer of the Wan-1.3B-shaped
+workload: the current chunk (3 latent frames x 1560 tokens = 4680 queries,
+12 heads, head_dim 128, bf16) attends under the frame-causal mask to
+[1 anchored reference frame | 21 window frames | itself]
+(``rtr_attn_frame_causal``), then its K/V are committed to the ring, evicting
+the 3 oldest frames (``rtr_kvcache_append_frame``).
+
+Prints one JSON line.  ``value`` is attention TFLOP/s of the whole job (the
+algorithmic flops: visible query-key pairs x 4 x head_dim, summed over
+heads, divided by the device time of the step); ``latent_frames_per_s_per_layer``
+and the roofline fraction of the attention kernel come with it.  Usage:
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one independent replica stream per GPU.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "frame-causal attn TFLOP/s & latent frames/s per layer; % of BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+PROFILE = os.path.join(ROOT, "profiles", "fc_attn_fwd_tc__wan13_layer.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "causal_attention_rtr_b200", "csrc", f) for f in ("attn_tc.cu", "ptx.cuh")]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ workload
+def workload():
+    from causal_attention_rtr_b200 import synth
+    return synth.WAN13_LAYER
+
+
+def visible_pairs_per_head(w):
+    """Query-key pairs the mask leaves visible for one chunk: every chunk
+    query sees all cached keys ((R + W) frames of k), and chunk frame c sees
+    chunk frames 0..c."""
+    cached = (w.ref_frames + w.window_frames) * w.k
+    nq = w.chunk_frames * w.k
+    chunk = sum(w.k * (c + 1) * w.k for c in range(w.chunk_frames))
+    return nq * cached + chunk
+
+
+def attn_flops(w):
+    return 4.0 * w.head_dim * w.heads * visible_pairs_per_head(w)
+
+
+def append_bytes(w):
+    """Algorithmic bytes of committing one chunk: read K and V of the chunk,
+    write them into their slots."""
+    return 2 * 2 * w.chunk_frames * w.k * w.heads * w.head_dim * 2
+
+
+def config_dict(w, world):
+    return {"workload": w.name, "heads": w.heads, "head_dim": w.head_dim, "tokens_per_frame": w.k,
+            "chunk_frames": w.chunk_frames, "ref_frames": w.ref_frames, "window_frames": w.window_frames,
+            "queries": w.chunk_frames * w.k,
+            "keys_per_head": (w.ref_frames + w.window_frames + w.chunk_frames) * w.k,
+            "l2": "flushed between steps (256 MiB write outside the step events)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def profiled_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    if not os.path.exists(PROFILE):
+        return None
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    digest = h.hexdigest()
+    vals = {}
+    with open(PROFILE) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip().strip("-* ")] = v.strip().strip("`")
+    if vals.get("source_sha256") != digest:
+        return None
+    try:
+        return int(float(vals["traffic_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = bus_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.bus_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        power = [num(r[3]) or 0.0 for r in rows]
+        pmax = max(power)
+        loaded = [r for r, p in zip(rows, power) if p >= 0.5 * pmax] or rows
+        sm = [num(r[1]) for r in loaded if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in loaded for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(loaded[0][2]),
+                "reasons": reasons, "samples": len(loaded), "power_w_max": pmax}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_cache_for(w, x):
+    import oracle
+    o = oracle.ReferenceCache(w.heads, w.head_dim, w.k, w.ref_frames, w.window_frames, w.dtype)
+    o.set_reference(x.ref_k, x.ref_v)
+    for fk, fv in zip(x.window_k, x.window_v):
+        o.append(fk, fv, 1)
+    return o
+
+
+def oracle_sample_flops(w, rows):
+    cached = (w.ref_frames + w.window_frames) * w.k
+    return sum(4.0 * w.head_dim * w.heads * (cached + (r // w.k + 1) * w.k) for r in rows)
+
+
+def time_oracle(w, x, o, seconds_target):
+    """Time the oracle on sampled query rows (all heads) of the chunk,
+    growing the sample until it takes about ``seconds_target``.  Returns
+    (flops, seconds, rows)."""
+    import numpy as np
+    import oracle
+    nq = w.chunk_frames * w.k
+    rng = np.random.default_rng(123)
+    n = 2
+    while True:
+        rows = np.sort(rng.choice(nq, size=min(n, nq), replace=False))
+        t0 = time.perf_counter()
+        o.stream_attention(x.q, x.k_cur, x.v_cur, w.chunk_frames, rows=rows)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * seconds_target or n >= nq:
+            return oracle_sample_flops(w, rows), dt, rows
+        n = min(nq, max(n * 2, int(n * seconds_target / max(dt, 1e-3) * 0.9)))
+
+
+def cpu_baseline_entry(flops, seconds, rows, w):
+    import oracle
+    return {"value": flops / seconds / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} query rows x {w.heads} heads of the chunk (of {w.chunk_frames * w.k}), "
+                      f"fp64 C/OpenMP oracle, {flops / 1e9:.1f} GFLOP in {seconds:.2f} s",
+            "cpu_model": cpu_model()}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from causal_attention_rtr_b200 import synth
+    w = workload()
+    x = synth.stream_layer_inputs(w)
+    o = oracle_cache_for(w, x)
+    per_step = max(0.05, 150.0 / max(1, args.steps + args.warmup))
+    flops, dt, rows = time_oracle(w, x, o, per_step)
+    for _ in range(args.warmup):
+        o.stream_attention(x.q, x.k_cur, x.v_cur, w.chunk_frames, rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        o.stream_attention(x.q, x.k_cur, x.v_cur, w.chunk_frames, rows=rows)
+    total = time.perf_counter() - t0
+    value = flops * args.steps / total / 1e12
+    cb = cpu_baseline_entry(flops * args.steps, total, rows, w)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: N(0,1)*0.5 rounded to bf16, seed 1", "config": config_dict(w, world),
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "note": "each step is the fp64 oracle on a bounded sample of the step's query rows"}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from causal_attention_rtr_b200 import rtr, synth
+
+    torch.cuda.set_device(local_rank)
+    dev_id = local_rank
+    w = workload()
+    x = synth.stream_layer_inputs(w, seed=w.seed + rank)
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).cuda()
+
+    c = rtr.rtr_kvcache_create(1, w.heads, w.head_dim, w.k, w.ref_frames, w.window_frames, "bf16", dev_id)
+    rtr.rtr_kvcache_set_reference(c, 0, dev(x.ref_k), dev(x.ref_v))
+    for fk, fv in zip(x.window_k, x.window_v):
+        rtr.rtr_kvcache_append_frame(c, 0, dev(fk), dev(fv), 1)
+    q, kc, vc = dev(x.q), dev(x.k_cur), dev(x.v_cur)
+    out = torch.empty_like(q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    C = w.chunk_frames
+
+    def step():
+        rtr.rtr_attn_frame_causal(c, 0, q, kc, vc, C, out, 0.0, sh)
+        rtr.rtr_kvcache_append_frame(c, 0, kc, vc, C, sh)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if rtr.rtr_get_device_status(dev_id, sh) != rtr.RTR_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    props = torch.cuda.get_device_properties(dev_id)
+    try:
+        bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    except AttributeError:
+        bus = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0]
+    clocks = ClockSampler(bus)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for s in range(K):
+        flush.zero_()
+        ev[s][0].record(stream)
+        rtr.rtr_attn_frame_causal(c, 0, q, kc, vc, C, out, 0.0, sh)
+        ev[s][1].record(stream)
+        rtr.rtr_kvcache_append_frame(c, 0, kc, vc, C, sh)
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    attn_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    app_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    step_ms = [a + b for a, b in zip(attn_ms, app_ms)]
+    status = rtr.rtr_get_device_status(dev_id, sh)
+    if status != rtr.RTR_OK:
+        raise RuntimeError(f"device status {rtr.rtr_status_string(status)}")
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside
+    hq = torch.from_numpy(x.q.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(x.k_cur.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(x.v_cur.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
+    Ke = min(K, 100)
+    e_start = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    e_end = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(Ke):
+        flush.zero_()
+        e_start[s].record(stream)
+        q.copy_(hq, non_blocking=True)
+        kc.copy_(hk, non_blocking=True)
+        vc.copy_(hv, non_blocking=True)
+        rtr.rtr_attn_frame_causal(c, 0, q, kc, vc, C, out, 0.0, sh)
+        rtr.rtr_kvcache_append_frame(c, 0, kc, vc, C, sh)
+        ho.copy_(out, non_blocking=True)
+        e_end[s].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = [a.elapsed_time(b) for a, b in zip(e_start, e_end)]
+
+    stats = torch.tensor([statistics.mean(step_ms), statistics.mean(attn_ms), statistics.mean(app_ms),
+                          statistics.mean(e2e_ms)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    step_mean, attn_mean, app_mean, e2e_mean = stats.tolist()
+
+    rtr.rtr_kvcache_destroy(c)
+    if rank != 0:
+        return
+
+    flops = attn_flops(w)
+    peaks = measured_peaks()
+    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    value = world * flops / (step_mean * 1e-3) / 1e12
+    attn_tflops = flops / (attn_mean * 1e-3) / 1e12
+    app_gbs = append_bytes(w) / (app_mean * 1e-3) / 1e9
+    traffic = profiled_traffic()
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": step_mean, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: N(0,1)*0.5 rounded to bf16 (seed 1 + rank); stands in for projected Q/K/V of "
+                "832x640 clips",
+        "config": config_dict(w, world),
+        "latent_frames_per_s_per_layer": world * w.chunk_frames / (step_mean * 1e-3),
+        "pct_bf16_peak": 100.0 * attn_tflops / peak_tc,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak_tc, "unit": "TFLOP/s",
+                     "frac": attn_tflops / peak_tc, "traffic": traffic,
+                     "kernel": "attn_fwd_tc<128> (rtr_attn_frame_causal)",
+                     "peak_source": f"{peaks.get('source')} bf16_tflops (burst cuBLAS)",
+                     "flops_per_launch": flops, "ms_per_launch": attn_mean},
+        "cache_update": {"kernel": "kv_scatter (rtr_kvcache_append_frame)", "bytes_per_launch": append_bytes(w),
+                         "ms_per_launch": app_mean, "achieved_gbs": app_gbs, "peak_gbs": peak_hbm,
+                         "frac": app_gbs / peak_hbm, "peak_source": f"{peaks.get('source')} hbm_gbs"},
+        "e2e": {"value": world * flops / (e2e_mean * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(3 * hq.numel() * 2), "d2h_bytes_per_step": int(ho.numel() * 2),
+                "ms_per_step": e2e_mean},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+        "when": datetime.datetime.utcnow().isoformat() + "Z",
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        o = oracle_cache_for(w, x)
+        fl, dt, rows = time_oracle(w, x, o, 12.0)
+        line["cpu_baseline"] = cpu_baseline_entry(fl, dt, rows, w)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,461 @@
+// api.cu -- host side of librtr: the C ABI declared in include/rtr.h.
+//
+// Owns the KV-cache and cross-attention buffers, keeps the host-side index
+// maps of the reference-preserving rolling cache (papernotes.org note "DiT as
+// Real-Time Rerenderer", Method > Key Designs 4), validates every argument
+// before anything is enqueued, turns the cache state into the list of key runs
+// the attention kernels read, and launches the kernels.  No compute happens
+// here and there is no host fallback: every data operation is a kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <utility>
+#include <vector>
+
+#include "internal.h"
+#include "rtr.h"
+
+namespace rtr {
+
+// ------------------------------------------------------------------ tensor maps
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = false;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) return;
+        ok = cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+};
+
+bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elt_size(rtr_dtype dt) { return dt == RTR_BF16 ? 2 : 4; }
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, uint64_t outer,
+                    uint32_t box_mid, uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || !aligned16(base)) return false;
+    cuuint64_t dims[3] = {d, mid, outer};
+    cuuint64_t strides[2] = {d * 2, mid * d * 2};
+    cuuint32_t box[3] = {64, box_mid, box_outer};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace rtr
+
+using namespace rtr;
+
+// ------------------------------------------------------------------ handles
+struct rtr_kvcache {
+    int layers, heads, head_dim, k, R, W;
+    rtr_dtype dt;
+    int device;
+    long long rows;          // (R + W) * k rows per head
+    size_t layer_bytes;      // heads * rows * head_dim * elt
+    char *kbuf = nullptr, *vbuf = nullptr;
+    std::vector<int> ref_valid, count;
+    std::vector<long long> g;
+    std::vector<CUtensorMap> tmk, tmv;
+};
+
+struct rtr_xattn {
+    int layers, heads, head_dim, max_text;
+    rtr_dtype dt;
+    int device;
+    size_t layer_bytes;
+    char *kbuf = nullptr, *vbuf = nullptr;
+    std::vector<int> n_text;
+    std::vector<CUtensorMap> tmk, tmv;
+};
+
+namespace {
+
+bool shape_ok(int heads, int head_dim) { return heads >= 1 && (head_dim == 64 || head_dim == 128); }
+
+rtr_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return RTR_OK;
+    if (e == cudaErrorMemoryAllocation) return RTR_E_NOMEM;
+    return RTR_E_CUDA;
+}
+
+float resolve_scale(float scale, int head_dim) { return scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim); }
+
+// Launch the attention for a problem; picks the kernel for the element type.
+rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0, const CUtensorMap *tm_v0,
+                         int device, cudaStream_t s) {
+    if (pb.nq == 0) return RTR_OK;
+    for (int i = 0; i < pb.nseg; ++i)
+        if (pb.seg[i].len <= 0) return RTR_E_INVAL;
+    if (pb.nseg < 1) return RTR_E_INVAL;
+    cudaError_t e;
+    if (dt == RTR_BF16) {
+        unsigned *st = device_status_ptr(device);
+        if (!st) return RTR_E_CUDA;
+        e = launch_attn_bf16(pb, tm_k0, tm_v0, st, s);
+    } else {
+        e = launch_attn_f32(pb, s);
+    }
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *rtr_status_string(rtr_status s) {
+    switch (s) {
+        case RTR_OK: return "RTR_OK";
+        case RTR_E_INVAL: return "RTR_E_INVAL: invalid argument";
+        case RTR_E_NOMEM: return "RTR_E_NOMEM: device allocation failed";
+        case RTR_E_STATE: return "RTR_E_STATE: call not valid in the current state";
+        case RTR_E_CUDA: return "RTR_E_CUDA: CUDA call failed";
+        case RTR_E_TIMEOUT: return "RTR_E_TIMEOUT: a kernel's bounded wait expired";
+        case RTR_E_UNSUPPORTED: return "RTR_E_UNSUPPORTED: not implemented";
+    }
+    return "unknown rtr_status";
+}
+
+const char *rtr_build_info(void) {
+    return "librtr: sm_100a tcgen05/TMEM/TMA frame-causal attention, fp32 CUDA-core path, "
+           "vectorised KV-cache scatter";
+}
+
+rtr_status rtr_kvcache_create(int layers, int heads, int head_dim, int k, int ref_frames, int window_frames,
+                              rtr_dtype dt, int device, rtr_kvcache **out) {
+    if (!out) return RTR_E_INVAL;
+    *out = nullptr;
+    if (layers < 1 || !shape_ok(heads, head_dim) || k < 1 || ref_frames < 0 || window_frames < 1 ||
+        (dt != RTR_BF16 && dt != RTR_F32) || device < 0)
+        return RTR_E_INVAL;
+    const long long rows = (long long)(ref_frames + window_frames) * k;
+    if (rows > (1ll << 30) || (long long)heads * rows * head_dim >= (1ll << 40)) return RTR_E_INVAL;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    rtr_kvcache *c = new (std::nothrow) rtr_kvcache();
+    if (!c) return RTR_E_NOMEM;
+    c->layers = layers; c->heads = heads; c->head_dim = head_dim; c->k = k;
+    c->R = ref_frames; c->W = window_frames; c->dt = dt; c->device = device;
+    c->rows = rows;
+    c->layer_bytes = (size_t)heads * rows * head_dim * elt_size(dt);
+    const size_t total = c->layer_bytes * layers;
+    if (cudaMalloc(&c->kbuf, total) != cudaSuccess || cudaMalloc(&c->vbuf, total) != cudaSuccess) {
+        cudaGetLastError();
+        if (c->kbuf) cudaFree(c->kbuf);
+        delete c;
+        return RTR_E_NOMEM;
+    }
+    if (cudaMemset(c->kbuf, 0, total) != cudaSuccess || cudaMemset(c->vbuf, 0, total) != cudaSuccess) {
+        cudaFree(c->kbuf); cudaFree(c->vbuf); delete c;
+        return RTR_E_CUDA;
+    }
+    c->ref_valid.assign(layers, 0);
+    c->count.assign(layers, 0);
+    c->g.assign(layers, 0);
+    if (dt == RTR_BF16) {
+        c->tmk.resize(layers);
+        c->tmv.resize(layers);
+        for (int l = 0; l < layers; ++l) {
+            if (!make_tmap_bf16(&c->tmk[l], c->kbuf + l * c->layer_bytes, head_dim, rows, heads, 128, 1) ||
+                !make_tmap_bf16(&c->tmv[l], c->vbuf + l * c->layer_bytes, head_dim, rows, heads, 128, 1)) {
+                cudaFree(c->kbuf); cudaFree(c->vbuf); delete c;
+                return RTR_E_CUDA;
+            }
+        }
+    }
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        cudaFree(c->kbuf); cudaFree(c->vbuf); delete c;
+        return RTR_E_CUDA;
+    }
+    *out = c;
+    return RTR_OK;
+}
+
+void rtr_kvcache_destroy(rtr_kvcache *c) {
+    if (!c) return;
+    DeviceGuard dg(c->device);
+    cudaDeviceSynchronize();
+    cudaFree(c->kbuf);
+    cudaFree(c->vbuf);
+    delete c;
+}
+
+rtr_status rtr_kvcache_set_reference(rtr_kvcache *c, int layer, const void *k_ref, const void *v_ref,
+                                     rtr_stream_t stream) {
+    if (!c || layer < 0 || layer >= c->layers || !aligned16(k_ref) || !aligned16(v_ref)) return RTR_E_INVAL;
+    if (c->R == 0) return RTR_E_STATE;
+    DeviceGuard dg(c->device);
+    ScatterArgs a;
+    a.src_k = k_ref; a.src_v = v_ref;
+    a.dst_k = c->kbuf + layer * c->layer_bytes;
+    a.dst_v = c->vbuf + layer * c->layer_bytes;
+    a.n_tok = c->R * c->k; a.heads = c->heads; a.row_bytes = c->head_dim * (int)elt_size(c->dt);
+    a.k_frame = c->k; a.first_slot = 0; a.slot_mod = c->R; a.slot_off = 0;
+    a.rows_per_head = c->rows;
+    rtr_status st = cuda_status(launch_kv_scatter(a, (cudaStream_t)stream));
+    if (st == RTR_OK) c->ref_valid[layer] = 1;
+    return st;
+}
+
+rtr_status rtr_kvcache_clear_reference(rtr_kvcache *c, int layer) {
+    if (!c || layer < -1 || layer >= c->layers) return RTR_E_INVAL;
+    for (int l = 0; l < c->layers; ++l)
+        if (layer == -1 || l == layer) c->ref_valid[l] = 0;
+    return RTR_OK;
+}
+
+rtr_status rtr_kvcache_append_frame(rtr_kvcache *c, int layer, const void *k_new, const void *v_new, int n_frames,
+                                    rtr_stream_t stream) {
+    if (!c || layer < 0 || layer >= c->layers || !aligned16(k_new) || !aligned16(v_new)) return RTR_E_INVAL;
+    if (n_frames < 1 || n_frames > c->W) return RTR_E_INVAL;
+    DeviceGuard dg(c->device);
+    ScatterArgs a;
+    a.src_k = k_new; a.src_v = v_new;
+    a.dst_k = c->kbuf + layer * c->layer_bytes;
+    a.dst_v = c->vbuf + layer * c->layer_bytes;
+    a.n_tok = n_frames * c->k; a.heads = c->heads; a.row_bytes = c->head_dim * (int)elt_size(c->dt);
+    a.k_frame = c->k; a.first_slot = (int)(c->g[layer] % c->W); a.slot_mod = c->W; a.slot_off = c->R;
+    a.rows_per_head = c->rows;
+    rtr_status st = cuda_status(launch_kv_scatter(a, (cudaStream_t)stream));
+    if (st == RTR_OK) {
+        c->g[layer] += n_frames;
+        c->count[layer] = std::min(c->W, c->count[layer] + n_frames);
+    }
+    return st;
+}
+
+rtr_status rtr_kvcache_retain_last(rtr_kvcache *c, int layer, int n_frames) {
+    if (!c || layer < -1 || layer >= c->layers || n_frames < 0) return RTR_E_INVAL;
+    for (int l = 0; l < c->layers; ++l)
+        if (layer == -1 || l == layer) c->count[l] = std::min(c->count[l], n_frames);
+    return RTR_OK;
+}
+
+rtr_status rtr_kvcache_get_index_map(const rtr_kvcache *c, int layer, int32_t *slot_frame, int32_t *ref_valid,
+                                     int64_t *frames_appended, int32_t *count) {
+    if (!c || layer < 0 || layer >= c->layers) return RTR_E_INVAL;
+    const long long g = c->g[layer];
+    const int cnt = c->count[layer];
+    if (slot_frame) {
+        for (int s = 0; s < c->W; ++s) slot_frame[s] = -1;
+        for (long long f = g - cnt; f < g; ++f) slot_frame[f % c->W] = (int32_t)f;
+    }
+    if (ref_valid) *ref_valid = c->ref_valid[layer];
+    if (frames_appended) *frames_appended = g;
+    if (count) *count = cnt;
+    return RTR_OK;
+}
+
+rtr_status rtr_kvcache_device_ptrs(const rtr_kvcache *c, int layer, void **k, void **v) {
+    if (!c || layer < 0 || layer >= c->layers || !k || !v) return RTR_E_INVAL;
+    *k = c->kbuf + layer * c->layer_bytes;
+    *v = c->vbuf + layer * c->layer_bytes;
+    return RTR_OK;
+}
+
+rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q, const void *k_cur,
+                                 const void *v_cur, int n_cur_frames, void *out, float scale, rtr_stream_t stream) {
+    if (!c || layer < 0 || layer >= c->layers || n_cur_frames < 1) return RTR_E_INVAL;
+    if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out)) return RTR_E_INVAL;
+    const long long nq = (long long)n_cur_frames * c->k;
+    if (nq > (1ll << 30)) return RTR_E_INVAL;
+    // Physical row intervals of the cached keys: the reference slot and the
+    // held window frames.  Every cached key is visible to every chunk query,
+    // so adjacent intervals merge and their order is free.
+    std::vector<std::pair<long long, long long>> iv;
+    if (c->ref_valid[layer] && c->R > 0) iv.push_back({0, (long long)c->R * c->k});
+    const long long g = c->g[layer];
+    for (long long f = g - c->count[layer]; f < g; ++f) {
+        const long long s = f % c->W;
+        iv.push_back({(c->R + s) * c->k, (c->R + s + 1) * c->k});
+    }
+    std::sort(iv.begin(), iv.end());
+    std::vector<std::pair<long long, long long>> merged;
+    for (auto &x : iv) {
+        if (!merged.empty() && merged.back().second == x.first)
+            merged.back().second = x.second;
+        else
+            merged.push_back(x);
+    }
+    if (merged.size() > (size_t)kMaxSegs - 1) return RTR_E_UNSUPPORTED;   // cannot happen: <= 3 runs
+    AttnProblem pb;
+    memset(&pb, 0, sizeof(pb));
+    pb.nq = (int)nq; pb.heads = c->heads; pb.head_dim = c->head_dim; pb.kpf = c->k;
+    for (auto &x : merged) pb.seg[pb.nseg++] = KvSeg{0, (int)x.first, (int)(x.second - x.first), 0};
+    pb.seg[pb.nseg++] = KvSeg{1, 0, (int)nq, 1};
+    pb.scale = resolve_scale(scale, c->head_dim);
+    pb.q = q; pb.o = out;
+    pb.k0 = c->kbuf + layer * c->layer_bytes; pb.v0 = c->vbuf + layer * c->layer_bytes; pb.rows0 = c->rows;
+    pb.k1 = k_cur; pb.v1 = v_cur; pb.rows1 = nq;
+    DeviceGuard dg(c->device);
+    const CUtensorMap *tk = c->dt == RTR_BF16 ? &c->tmk[layer] : nullptr;
+    const CUtensorMap *tv = c->dt == RTR_BF16 ? &c->tmv[layer] : nullptr;
+    return run_attention(pb, c->dt, tk, tv, c->device, (cudaStream_t)stream);
+}
+
+rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k, const void *v, int n_tokens, int heads,
+                                         int head_dim, int k_per_frame, rtr_dtype dt, void *out, float scale,
+                                         int device, rtr_stream_t stream) {
+    if (n_tokens < 0 || !shape_ok(heads, head_dim) || k_per_frame < 1 || (dt != RTR_BF16 && dt != RTR_F32) ||
+        device < 0)
+        return RTR_E_INVAL;
+    if (n_tokens == 0) return RTR_OK;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return RTR_E_INVAL;
+    if (n_tokens > (1 << 30)) return RTR_E_INVAL;
+    AttnProblem pb;
+    memset(&pb, 0, sizeof(pb));
+    pb.nq = n_tokens; pb.heads = heads; pb.head_dim = head_dim; pb.kpf = k_per_frame;
+    pb.nseg = 1;
+    pb.seg[0] = KvSeg{1, 0, n_tokens, 1};
+    pb.scale = resolve_scale(scale, head_dim);
+    pb.q = q; pb.o = out; pb.k1 = k; pb.v1 = v; pb.rows1 = n_tokens;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    return run_attention(pb, dt, nullptr, nullptr, device, (cudaStream_t)stream);
+}
+
+rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_text, rtr_dtype dt, int device,
+                                rtr_xattn **out) {
+    if (!out) return RTR_E_INVAL;
+    *out = nullptr;
+    if (layers < 1 || !shape_ok(heads, head_dim) || max_text < 1 || max_text > (1 << 24) ||
+        (dt != RTR_BF16 && dt != RTR_F32) || device < 0)
+        return RTR_E_INVAL;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    rtr_xattn *x = new (std::nothrow) rtr_xattn();
+    if (!x) return RTR_E_NOMEM;
+    x->layers = layers; x->heads = heads; x->head_dim = head_dim; x->max_text = max_text;
+    x->dt = dt; x->device = device;
+    x->layer_bytes = (size_t)heads * max_text * head_dim * elt_size(dt);
+    const size_t total = x->layer_bytes * layers;
+    if (cudaMalloc(&x->kbuf, total) != cudaSuccess || cudaMalloc(&x->vbuf, total) != cudaSuccess) {
+        cudaGetLastError();
+        if (x->kbuf) cudaFree(x->kbuf);
+        delete x;
+        return RTR_E_NOMEM;
+    }
+    if (cudaMemset(x->kbuf, 0, total) != cudaSuccess || cudaMemset(x->vbuf, 0, total) != cudaSuccess) {
+        cudaFree(x->kbuf); cudaFree(x->vbuf); delete x;
+        return RTR_E_CUDA;
+    }
+    x->n_text.assign(layers, 0);
+    if (dt == RTR_BF16) {
+        x->tmk.resize(layers);
+        x->tmv.resize(layers);
+        for (int l = 0; l < layers; ++l) {
+            if (!make_tmap_bf16(&x->tmk[l], x->kbuf + l * x->layer_bytes, head_dim, max_text, heads, 128, 1) ||
+                !make_tmap_bf16(&x->tmv[l], x->vbuf + l * x->layer_bytes, head_dim, max_text, heads, 128, 1)) {
+                cudaFree(x->kbuf); cudaFree(x->vbuf); delete x;
+                return RTR_E_CUDA;
+            }
+        }
+    }
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        cudaFree(x->kbuf); cudaFree(x->vbuf); delete x;
+        return RTR_E_CUDA;
+    }
+    *out = x;
+    return RTR_OK;
+}
+
+void rtr_crossattn_destroy(rtr_xattn *x) {
+    if (!x) return;
+    DeviceGuard dg(x->device);
+    cudaDeviceSynchronize();
+    cudaFree(x->kbuf);
+    cudaFree(x->vbuf);
+    delete x;
+}
+
+rtr_status rtr_crossattn_set_text(rtr_xattn *x, int layer, const void *k_text, const void *v_text, int n_text,
+                                  rtr_stream_t stream) {
+    if (!x || layer < 0 || layer >= x->layers || !aligned16(k_text) || !aligned16(v_text)) return RTR_E_INVAL;
+    if (n_text < 1 || n_text > x->max_text) return RTR_E_INVAL;
+    DeviceGuard dg(x->device);
+    ScatterArgs a;
+    a.src_k = k_text; a.src_v = v_text;
+    a.dst_k = x->kbuf + layer * x->layer_bytes;
+    a.dst_v = x->vbuf + layer * x->layer_bytes;
+    a.n_tok = n_text; a.heads = x->heads; a.row_bytes = x->head_dim * (int)elt_size(x->dt);
+    a.k_frame = n_text; a.first_slot = 0; a.slot_mod = 1; a.slot_off = 0;
+    a.rows_per_head = x->max_text;
+    rtr_status st = cuda_status(launch_kv_scatter(a, (cudaStream_t)stream));
+    if (st == RTR_OK) x->n_text[layer] = n_text;
+    return st;
+}
+
+rtr_status rtr_crossattn_reset(rtr_xattn *x) {
+    if (!x) return RTR_E_INVAL;
+    std::fill(x->n_text.begin(), x->n_text.end(), 0);
+    return RTR_OK;
+}
+
+rtr_status rtr_attn_cross(const rtr_xattn *x, int layer, const void *q, int n_q, void *out, float scale,
+                          rtr_stream_t stream) {
+    if (!x || layer < 0 || layer >= x->layers || n_q < 0) return RTR_E_INVAL;
+    if (x->n_text[layer] == 0) return RTR_E_STATE;
+    if (n_q == 0) return RTR_OK;
+    if (!aligned16(q) || !aligned16(out)) return RTR_E_INVAL;
+    AttnProblem pb;
+    memset(&pb, 0, sizeof(pb));
+    pb.nq = n_q; pb.heads = x->heads; pb.head_dim = x->head_dim; pb.kpf = 1;
+    pb.nseg = 1;
+    pb.seg[0] = KvSeg{0, 0, x->n_text[layer], 0};
+    pb.scale = resolve_scale(scale, x->head_dim);
+    pb.q = q; pb.o = out;
+    pb.k0 = x->kbuf + layer * x->layer_bytes; pb.v0 = x->vbuf + layer * x->layer_bytes; pb.rows0 = x->max_text;
+    DeviceGuard dg(x->device);
+    const CUtensorMap *tk = x->dt == RTR_BF16 ? &x->tmk[layer] : nullptr;
+    const CUtensorMap *tv = x->dt == RTR_BF16 ? &x->tmv[layer] : nullptr;
+    return run_attention(pb, x->dt, tk, tv, x->device, (cudaStream_t)stream);
+}
+
+rtr_status rtr_get_device_status(int device, rtr_stream_t stream) {
+    if (device < 0) return RTR_E_INVAL;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    unsigned *p = device_status_ptr(device);
+    if (!p) return RTR_E_CUDA;
+    unsigned h = 0;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RTR_E_CUDA;
+    if (cudaMemcpy(&h, p, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return RTR_E_CUDA;
+    const unsigned zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return RTR_E_CUDA;
+    return h == 0 ? RTR_OK : (rtr_status)h;
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// internal.h -- declarations shared by the host side of librtr and its
+// kernels (not part of the public C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "rtr.h"
+
+namespace rtr {
+
+// One contiguous run of keys the query rows attend to.
+//   src 0: head-major source [heads][rows][d] (KV cache, text cache)
+//   src 1: token-major source [rows][heads][d] (current chunk, prefill
+//          sequence)
+//   causal: key j of the run (0-based) is visible to query row i (0-based)
+//          iff floor(j / kpf) <= floor(i / kpf); the run and the query rows
+//          start on the same frame boundary.  Otherwise every key is visible.
+struct KvSeg {
+    int src;
+    int row0;
+    int len;
+    int causal;
+};
+
+constexpr int kMaxSegs = 4;
+
+// Work description shared by the tensor-core and the fp32 attention kernels.
+struct AttnProblem {
+    int nq;          // query rows (token-major [nq][heads][d])
+    int heads;
+    int head_dim;
+    int kpf;         // tokens per latent frame for causal runs
+    int nseg;
+    KvSeg seg[kMaxSegs];
+    float scale;     // multiplies q.k
+    // raw pointers (fp32 path) / bases for the tensor maps (bf16 path)
+    const void *q;
+    void *o;
+    const void *k0, *v0;   // head-major source
+    long long rows0;       // rows per head of the head-major source
+    const void *k1, *v1;   // token-major source
+    long long rows1;       // rows of the token-major source
+};
+
+// Kernel launchers; return cudaSuccess or the launch error.
+cudaError_t launch_attn_bf16(const AttnProblem &p, const CUtensorMap *tm_k0, const CUtensorMap *tm_v0,
+                             unsigned *status, cudaStream_t s);
+cudaError_t launch_attn_f32(const AttnProblem &p, cudaStream_t s);
+
+// Copy n_tok rows of [n_tok][heads][d] into a head-major buffer
+// [heads][rows_per_head][d]: token t of frame f = t / k_frame goes to row
+// ((first_slot + f) mod slot_mod + slot_off) * k_frame + t mod k_frame.
+// K and V move in one launch.
+struct ScatterArgs {
+    const void *src_k, *src_v;
+    void *dst_k, *dst_v;
+    int n_tok, heads, row_bytes, k_frame;
+    int first_slot, slot_mod, slot_off;
+    long long rows_per_head;
+};
+cudaError_t launch_kv_scatter(const ScatterArgs &a, cudaStream_t s);
+
+// Tensor map for a 3-D tensor of bf16 [outer][mid][d] with a box of
+// (64, box_mid, box_outer) elements and 128-byte swizzle.
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, uint64_t outer,
+                    uint32_t box_mid, uint32_t box_outer);
+
+unsigned *device_status_ptr(int device);
+
+}  // namespace rtr

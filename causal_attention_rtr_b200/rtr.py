@@ -1,0 +1,206 @@
+"""ctypes binding of librtr (``include/rtr.h``): one Python function per C
+entry point, same names and argument order.  Argument marshalling only --
+every step of the path runs in librtr's kernels.  Device buffers may be given
+as torch tensors (their ``data_ptr()`` is passed) or as integers; streams as
+``torch.cuda.Stream`` objects, raw handles or ``None`` (legacy default
+stream).
+
+Importing this module loads ``librtr.so`` and raises ``ImportError`` if it has
+not been built: there is no fallback.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librtr.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "librtr.so is not built; run `python -c 'import __graft_entry__ as g; g.build()'` "
+        "or `python causal_attention_rtr_b200/build.py`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+RTR_OK, RTR_E_INVAL, RTR_E_NOMEM, RTR_E_STATE, RTR_E_CUDA, RTR_E_TIMEOUT, RTR_E_UNSUPPORTED = range(7)
+RTR_BF16, RTR_F32 = 0, 1
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+# (name, restype, argtypes) for every symbol of include/rtr.h
+_SIGNATURES = [
+    ("rtr_status_string", ctypes.c_char_p, [_i]),
+    ("rtr_build_info", ctypes.c_char_p, []),
+    ("rtr_kvcache_create", _i, [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
+    ("rtr_kvcache_destroy", None, [_vp]),
+    ("rtr_kvcache_set_reference", _i, [_vp, _i, _vp, _vp, _vp]),
+    ("rtr_kvcache_clear_reference", _i, [_vp, _i]),
+    ("rtr_kvcache_append_frame", _i, [_vp, _i, _vp, _vp, _i, _vp]),
+    ("rtr_kvcache_retain_last", _i, [_vp, _i, _i]),
+    ("rtr_kvcache_get_index_map", _i, [_vp, _i, ctypes.POINTER(ctypes.c_int32),
+                                       ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.POINTER(ctypes.c_int32)]),
+    ("rtr_kvcache_device_ptrs", _i, [_vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
+    ("rtr_attn_frame_causal", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
+    ("rtr_attn_block_causal_prefill", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
+    ("rtr_crossattn_create", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
+    ("rtr_crossattn_destroy", None, [_vp]),
+    ("rtr_crossattn_set_text", _i, [_vp, _i, _vp, _vp, _i, _vp]),
+    ("rtr_crossattn_reset", _i, [_vp]),
+    ("rtr_attn_cross", _i, [_vp, _i, _vp, _i, _vp, _f, _vp]),
+    ("rtr_get_device_status", _i, [_i, _vp]),
+]
+
+for _name, _res, _args in _SIGNATURES:
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = [s[0] for s in _SIGNATURES]
+
+
+class RtrError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {rtr_status_string(status)}")
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if isinstance(x, ctypes.c_void_p):
+        return x.value
+    raise TypeError(f"cannot pass {type(x).__name__} as a device pointer")
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    if hasattr(s, "cuda_stream"):
+        return s.cuda_stream
+    raise TypeError("stream must be None, an int handle or a torch.cuda.Stream")
+
+
+def _check(st, where):
+    if st != RTR_OK:
+        raise RtrError(st, where)
+    return st
+
+
+def _dtype(dt):
+    if dt in ("bf16", RTR_BF16):
+        return RTR_BF16
+    if dt in ("f32", RTR_F32):
+        return RTR_F32
+    raise ValueError("dtype must be 'bf16' or 'f32'")
+
+
+# ---------------------------------------------------------------- raw calls
+def rtr_status_string(status):
+    return _lib.rtr_status_string(int(status)).decode()
+
+
+def rtr_build_info():
+    return _lib.rtr_build_info().decode()
+
+
+def rtr_kvcache_create(layers, heads, head_dim, k, ref_frames, window_frames, dt, device):
+    h = _vp()
+    _check(_lib.rtr_kvcache_create(layers, heads, head_dim, k, ref_frames, window_frames, _dtype(dt),
+                                   device, ctypes.byref(h)), "rtr_kvcache_create")
+    return h.value
+
+
+def rtr_kvcache_destroy(c):
+    _lib.rtr_kvcache_destroy(c)
+
+
+def rtr_kvcache_set_reference(c, layer, k_ref, v_ref, stream=None):
+    return _check(_lib.rtr_kvcache_set_reference(c, layer, _ptr(k_ref), _ptr(v_ref), _stream(stream)),
+                  "rtr_kvcache_set_reference")
+
+
+def rtr_kvcache_clear_reference(c, layer=-1):
+    return _check(_lib.rtr_kvcache_clear_reference(c, layer), "rtr_kvcache_clear_reference")
+
+
+def rtr_kvcache_append_frame(c, layer, k_new, v_new, n_frames, stream=None):
+    return _check(_lib.rtr_kvcache_append_frame(c, layer, _ptr(k_new), _ptr(v_new), n_frames,
+                                                _stream(stream)), "rtr_kvcache_append_frame")
+
+
+def rtr_kvcache_retain_last(c, layer, n_frames):
+    return _check(_lib.rtr_kvcache_retain_last(c, layer, n_frames), "rtr_kvcache_retain_last")
+
+
+def rtr_kvcache_get_index_map(c, layer, window_frames):
+    """Returns (slot_frame list, ref_valid, frames_appended, count)."""
+    slots = (ctypes.c_int32 * window_frames)()
+    ref = ctypes.c_int32()
+    g = ctypes.c_int64()
+    cnt = ctypes.c_int32()
+    _check(_lib.rtr_kvcache_get_index_map(c, layer, slots, ctypes.byref(ref), ctypes.byref(g),
+                                          ctypes.byref(cnt)), "rtr_kvcache_get_index_map")
+    return list(slots), ref.value, g.value, cnt.value
+
+
+def rtr_kvcache_device_ptrs(c, layer):
+    k, v = _vp(), _vp()
+    _check(_lib.rtr_kvcache_device_ptrs(c, layer, ctypes.byref(k), ctypes.byref(v)), "rtr_kvcache_device_ptrs")
+    return k.value, v.value
+
+
+def rtr_attn_frame_causal(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale=0.0, stream=None):
+    return _check(_lib.rtr_attn_frame_causal(c, layer, _ptr(q), _ptr(k_cur), _ptr(v_cur), n_cur_frames,
+                                             _ptr(out), float(scale), _stream(stream)), "rtr_attn_frame_causal")
+
+
+def rtr_attn_block_causal_prefill(q, k, v, n_tokens, heads, head_dim, k_per_frame, dt, out, scale=0.0,
+                                  device=0, stream=None):
+    return _check(_lib.rtr_attn_block_causal_prefill(_ptr(q), _ptr(k), _ptr(v), n_tokens, heads, head_dim,
+                                                     k_per_frame, _dtype(dt), _ptr(out), float(scale),
+                                                     device, _stream(stream)),
+                  "rtr_attn_block_causal_prefill")
+
+
+def rtr_crossattn_create(layers, heads, head_dim, max_text, dt, device):
+    h = _vp()
+    _check(_lib.rtr_crossattn_create(layers, heads, head_dim, max_text, _dtype(dt), device, ctypes.byref(h)),
+           "rtr_crossattn_create")
+    return h.value
+
+
+def rtr_crossattn_destroy(x):
+    _lib.rtr_crossattn_destroy(x)
+
+
+def rtr_crossattn_set_text(x, layer, k_text, v_text, n_text, stream=None):
+    return _check(_lib.rtr_crossattn_set_text(x, layer, _ptr(k_text), _ptr(v_text), n_text, _stream(stream)),
+                  "rtr_crossattn_set_text")
+
+
+def rtr_crossattn_reset(x):
+    return _check(_lib.rtr_crossattn_reset(x), "rtr_crossattn_reset")
+
+
+def rtr_attn_cross(x, layer, q, n_q, out, scale=0.0, stream=None):
+    return _check(_lib.rtr_attn_cross(x, layer, _ptr(q), n_q, _ptr(out), float(scale), _stream(stream)),
+                  "rtr_attn_cross")
+
+
+def rtr_get_device_status(device=0, stream=None):
+    """Latched device-side status (RTR_OK or RTR_E_TIMEOUT); clears it."""
+    return _lib.rtr_get_device_status(device, _stream(stream))
+
+
+def raw_status(fn_name, *args):
+    """Call a C entry point and return its status without raising (tests of
+    the error paths)."""
+    return getattr(_lib, fn_name)(*args)

@@ -1,0 +1,205 @@
+/*
+ * rtr.h -- C ABI of librtr: frame-causal attention with a reference-preserving
+ * rolling KV cache on NVIDIA B200 (sm_100a).
+ *
+ * The method is RTR-DiT's streaming rerenderer, as described by the
+ * papernotes.org note "DiT as Real-Time Rerenderer: Streaming Video
+ * Stylization with Autoregressive Diffusion Transformer":
+ *
+ *   - Method > Key Designs 2: 3D self-attention under a temporal causal mask,
+ *       Attn(Q,K,V) = softmax(Q K^T / sqrt(d) + M) V,
+ *       M_ij = 0 iff floor(j/k) <= floor(i/k), else -inf,
+ *     d = head dimension, k = spatial tokens per latent frame.
+ *   - Method > Key Designs 4: a fixed-length rolling KV cache (new frames
+ *     appended, oldest evicted) whose reference-image tokens live in a
+ *     resident slot at the front that eviction never touches; a fixed-length
+ *     cross-attention cache that is reinitialised when the text prompt or the
+ *     reference image is switched, while the 3D cache keeps its most recent
+ *     frame and a new reference image is anchored at the front.
+ *   - Method > Key Designs 1: the reference latent is one extra latent frame
+ *     placed before the first frame; text enters through cross-attention;
+ *     TV2V runs without a reference.
+ *
+ * Conventions shared by every call
+ *   - Device tensors are row-major.  Q, K, V and outputs use the layout
+ *     [tokens][heads][head_dim] (what a DiT's QKV projection produces).
+ *   - Element types: RTR_BF16 (bfloat16, arithmetic in fp32 with fp32
+ *     accumulation on the tensor cores) or RTR_F32 (float32 storage, fp32
+ *     arithmetic).  head_dim is 64 or 128.
+ *   - Ownership: the library owns cache and cross-attention buffers; the
+ *     caller owns every q/k/v/out pointer.  Those must be device pointers on
+ *     the handle's device, 16-byte aligned, and stay valid until the work
+ *     enqueued on `stream` has finished.
+ *   - Asynchrony: data work is enqueued on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Host-side cache state (index maps, valid
+ *     flags) changes when the call returns.  Calls on one handle must be
+ *     ordered by the caller (one stream, or events).
+ *   - Errors: arguments are checked before anything is enqueued; a failing
+ *     call returns a status and leaves the handle unchanged.  Nothing aborts.
+ *     Device-side failures (a bounded wait that expired) are latched in a
+ *     per-device status word read by rtr_get_device_status.
+ *   - Not thread-safe per handle; distinct handles may be used concurrently.
+ */
+#ifndef RTR_H
+#define RTR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RTR_OK = 0,
+    RTR_E_INVAL = 1,        /* bad argument (shape, pointer, alignment, range) */
+    RTR_E_NOMEM = 2,        /* device allocation failed */
+    RTR_E_STATE = 3,        /* call not valid in the handle's current state */
+    RTR_E_CUDA = 4,         /* a CUDA runtime/driver call failed */
+    RTR_E_TIMEOUT = 5,      /* a kernel's bounded wait expired (device status) */
+    RTR_E_UNSUPPORTED = 6   /* valid request this build does not implement */
+} rtr_status;
+
+typedef enum { RTR_BF16 = 0, RTR_F32 = 1 } rtr_dtype;
+
+/* Same type as cudaStream_t, spelled without the CUDA headers. */
+typedef struct CUstream_st *rtr_stream_t;
+
+typedef struct rtr_kvcache rtr_kvcache;
+typedef struct rtr_xattn rtr_xattn;
+
+/* Human-readable name of a status code (static storage). */
+const char *rtr_status_string(rtr_status s);
+
+/* ---------------------------------------------------------------------------
+ * Reference-preserving rolling KV cache (Key Designs 4; reference frame from
+ * Key Designs 1).
+ *
+ * Per layer the cache holds K and V, each [heads][(ref_frames +
+ * window_frames) * k][head_dim]: rows [0, ref_frames*k) are the anchored
+ * reference slot, window slot s occupies rows (ref_frames+s)*k ... +k-1.
+ * Frame f (counted from creation) lives in slot f mod window_frames.  All
+ * slots start empty and the reference starts invalid.  Buffers are zeroed at
+ * creation.
+ *
+ * rtr_kvcache_create: layers >= 1, heads >= 1, head_dim in {64, 128}, k >= 1,
+ *   ref_frames >= 0, window_frames >= 1, dt RTR_BF16 or RTR_F32, device a
+ *   CUDA ordinal.  On success *out receives the handle.  RTR_E_NOMEM if the
+ *   device allocation fails.
+ */
+rtr_status rtr_kvcache_create(int layers, int heads, int head_dim, int k,
+                              int ref_frames, int window_frames, rtr_dtype dt,
+                              int device, rtr_kvcache **out);
+
+/* Frees the buffers after synchronising the device.  NULL is ignored. */
+void rtr_kvcache_destroy(rtr_kvcache *c);
+
+/* Anchor (or overwrite in place) layer `layer`'s reference: copies
+ * k_ref / v_ref, each [ref_frames*k][heads][head_dim], into the reference
+ * slot and marks it valid.  The window is untouched.  RTR_E_STATE if the
+ * cache has ref_frames == 0. */
+rtr_status rtr_kvcache_set_reference(rtr_kvcache *c, int layer,
+                                     const void *k_ref, const void *v_ref,
+                                     rtr_stream_t stream);
+
+/* Mark the reference of `layer` (or of every layer if layer == -1) absent:
+ * TV2V, or a switch to a text-only condition.  No data moves. */
+rtr_status rtr_kvcache_clear_reference(rtr_kvcache *c, int layer);
+
+/* Append n_frames latent frames to layer `layer`: k_new / v_new are
+ * [n_frames*k][heads][head_dim].  Frame f = frames_appended + i goes to slot
+ * f mod window_frames, overwriting (evicting) the oldest frame once the
+ * window is full; the reference slot is never written.  Then
+ * frames_appended += n_frames and count = min(window_frames, count +
+ * n_frames).  1 <= n_frames <= window_frames, else RTR_E_INVAL. */
+rtr_status rtr_kvcache_append_frame(rtr_kvcache *c, int layer,
+                                    const void *k_new, const void *v_new,
+                                    int n_frames, rtr_stream_t stream);
+
+/* Condition switch: keep only the n_frames most recent window frames of
+ * `layer` (every layer if layer == -1): count = min(count, n_frames).  The
+ * page keeps one frame as the bridge (n_frames = 1).  Index-map work only. */
+rtr_status rtr_kvcache_retain_last(rtr_kvcache *c, int layer, int n_frames);
+
+/* Host copy of layer `layer`'s index map.  slot_frame (window_frames
+ * entries, may be NULL): frame index held by each slot, -1 if empty.
+ * ref_valid (may be NULL): 1 if a reference is anchored.  frames_appended
+ * (may be NULL): frames appended since creation.  count (may be NULL): frames
+ * currently held. */
+rtr_status rtr_kvcache_get_index_map(const rtr_kvcache *c, int layer,
+                                     int32_t *slot_frame, int32_t *ref_valid,
+                                     int64_t *frames_appended, int32_t *count);
+
+/* Device pointers of layer `layer`'s K and V buffers (layout above), for
+ * inspection and snapshotting.  The library keeps ownership. */
+rtr_status rtr_kvcache_device_ptrs(const rtr_kvcache *c, int layer,
+                                   void **k, void **v);
+
+/* ---------------------------------------------------------------------------
+ * Frame-causal attention of the current chunk (Key Designs 2 and 4).
+ *
+ * The chunk's queries q ([n_cur_frames*k][heads][head_dim]) attend to the
+ * logical key sequence [reference (if anchored) | window frames oldest to
+ * newest | the chunk's own k_cur / v_cur (same layout as q)].  Chunk frame c
+ * sits at logical frame R' + count + c (R' = ref_frames if the reference is
+ * valid, else 0), so under M it sees every cached key and chunk frames
+ * 0..c.  out receives [n_cur_frames*k][heads][head_dim] in the cache's
+ * element type.  scale <= 0 selects 1/sqrt(head_dim).  The cache is not
+ * modified; commit the chunk afterwards with rtr_kvcache_append_frame.
+ * Softmax is a permutation-invariant sum, so the kernel visits cached keys
+ * in physical slot order; only the rounding order differs from the logical
+ * order.
+ */
+rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer,
+                                 const void *q, const void *k_cur,
+                                 const void *v_cur, int n_cur_frames,
+                                 void *out, float scale, rtr_stream_t stream);
+
+/* Block-causal attention over one whole sequence (Key Designs 2: training
+ * sees all frames at once under M).  q, k, v, out: [n_tokens][heads]
+ * [head_dim]; token i belongs to frame floor(i / k_per_frame).  scale <= 0
+ * selects 1/sqrt(head_dim).  n_tokens == 0 is a no-op. */
+rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k,
+                                         const void *v, int n_tokens,
+                                         int heads, int head_dim,
+                                         int k_per_frame, rtr_dtype dt,
+                                         void *out, float scale,
+                                         int device, rtr_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Cross-attention cache for the text condition (Key Designs 1 and 4).
+ * Per layer K and V, each [heads][max_text][head_dim]; starts empty.
+ */
+rtr_status rtr_crossattn_create(int layers, int heads, int head_dim,
+                                int max_text, rtr_dtype dt, int device,
+                                rtr_xattn **out);
+void rtr_crossattn_destroy(rtr_xattn *x);
+
+/* Copy the projected text K / V ([n_text][heads][head_dim]) of `layer` into
+ * the cache and mark it valid with n_text tokens (1 <= n_text <= max_text). */
+rtr_status rtr_crossattn_set_text(rtr_xattn *x, int layer, const void *k_text,
+                                  const void *v_text, int n_text,
+                                  rtr_stream_t stream);
+
+/* Condition switch: mark every layer's text cache empty (no data moves). */
+rtr_status rtr_crossattn_reset(rtr_xattn *x);
+
+/* Unmasked softmax attention of q ([n_q][heads][head_dim]) against layer
+ * `layer`'s text keys; out as q.  RTR_E_STATE if the layer is empty. */
+rtr_status rtr_attn_cross(const rtr_xattn *x, int layer, const void *q,
+                          int n_q, void *out, float scale,
+                          rtr_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Device status: synchronises `stream`, returns the latched device-side
+ * status of `device` (RTR_OK or RTR_E_TIMEOUT) and clears it.
+ */
+rtr_status rtr_get_device_status(int device, rtr_stream_t stream);
+
+/* Library build information (static string). */
+const char *rtr_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RTR_H */

@@ -1,0 +1,91 @@
+"""CPU checks of the C-ABI library: it builds, loads without a GPU, exports
+every function ``include/rtr.h`` declares, the Python binding covers exactly
+those names, and argument validation answers before any device work."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rtr.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rtr_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from causal_attention_rtr_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path), path
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("rtr_kvcache_create", "rtr_kvcache_set_reference", "rtr_kvcache_append_frame",
+                     "rtr_attn_frame_causal", "rtr_attn_block_causal_prefill", "rtr_crossattn_set_text",
+                     "rtr_crossattn_reset"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    handle, path = lib
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in declared_functions():
+        getattr(handle, n)
+
+
+def test_binding_matches_header(lib):
+    from causal_attention_rtr_b200 import rtr
+    assert sorted(rtr.EXPORTED) == declared_functions()
+    for n in rtr.EXPORTED:
+        assert callable(getattr(rtr, n))
+
+
+def test_status_strings(lib):
+    from causal_attention_rtr_b200 import rtr
+    assert rtr.rtr_status_string(rtr.RTR_OK) == "RTR_OK"
+    assert "invalid" in rtr.rtr_status_string(rtr.RTR_E_INVAL)
+    assert "sm_100a" in rtr.rtr_build_info()
+
+
+def test_validation_before_device_work(lib):
+    """Bad shapes are rejected on the host, so these answer without a GPU."""
+    from causal_attention_rtr_b200 import rtr
+    h = ctypes.c_void_p()
+    bad = [
+        (0, 2, 128, 16, 1, 4, 0, 0),      # layers
+        (1, 0, 128, 16, 1, 4, 0, 0),      # heads
+        (1, 2, 96, 16, 1, 4, 0, 0),       # head_dim not 64/128
+        (1, 2, 128, 0, 1, 4, 0, 0),       # k
+        (1, 2, 128, 16, -1, 4, 0, 0),     # ref_frames
+        (1, 2, 128, 16, 1, 0, 0, 0),      # window_frames
+        (1, 2, 128, 16, 1, 4, 7, 0),      # dtype
+        (1, 2, 128, 16, 1, 4, 0, -1),     # device
+    ]
+    for args in bad:
+        st = rtr.raw_status("rtr_kvcache_create", *args, ctypes.byref(h))
+        assert st == rtr.RTR_E_INVAL, args
+        assert h.value is None
+    assert rtr.raw_status("rtr_kvcache_create", 1, 2, 128, 16, 1, 4, 0, 0, None) == rtr.RTR_E_INVAL
+    # null handles
+    assert rtr.raw_status("rtr_kvcache_append_frame", None, 0, None, None, 1, None) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_attn_frame_causal", None, 0, None, None, None, 1, None, 0.0, None) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_kvcache_retain_last", None, 0, 1) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_crossattn_reset", None) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_attn_cross", None, 0, None, 1, None, 0.0, None) == rtr.RTR_E_INVAL
+    # prefill: bad shapes, and n_tokens == 0 is a no-op
+    assert rtr.raw_status("rtr_attn_block_causal_prefill", None, None, None, 10, 2, 100, 4, 0, None, 0.0, 0,
+                          None) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_attn_block_causal_prefill", None, None, None, 0, 2, 128, 4, 0, None, 0.0, 0,
+                          None) == rtr.RTR_OK
+    assert rtr.raw_status("rtr_attn_block_causal_prefill", 16, 16, 16, 10, 2, 128, 0, 0, 16, 0.0, 0,
+                          None) == rtr.RTR_E_INVAL
