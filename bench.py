@@ -37,7 +37,8 @@ if ROOT not in sys.path:
 METRIC = "frame-causal attn TFLOP/s & latent frames/s per layer; % of BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 PROFILE = os.path.join(ROOT, "profiles", "fc_attn_fwd_tc__wan13_layer.md")
-KERNEL_SOURCES = [os.path.join(ROOT, "causal_attention_rtr_b200", "csrc", f) for f in ("attn_tc.cu", "ptx.cuh")]
+KERNEL_SOURCES = [os.path.join(ROOT, "causal_attention_rtr_b200", "csrc", f)
+                  for f in ("attn_tc.cu", "ptx.cuh", "exp2_poly.h", "internal.h")]
 
 
 def parse_args():
@@ -389,7 +390,7 @@ def run_ours(args, rank, world, local_rank):
                 "ms_per_step": e2e_mean},
         "gpu_launches": 2 * K,
         "clocks": clk,
-        "when": datetime.datetime.utcnow().isoformat() + "Z",
+        "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
     }
     if world == 1 and not args.no_cpu_baseline:
         o = oracle_cache_for(w, x)

@@ -11,6 +11,8 @@
 
 #include <algorithm>
 #include <cmath>
+#include <map>
+#include <mutex>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -114,6 +116,40 @@ rtr_status cuda_status(cudaError_t e) {
 
 float resolve_scale(float scale, int head_dim) { return scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim); }
 
+int sm_count(int device) {
+    static int cache[64] = {};
+    if (device < 0 || device >= 64) return 148;
+    if (!cache[device]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) n = 148;
+        cache[device] = n;
+    }
+    return cache[device];
+}
+
+// Scratch for the partial results of split attention units, one buffer per
+// (device, stream) so that calls on different streams never share it.  Grown
+// on demand (cudaFree synchronises the device, so no kernel still uses the old
+// buffer) and kept until the process exits.
+void *stream_workspace(int device, cudaStream_t s, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<int, cudaStream_t>, std::pair<void *, size_t>> ws;
+    std::lock_guard<std::mutex> lock(mu);
+    auto &w = ws[{device, s}];
+    if (w.second < bytes) {
+        if (w.first) cudaFree(w.first);
+        w.first = nullptr;
+        w.second = 0;
+        if (cudaMalloc(&w.first, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            w.first = nullptr;
+            return nullptr;
+        }
+        w.second = bytes;
+    }
+    return w.first;
+}
+
 // Launch the attention for a problem; picks the kernel for the element type.
 rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0, const CUtensorMap *tm_v0,
                          int device, cudaStream_t s) {
@@ -125,7 +161,11 @@ rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0
     if (dt == RTR_BF16) {
         unsigned *st = device_status_ptr(device);
         if (!st) return RTR_E_CUDA;
-        e = launch_attn_bf16(pb, tm_k0, tm_v0, st, s);
+        AttnPlan plan;
+        plan_attn_bf16(pb, sm_count(device), plan);
+        void *scratch = stream_workspace(device, s, plan.scratch_bytes);
+        if (!scratch) return RTR_E_NOMEM;
+        e = launch_attn_bf16(pb, plan, tm_k0, tm_v0, st, scratch, s);
     } else {
         e = launch_attn_f32(pb, s);
     }

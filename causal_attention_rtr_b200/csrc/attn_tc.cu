@@ -12,30 +12,54 @@
 // never loaded, fully visible tiles take no mask work, and only tiles that
 // straddle a frame boundary or a run's end mask element-wise.
 //
-// Structure of one CTA (one head, 256 query rows = two 128-row tiles Q0, Q1):
-//   warp 0      TMA producer: Q0/Q1 once, then K_j, V_j into a 4-slot ring
+// Work unit: one head x 256 query rows (two 128-row tiles Q0, Q1 sharing one
+// K/V stream).  The kernel is persistent, one CTA per SM.  Units are ordered
+// largest first; CTA c takes units c, c+G, c+2G, ... for as many full rounds as
+// there are units for every CTA, then an equal share of the remaining units'
+// key tiles.  A unit split across CTAs writes an unnormalised fp32 partial
+// (O, running max, row sum) to scratch and attn_combine merges the parts.
+// Full rounds start every CTA at key tile 0 of a unit, so CTAs that work on
+// the same head sweep its cache together and share it through L2.
+//
+// One CTA, 384 threads:
+//   warp 0      TMA producer: Q0/Q1 per unit, then K_j, V_j into a 4-slot ring
 //   warp 1      tcgen05 issuer (one thread): S_i = Q_i K_j^T into TMEM,
 //               O_i += P_i V_j with P_i read from TMEM (the "A in tensor
 //               memory" form), commits to mbarriers
 //   warps 4-7   softmax for Q0, warps 8-11 softmax for Q1: one thread per
 //               query row reads its S row from TMEM, online softmax in fp32
-//               (exp2 domain, rescale of O only when the running max grows by
-//               more than 2^8 -- exact after the final division), writes P
+//               (exp2 domain; O is rescaled only when the running max grows
+//               by more than 2^8 -- exact after the final division), writes P
 //               as bf16 back over its S columns, and finally normalises O and
-//               stores it with TMA.
+//               stores it with TMA (or writes the fp32 partial).
 // The two softmax groups ping-pong: while one works on its S tile the tensor
-// core runs the other tile's QK^T or PV.
+// core runs the other tile's QK^T or PV.  Part of the exponentials run as a
+// polynomial on the FMA pipe (exp2_poly) so that the special-function unit
+// is not the bottleneck.
 //
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 // Shared memory: Q0, Q1 and 4 K/V slots, each 128 rows x D bf16 stored as D/64
 // boxes of 128 rows x 128 bytes with the 128-byte swizzle that TMA writes and
 // the tcgen05 descriptors read.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
-#include <cstdint>
 
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "exp2_poly.h"
 #include "internal.h"
 #include "ptx.cuh"
+
+#ifndef RTR_REGS_LOW
+#define RTR_REGS_LOW 88      // producer / MMA warpgroup after setmaxnreg
+#endif
+#define RTR_REGS_HIGH (168 + (168 - RTR_REGS_LOW) / 2)   // each softmax warpgroup
+#ifndef RTR_EXP2_POLY_PER8
+#define RTR_EXP2_POLY_PER8 0   // of every 8 scores, how many use exp2_poly (0 measured fastest so far)
+#endif
 
 namespace rtr {
 
@@ -45,6 +69,7 @@ namespace {
 
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per tile
+constexpr int kPairRows = 2 * kBM;
 constexpr int kSlots = 4;         // K/V ring depth
 constexpr int kThreads = 384;     // 12 warps
 constexpr uint64_t kWaitNs = 1000000000ull;   // bounded waits: 1 s
@@ -60,6 +85,12 @@ struct TcParams {
     KvSeg seg[kMaxSegs];
     float scale_log2;   // scale * log2(e)
     unsigned *status;
+    // schedule
+    int n_pairs, n_units, grid, full_rounds;
+    long long rem_per_cta, rem_total;
+    float4 *part_o;     // [grid][2][D/4][256]
+    float2 *part_ml;    // [grid][2][256]: running max (log2 units), row sum
+    __nv_bfloat16 *out; // token-major output (combine kernel)
 };
 
 template <int D>
@@ -68,27 +99,138 @@ struct Layout {
     static constexpr int kQ = 0;                            // Q0, Q1
     static constexpr int kKV = 2 * kTileBytes;              // ring slots
     static constexpr int kBars = kKV + kSlots * kTileBytes; // mbarriers
-    // barrier indices
-    static constexpr int bQ = 0, bFull = 1, bEmpty = bFull + kSlots, bS = bEmpty + kSlots,
+    static constexpr int bQ = 0, bQfree = 1, bFull = 2, bEmpty = bFull + kSlots, bS = bEmpty + kSlots,
                          bP = bS + 2, bO = bP + 2, bEpi = bO + 2, bDrain = bEpi + 2, kNumBars = bDrain + 1;
     static constexpr int kMisc = kBars + kNumBars * 8;      // tmem holder, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1 KB alignment
 };
 
-__device__ __forceinline__ int seg_len_for(const TcParams &p, int s, int q_last) {
+// Key tiles of one run for the query pair starting at q0.
+__device__ __forceinline__ int seg_tiles(const TcParams &p, int s, int q0) {
     const KvSeg &g = p.seg[s];
     int len = g.len;
     if (g.causal) {
+        const int q_last = min(q0 + kPairRows - 1, p.nq - 1);
         const int lim = (q_last / p.kpf + 1) * p.kpf;
         len = len < lim ? len : lim;
     }
-    return len;
+    return (len + kBN - 1) / kBN;
+}
+
+__device__ __forceinline__ int pair_tiles(const TcParams &p, int pair) {
+    int t = 0;
+    for (int s = 0; s < p.nseg; ++s) t += seg_tiles(p, s, pair * kPairRows);
+    return t;
+}
+
+// Unit u -> (pair, head), largest pairs (most key tiles) first.
+__device__ __forceinline__ void unit_coords(const TcParams &p, int u, int &pair, int &head) {
+    pair = p.n_pairs - 1 - u / p.heads;
+    head = u % p.heads;
+}
+
+struct Item {
+    int unit, t0, t1, slot;   // slot -1: whole unit (final output); 0/1: partial
+    int T;                    // key tiles of the whole unit
+};
+
+// Deterministic per-CTA work sequence; every role walks the same sequence.
+struct Sched {
+    int r = 0, ru = 0;
+    long long U = 0;
+    bool first_rem = true;
+};
+
+__device__ bool sched_next(const TcParams &p, Sched &s, Item &it) {
+    const int c = blockIdx.x;
+    if (s.r < p.full_rounds) {
+        it.unit = c + s.r * p.grid;
+        int pair, head;
+        unit_coords(p, it.unit, pair, head);
+        it.T = pair_tiles(p, pair);
+        it.t0 = 0;
+        it.t1 = it.T;
+        it.slot = -1;
+        ++s.r;
+        if (s.r == p.full_rounds) s.ru = p.full_rounds * p.grid;
+        return true;
+    }
+    const long long lo = (long long)c * p.rem_per_cta;
+    const long long hi = min(lo + p.rem_per_cta, p.rem_total);
+    while (s.ru < p.n_units && s.U < hi) {
+        int pair, head;
+        unit_coords(p, s.ru, pair, head);
+        const int T = pair_tiles(p, pair);
+        const long long a = max(s.U, lo), b = min(s.U + T, hi);
+        const int u = s.ru;
+        const long long U0 = s.U;
+        ++s.ru;
+        s.U += T;
+        if (a < b) {
+            it.unit = u;
+            it.T = T;
+            it.t0 = (int)(a - U0);
+            it.t1 = (int)(b - U0);
+            it.slot = (it.t0 == 0 && it.t1 == T) ? -1 : (s.first_rem ? 0 : 1);
+            s.first_rem = false;
+            return true;
+        }
+    }
+    return false;
 }
 
 __device__ __forceinline__ void raise_timeout(const TcParams &p, volatile int *abort_flag) {
     *abort_flag = 1;
     atomicExch(p.status, (unsigned)RTR_E_TIMEOUT);
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void set_max_regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <uint32_t N>
+__device__ __forceinline__ void set_max_regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
+// Walk the key runs to the run holding unit tile t: returns the run and the
+// tile's index within it.
+__device__ __forceinline__ void locate_tile(const TcParams &p, int q0, int t, int &s, int &tt) {
+    s = 0;
+    while (s < p.nseg - 1) {
+        const int n = seg_tiles(p, s, q0);
+        if (t < n) break;
+        t -= n;
+        ++s;
+    }
+    tt = t;
+}
+
+// P = exp2(s * scale_log2 - m) for one row of 128 scores, packed to bf16
+// pairs and stored over the row's first 64 TMEM columns; row sums into acc.
+template <bool POLY>
+__device__ __forceinline__ void softmax_probs(const uint32_t (&sr)[128], float sl2, float neg_m, uint32_t tS,
+                                              float (&acc)[8]) {
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c = 32 * q4 + 2 * e;
+            const float x0 = fmaf(__uint_as_float(sr[c]), sl2, neg_m);
+            const float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, neg_m);
+            const bool poly = POLY && (e % 4) < (RTR_EXP2_POLY_PER8 / 2);
+            const float p0 = poly ? exp2_poly(x0) : fast_exp2(x0);
+            const float p1 = poly ? exp2_poly(x1) : fast_exp2(x1);
+            acc[(2 * e) & 7] += p0;
+            acc[(2 * e + 1) & 7] += p1;
+            pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + 16 * q4, pk);
+    }
 }
 
 template <int D>
@@ -106,15 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int head = blockIdx.y;
-    const int q0 = blockIdx.x * 2 * kBM;
-    const int q_last = min(q0 + 2 * kBM - 1, p.nq - 1);
-
-    int T = 0;
-    for (int s = 0; s < p.nseg; ++s) T += (seg_len_for(p, s, q_last) + kBN - 1) / kBN;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(L::bQ), 1);
+        mbar_init(bar(L::bQfree), 2);          // one arrive per softmax group
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(bar(L::bFull + i), 1);
             mbar_init(bar(L::bEmpty + i), 1);
@@ -131,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&p.tm_q);
+        prefetch_tmap(&p.tm_o);
         prefetch_tmap(&p.tm_k0);
         prefetch_tmap(&p.tm_v0);
         prefetch_tmap(&p.tm_k1);
@@ -145,29 +283,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    // Registers: the producer / MMA warpgroup gives up what the softmax
+    // warpgroups take: 4*32*(168-RTR_REGS_LOW) == 8*32*(RTR_REGS_HIGH-168).
+    if (warp < 4) {
+    set_max_regs_dec<RTR_REGS_LOW>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_tx(bar(L::bQ), 2 * L::kTileBytes);
-            for (int i = 0; i < 2; ++i)
-                for (int b = 0; b < NBOX; ++b)
-                    tma_load_3d(sQ + i * L::kTileBytes + b * 16384, &p.tm_q, bar(L::bQ), b * 64, head,
-                                q0 + i * kBM);
-            int n = 0;
+            Sched sc;
+            Item it;
+            int n = 0, k = 0;
             bool ok = true;
-            for (int s = 0; s < p.nseg && ok; ++s) {
-                const KvSeg g = p.seg[s];
-                const int ntile = (seg_len_for(p, s, q_last) + kBN - 1) / kBN;
-                for (int t = 0; t < ntile && ok; ++t) {
-                    const int row = g.row0 + t * kBN;
+            while (ok && sched_next(p, sc, it)) {
+                int pair, head;
+                unit_coords(p, it.unit, pair, head);
+                const int q0 = pair * kPairRows;
+                if (k > 0 && !mbar_wait(bar(L::bQfree), (k - 1) & 1, kWaitNs)) {
+                    raise_timeout(p, abort_flag);
+                    break;
+                }
+                mbar_arrive_tx(bar(L::bQ), 2 * L::kTileBytes);
+                for (int i = 0; i < 2; ++i)
+                    for (int b = 0; b < NBOX; ++b)
+                        tma_load_3d(sQ + i * L::kTileBytes + b * 16384, &p.tm_q, bar(L::bQ), b * 64, head,
+                                    q0 + i * kBM);
+                int s, tt;
+                locate_tile(p, q0, it.t0, s, tt);
+                int ntile = seg_tiles(p, s, q0);
+                for (int t = it.t0; t < it.t1 && ok; ++t) {
+                    while (tt >= ntile) {
+                        ++s;
+                        tt = 0;
+                        ntile = seg_tiles(p, s, q0);
+                    }
+                    const KvSeg g = p.seg[s];
+                    const int row = g.row0 + tt * kBN;
                     for (int kv = 0; kv < 2; ++kv, ++n) {
                         const int slot = n % kSlots, use = n / kSlots;
+                        if (*abort_flag) { ok = false; break; }
                         if (use > 0 && !mbar_wait(bar(L::bEmpty + slot), (use - 1) & 1, kWaitNs)) {
                             raise_timeout(p, abort_flag);
                             ok = false;
                             break;
                         }
-                        if (*abort_flag) { ok = false; break; }
                         const uint32_t dst = sKV + slot * L::kTileBytes;
                         mbar_arrive_tx(bar(L::bFull + slot), L::kTileBytes);
                         const CUtensorMap *map =
@@ -179,7 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                                 tma_load_3d(dst + b * 16384, map, bar(L::bFull + slot), b * 64, head, row);
                         }
                     }
+                    ++tt;
                 }
+                ++k;
             }
         }
         __syncwarp();
@@ -204,56 +364,60 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     mma_ts(tmem + 256 + i * D, tmem + i * 128 + kk * 8, b, idesc_o, (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            int n = 0;
-            bool ok = mbar_wait(bar(L::bQ), 0, kWaitNs);
-            uint32_t kslot = 0;
-            if (ok) {
-                const int slot = n % kSlots;
-                ok = mbar_wait(bar(L::bFull + slot), (n / kSlots) & 1, kWaitNs);
-                if (ok) {
-                    tc_fence_after();
-                    kslot = sKV + slot * L::kTileBytes;
-                    issue_s(0, kslot);
-                    tc_commit(bar(L::bS + 0));
-                    issue_s(1, kslot);
-                    tc_commit(bar(L::bS + 1));
-                    tc_commit(bar(L::bEmpty + slot));
-                    ++n;
-                }
-            }
-            for (int j = 0; j < T && ok; ++j) {
-                const int vs = n % kSlots;
-                ok = mbar_wait(bar(L::bFull + vs), (n / kSlots) & 1, kWaitNs);
+            Sched sc;
+            Item it;
+            int n = 0, k = 0, jj = 0;   // ring loads consumed, items, tiles (S/P phases)
+            bool ok = true;
+            while (ok && sched_next(p, sc, it)) {
+                const int T = it.t1 - it.t0;
+                ok = mbar_wait(bar(L::bQ), k & 1, kWaitNs) && !*abort_flag;
                 if (!ok) break;
-                ++n;
-                const uint32_t vslot = sKV + vs * L::kTileBytes;
-                ok = mbar_wait(bar(L::bP + 0), j & 1, kWaitNs) && !*abort_flag;
+                int slot = n % kSlots;
+                ok = mbar_wait(bar(L::bFull + slot), (n / kSlots) & 1, kWaitNs);
                 if (!ok) break;
                 tc_fence_after();
-                issue_pv(0, vslot, j > 0);
-                if (j == T - 1) tc_commit(bar(L::bO + 0));
-                int ks = -1;
-                if (j + 1 < T) {
-                    ks = n % kSlots;
-                    ok = mbar_wait(bar(L::bFull + ks), (n / kSlots) & 1, kWaitNs);
+                uint32_t kslot = sKV + slot * L::kTileBytes;
+                issue_s(0, kslot);
+                tc_commit(bar(L::bS + 0));
+                issue_s(1, kslot);
+                tc_commit(bar(L::bS + 1));
+                tc_commit(bar(L::bEmpty + slot));
+                ++n;
+                for (int j = 0; j < T; ++j, ++jj) {
+                    const int vs = n % kSlots;
+                    ok = mbar_wait(bar(L::bFull + vs), (n / kSlots) & 1, kWaitNs);
+                    if (!ok) break;
+                    ++n;
+                    const uint32_t vslot = sKV + vs * L::kTileBytes;
+                    ok = mbar_wait(bar(L::bP + 0), jj & 1, kWaitNs) && !*abort_flag;
                     if (!ok) break;
                     tc_fence_after();
-                    kslot = sKV + ks * L::kTileBytes;
-                    issue_s(0, kslot);
-                    tc_commit(bar(L::bS + 0));
+                    issue_pv(0, vslot, j > 0);
+                    if (j == T - 1) tc_commit(bar(L::bO + 0));
+                    int ks = -1;
+                    if (j + 1 < T) {
+                        ks = n % kSlots;
+                        ok = mbar_wait(bar(L::bFull + ks), (n / kSlots) & 1, kWaitNs);
+                        if (!ok) break;
+                        tc_fence_after();
+                        kslot = sKV + ks * L::kTileBytes;
+                        issue_s(0, kslot);
+                        tc_commit(bar(L::bS + 0));
+                    }
+                    ok = mbar_wait(bar(L::bP + 1), jj & 1, kWaitNs) && !*abort_flag;
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(1, vslot, j > 0);
+                    tc_commit(bar(L::bEmpty + vs));
+                    if (j == T - 1) tc_commit(bar(L::bO + 1));
+                    if (j + 1 < T) {
+                        issue_s(1, kslot);
+                        tc_commit(bar(L::bS + 1));
+                        tc_commit(bar(L::bEmpty + ks));
+                        ++n;
+                    }
                 }
-                ok = mbar_wait(bar(L::bP + 1), j & 1, kWaitNs) && !*abort_flag;
-                if (!ok) break;
-                tc_fence_after();
-                issue_pv(1, vslot, j > 0);
-                tc_commit(bar(L::bEmpty + vs));
-                if (j == T - 1) tc_commit(bar(L::bO + 1));
-                if (j + 1 < T) {
-                    issue_s(1, kslot);
-                    tc_commit(bar(L::bS + 1));
-                    tc_commit(bar(L::bEmpty + ks));
-                    ++n;
-                }
+                ++k;
             }
             if (!ok) raise_timeout(p, abort_flag);
             // Drain: every MMA issued above has completed before TMEM is freed.
@@ -261,27 +425,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             mbar_wait(bar(L::bDrain), 0, kWaitNs);
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    }
+    } else {
+        set_max_regs_inc<RTR_REGS_HIGH>();
         // ------------------------------------------------------------ softmax
-        const int i = (warp - 4) >> 2;                  // which query tile
+        const int i = (warp - 4) >> 2;                  // which query tile of the pair
         const int sub = warp & 3;                       // TMEM lane quarter
         const int row_local = sub * 32 + lane;
-        const int q_row = q0 + i * kBM + row_local;
-        const int row_vis_end = (q_row / p.kpf + 1) * p.kpf;
         const uint32_t lane_bits = (uint32_t)(sub * 32) << 16;
         const uint32_t tS = tmem + lane_bits + i * 128;
         const uint32_t tO = tmem + lane_bits + 256 + i * D;
+        const uint32_t sOut = sQ + i * L::kTileBytes;   // Q_i is dead once O_i is final
         const float sl2 = p.scale_log2;
-        float m_run = -INFINITY, l_run = 0.f;
+        Sched sc;
+        Item it;
+        int k = 0, jj = 0;
         bool ok = true;
-        int j = 0;
-        for (int s = 0; s < p.nseg && ok; ++s) {
-            const KvSeg g = p.seg[s];
-            const int ntile = (seg_len_for(p, s, q_last) + kBN - 1) / kBN;
-            const int row_len = g.causal ? min(g.len, row_vis_end) : g.len;
-            for (int t = 0; t < ntile; ++t, ++j) {
-                const int lim = row_len - t * kBN;      // visible columns of this row
-                bool w = !*abort_flag && mbar_wait(bar(L::bS + i), j & 1, kWaitNs);
+        while (ok && sched_next(p, sc, it)) {
+            int pair, head;
+            unit_coords(p, it.unit, pair, head);
+            const int q0 = pair * kPairRows;
+            const int q_row = q0 + i * kBM + row_local;
+            const int row_vis_end = (q_row / p.kpf + 1) * p.kpf;
+            float m_run = -INFINITY, l_run = 0.f;
+            int s, tt;
+            locate_tile(p, q0, it.t0, s, tt);
+            int ntile = seg_tiles(p, s, q0);
+            for (int t = it.t0; t < it.t1; ++t, ++jj, ++tt) {
+                while (tt >= ntile) {
+                    ++s;
+                    tt = 0;
+                    ntile = seg_tiles(p, s, q0);
+                }
+                const KvSeg g = p.seg[s];
+                const int row_len = g.causal ? min(g.len, row_vis_end) : g.len;
+                const int lim = row_len - tt * kBN;     // visible columns of this row
+                bool w = !*abort_flag && mbar_wait(bar(L::bS + i), jj & 1, kWaitNs);
                 w = __all_sync(0xffffffffu, w);
                 if (!w) { ok = false; break; }
                 tc_fence_after();
@@ -291,15 +470,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
                 tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
                 tmem_wait_ld();
-                float *sv = reinterpret_cast<float *>(sr);
-                if (lim < kBN) {
+                // Warp-uniform: the code below holds tcgen05.st.sync.aligned,
+                // which every lane of the warp must execute together.
+                const bool masked = __any_sync(0xffffffffu, lim < kBN);
+                if (masked) {
 #pragma unroll
                     for (int c = 0; c < kBN; ++c)
-                        if (c >= lim) sv[c] = -INFINITY;
+                        if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
                 }
-                float mx = sv[0];
+#define SV(c) __uint_as_float(sr[c])
+                float mx0 = max3f(SV(0), SV(1), SV(2)), mx1 = max3f(SV(3), SV(4), SV(5));
+                float mx2 = max3f(SV(6), SV(7), SV(8)), mx3 = max3f(SV(9), SV(10), SV(11));
 #pragma unroll
-                for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, sv[c]);
+                for (int c = 12; c < 124; c += 8) {
+                    mx0 = max3f(mx0, SV(c + 0), SV(c + 1));
+                    mx1 = max3f(mx1, SV(c + 2), SV(c + 3));
+                    mx2 = max3f(mx2, SV(c + 4), SV(c + 5));
+                    mx3 = max3f(mx3, SV(c + 6), SV(c + 7));
+                }
+                mx0 = max3f(mx0, SV(124), SV(125));
+                mx1 = max3f(mx1, SV(126), SV(127));
+#undef SV
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
                 const float m_new = fmaxf(m_run, mx * sl2);
                 const bool upd = m_new > m_run + 8.0f;
                 float factor = 1.f;
@@ -308,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     m_run = m_new;
                     l_run *= factor;
                 }
-                if (j > 0 && __any_sync(0xffffffffu, upd)) {
+                if (t > it.t0 && __any_sync(0xffffffffu, upd)) {
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
@@ -320,66 +512,83 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     }
                 }
                 const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-                float sum = 0.f;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float p0 = fast_exp2(fmaf(sv[64 * h + 2 * e], sl2, neg_m));
-                        const float p1 = fast_exp2(fmaf(sv[64 * h + 2 * e + 1], sl2, neg_m));
-                        sum += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st32(tS + 32 * h, pk);
-                }
-                l_run += sum;
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                // The polynomial exp2 runs only on tiles without masked
+                // entries (every input finite); ex2 maps -inf to exactly 0.
+                if (masked)
+                    softmax_probs<false>(sr, sl2, neg_m, tS, acc);
+                else
+                    softmax_probs<true>(sr, sl2, neg_m, tS, acc);
+                l_run += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(L::bP + i));
             }
-        }
-        // ------------------------------------------------------------ epilogue
-        const uint32_t sOut = sQ + i * L::kTileBytes;   // Q_i is dead once O_i is final
-        bool w = ok && !*abort_flag && mbar_wait(bar(L::bO + i), 0, kWaitNs);
-        w = __all_sync(0xffffffffu, w);
-        if (w) {
+            if (!ok) break;
+            // -------------------------------------------------------- epilogue
+            bool w = !*abort_flag && mbar_wait(bar(L::bO + i), k & 1, kWaitNs);
+            w = __all_sync(0xffffffffu, w);
+            if (!w) { ok = false; break; }
             tc_fence_after();
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            const int prow = i * kBM + row_local;       // row within the pair
+            if (it.slot < 0) {
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tO + 32 * c, o);
-                tmem_wait_ld();
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(o[8 * t + 0]) * inv, __uint_as_float(o[8 * t + 1]) * inv);
-                    v.y = pack_bf16x2(__uint_as_float(o[8 * t + 2]) * inv, __uint_as_float(o[8 * t + 3]) * inv);
-                    v.z = pack_bf16x2(__uint_as_float(o[8 * t + 4]) * inv, __uint_as_float(o[8 * t + 5]) * inv);
-                    v.w = pack_bf16x2(__uint_as_float(o[8 * t + 6]) * inv, __uint_as_float(o[8 * t + 7]) * inv);
-                    const int col = 32 * c + 8 * t;
-                    const int box = col / 64, cc = (col % 64) / 8;
-                    const uint32_t addr = sOut + box * 16384 + row_local * 128 + ((cc ^ (row_local & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-                                 "r"(v.z), "r"(v.w)
-                                 : "memory");
+                    for (int t4 = 0; t4 < 4; ++t4) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(o[8 * t4 + 0]) * inv, __uint_as_float(o[8 * t4 + 1]) * inv);
+                        v.y = pack_bf16x2(__uint_as_float(o[8 * t4 + 2]) * inv, __uint_as_float(o[8 * t4 + 3]) * inv);
+                        v.z = pack_bf16x2(__uint_as_float(o[8 * t4 + 4]) * inv, __uint_as_float(o[8 * t4 + 5]) * inv);
+                        v.w = pack_bf16x2(__uint_as_float(o[8 * t4 + 6]) * inv, __uint_as_float(o[8 * t4 + 7]) * inv);
+                        const int col = 32 * c + 8 * t4;
+                        const int box = col / 64, cc = (col % 64) / 8;
+                        const uint32_t addr = sOut + box * 16384 + row_local * 128 + ((cc ^ (row_local & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                                     "r"(v.z), "r"(v.w)
+                                     : "memory");
+                    }
                 }
+                fence_proxy_async_smem();
+            } else {
+                // Partial: unnormalised O, running max and row sum, laid out so
+                // that consecutive rows are consecutive float4s.
+                const size_t base = ((size_t)blockIdx.x * 2 + it.slot);
+                float4 *po = p.part_o + base * (D / 4) * kPairRows;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int t4 = 0; t4 < 8; ++t4)
+                        po[(size_t)(8 * c + t4) * kPairRows + prow] =
+                            make_float4(__uint_as_float(o[4 * t4 + 0]), __uint_as_float(o[4 * t4 + 1]),
+                                        __uint_as_float(o[4 * t4 + 2]), __uint_as_float(o[4 * t4 + 3]));
+                }
+                p.part_ml[base * kPairRows + prow] = make_float2(m_run, l_run);
             }
-            fence_proxy_async_smem();
-        } else if (ok) {
-            raise_timeout(p, abort_flag);
-        }
-        mbar_arrive(bar(L::bEpi + i));
-        if (row_local == 0) {
-            const bool all = mbar_wait(bar(L::bEpi + i), 0, kWaitNs);
-            if (all && w && !*abort_flag && q0 + i * kBM < p.nq) {
-                for (int b = 0; b < NBOX; ++b) tma_store_3d(&p.tm_o, sOut + b * 16384, b * 64, head, q0 + i * kBM);
-                bulk_commit();
-                bulk_wait_read0();
+            tc_fence_before();
+            mbar_arrive(bar(L::bEpi + i));
+            if (row_local == 0) {
+                const bool all = mbar_wait(bar(L::bEpi + i), k & 1, kWaitNs);
+                if (!all) raise_timeout(p, abort_flag);
+                if (all && it.slot < 0 && q0 + i * kBM < p.nq) {
+                    for (int b = 0; b < NBOX; ++b)
+                        tma_store_3d(&p.tm_o, sOut + b * 16384, b * 64, head, q0 + i * kBM);
+                    bulk_commit();
+                    bulk_wait_read0();
+                }
+                mbar_arrive(bar(L::bQfree));
             }
+            ++k;
         }
+        if (!ok) raise_timeout(p, abort_flag);
     }
     tc_fence_before();
     __syncthreads();
@@ -389,8 +598,67 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     }
 }
 
+// Merge the partial results of units split across CTAs: one block per unit
+// of the last (shared) round, one thread per query row of the pair.
 template <int D>
-cudaError_t launch_tc(const TcParams &tp, int nq, int heads, cudaStream_t s) {
+__global__ void __launch_bounds__(kPairRows) attn_combine(const __grid_constant__ TcParams p) {
+    const int ru = p.full_rounds * p.grid + blockIdx.x;
+    if (ru >= p.n_units) return;
+    long long U = 0;
+    for (int u = p.full_rounds * p.grid; u < ru; ++u) {
+        int pr, hd;
+        unit_coords(p, u, pr, hd);
+        U += pair_tiles(p, pr);
+    }
+    int pair, head;
+    unit_coords(p, ru, pair, head);
+    const int T = pair_tiles(p, pair);
+    const long long B = p.rem_per_cta;
+    const int c0 = (int)(U / B), c1 = (int)((U + T - 1) / B);
+    if (c0 == c1) return;                           // whole unit: written by its CTA
+    const int row = threadIdx.x;
+    const int q = pair * kPairRows + row;
+    if (q >= p.nq) return;
+    float M = -INFINITY;
+    for (int c = c0; c <= c1; ++c) {
+        const int slot = (c == c0 && U != (long long)c0 * B) ? 1 : 0;
+        M = fmaxf(M, p.part_ml[((size_t)c * 2 + slot) * kPairRows + row].x);
+    }
+    float l = 0.f;
+    float4 acc[D / 4];
+#pragma unroll
+    for (int e = 0; e < D / 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = c0; c <= c1; ++c) {
+        const int slot = (c == c0 && U != (long long)c0 * B) ? 1 : 0;
+        const size_t base = (size_t)c * 2 + slot;
+        const float2 ml = p.part_ml[base * kPairRows + row];
+        const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+        l += w * ml.y;
+        const float4 *po = p.part_o + base * (D / 4) * kPairRows;
+#pragma unroll
+        for (int e = 0; e < D / 4; ++e) {
+            const float4 v = po[(size_t)e * kPairRows + row];
+            acc[e].x += w * v.x;
+            acc[e].y += w * v.y;
+            acc[e].z += w * v.z;
+            acc[e].w += w * v.w;
+        }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)q * p.heads + head) * D);
+#pragma unroll
+    for (int e = 0; e < D / 8; ++e) {
+        uint4 v;
+        v.x = pack_bf16x2(acc[2 * e].x * inv, acc[2 * e].y * inv);
+        v.y = pack_bf16x2(acc[2 * e].z * inv, acc[2 * e].w * inv);
+        v.z = pack_bf16x2(acc[2 * e + 1].x * inv, acc[2 * e + 1].y * inv);
+        v.w = pack_bf16x2(acc[2 * e + 1].z * inv, acc[2 * e + 1].w * inv);
+        dst[e] = v;
+    }
+}
+
+template <int D>
+cudaError_t launch_tc(const TcParams &tp, cudaStream_t s) {
     using L = Layout<D>;
     static int configured_mask = 0;   // per device bit (up to 32 devices)
     int dev = 0;
@@ -400,9 +668,31 @@ cudaError_t launch_tc(const TcParams &tp, int nq, int heads, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         configured_mask |= 1 << dev;
     }
-    dim3 grid((nq + 2 * kBM - 1) / (2 * kBM), heads);
-    attn_fwd_tc<D><<<grid, kThreads, L::kAlloc, s>>>(tp);
-    return cudaGetLastError();
+    attn_fwd_tc<D><<<tp.grid, kThreads, L::kAlloc, s>>>(tp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int rem_units = tp.n_units - tp.full_rounds * tp.grid;
+    if (rem_units > 0 && tp.rem_per_cta < tp.rem_total) {
+        attn_combine<D><<<rem_units, kPairRows, 0, s>>>(tp);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+// Host copy of the device's tile count per pair.
+int host_pair_tiles(const AttnProblem &p, int pair) {
+    int t = 0;
+    const int q0 = pair * kPairRows;
+    for (int s = 0; s < p.nseg; ++s) {
+        int len = p.seg[s].len;
+        if (p.seg[s].causal) {
+            const int q_last = std::min(q0 + kPairRows - 1, p.nq - 1);
+            const int lim = (q_last / p.kpf + 1) * p.kpf;
+            len = std::min(len, lim);
+        }
+        t += (len + kBN - 1) / kBN;
+    }
+    return t;
 }
 
 }  // namespace
@@ -418,8 +708,29 @@ unsigned *device_status_ptr(int device) {
     return ptrs[device];
 }
 
-cudaError_t launch_attn_bf16(const AttnProblem &p, const CUtensorMap *tm_k0, const CUtensorMap *tm_v0,
-                             unsigned *status, cudaStream_t s) {
+// Scheduling of the persistent kernel (mirrors sched_next on the device).
+void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan) {
+    plan.n_pairs = (p.nq + kPairRows - 1) / kPairRows;
+    plan.n_units = plan.n_pairs * p.heads;
+    const int G = std::max(1, sms);
+    plan.full_rounds = plan.n_units / G;
+    long long rem_total = 0;
+    for (int u = plan.full_rounds * G; u < plan.n_units; ++u)
+        rem_total += host_pair_tiles(p, plan.n_pairs - 1 - u / p.heads);
+    plan.rem_total = rem_total;
+    // Share of the remainder per CTA; at least 8 key tiles so that a split
+    // part amortises its Q load and epilogue.
+    long long per = rem_total > 0 ? (rem_total + G - 1) / G : 1;
+    per = std::max<long long>(per, 8);
+    plan.rem_per_cta = per;
+    const int rem_ctas = rem_total > 0 ? (int)((rem_total + per - 1) / per) : 0;
+    plan.grid = plan.full_rounds > 0 ? G : std::max(1, rem_ctas);
+    if (plan.full_rounds > 0 && rem_ctas > G) plan.grid = G;   // cannot happen: per >= rem_total / G
+    plan.scratch_bytes = (size_t)plan.grid * 2 * ((size_t)kPairRows * p.head_dim * 4 + (size_t)kPairRows * 8);
+}
+
+cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const CUtensorMap *tm_k0,
+                             const CUtensorMap *tm_v0, unsigned *status, void *scratch, cudaStream_t s) {
     TcParams tp;
     memset(&tp, 0, sizeof(tp));
     const uint64_t D = (uint64_t)p.head_dim;
@@ -448,8 +759,18 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const CUtensorMap *tm_k0, con
     for (int i = 0; i < p.nseg; ++i) tp.seg[i] = p.seg[i];
     tp.scale_log2 = p.scale * 1.4426950408889634f;
     tp.status = status;
-    if (p.head_dim == 128) return launch_tc<128>(tp, p.nq, p.heads, s);
-    if (p.head_dim == 64) return launch_tc<64>(tp, p.nq, p.heads, s);
+    tp.n_pairs = plan.n_pairs;
+    tp.n_units = plan.n_units;
+    tp.grid = plan.grid;
+    tp.full_rounds = plan.full_rounds;
+    tp.rem_per_cta = plan.rem_per_cta;
+    tp.rem_total = plan.rem_total;
+    const size_t part_o_bytes = (size_t)plan.grid * 2 * kPairRows * p.head_dim * 4;
+    tp.part_o = static_cast<float4 *>(scratch);
+    tp.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(scratch) + part_o_bytes);
+    tp.out = static_cast<__nv_bfloat16 *>(p.o);
+    if (p.head_dim == 128) return launch_tc<128>(tp, s);
+    if (p.head_dim == 64) return launch_tc<64>(tp, s);
     return cudaErrorInvalidValue;
 }
 

@@ -1,0 +1,32 @@
+// exp2_poly.h -- 2^x on the FMA pipe, for part of the softmax exponentials.
+//
+// Method: Cody-Waite style range reduction for base 2 (x = n + f with n the
+// nearest integer, f in [-0.5, 0.5]), a degree-3 polynomial for 2^f, and the
+// exponent n added to the result's exponent field.  The polynomial is the
+// minimax approximation of 2^f on [-0.5, 0.5] in relative error, computed for
+// this library by the Remez exchange algorithm; its maximum relative error is
+// 7.5e-5 (fp32 Horner evaluation), far below the 2^-9 rounding of the bf16
+// probabilities it feeds.  n is taken with the round-to-nearest "magic
+// number" addition 1.5 * 2^23.  Valid for finite x <= 64; inputs below -125
+// are clamped (their result, < 2^-125, is negligible next to the row sum).
+#pragma once
+
+#define RTR_EXP2_C0 0.9999280571937561f
+#define RTR_EXP2_C1 0.6932609677314758f
+#define RTR_EXP2_C2 0.2426111251115799f
+#define RTR_EXP2_C3 0.0551716685295105f
+
+namespace rtr {
+
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;           // 1.5 * 2^23: low mantissa bits hold round(x)
+    const float n = t - 12582912.0f;
+    const float f = x - n;                      // [-0.5, 0.5]
+    float p = fmaf(RTR_EXP2_C3, f, RTR_EXP2_C2);
+    p = fmaf(p, f, RTR_EXP2_C1);
+    p = fmaf(p, f, RTR_EXP2_C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+}  // namespace rtr

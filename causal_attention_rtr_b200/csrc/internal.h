@@ -43,9 +43,20 @@ struct AttnProblem {
     long long rows1;       // rows of the token-major source
 };
 
+// Schedule of the persistent tensor-core kernel for one problem: units are
+// (head, 256-row query pair); full rounds give every CTA one whole unit, the
+// remaining units' key tiles are shared equally (rem_per_cta tiles per CTA).
+struct AttnPlan {
+    int n_pairs, n_units, grid, full_rounds;
+    long long rem_per_cta, rem_total;
+    size_t scratch_bytes;   // partial results of split units
+};
+
+void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan);
+
 // Kernel launchers; return cudaSuccess or the launch error.
-cudaError_t launch_attn_bf16(const AttnProblem &p, const CUtensorMap *tm_k0, const CUtensorMap *tm_v0,
-                             unsigned *status, cudaStream_t s);
+cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const CUtensorMap *tm_k0,
+                             const CUtensorMap *tm_v0, unsigned *status, void *scratch, cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnProblem &p, cudaStream_t s);
 
 // Copy n_tok rows of [n_tok][heads][d] into a head-major buffer

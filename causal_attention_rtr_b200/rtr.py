@@ -12,7 +12,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "librtr.so")
+# RTR_LIBRARY selects another build of the same library (e.g. one compiled
+# with different tuning macros); the default is the in-tree build.
+LIB_PATH = os.environ.get("RTR_LIBRARY", os.path.join(_HERE, "librtr.so"))
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

@@ -17,7 +17,7 @@ class _DevArray:
     """__cuda_array_interface__ view of a library-owned device buffer."""
 
     def __init__(self, ptr, n, typestr):
-        self.__cuda_array_interface__ = {"shape": (n,), "typestr": typestr, "data": (ptr, True),
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": typestr, "data": (ptr, False),
                                          "version": 3, "strides": None}
 
 
