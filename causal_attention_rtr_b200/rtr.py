@@ -46,6 +46,7 @@ _SIGNATURES = [
     ("rtr_kvcache_device_ptrs", _i, [_vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
     ("rtr_attn_frame_causal", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
     ("rtr_attn_block_causal_prefill", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
+    ("rtr_attn_block_causal_prefill_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     ("rtr_crossattn_create", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
     ("rtr_crossattn_destroy", None, [_vp]),
     ("rtr_crossattn_set_text", _i, [_vp, _i, _vp, _vp, _i, _vp]),
@@ -170,6 +171,17 @@ def rtr_attn_block_causal_prefill(q, k, v, n_tokens, heads, head_dim, k_per_fram
                                                      k_per_frame, _dtype(dt), _ptr(out), float(scale),
                                                      device, _stream(stream)),
                   "rtr_attn_block_causal_prefill")
+
+
+def rtr_attn_block_causal_prefill_noalloc(q, k, v, n_tokens, heads, head_dim, k_per_frame, dt, out, scale=0.0,
+                                          device=0, stream=None):
+    """Same as rtr_attn_block_causal_prefill, with its scratch in the
+    library's static device array instead of a buffer it allocates (for
+    callers that cannot allocate device memory)."""
+    return _check(_lib.rtr_attn_block_causal_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), n_tokens, heads,
+                                                             head_dim, k_per_frame, _dtype(dt), _ptr(out),
+                                                             float(scale), device, _stream(stream)),
+                  "rtr_attn_block_causal_prefill_noalloc")
 
 
 def rtr_crossattn_create(layers, heads, head_dim, max_text, dt, device):

@@ -166,6 +166,32 @@ rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k,
                                          void *out, float scale,
                                          int device, rtr_stream_t stream);
 
+/* Block-causal prefill that allocates no device memory.  The paper has no
+ * counterpart: this is a library addition for callers that cannot let a
+ * library allocate -- e.g. a serving process whose device memory is reserved
+ * up front by its own caching allocator, or a frame loop that must not stall
+ * on the device-wide wait of cudaFree when rtr_attn_block_causal_prefill
+ * grows its scratch buffer.
+ *
+ * Same arguments, layouts and results as rtr_attn_block_causal_prefill.  The
+ * scratch (partial results of work split across SMs) lives in a static device
+ * array of RTR_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds
+ * until process exit; a problem whose schedule needs more returns
+ * RTR_E_INVAL (bf16, head_dim 128 on a 148-SM B200 needs 37.6 MiB at most).
+ * The first call on a device looks up the array's device address; make that
+ * first call before any stream capture.  All calls share the array: calls
+ * that overlap on the GPU (different streams or host threads) race and must
+ * be ordered by the caller.  No cudaMalloc, cudaFree or allocating library
+ * routine is called. */
+#define RTR_NOALLOC_SCRATCH_BYTES (40u << 20)
+rtr_status rtr_attn_block_causal_prefill_noalloc(const void *q, const void *k,
+                                                 const void *v, int n_tokens,
+                                                 int heads, int head_dim,
+                                                 int k_per_frame, rtr_dtype dt,
+                                                 void *out, float scale,
+                                                 int device,
+                                                 rtr_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Cross-attention cache for the text condition (Key Designs 1 and 4).
  * Per layer K and V, each [heads][max_text][head_dim]; starts empty.
