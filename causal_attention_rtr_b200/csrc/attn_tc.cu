@@ -48,6 +48,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #include "exp2_poly.h"
 #include "internal.h"
@@ -57,6 +58,9 @@
 #define RTR_REGS_LOW 88      // producer / MMA warpgroup after setmaxnreg
 #endif
 #define RTR_REGS_HIGH (168 + (168 - RTR_REGS_LOW) / 2)   // each softmax warpgroup
+#ifndef RTR_UNIT_ORDER_RATIO
+#define RTR_UNIT_ORDER_RATIO 1.25   // head-major unit order when max/min key tiles per pair <= this
+#endif
 #ifndef RTR_EXP2_POLY_PER8
 #define RTR_EXP2_POLY_PER8 0   // of every 8 scores, how many use exp2_poly (0 measured fastest so far)
 #endif
@@ -72,6 +76,7 @@ constexpr int kBN = 128;          // keys per tile
 constexpr int kPairRows = 2 * kBM;
 constexpr int kSlots = 4;         // K/V ring depth
 constexpr int kThreads = 384;     // 12 warps
+constexpr int kMaxGrid = 160;     // persistent CTAs at most (B200: 148 SMs)
 constexpr uint64_t kWaitNs = 1000000000ull;   // bounded waits: 1 s
 
 struct TcParams {
@@ -85,9 +90,10 @@ struct TcParams {
     KvSeg seg[kMaxSegs];
     float scale_log2;   // scale * log2(e)
     unsigned *status;
-    // schedule
-    int n_pairs, n_units, grid, full_rounds;
-    long long rem_per_cta, rem_total;
+    // schedule: full rounds, then CTA c takes tiles [rem_lo[c], rem_lo[c+1])
+    // of the remaining units' key tiles
+    int n_pairs, n_units, grid, full_rounds, head_major;
+    int rem_lo[kMaxGrid + 1];
     float4 *part_o;     // [grid][2][D/4][256]
     float2 *part_ml;    // [grid][2][256]: running max (log2 units), row sum
     __nv_bfloat16 *out; // token-major output (combine kernel)
@@ -124,10 +130,24 @@ __device__ __forceinline__ int pair_tiles(const TcParams &p, int pair) {
     return t;
 }
 
-// Unit u -> (pair, head), largest pairs (most key tiles) first.
+// Unit u -> (pair, head).  Pairs of similar size: head-major (a head's pairs
+// are consecutive units, so a full round sweeps whole heads together and the
+// shared remainder covers few heads); very unequal pairs (block-causal
+// prefill): largest pairs first across heads, so a round's units are alike.
 __device__ __forceinline__ void unit_coords(const TcParams &p, int u, int &pair, int &head) {
-    pair = p.n_pairs - 1 - u / p.heads;
-    head = u % p.heads;
+    if (p.head_major) {
+        head = u / p.n_pairs;
+        pair = p.n_pairs - 1 - u % p.n_pairs;
+    } else {
+        pair = p.n_pairs - 1 - u / p.heads;
+        head = u % p.heads;
+    }
+}
+
+// Unit of CTA c in full round r: rounds alternate direction so that CTAs that
+// get a larger unit in one round get a smaller one in the next.
+__host__ __device__ __forceinline__ int full_round_unit(int G, int c, int r) {
+    return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
 struct Item {
@@ -145,7 +165,7 @@ struct Sched {
 __device__ bool sched_next(const TcParams &p, Sched &s, Item &it) {
     const int c = blockIdx.x;
     if (s.r < p.full_rounds) {
-        it.unit = c + s.r * p.grid;
+        it.unit = full_round_unit(p.grid, c, s.r);
         int pair, head;
         unit_coords(p, it.unit, pair, head);
         it.T = pair_tiles(p, pair);
@@ -156,8 +176,8 @@ __device__ bool sched_next(const TcParams &p, Sched &s, Item &it) {
         if (s.r == p.full_rounds) s.ru = p.full_rounds * p.grid;
         return true;
     }
-    const long long lo = (long long)c * p.rem_per_cta;
-    const long long hi = min(lo + p.rem_per_cta, p.rem_total);
+    const long long lo = p.rem_lo[c];
+    const long long hi = p.rem_lo[c + 1];
     while (s.ru < p.n_units && s.U < hi) {
         int pair, head;
         unit_coords(p, s.ru, pair, head);
@@ -598,10 +618,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     }
 }
 
-// Merge the partial results of units split across CTAs: one block per unit
-// of the last (shared) round, one thread per query row of the pair.
+// Merge the partial results of units split across CTAs.  Grid: (units of the
+// shared remainder, 4); each block covers 64 query rows of one unit, each
+// thread one row and a quarter of the head dimension.
 template <int D>
-__global__ void __launch_bounds__(kPairRows) attn_combine(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcParams p) {
     const int ru = p.full_rounds * p.grid + blockIdx.x;
     if (ru >= p.n_units) return;
     long long U = 0;
@@ -613,31 +634,43 @@ __global__ void __launch_bounds__(kPairRows) attn_combine(const __grid_constant_
     int pair, head;
     unit_coords(p, ru, pair, head);
     const int T = pair_tiles(p, pair);
-    const long long B = p.rem_per_cta;
-    const int c0 = (int)(U / B), c1 = (int)((U + T - 1) / B);
+    // CTA whose range holds tile x: rem_lo[c] <= x < rem_lo[c+1]
+    auto owner = [&](long long x) {
+        int lo = 0, hi = p.grid - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (p.rem_lo[mid] <= x) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
+    const int c0 = owner(U), c1 = owner(U + T - 1);
     if (c0 == c1) return;                           // whole unit: written by its CTA
-    const int row = threadIdx.x;
+    const int row = blockIdx.y * 64 + (threadIdx.x >> 2);
+    const int quarter = threadIdx.x & 3;            // D/4 columns each
     const int q = pair * kPairRows + row;
     if (q >= p.nq) return;
     float M = -INFINITY;
     for (int c = c0; c <= c1; ++c) {
-        const int slot = (c == c0 && U != (long long)c0 * B) ? 1 : 0;
+        if (p.rem_lo[c] == p.rem_lo[c + 1]) continue;
+        const int slot = (c == c0 && U != p.rem_lo[c0]) ? 1 : 0;
         M = fmaxf(M, p.part_ml[((size_t)c * 2 + slot) * kPairRows + row].x);
     }
+    constexpr int NV = D / 16;                       // float4 per thread
     float l = 0.f;
-    float4 acc[D / 4];
+    float4 acc[NV];
 #pragma unroll
-    for (int e = 0; e < D / 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < NV; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int c = c0; c <= c1; ++c) {
-        const int slot = (c == c0 && U != (long long)c0 * B) ? 1 : 0;
+        if (p.rem_lo[c] == p.rem_lo[c + 1]) continue;
+        const int slot = (c == c0 && U != p.rem_lo[c0]) ? 1 : 0;
         const size_t base = (size_t)c * 2 + slot;
         const float2 ml = p.part_ml[base * kPairRows + row];
         const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
         l += w * ml.y;
         const float4 *po = p.part_o + base * (D / 4) * kPairRows;
 #pragma unroll
-        for (int e = 0; e < D / 4; ++e) {
-            const float4 v = po[(size_t)e * kPairRows + row];
+        for (int e = 0; e < NV; ++e) {
+            const float4 v = po[(size_t)(quarter * NV + e) * kPairRows + row];
             acc[e].x += w * v.x;
             acc[e].y += w * v.y;
             acc[e].z += w * v.z;
@@ -645,9 +678,9 @@ __global__ void __launch_bounds__(kPairRows) attn_combine(const __grid_constant_
         }
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)q * p.heads + head) * D);
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)q * p.heads + head) * D + quarter * (D / 4));
 #pragma unroll
-    for (int e = 0; e < D / 8; ++e) {
+    for (int e = 0; e < NV / 2; ++e) {
         uint4 v;
         v.x = pack_bf16x2(acc[2 * e].x * inv, acc[2 * e].y * inv);
         v.y = pack_bf16x2(acc[2 * e].z * inv, acc[2 * e].w * inv);
@@ -658,7 +691,7 @@ __global__ void __launch_bounds__(kPairRows) attn_combine(const __grid_constant_
 }
 
 template <int D>
-cudaError_t launch_tc(const TcParams &tp, cudaStream_t s) {
+cudaError_t launch_tc(const TcParams &tp, bool has_split, cudaStream_t s) {
     using L = Layout<D>;
     static int configured_mask = 0;   // per device bit (up to 32 devices)
     int dev = 0;
@@ -672,8 +705,8 @@ cudaError_t launch_tc(const TcParams &tp, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int rem_units = tp.n_units - tp.full_rounds * tp.grid;
-    if (rem_units > 0 && tp.rem_per_cta < tp.rem_total) {
-        attn_combine<D><<<rem_units, kPairRows, 0, s>>>(tp);
+    if (rem_units > 0 && has_split) {
+        attn_combine<D><<<dim3(rem_units, kPairRows / 64), 256, 0, s>>>(tp);
         e = cudaGetLastError();
     }
     return e;
@@ -708,24 +741,63 @@ unsigned *device_status_ptr(int device) {
     return ptrs[device];
 }
 
-// Scheduling of the persistent kernel (mirrors sched_next on the device).
+// Scheduling of the persistent kernel (mirrors sched_next on the device):
+// full rounds of one unit per CTA, then the remaining units' key tiles cut
+// into per-CTA ranges sized so that every CTA's total (its full-round units
+// plus its range) is as equal as possible.
 void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan) {
     plan.n_pairs = (p.nq + kPairRows - 1) / kPairRows;
     plan.n_units = plan.n_pairs * p.heads;
-    const int G = std::max(1, sms);
+    const int G = std::max(1, std::min(sms, kMaxGrid));
     plan.full_rounds = plan.n_units / G;
+    std::vector<int> pt(plan.n_pairs);
+    int tmin = 1 << 30, tmax = 0;
+    for (int pr = 0; pr < plan.n_pairs; ++pr) {
+        pt[pr] = host_pair_tiles(p, pr);
+        tmin = std::min(tmin, pt[pr]);
+        tmax = std::max(tmax, pt[pr]);
+    }
+    plan.head_major = (double)tmax <= RTR_UNIT_ORDER_RATIO * (double)tmin ? 1 : 0;
+    auto unit_T = [&](int u) {
+        const int pair = plan.head_major ? plan.n_pairs - 1 - u % plan.n_pairs : plan.n_pairs - 1 - u / p.heads;
+        return pt[pair];
+    };
     long long rem_total = 0;
-    for (int u = plan.full_rounds * G; u < plan.n_units; ++u)
-        rem_total += host_pair_tiles(p, plan.n_pairs - 1 - u / p.heads);
-    plan.rem_total = rem_total;
-    // Share of the remainder per CTA; at least 8 key tiles so that a split
-    // part amortises its Q load and epilogue.
-    long long per = rem_total > 0 ? (rem_total + G - 1) / G : 1;
-    per = std::max<long long>(per, 8);
-    plan.rem_per_cta = per;
-    const int rem_ctas = rem_total > 0 ? (int)((rem_total + per - 1) / per) : 0;
-    plan.grid = plan.full_rounds > 0 ? G : std::max(1, rem_ctas);
-    if (plan.full_rounds > 0 && rem_ctas > G) plan.grid = G;   // cannot happen: per >= rem_total / G
+    for (int u = plan.full_rounds * G; u < plan.n_units; ++u) rem_total += unit_T(u);
+    std::vector<long long> load(G, 0);
+    long long total = rem_total;
+    for (int c = 0; c < G; ++c)
+        for (int r = 0; r < plan.full_rounds; ++r) {
+            load[c] += unit_T(full_round_unit(G, c, r));
+            total += unit_T(full_round_unit(G, c, r));
+        }
+    long long budget = (total + G - 1) / G;
+    // A split part costs a Q load and an epilogue: with no full rounds, give
+    // each CTA at least 8 key tiles.
+    if (plan.full_rounds == 0) budget = std::max<long long>(budget, 8);
+    plan.rem_lo.assign(G + 1, 0);
+    for (int c = 0; c < G; ++c) {
+        const long long share = std::max<long long>(0, budget - load[c]);
+        plan.rem_lo[c + 1] = (int)std::min(rem_total, plan.rem_lo[c] + share);
+    }
+    plan.grid = G;
+    if (plan.full_rounds == 0) {
+        int used = 1;
+        while (used < G && plan.rem_lo[used] < rem_total) ++used;
+        plan.grid = used;
+        plan.rem_lo.resize(used + 1);
+    }
+    plan.rem_lo.back() = (int)rem_total;
+    // Any remainder unit split across CTAs?
+    plan.has_split = false;
+    long long U = 0;
+    int c = 0;
+    for (int u = plan.full_rounds * G; u < plan.n_units && !plan.has_split; ++u) {
+        const int T = unit_T(u);
+        while (c + 1 < plan.grid && plan.rem_lo[c + 1] <= U) ++c;
+        if (U + T > plan.rem_lo[c + 1]) plan.has_split = true;
+        U += T;
+    }
     plan.scratch_bytes = (size_t)plan.grid * 2 * ((size_t)kPairRows * p.head_dim * 4 + (size_t)kPairRows * 8);
 }
 
@@ -763,14 +835,15 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
     tp.n_units = plan.n_units;
     tp.grid = plan.grid;
     tp.full_rounds = plan.full_rounds;
-    tp.rem_per_cta = plan.rem_per_cta;
-    tp.rem_total = plan.rem_total;
+    tp.head_major = plan.head_major;
+    if ((int)plan.rem_lo.size() != plan.grid + 1 || plan.grid > kMaxGrid) return cudaErrorInvalidValue;
+    for (int c = 0; c <= plan.grid; ++c) tp.rem_lo[c] = plan.rem_lo[c];
     const size_t part_o_bytes = (size_t)plan.grid * 2 * kPairRows * p.head_dim * 4;
     tp.part_o = static_cast<float4 *>(scratch);
     tp.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(scratch) + part_o_bytes);
     tp.out = static_cast<__nv_bfloat16 *>(p.o);
-    if (p.head_dim == 128) return launch_tc<128>(tp, s);
-    if (p.head_dim == 64) return launch_tc<64>(tp, s);
+    if (p.head_dim == 128) return launch_tc<128>(tp, plan.has_split, s);
+    if (p.head_dim == 64) return launch_tc<64>(tp, plan.has_split, s);
     return cudaErrorInvalidValue;
 }
 

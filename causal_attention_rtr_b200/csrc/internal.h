@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <vector>
 
 #include "rtr.h"
 
@@ -45,11 +46,13 @@ struct AttnProblem {
 
 // Schedule of the persistent tensor-core kernel for one problem: units are
 // (head, 256-row query pair); full rounds give every CTA one whole unit, the
-// remaining units' key tiles are shared equally (rem_per_cta tiles per CTA).
+// remaining units' key tiles are cut into per-CTA ranges that even out the
+// CTAs' totals.
 struct AttnPlan {
-    int n_pairs, n_units, grid, full_rounds;
-    long long rem_per_cta, rem_total;
-    size_t scratch_bytes;   // partial results of split units
+    int n_pairs, n_units, grid, full_rounds, head_major;
+    std::vector<int> rem_lo;   // grid + 1 boundaries of the per-CTA remainder ranges
+    bool has_split;            // some unit is shared by two CTAs (combine kernel runs)
+    size_t scratch_bytes;      // partial results of split units
 };
 
 void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan);
