@@ -94,6 +94,7 @@ struct TcParams {
     // of the remaining units' key tiles
     int n_pairs, n_units, grid, full_rounds, head_major;
     int rem_lo[kMaxGrid + 1];
+    int rem_U[kMaxGrid];   // key tiles of the remainder before its unit i (fewer than kMaxGrid units)
     float4 *part_o;     // [grid][2][D/4][256]
     float2 *part_ml;    // [grid][2][256]: running max (log2 units), row sum
     __nv_bfloat16 *out; // token-major output (combine kernel)
@@ -231,23 +232,23 @@ __device__ __forceinline__ void locate_tile(const TcParams &p, int q0, int t, in
 
 // P = exp2(s * scale_log2 - m) for one row of 128 scores, packed to bf16
 // pairs and stored over the row's first 64 TMEM columns; row sums into acc.
+// The scale-and-shift and the sums use packed f32x2 instructions.
 template <bool POLY>
 __device__ __forceinline__ void softmax_probs(const uint32_t (&sr)[128], float sl2, float neg_m, uint32_t tS,
-                                              float (&acc)[8]) {
+                                              float2 (&acc)[4]) {
+    const float2 sl2x2 = make_float2(sl2, sl2), negm2 = make_float2(neg_m, neg_m);
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int c = 32 * q4 + 2 * e;
-            const float x0 = fmaf(__uint_as_float(sr[c]), sl2, neg_m);
-            const float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, neg_m);
+            const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
             const bool poly = POLY && (e % 4) < (RTR_EXP2_POLY_PER8 / 2);
-            const float p0 = poly ? exp2_poly(x0) : fast_exp2(x0);
-            const float p1 = poly ? exp2_poly(x1) : fast_exp2(x1);
-            acc[(2 * e) & 7] += p0;
-            acc[(2 * e + 1) & 7] += p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            const float2 pr = make_float2(poly ? exp2_poly(x.x) : fast_exp2(x.x),
+                                          poly ? exp2_poly(x.y) : fast_exp2(x.y));
+            acc[e & 3] = fadd2(acc[e & 3], pr);
+            pk[e] = pack_bf16x2(pr.x, pr.y);
         }
         tmem_st16(tS + 16 * q4, pk);
     }
@@ -368,21 +369,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 0, 1);
-            auto issue_s = [&](int i, uint32_t kslot) {
+            // Descriptors depend only on the buffer: build them once, then
+            // step along K by adding the byte offset >> 4 to the start-address
+            // field (no carry: every address is below 256 KB).
+            const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t dq1 = smem_desc_sw128(sQ + L::kTileBytes, 16, 1024);
+            const uint64_t dk0 = smem_desc_sw128(sKV, 16, 1024);
+            const uint64_t dv0 = smem_desc_sw128(sKV, 16384, 1024);
+            auto issue_s = [&](int i, int slot) {
+                const uint64_t a0 = i ? dq1 : dq0;
+                const uint64_t b0 = dk0 + (uint64_t)((slot * L::kTileBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-                    const uint64_t a = smem_desc_sw128(sQ + i * L::kTileBytes + off, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(kslot + off, 16, 1024);
-                    mma_ss(tmem + i * 128, a, b, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem + i * 128, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](int i, uint32_t vslot, bool acc) {
+            auto issue_pv = [&](int i, int slot, bool acc) {
+                const uint64_t b0 = dv0 + (uint64_t)((slot * L::kTileBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint64_t b = smem_desc_sw128(vslot + kk * 2048, 16384, 1024);
-                    mma_ts(tmem + 256 + i * D, tmem + i * 128 + kk * 8, b, idesc_o, (acc || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_ts(tmem + 256 + i * D, tmem + i * 128 + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_o,
+                           (acc || kk > 0) ? 1u : 0u);
             };
             Sched sc;
             Item it;
@@ -396,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 ok = mbar_wait(bar(L::bFull + slot), (n / kSlots) & 1, kWaitNs);
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t kslot = sKV + slot * L::kTileBytes;
+                int kslot = slot;
                 issue_s(0, kslot);
                 tc_commit(bar(L::bS + 0));
                 issue_s(1, kslot);
@@ -408,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     ok = mbar_wait(bar(L::bFull + vs), (n / kSlots) & 1, kWaitNs);
                     if (!ok) break;
                     ++n;
-                    const uint32_t vslot = sKV + vs * L::kTileBytes;
+                    const int vslot = vs;
                     ok = mbar_wait(bar(L::bP + 0), jj & 1, kWaitNs) && !*abort_flag;
                     if (!ok) break;
                     tc_fence_after();
@@ -420,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                         ok = mbar_wait(bar(L::bFull + ks), (n / kSlots) & 1, kWaitNs);
                         if (!ok) break;
                         tc_fence_after();
-                        kslot = sKV + ks * L::kTileBytes;
+                        kslot = ks;
                         issue_s(0, kslot);
                         tc_commit(bar(L::bS + 0));
                     }
@@ -532,14 +540,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     }
                 }
                 const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f)};
                 // The polynomial exp2 runs only on tiles without masked
                 // entries (every input finite); ex2 maps -inf to exactly 0.
                 if (masked)
                     softmax_probs<false>(sr, sl2, neg_m, tS, acc);
                 else
                     softmax_probs<true>(sr, sl2, neg_m, tS, acc);
-                l_run += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+                const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+                const float2 a4 = fadd2(a01, a23);
+                l_run += a4.x + a4.y;
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -625,12 +636,7 @@ template <int D>
 __global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcParams p) {
     const int ru = p.full_rounds * p.grid + blockIdx.x;
     if (ru >= p.n_units) return;
-    long long U = 0;
-    for (int u = p.full_rounds * p.grid; u < ru; ++u) {
-        int pr, hd;
-        unit_coords(p, u, pr, hd);
-        U += pair_tiles(p, pr);
-    }
+    const long long U = p.rem_U[blockIdx.x];
     int pair, head;
     unit_coords(p, ru, pair, head);
     const int T = pair_tiles(p, pair);
@@ -788,12 +794,14 @@ void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan) {
         plan.rem_lo.resize(used + 1);
     }
     plan.rem_lo.back() = (int)rem_total;
-    // Any remainder unit split across CTAs?
+    // Tile offsets of the remainder units; any unit split across CTAs?
     plan.has_split = false;
+    plan.rem_U.clear();
     long long U = 0;
     int c = 0;
-    for (int u = plan.full_rounds * G; u < plan.n_units && !plan.has_split; ++u) {
+    for (int u = plan.full_rounds * G; u < plan.n_units; ++u) {
         const int T = unit_T(u);
+        plan.rem_U.push_back((int)U);
         while (c + 1 < plan.grid && plan.rem_lo[c + 1] <= U) ++c;
         if (U + T > plan.rem_lo[c + 1]) plan.has_split = true;
         U += T;
@@ -838,6 +846,8 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
     tp.head_major = plan.head_major;
     if ((int)plan.rem_lo.size() != plan.grid + 1 || plan.grid > kMaxGrid) return cudaErrorInvalidValue;
     for (int c = 0; c <= plan.grid; ++c) tp.rem_lo[c] = plan.rem_lo[c];
+    if (plan.rem_U.size() > (size_t)kMaxGrid) return cudaErrorInvalidValue;
+    for (size_t i = 0; i < plan.rem_U.size(); ++i) tp.rem_U[i] = plan.rem_U[i];
     const size_t part_o_bytes = (size_t)plan.grid * 2 * kPairRows * p.head_dim * 4;
     tp.part_o = static_cast<float4 *>(scratch);
     tp.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(scratch) + part_o_bytes);

@@ -51,6 +51,7 @@ struct AttnProblem {
 struct AttnPlan {
     int n_pairs, n_units, grid, full_rounds, head_major;
     std::vector<int> rem_lo;   // grid + 1 boundaries of the per-CTA remainder ranges
+    std::vector<int> rem_U;    // key-tile offset of each remainder unit
     bool has_split;            // some unit is shared by two CTAs (combine kernel runs)
     size_t scratch_bytes;      // partial results of split units
 };
