@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--workload", default="wan13_layer",
+                    choices=["wan13_layer", "prefill_22", "long_stream", "switch_14b", "tiny_f32"],
+                    help="wan13_layer is the headline step; the others print one line each for reference")
     return ap.parse_args()
 
 
@@ -399,8 +402,164 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ other workloads
+def _events(n):
+    import torch
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def run_other(args):
+    """One JSON line per workload other than the headline one (single GPU)."""
+    import numpy as np
+    import torch
+
+    from causal_attention_rtr_b200 import rtr, synth
+
+    torch.cuda.set_device(0)
+    sh = torch.cuda.current_stream().cuda_stream
+    peaks = measured_peaks()
+    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(0)
+
+    def rnd(shape, dtype=torch.bfloat16, scale=0.5):
+        return (torch.randn(shape, generator=gen, device="cuda", dtype=torch.float32) * scale).to(dtype)
+
+    def stream_flops(H, d, k, cached_frames, C):
+        nq = C * k
+        return 4.0 * d * H * (nq * cached_frames * k + sum(k * (c + 1) * k for c in range(C)))
+
+    line = {"workload": args.workload, "n_gpus": 1, "dtype": "bf16", "data": "synthetic (torch.randn * 0.5 on device)"}
+    if args.workload == "prefill_22":
+        w = synth.PREFILL_22
+        n = w.chunk_frames * w.k
+        q, k, v = rnd((n, w.heads, w.head_dim)), rnd((n, w.heads, w.head_dim)), rnd((n, w.heads, w.head_dim))
+        out = torch.empty_like(q)
+        vis = sum(min(n, (i // w.k + 1) * w.k) for i in range(0, n, 1))
+        flops = 4.0 * w.head_dim * w.heads * vis
+        for _ in range(3):
+            rtr.rtr_attn_block_causal_prefill(q, k, v, n, w.heads, w.head_dim, w.k, "bf16", out, 0.0, 0, sh)
+        ts = []
+        for _ in range(max(1, args.steps)):
+            flush.zero_()
+            a, b = _events(2)
+            a.record()
+            rtr.rtr_attn_block_causal_prefill(q, k, v, n, w.heads, w.head_dim, w.k, "bf16", out, 0.0, 0, sh)
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.mean(ts)
+        line.update({"config": w.name, "ms_per_call": ms, "tflop_per_call": flops / 1e12,
+                     "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc})
+    elif args.workload == "long_stream":
+        w = synth.LONG_STREAM
+        L, H, d, k, C, W = w.layers, w.heads, w.head_dim, w.k, w.chunk_frames, w.window_frames
+        c = rtr.rtr_kvcache_create(L, H, d, k, 1, W, "bf16", 0)
+        ref = rnd((k, H, d))
+        for l in range(L):
+            rtr.rtr_kvcache_set_reference(c, l, ref, ref, sh)
+        chunks = [tuple(rnd((C * k, H, d)) for _ in range(3)) for _ in range(2)]  # reused inputs
+        out = torch.empty_like(chunks[0][0])
+        n_chunks = w.frames_total // C
+        flops = 0.0
+        torch.cuda.synchronize()
+        a, b = _events(2)
+        a.record()
+        for ch in range(n_chunks):
+            cached = 1 + min(W, ch * C)
+            for step_ in range(w.steps_per_chunk):
+                q, kk, vv = chunks[(ch + step_) % 2]
+                for l in range(L):
+                    rtr.rtr_attn_frame_causal(c, l, q, kk, vv, C, out, 0.0, sh)
+                    flops += stream_flops(H, d, k, cached, C)
+            for l in range(L):
+                rtr.rtr_kvcache_append_frame(c, l, kk, vv, C, sh)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        st = rtr.rtr_get_device_status(0, sh)
+        rtr.rtr_kvcache_destroy(c)
+        line.update({"config": w.name, "total_ms": ms, "attention_tflop": flops / 1e12,
+                     "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
+                     "latent_frames_per_s_per_layer": w.frames_total / (ms / 1e3 / L),
+                     "latent_frames_per_s_all_layers": w.frames_total / (ms / 1e3),
+                     "device_status": rtr.rtr_status_string(st),
+                     "note": "attention calls + appends of 30 layers x 40 chunks x 2 steps, one stream"})
+    elif args.workload == "switch_14b":
+        w = synth.SWITCH_14B
+        H, d, k, W, T = w.heads, w.head_dim, w.k, w.window_frames, w.text_tokens
+        c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "bf16", 0)
+        x = rtr.rtr_crossattn_create(1, H, d, T, "bf16", 0)
+        ref, kt, vt = rnd((k, H, d)), rnd((T, H, d)), rnd((T, H, d))
+        frames = [tuple(rnd((k, H, d)) for _ in range(3)) for _ in range(2)]
+        out = torch.empty_like(frames[0][0])
+        xout = torch.empty_like(out)
+        rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
+        rtr.rtr_crossattn_set_text(x, 0, kt, vt, T, sh)
+        torch.cuda.synchronize()
+        flops = 0.0
+        count = 0
+        a, b = _events(2)
+        sw_ev = []
+        a.record()
+        for f in range(w.frames_total):
+            if f > 0 and f % w.switch_every == 0:
+                e0, e1 = _events(2)
+                e0.record()
+                rtr.rtr_crossattn_reset(x)
+                rtr.rtr_crossattn_set_text(x, 0, vt, kt, T, sh)
+                rtr.rtr_kvcache_retain_last(c, 0, 1)
+                count = min(count, 1)
+                rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
+                e1.record()
+                sw_ev.append((e0, e1))
+            q, kk, vv = frames[f % 2]
+            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, 1, out, 0.0, sh)
+            rtr.rtr_attn_cross(x, 0, q, k, xout, 0.0, sh)
+            rtr.rtr_kvcache_append_frame(c, 0, kk, vv, 1, sh)
+            flops += stream_flops(H, d, k, 1 + count, 1) + 4.0 * d * H * k * T
+            count = min(W, count + 1)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        sw_ms = [e0.elapsed_time(e1) for e0, e1 in sw_ev]
+        rtr.rtr_kvcache_destroy(c)
+        rtr.rtr_crossattn_destroy(x)
+        line.update({"config": w.name, "total_ms": ms, "ms_per_frame": ms / w.frames_total,
+                     "attention_tflop": flops / 1e12, "tflops": flops / ms / 1e9,
+                     "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
+                     "latent_frames_per_s": w.frames_total / (ms / 1e3),
+                     "switch_ms": sw_ms,
+                     "note": "per frame: self-attention (ref + window + frame), cross-attention to 512 text "
+                             "tokens, append; switches at frames 16/32/48 reset+set text, retain 1, set ref"})
+    elif args.workload == "tiny_f32":
+        w = synth.TINY_F32
+        H, d, k, W = w.heads, w.head_dim, w.k, w.window_frames
+        c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "f32", 0)
+        ref = rnd((k, H, d), torch.float32, 1.0)
+        rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
+        fr = [tuple(rnd((k, H, d), torch.float32, 1.0) for _ in range(3)) for _ in range(w.frames_total)]
+        out = torch.empty_like(fr[0][0])
+        torch.cuda.synchronize()
+        a, b = _events(2)
+        a.record()
+        for q, kk, vv in fr:
+            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, 1, out, 0.0, sh)
+            rtr.rtr_kvcache_append_frame(c, 0, kk, vv, 1, sh)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        rtr.rtr_kvcache_destroy(c)
+        line.update({"config": w.name, "dtype": "f32", "total_ms": ms, "ms_per_frame": ms / w.frames_total,
+                     "note": "correctness workload; time is launch-bound"})
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.workload != "wan13_layer":
+        run_other(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -484,6 +484,12 @@ rtr_status rtr_attn_cross(const rtr_xattn *x, int layer, const void *q, int n_q,
     return run_attention(pb, x->dt, tk, tv, x->device, (cudaStream_t)stream);
 }
 
+rtr_status rtr_test_inject_wait_timeout(int device, int launches) {
+    if (device < 0 || device >= 64 || launches < 0) return RTR_E_INVAL;
+    inject_wait_timeouts(device, launches);
+    return RTR_OK;
+}
+
 rtr_status rtr_get_device_status(int device, rtr_stream_t stream) {
     if (device < 0) return RTR_E_INVAL;
     DeviceGuard dg(device);

@@ -90,6 +90,7 @@ struct TcParams {
     KvSeg seg[kMaxSegs];
     float scale_log2;   // scale * log2(e)
     unsigned *status;
+    int test_skip_loads;   // test hook: issue no loads, so the bounded waits expire
     // schedule: full rounds, then CTA c takes tiles [rem_lo[c], rem_lo[c+1])
     // of the remaining units' key tiles
     int n_pairs, n_units, grid, full_rounds, head_major;
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     set_max_regs_dec<RTR_REGS_LOW>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
+        if (lane == 0 && !p.test_skip_loads) {
             Sched sc;
             Item it;
             int n = 0, k = 0;
@@ -809,10 +810,23 @@ void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan) {
     plan.scratch_bytes = (size_t)plan.grid * 2 * ((size_t)kPairRows * p.head_dim * 4 + (size_t)kPairRows * 8);
 }
 
+namespace {
+int g_inject_timeouts[64] = {};   // per device: launches left that skip their loads
+}
+
+void inject_wait_timeouts(int device, int launches) {
+    if (device >= 0 && device < 64) g_inject_timeouts[device] = launches > 0 ? launches : 0;
+}
+
 cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const CUtensorMap *tm_k0,
                              const CUtensorMap *tm_v0, unsigned *status, void *scratch, cudaStream_t s) {
     TcParams tp;
     memset(&tp, 0, sizeof(tp));
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && g_inject_timeouts[dev] > 0) {
+        --g_inject_timeouts[dev];
+        tp.test_skip_loads = 1;
+    }
     const uint64_t D = (uint64_t)p.head_dim;
     if (!make_tmap_bf16(&tp.tm_q, p.q, D, p.heads, p.nq, 1, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&tp.tm_o, p.o, D, p.heads, p.nq, 1, kBM)) return cudaErrorInvalidValue;

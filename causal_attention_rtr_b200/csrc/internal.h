@@ -83,4 +83,8 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, 
 
 unsigned *device_status_ptr(int device);
 
+// Test hook: the next `launches` tensor-core attention launches on `device`
+// issue no loads, so their bounded waits expire and latch RTR_E_TIMEOUT.
+void inject_wait_timeouts(int device, int launches);
+
 }  // namespace rtr

@@ -53,6 +53,7 @@ _SIGNATURES = [
     ("rtr_crossattn_reset", _i, [_vp]),
     ("rtr_attn_cross", _i, [_vp, _i, _vp, _i, _vp, _f, _vp]),
     ("rtr_get_device_status", _i, [_i, _vp]),
+    ("rtr_test_inject_wait_timeout", _i, [_i, _i]),
 ]
 
 for _name, _res, _args in _SIGNATURES:
@@ -218,3 +219,10 @@ def raw_status(fn_name, *args):
     """Call a C entry point and return its status without raising (tests of
     the error paths)."""
     return getattr(_lib, fn_name)(*args)
+
+
+def rtr_test_inject_wait_timeout(device, launches):
+    """Test hook: the next `launches` bf16 attention launches on `device`
+    issue no loads, so their bounded waits expire and RTR_E_TIMEOUT is
+    latched (see include/rtr.h)."""
+    return _check(_lib.rtr_test_inject_wait_timeout(device, launches), "rtr_test_inject_wait_timeout")

@@ -222,6 +222,15 @@ rtr_status rtr_attn_cross(const rtr_xattn *x, int layer, const void *q,
  */
 rtr_status rtr_get_device_status(int device, rtr_stream_t stream);
 
+/* Test hook for the failure path: the next `launches` bf16 attention
+ * launches on `device` (any of the attention calls) deliberately issue no
+ * loads.  Their bounded waits then expire after about one second each, the
+ * kernel stops, frees its tensor memory and returns, and RTR_E_TIMEOUT is
+ * latched for rtr_get_device_status.  The outputs of those launches are
+ * unspecified.  No fault, trap or hang is involved; later launches run
+ * normally.  launches == 0 cancels.  For tests only. */
+rtr_status rtr_test_inject_wait_timeout(int device, int launches);
+
 /* Library build information (static string). */
 const char *rtr_build_info(void);
 
