@@ -6,7 +6,7 @@
 //
 // Source rows are [tokens][heads][d] (the layout a QKV projection produces);
 // the cache is head-major [heads][rows][d].  The kernel is a pure HBM-bound
-// copy: every thread moves eight 16-byte vectors, all loads in flight before
+// copy: every thread moves four 16-byte vectors, all loads in flight before
 // the matching stores, and one grid pass covers K and V together.  Index
 // arithmetic uses multiply-high division by run-time constants (Granlund and
 // Montgomery, "Division by Invariant Integers using Multiplication", 1994).
@@ -48,7 +48,7 @@ struct ScatterDev {
     uint64_t rows_per_head;
 };
 
-constexpr int kUnroll = 8;
+constexpr int kUnroll = 4;
 constexpr int kBlock = 256;
 
 // K and V form one index space of 2 * per_tensor vectors; every thread moves
