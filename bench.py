@@ -123,6 +123,23 @@ def profiled_traffic():
         return None
 
 
+def max_over_ranks(values, world, device):
+    """Per-rank mean times -> the slowest rank's, identical on every rank
+    (the job finishes when its slowest replica does)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(flops_per_step_per_rank, step_ms, world):
+    """Whole-job TFLOP/s: every replica does the same work per step, timed
+    by the slowest rank."""
+    return world * flops_per_step_per_rank / (step_ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
@@ -352,21 +369,19 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = [a.elapsed_time(b) for a, b in zip(e_start, e_end)]
 
-    stats = torch.tensor([statistics.mean(step_ms), statistics.mean(attn_ms), statistics.mean(app_ms),
-                          statistics.mean(e2e_ms)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-    step_mean, attn_mean, app_mean, e2e_mean = stats.tolist()
+    step_mean, attn_mean, app_mean, e2e_mean = max_over_ranks(
+        [statistics.mean(step_ms), statistics.mean(attn_ms), statistics.mean(app_ms), statistics.mean(e2e_ms)],
+        world, "cuda")
 
     rtr.rtr_kvcache_destroy(c)
     if rank != 0:
         return
 
     flops = attn_flops(w)
+    value = job_throughput(flops, step_mean, world)
     peaks = measured_peaks()
     peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    value = world * flops / (step_mean * 1e-3) / 1e12
     attn_tflops = flops / (attn_mean * 1e-3) / 1e12
     app_gbs = append_bytes(w) / (app_mean * 1e-3) / 1e9
     traffic = profiled_traffic()
