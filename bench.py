@@ -327,6 +327,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
+    launches_before = rtr.rtr_kernel_launches()
     for s in range(K):
         flush.zero_()
         ev[s][0].record(stream)
@@ -335,6 +336,7 @@ def run_ours(args, rank, world, local_rank):
         rtr.rtr_kvcache_append_frame(c, 0, kc, vc, C, sh)
         ev[s][2].record(stream)
     torch.cuda.synchronize()
+    launches_timed = rtr.rtr_kernel_launches() - launches_before
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
@@ -346,28 +348,55 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {rtr.rtr_status_string(status)}")
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside
+    # the timed region: every step uploads its Q, K, V from pinned host memory
+    # and reads its output back.  Two device buffer sets and a copy stream let
+    # step s+1's uploads and step s-1's download overlap step s's kernels.
     hq = torch.from_numpy(x.q.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
     hk = torch.from_numpy(x.k_cur.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
     hv = torch.from_numpy(x.v_cur.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
-    ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
     Ke = min(K, 100)
-    e_start = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
-    e_end = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    ho = [torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    bufs = [(torch.empty_like(q), torch.empty_like(kc), torch.empty_like(vc), torch.empty_like(out)) for _ in range(2)]
+    copy_stream = torch.cuda.Stream()
+    up_done = [torch.cuda.Event() for _ in range(Ke)]
+    comp_done = [torch.cuda.Event() for _ in range(Ke)]
+    down_done = [torch.cuda.Event() for _ in range(Ke)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def upload(s_):
+        bq, bk, bv, _ = bufs[s_ % 2]
+        with torch.cuda.stream(copy_stream):
+            if s_ >= 2:
+                copy_stream.wait_event(comp_done[s_ - 2])      # buffer set free again
+            bq.copy_(hq, non_blocking=True)
+            bk.copy_(hk, non_blocking=True)
+            bv.copy_(hv, non_blocking=True)
+            up_done[s_].record(copy_stream)
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    e_start.record(stream)
+    copy_stream.wait_stream(stream)
+    upload(0)
     for s in range(Ke):
-        flush.zero_()
-        e_start[s].record(stream)
-        q.copy_(hq, non_blocking=True)
-        kc.copy_(hk, non_blocking=True)
-        vc.copy_(hv, non_blocking=True)
-        rtr.rtr_attn_frame_causal(c, 0, q, kc, vc, C, out, 0.0, sh)
-        rtr.rtr_kvcache_append_frame(c, 0, kc, vc, C, sh)
-        ho.copy_(out, non_blocking=True)
-        e_end[s].record(stream)
+        if s + 1 < Ke:
+            upload(s + 1)
+        bq, bk, bv, bo = bufs[s % 2]
+        stream.wait_event(up_done[s])
+        if s >= 2:
+            stream.wait_event(down_done[s - 2])                 # output buffer read back
+        rtr.rtr_attn_frame_causal(c, 0, bq, bk, bv, C, bo, 0.0, sh)
+        rtr.rtr_kvcache_append_frame(c, 0, bk, bv, C, sh)
+        comp_done[s].record(stream)
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(comp_done[s])
+            ho[s % 2].copy_(bo, non_blocking=True)
+            down_done[s].record(copy_stream)
+    stream.wait_event(down_done[Ke - 1])
+    e_end.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = [a.elapsed_time(b) for a, b in zip(e_start, e_end)]
+    e2e_ms = [e_start.elapsed_time(e_end) / Ke]
 
     step_mean, attn_mean, app_mean, e2e_mean = max_over_ranks(
         [statistics.mean(step_ms), statistics.mean(attn_ms), statistics.mean(app_ms), statistics.mean(e2e_ms)],
@@ -404,9 +433,11 @@ def run_ours(args, rank, world, local_rank):
                          "ms_per_launch": app_mean, "achieved_gbs": app_gbs, "peak_gbs": peak_hbm,
                          "frac": app_gbs / peak_hbm, "peak_source": f"{peaks.get('source')} hbm_gbs"},
         "e2e": {"value": world * flops / (e2e_mean * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(3 * hq.numel() * 2), "d2h_bytes_per_step": int(ho.numel() * 2),
-                "ms_per_step": e2e_mean},
-        "gpu_launches": 2 * K,
+                "h2d_bytes_per_step": int(3 * hq.numel() * 2), "d2h_bytes_per_step": int(ho[0].numel() * 2),
+                "ms_per_step": e2e_mean,
+                "how": "pinned host Q/K/V uploaded and output read back every step; copies of neighbouring "
+                       "steps overlap the kernels (copy stream, two buffer sets)"},
+        "gpu_launches": launches_timed,
         "clocks": clk,
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
     }

@@ -10,7 +10,9 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <cstdint>
@@ -21,6 +23,10 @@
 
 #include "internal.h"
 #include "rtr.h"
+
+#ifndef RTR_DEFAULT_CTA_GROUP
+#define RTR_DEFAULT_CTA_GROUP 1   // the CTA-pair kernel (2) measured slower on every workload
+#endif
 
 namespace rtr {
 
@@ -77,6 +83,19 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, 
     return r == CUDA_SUCCESS;
 }
 
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+int attn_cta_group() {
+    const char *e = std::getenv("RTR_CTA_GROUP");
+    if (e && e[0] == '1') return 1;
+    if (e && e[0] == '2') return 2;
+    return RTR_DEFAULT_CTA_GROUP;
+}
+
 }  // namespace rtr
 
 using namespace rtr;
@@ -92,6 +111,7 @@ struct rtr_kvcache {
     std::vector<int> ref_valid, count;
     std::vector<long long> g;
     std::vector<CUtensorMap> tmk, tmv;
+    std::vector<CUtensorMap> tmk64;   // K maps with 64-row boxes (CTA-pair attention)
 };
 
 struct rtr_xattn {
@@ -102,6 +122,7 @@ struct rtr_xattn {
     char *kbuf = nullptr, *vbuf = nullptr;
     std::vector<int> n_text;
     std::vector<CUtensorMap> tmk, tmv;
+    std::vector<CUtensorMap> tmk64;   // K maps with 64-row boxes (CTA-pair attention)
 };
 
 namespace {
@@ -151,8 +172,8 @@ void *stream_workspace(int device, cudaStream_t s, size_t bytes) {
 }
 
 // Launch the attention for a problem; picks the kernel for the element type.
-rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0, const CUtensorMap *tm_v0,
-                         int device, cudaStream_t s) {
+rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0, const CUtensorMap *tm_k0h,
+                         const CUtensorMap *tm_v0, int device, cudaStream_t s) {
     if (pb.nq == 0) return RTR_OK;
     for (int i = 0; i < pb.nseg; ++i)
         if (pb.seg[i].len <= 0) return RTR_E_INVAL;
@@ -162,10 +183,10 @@ rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0
         unsigned *st = device_status_ptr(device);
         if (!st) return RTR_E_CUDA;
         AttnPlan plan;
-        plan_attn_bf16(pb, sm_count(device), plan);
+        plan_attn_bf16(pb, sm_count(device), attn_cta_group(), plan);
         void *scratch = stream_workspace(device, s, plan.scratch_bytes);
         if (!scratch) return RTR_E_NOMEM;
-        e = launch_attn_bf16(pb, plan, tm_k0, tm_v0, st, scratch, s);
+        e = launch_attn_bf16(pb, plan, tm_k0, tm_k0h, tm_v0, st, scratch, s);
     } else {
         e = launch_attn_f32(pb, s);
     }
@@ -228,8 +249,10 @@ rtr_status rtr_kvcache_create(int layers, int heads, int head_dim, int k, int re
     if (dt == RTR_BF16) {
         c->tmk.resize(layers);
         c->tmv.resize(layers);
+        c->tmk64.resize(layers);
         for (int l = 0; l < layers; ++l) {
             if (!make_tmap_bf16(&c->tmk[l], c->kbuf + l * c->layer_bytes, head_dim, rows, heads, 128, 1) ||
+                !make_tmap_bf16(&c->tmk64[l], c->kbuf + l * c->layer_bytes, head_dim, rows, heads, 64, 1) ||
                 !make_tmap_bf16(&c->tmv[l], c->vbuf + l * c->layer_bytes, head_dim, rows, heads, 128, 1)) {
                 cudaFree(c->kbuf); cudaFree(c->vbuf); delete c;
                 return RTR_E_CUDA;
@@ -362,8 +385,9 @@ rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q,
     pb.k1 = k_cur; pb.v1 = v_cur; pb.rows1 = nq;
     DeviceGuard dg(c->device);
     const CUtensorMap *tk = c->dt == RTR_BF16 ? &c->tmk[layer] : nullptr;
+    const CUtensorMap *tkh = c->dt == RTR_BF16 ? &c->tmk64[layer] : nullptr;
     const CUtensorMap *tv = c->dt == RTR_BF16 ? &c->tmv[layer] : nullptr;
-    return run_attention(pb, c->dt, tk, tv, c->device, (cudaStream_t)stream);
+    return run_attention(pb, c->dt, tk, tkh, tv, c->device, (cudaStream_t)stream);
 }
 
 rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k, const void *v, int n_tokens, int heads,
@@ -384,7 +408,7 @@ rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k, const voi
     pb.q = q; pb.o = out; pb.k1 = k; pb.v1 = v; pb.rows1 = n_tokens;
     DeviceGuard dg(device);
     if (!dg.ok) return RTR_E_INVAL;
-    return run_attention(pb, dt, nullptr, nullptr, device, (cudaStream_t)stream);
+    return run_attention(pb, dt, nullptr, nullptr, nullptr, device, (cudaStream_t)stream);
 }
 
 rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_text, rtr_dtype dt, int device,
@@ -416,8 +440,10 @@ rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_tex
     if (dt == RTR_BF16) {
         x->tmk.resize(layers);
         x->tmv.resize(layers);
+        x->tmk64.resize(layers);
         for (int l = 0; l < layers; ++l) {
             if (!make_tmap_bf16(&x->tmk[l], x->kbuf + l * x->layer_bytes, head_dim, max_text, heads, 128, 1) ||
+                !make_tmap_bf16(&x->tmk64[l], x->kbuf + l * x->layer_bytes, head_dim, max_text, heads, 64, 1) ||
                 !make_tmap_bf16(&x->tmv[l], x->vbuf + l * x->layer_bytes, head_dim, max_text, heads, 128, 1)) {
                 cudaFree(x->kbuf); cudaFree(x->vbuf); delete x;
                 return RTR_E_CUDA;
@@ -480,9 +506,12 @@ rtr_status rtr_attn_cross(const rtr_xattn *x, int layer, const void *q, int n_q,
     pb.k0 = x->kbuf + layer * x->layer_bytes; pb.v0 = x->vbuf + layer * x->layer_bytes; pb.rows0 = x->max_text;
     DeviceGuard dg(x->device);
     const CUtensorMap *tk = x->dt == RTR_BF16 ? &x->tmk[layer] : nullptr;
+    const CUtensorMap *tkh = x->dt == RTR_BF16 ? &x->tmk64[layer] : nullptr;
     const CUtensorMap *tv = x->dt == RTR_BF16 ? &x->tmv[layer] : nullptr;
-    return run_attention(pb, x->dt, tk, tv, x->device, (cudaStream_t)stream);
+    return run_attention(pb, x->dt, tk, tkh, tv, x->device, (cudaStream_t)stream);
 }
+
+unsigned long long rtr_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 rtr_status rtr_test_inject_wait_timeout(int device, int launches) {
     if (device < 0 || device >= 64 || launches < 0) return RTR_E_INVAL;

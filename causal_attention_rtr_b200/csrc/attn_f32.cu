@@ -80,7 +80,9 @@ cudaError_t launch_attn_f32(const AttnProblem &p, cudaStream_t s) {
         attn_fwd_f32<128><<<(unsigned)blocks, 256, 0, s>>>(p);
     else
         return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launch();
+    return e;
 }
 
 }  // namespace rtr

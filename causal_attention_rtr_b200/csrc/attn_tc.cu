@@ -73,8 +73,7 @@ namespace {
 
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // keys per tile
-constexpr int kPairRows = 2 * kBM;
-constexpr int kSlots = 4;         // K/V ring depth
+constexpr int kPairRows = 2 * kBM;   // query rows per CTA (two tiles)
 constexpr int kThreads = 384;     // 12 warps
 constexpr int kMaxGrid = 160;     // persistent CTAs at most (B200: 148 SMs)
 constexpr uint64_t kWaitNs = 1000000000ull;   // bounded waits: 1 s
@@ -86,27 +85,35 @@ struct TcParams {
     CUtensorMap tm_v0;
     CUtensorMap tm_k1;  // token-major [rows][H][D], box (64, 1, 128)
     CUtensorMap tm_v1;
+    CUtensorMap tm_k0h; // K maps with 64-row boxes (CTA-pair mode: each CTA loads half a key tile)
+    CUtensorMap tm_k1h;
     int nq, heads, kpf, nseg;
+    int unit_rows;      // query rows per work unit: 256 per CTA of the cluster
     KvSeg seg[kMaxSegs];
     float scale_log2;   // scale * log2(e)
     unsigned *status;
     int test_skip_loads;   // test hook: issue no loads, so the bounded waits expire
     // schedule: full rounds, then CTA c takes tiles [rem_lo[c], rem_lo[c+1])
     // of the remaining units' key tiles
-    int n_pairs, n_units, grid, full_rounds, head_major;
+    int n_pairs, n_units, grid, full_rounds, head_major;   // n_pairs: row blocks of unit_rows per head; grid: clusters
     int rem_lo[kMaxGrid + 1];
     int rem_U[kMaxGrid];   // key tiles of the remainder before its unit i (fewer than kMaxGrid units)
-    float4 *part_o;     // [grid][2][D/4][256]
-    float2 *part_ml;    // [grid][2][256]: running max (log2 units), row sum
+    float4 *part_o;     // [CTAs][2][D/4][256]
+    float2 *part_ml;    // [CTAs][2][256]: running max (log2 units), row sum
     __nv_bfloat16 *out; // token-major output (combine kernel)
 };
 
-template <int D>
+// CG = CTAs per cluster working one MMA: 1, or 2 for the CTA-pair MMA
+// (tcgen05 cta_group::2: M = 256 rows across the pair, each CTA holding half
+// of every key / value tile).
+template <int D, int CG>
 struct Layout {
     static constexpr int kTileBytes = kBM * D * 2;          // one Q / K / V tile
+    static constexpr int kSlotBytes = kTileBytes / CG;      // this CTA's part of a K or V tile
+    static constexpr int kSlots = 4 * CG;                   // ring: 128 KB of K/V in flight
     static constexpr int kQ = 0;                            // Q0, Q1
     static constexpr int kKV = 2 * kTileBytes;              // ring slots
-    static constexpr int kBars = kKV + kSlots * kTileBytes; // mbarriers
+    static constexpr int kBars = kKV + kSlots * kSlotBytes; // mbarriers
     static constexpr int bQ = 0, bQfree = 1, bFull = 2, bEmpty = bFull + kSlots, bS = bEmpty + kSlots,
                          bP = bS + 2, bO = bP + 2, bEpi = bO + 2, bDrain = bEpi + 2, kNumBars = bDrain + 1;
     static constexpr int kMisc = kBars + kNumBars * 8;      // tmem holder, abort flag
@@ -114,12 +121,12 @@ struct Layout {
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1 KB alignment
 };
 
-// Key tiles of one run for the query pair starting at q0.
+// Key tiles of one run for the unit whose rows start at q0.
 __device__ __forceinline__ int seg_tiles(const TcParams &p, int s, int q0) {
     const KvSeg &g = p.seg[s];
     int len = g.len;
     if (g.causal) {
-        const int q_last = min(q0 + kPairRows - 1, p.nq - 1);
+        const int q_last = min(q0 + p.unit_rows - 1, p.nq - 1);
         const int lim = (q_last / p.kpf + 1) * p.kpf;
         len = len < lim ? len : lim;
     }
@@ -128,7 +135,7 @@ __device__ __forceinline__ int seg_tiles(const TcParams &p, int s, int q0) {
 
 __device__ __forceinline__ int pair_tiles(const TcParams &p, int pair) {
     int t = 0;
-    for (int s = 0; s < p.nseg; ++s) t += seg_tiles(p, s, pair * kPairRows);
+    for (int s = 0; s < p.nseg; ++s) t += seg_tiles(p, s, pair * p.unit_rows);
     return t;
 }
 
@@ -164,8 +171,9 @@ struct Sched {
     bool first_rem = true;
 };
 
+template <int CG>
 __device__ bool sched_next(const TcParams &p, Sched &s, Item &it) {
-    const int c = blockIdx.x;
+    const int c = blockIdx.x / CG;   // cluster
     if (s.r < p.full_rounds) {
         it.unit = full_round_unit(p.grid, c, s.r);
         int pair, head;
@@ -255,10 +263,11 @@ __device__ __forceinline__ void softmax_probs(const uint32_t (&sr)[128], float s
     }
 }
 
-template <int D>
+template <int D, int CG>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant__ TcParams p) {
-    using L = Layout<D>;
+    using L = Layout<D, CG>;
     constexpr int NBOX = D / 64;
+    constexpr int kKRows = kBN / CG;                        // key rows of this CTA's K part
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_u32(smem);
@@ -270,17 +279,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // CTA pair: rank 0 issues every MMA for both CTAs; loads and P hand-offs
+    // of both CTAs count on rank 0's barriers (`lead`).
+    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+    auto lead = [&](int i) -> uint32_t { return CG == 2 ? mapa_shared(bar(i), 0) : bar(i); };
+    auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+        return CG == 2 ? mbar_wait_cluster(b, parity, kWaitNs) : mbar_wait(b, parity, kWaitNs);
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(L::bQ), 1);
         mbar_init(bar(L::bQfree), 2);          // one arrive per softmax group
-        for (int i = 0; i < kSlots; ++i) {
+        for (int i = 0; i < L::kSlots; ++i) {
             mbar_init(bar(L::bFull + i), 1);
             mbar_init(bar(L::bEmpty + i), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(L::bS + i), 1);
-            mbar_init(bar(L::bP + i), 4);      // one arrive per softmax warp
+            mbar_init(bar(L::bP + i), 4 * CG); // one arrive per softmax warp of the cluster
             mbar_init(bar(L::bO + i), 1);
             mbar_init(bar(L::bEpi + i), kBM);  // every softmax thread
         }
@@ -291,17 +307,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&p.tm_q);
         prefetch_tmap(&p.tm_o);
-        prefetch_tmap(&p.tm_k0);
+        prefetch_tmap(CG == 2 ? &p.tm_k0h : &p.tm_k0);
         prefetch_tmap(&p.tm_v0);
-        prefetch_tmap(&p.tm_k1);
+        prefetch_tmap(CG == 2 ? &p.tm_k1h : &p.tm_k1);
         prefetch_tmap(&p.tm_v1);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_holder), 512);
-        tmem_relinquish();
+        if (CG == 2) {
+            tmem_alloc_pair(smem_u32(tmem_holder), 512);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_holder), 512);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync();               // the peer's barriers exist before anything signals them
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
@@ -316,19 +338,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             Item it;
             int n = 0, k = 0;
             bool ok = true;
-            while (ok && sched_next(p, sc, it)) {
-                int pair, head;
-                unit_coords(p, it.unit, pair, head);
-                const int q0 = pair * kPairRows;
+            while (ok && sched_next<CG>(p, sc, it)) {
+                int unit_row, head;
+                unit_coords(p, it.unit, unit_row, head);
+                const int q0 = unit_row * p.unit_rows;            // first row of the unit
+                const int my_q0 = q0 + (int)rank * kPairRows;     // this CTA's rows
                 if (k > 0 && !mbar_wait(bar(L::bQfree), (k - 1) & 1, kWaitNs)) {
                     raise_timeout(p, abort_flag);
                     break;
                 }
-                mbar_arrive_tx(bar(L::bQ), 2 * L::kTileBytes);
+                if (rank == 0) mbar_arrive_tx(bar(L::bQ), CG * 2 * L::kTileBytes);
                 for (int i = 0; i < 2; ++i)
-                    for (int b = 0; b < NBOX; ++b)
-                        tma_load_3d(sQ + i * L::kTileBytes + b * 16384, &p.tm_q, bar(L::bQ), b * 64, head,
-                                    q0 + i * kBM);
+                    for (int b = 0; b < NBOX; ++b) {
+                        if (CG == 2)
+                            tma_load_3d_pair(sQ + i * L::kTileBytes + b * 16384, &p.tm_q, lead(L::bQ), b * 64, head,
+                                             my_q0 + i * kBM);
+                        else
+                            tma_load_3d(sQ + i * L::kTileBytes + b * 16384, &p.tm_q, bar(L::bQ), b * 64, head,
+                                        my_q0 + i * kBM);
+                    }
                 int s, tt;
                 locate_tile(p, q0, it.t0, s, tt);
                 int ntile = seg_tiles(p, s, q0);
@@ -341,22 +369,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     const KvSeg g = p.seg[s];
                     const int row = g.row0 + tt * kBN;
                     for (int kv = 0; kv < 2; ++kv, ++n) {
-                        const int slot = n % kSlots, use = n / kSlots;
+                        const int slot = n % L::kSlots, use = n / L::kSlots;
                         if (*abort_flag) { ok = false; break; }
                         if (use > 0 && !mbar_wait(bar(L::bEmpty + slot), (use - 1) & 1, kWaitNs)) {
                             raise_timeout(p, abort_flag);
                             ok = false;
                             break;
                         }
-                        const uint32_t dst = sKV + slot * L::kTileBytes;
-                        mbar_arrive_tx(bar(L::bFull + slot), L::kTileBytes);
-                        const CUtensorMap *map =
-                            g.src == 0 ? (kv ? &p.tm_v0 : &p.tm_k0) : (kv ? &p.tm_v1 : &p.tm_k1);
-                        for (int b = 0; b < NBOX; ++b) {
+                        const uint32_t dst = sKV + slot * L::kSlotBytes;
+                        if (rank == 0) mbar_arrive_tx(bar(L::bFull + slot), CG * L::kSlotBytes);
+                        if (CG == 1) {
+                            const CUtensorMap *map =
+                                g.src == 0 ? (kv ? &p.tm_v0 : &p.tm_k0) : (kv ? &p.tm_v1 : &p.tm_k1);
+                            for (int b = 0; b < NBOX; ++b) {
+                                if (g.src == 0)
+                                    tma_load_3d(dst + b * 16384, map, bar(L::bFull + slot), b * 64, row, head);
+                                else
+                                    tma_load_3d(dst + b * 16384, map, bar(L::bFull + slot), b * 64, head, row);
+                            }
+                        } else if (kv == 0) {
+                            // K: this CTA's half of the key rows, all of d
+                            const CUtensorMap *map = g.src == 0 ? &p.tm_k0h : &p.tm_k1h;
+                            const int r = row + (int)rank * kKRows;
+                            for (int b = 0; b < NBOX; ++b) {
+                                const uint32_t d_b = dst + b * (kKRows * 128);
+                                if (g.src == 0)
+                                    tma_load_3d_pair(d_b, map, lead(L::bFull + slot), b * 64, r, head);
+                                else
+                                    tma_load_3d_pair(d_b, map, lead(L::bFull + slot), b * 64, head, r);
+                            }
+                        } else {
+                            // V: all key rows, this CTA's half of d (64 columns)
+                            const CUtensorMap *map = g.src == 0 ? &p.tm_v0 : &p.tm_v1;
                             if (g.src == 0)
-                                tma_load_3d(dst + b * 16384, map, bar(L::bFull + slot), b * 64, row, head);
+                                tma_load_3d_pair(dst, map, lead(L::bFull + slot), (int)rank * 64, row, head);
                             else
-                                tma_load_3d(dst + b * 16384, map, bar(L::bFull + slot), b * 64, head, row);
+                                tma_load_3d_pair(dst, map, lead(L::bFull + slot), (int)rank * 64, head, row);
                         }
                     }
                     ++tt;
@@ -367,90 +415,108 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, 0, 0);
-            constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, 0, 1);
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(kBM * CG, kBN, 0, 0);
+            constexpr uint32_t idesc_o = idesc_bf16_f32(kBM * CG, D, 0, 1);
             // Descriptors depend only on the buffer: build them once, then
             // step along K by adding the byte offset >> 4 to the start-address
-            // field (no carry: every address is below 256 KB).
+            // field (no carry: every address is below 256 KB).  In pair mode the
+            // same offsets address the peer CTA's half of each operand.
             const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
             const uint64_t dq1 = smem_desc_sw128(sQ + L::kTileBytes, 16, 1024);
             const uint64_t dk0 = smem_desc_sw128(sKV, 16, 1024);
             const uint64_t dv0 = smem_desc_sw128(sKV, 16384, 1024);
             auto issue_s = [&](int i, int slot) {
                 const uint64_t a0 = i ? dq1 : dq0;
-                const uint64_t b0 = dk0 + (uint64_t)((slot * L::kTileBytes) >> 4);
+                const uint64_t b0 = dk0 + (uint64_t)((slot * L::kSlotBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
-                    mma_ss(tmem + i * 128, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t a_off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
+                    const uint32_t b_off = ((kk / 4) * (kKRows * 128) + (kk % 4) * 32) >> 4;
+                    if (CG == 2)
+                        mma_ss_pair(tmem + i * 128, a0 + a_off, b0 + b_off, idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss(tmem + i * 128, a0 + a_off, b0 + b_off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int i, int slot, bool acc) {
-                const uint64_t b0 = dv0 + (uint64_t)((slot * L::kTileBytes) >> 4);
+                const uint64_t b0 = dv0 + (uint64_t)((slot * L::kSlotBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts(tmem + 256 + i * D, tmem + i * 128 + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_o,
-                           (acc || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    if (CG == 2)
+                        mma_ts_pair(tmem + 256 + i * D, tmem + i * 128 + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4),
+                                    idesc_o, (acc || kk > 0) ? 1u : 0u);
+                    else
+                        mma_ts(tmem + 256 + i * D, tmem + i * 128 + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4),
+                               idesc_o, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            auto commit = [&](int i) {
+                if (CG == 2) tc_commit_pair(bar(i));
+                else tc_commit(bar(i));
             };
             Sched sc;
             Item it;
             int n = 0, k = 0, jj = 0;   // ring loads consumed, items, tiles (S/P phases)
             bool ok = true;
-            while (ok && sched_next(p, sc, it)) {
+            while (ok && sched_next<CG>(p, sc, it)) {
                 const int T = it.t1 - it.t0;
-                ok = mbar_wait(bar(L::bQ), k & 1, kWaitNs) && !*abort_flag;
+                ok = wait(bar(L::bQ), k & 1) && !*abort_flag;
                 if (!ok) break;
-                int slot = n % kSlots;
-                ok = mbar_wait(bar(L::bFull + slot), (n / kSlots) & 1, kWaitNs);
+                int slot = n % L::kSlots;
+                ok = wait(bar(L::bFull + slot), (n / L::kSlots) & 1);
                 if (!ok) break;
                 tc_fence_after();
                 int kslot = slot;
                 issue_s(0, kslot);
-                tc_commit(bar(L::bS + 0));
+                commit(L::bS + 0);
                 issue_s(1, kslot);
-                tc_commit(bar(L::bS + 1));
-                tc_commit(bar(L::bEmpty + slot));
+                commit(L::bS + 1);
+                commit(L::bEmpty + slot);
                 ++n;
                 for (int j = 0; j < T; ++j, ++jj) {
-                    const int vs = n % kSlots;
-                    ok = mbar_wait(bar(L::bFull + vs), (n / kSlots) & 1, kWaitNs);
+                    const int vs = n % L::kSlots;
+                    ok = wait(bar(L::bFull + vs), (n / L::kSlots) & 1);
                     if (!ok) break;
                     ++n;
                     const int vslot = vs;
-                    ok = mbar_wait(bar(L::bP + 0), jj & 1, kWaitNs) && !*abort_flag;
+                    ok = wait(bar(L::bP + 0), jj & 1) && !*abort_flag;
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(0, vslot, j > 0);
-                    if (j == T - 1) tc_commit(bar(L::bO + 0));
+                    if (j == T - 1) commit(L::bO + 0);
                     int ks = -1;
                     if (j + 1 < T) {
-                        ks = n % kSlots;
-                        ok = mbar_wait(bar(L::bFull + ks), (n / kSlots) & 1, kWaitNs);
+                        ks = n % L::kSlots;
+                        ok = wait(bar(L::bFull + ks), (n / L::kSlots) & 1);
                         if (!ok) break;
                         tc_fence_after();
                         kslot = ks;
                         issue_s(0, kslot);
-                        tc_commit(bar(L::bS + 0));
+                        commit(L::bS + 0);
                     }
-                    ok = mbar_wait(bar(L::bP + 1), jj & 1, kWaitNs) && !*abort_flag;
+                    ok = wait(bar(L::bP + 1), jj & 1) && !*abort_flag;
                     if (!ok) break;
                     tc_fence_after();
                     issue_pv(1, vslot, j > 0);
-                    tc_commit(bar(L::bEmpty + vs));
-                    if (j == T - 1) tc_commit(bar(L::bO + 1));
+                    commit(L::bEmpty + vs);
+                    if (j == T - 1) commit(L::bO + 1);
                     if (j + 1 < T) {
                         issue_s(1, kslot);
-                        tc_commit(bar(L::bS + 1));
-                        tc_commit(bar(L::bEmpty + ks));
+                        commit(L::bS + 1);
+                        commit(L::bEmpty + ks);
                         ++n;
                     }
                 }
                 ++k;
             }
             if (!ok) raise_timeout(p, abort_flag);
-            // Drain: every MMA issued above has completed before TMEM is freed.
-            tc_commit(bar(L::bDrain));
+            // Drain: every MMA issued above has completed before TMEM is freed
+            // (in pair mode the commit also releases the peer CTA).
+            commit(L::bDrain);
+            mbar_wait(bar(L::bDrain), 0, kWaitNs);
+        } else if (lane == 0) {
+            // pair mode, rank 1: wait until rank 0's MMAs into this CTA's TMEM are done
             mbar_wait(bar(L::bDrain), 0, kWaitNs);
         }
         __syncwarp();
@@ -470,11 +536,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
         Item it;
         int k = 0, jj = 0;
         bool ok = true;
-        while (ok && sched_next(p, sc, it)) {
-            int pair, head;
-            unit_coords(p, it.unit, pair, head);
-            const int q0 = pair * kPairRows;
-            const int q_row = q0 + i * kBM + row_local;
+        while (ok && sched_next<CG>(p, sc, it)) {
+            int unit_row, head;
+            unit_coords(p, it.unit, unit_row, head);
+            const int q0 = unit_row * p.unit_rows;              // first row of the unit
+            const int my_q0 = q0 + (int)rank * kPairRows;       // this CTA's rows
+            const int q_row = my_q0 + i * kBM + row_local;
             const int row_vis_end = (q_row / p.kpf + 1) * p.kpf;
             float m_run = -INFINITY, l_run = 0.f;
             int s, tt;
@@ -555,7 +622,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(L::bP + i));
+                if (lane == 0) {
+                    if (CG == 2) mbar_arrive_cluster(lead(L::bP + i));
+                    else mbar_arrive(bar(L::bP + i));
+                }
             }
             if (!ok) break;
             // -------------------------------------------------------- epilogue
@@ -610,9 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             if (row_local == 0) {
                 const bool all = mbar_wait(bar(L::bEpi + i), k & 1, kWaitNs);
                 if (!all) raise_timeout(p, abort_flag);
-                if (all && it.slot < 0 && q0 + i * kBM < p.nq) {
+                if (all && it.slot < 0 && my_q0 + i * kBM < p.nq) {
                     for (int b = 0; b < NBOX; ++b)
-                        tma_store_3d(&p.tm_o, sOut + b * 16384, b * 64, head, q0 + i * kBM);
+                        tma_store_3d(&p.tm_o, sOut + b * 16384, b * 64, head, my_q0 + i * kBM);
                     bulk_commit();
                     bulk_wait_read0();
                 }
@@ -624,24 +694,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     }
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync();               // neither CTA leaves while the pair's MMAs may touch it
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        if (CG == 2) tmem_dealloc_pair(tmem, 512);
+        else tmem_dealloc(tmem, 512);
     }
 }
 
-// Merge the partial results of units split across CTAs.  Grid: (units of the
-// shared remainder, 4); each block covers 64 query rows of one unit, each
-// thread one row and a quarter of the head dimension.
-template <int D>
+// Merge the partial results of units split across clusters.  Grid: (units of
+// the shared remainder, CG * 4); each block covers 64 query rows of one CTA's
+// share of a unit, each thread one row and a quarter of the head dimension.
+template <int D, int CG>
 __global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcParams p) {
     const int ru = p.full_rounds * p.grid + blockIdx.x;
     if (ru >= p.n_units) return;
     const long long U = p.rem_U[blockIdx.x];
-    int pair, head;
-    unit_coords(p, ru, pair, head);
-    const int T = pair_tiles(p, pair);
-    // CTA whose range holds tile x: rem_lo[c] <= x < rem_lo[c+1]
+    int unit_row, head;
+    unit_coords(p, ru, unit_row, head);
+    const int T = pair_tiles(p, unit_row);
+    // cluster whose range holds tile x: rem_lo[c] <= x < rem_lo[c+1]
     auto owner = [&](long long x) {
         int lo = 0, hi = p.grid - 1;
         while (lo < hi) {
@@ -651,16 +723,17 @@ __global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcPa
         return lo;
     };
     const int c0 = owner(U), c1 = owner(U + T - 1);
-    if (c0 == c1) return;                           // whole unit: written by its CTA
-    const int row = blockIdx.y * 64 + (threadIdx.x >> 2);
+    if (c0 == c1) return;                           // whole unit: written by its cluster
+    const int r = blockIdx.y / 4;                   // CTA of the cluster
+    const int row = (blockIdx.y % 4) * 64 + (threadIdx.x >> 2);   // row within that CTA's share
     const int quarter = threadIdx.x & 3;            // D/4 columns each
-    const int q = pair * kPairRows + row;
+    const int q = unit_row * p.unit_rows + r * kPairRows + row;
     if (q >= p.nq) return;
     float M = -INFINITY;
     for (int c = c0; c <= c1; ++c) {
         if (p.rem_lo[c] == p.rem_lo[c + 1]) continue;
         const int slot = (c == c0 && U != p.rem_lo[c0]) ? 1 : 0;
-        M = fmaxf(M, p.part_ml[((size_t)c * 2 + slot) * kPairRows + row].x);
+        M = fmaxf(M, p.part_ml[((size_t)(c * CG + r) * 2 + slot) * kPairRows + row].x);
     }
     constexpr int NV = D / 16;                       // float4 per thread
     float l = 0.f;
@@ -670,7 +743,7 @@ __global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcPa
     for (int c = c0; c <= c1; ++c) {
         if (p.rem_lo[c] == p.rem_lo[c + 1]) continue;
         const int slot = (c == c0 && U != p.rem_lo[c0]) ? 1 : 0;
-        const size_t base = (size_t)c * 2 + slot;
+        const size_t base = (size_t)(c * CG + r) * 2 + slot;
         const float2 ml = p.part_ml[base * kPairRows + row];
         const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
         l += w * ml.y;
@@ -697,36 +770,56 @@ __global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcPa
     }
 }
 
-template <int D>
+template <int D, int CG>
 cudaError_t launch_tc(const TcParams &tp, bool has_split, cudaStream_t s) {
-    using L = Layout<D>;
+    using L = Layout<D, CG>;
     static int configured_mask = 0;   // per device bit (up to 32 devices)
     int dev = 0;
     cudaGetDevice(&dev);
     if (!(configured_mask & (1 << dev))) {
-        cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+        cudaError_t e =
+            cudaFuncSetAttribute(attn_fwd_tc<D, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
         if (e != cudaSuccess) return e;
         configured_mask |= 1 << dev;
     }
-    attn_fwd_tc<D><<<tp.grid, kThreads, L::kAlloc, s>>>(tp);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (CG == 2) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(tp.grid * 2);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = L::kAlloc;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, attn_fwd_tc<D, CG>, tp);
+    } else {
+        attn_fwd_tc<D, CG><<<tp.grid, kThreads, L::kAlloc, s>>>(tp);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
+    count_launch();
     const int rem_units = tp.n_units - tp.full_rounds * tp.grid;
     if (rem_units > 0 && has_split) {
-        attn_combine<D><<<dim3(rem_units, kPairRows / 64), 256, 0, s>>>(tp);
+        attn_combine<D, CG><<<dim3(rem_units, CG * 4), 256, 0, s>>>(tp);
         e = cudaGetLastError();
+        if (e == cudaSuccess) count_launch();
     }
     return e;
 }
 
-// Host copy of the device's tile count per pair.
-int host_pair_tiles(const AttnProblem &p, int pair) {
+// Host copy of the device's tile count per unit (rows [idx*unit_rows, ...)).
+int host_pair_tiles(const AttnProblem &p, int idx, int unit_rows) {
     int t = 0;
-    const int q0 = pair * kPairRows;
+    const int q0 = idx * unit_rows;
     for (int s = 0; s < p.nseg; ++s) {
         int len = p.seg[s].len;
         if (p.seg[s].causal) {
-            const int q_last = std::min(q0 + kPairRows - 1, p.nq - 1);
+            const int q_last = std::min(q0 + unit_rows - 1, p.nq - 1);
             const int lim = (q_last / p.kpf + 1) * p.kpf;
             len = std::min(len, lim);
         }
@@ -752,15 +845,17 @@ unsigned *device_status_ptr(int device) {
 // full rounds of one unit per CTA, then the remaining units' key tiles cut
 // into per-CTA ranges sized so that every CTA's total (its full-round units
 // plus its range) is as equal as possible.
-void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan) {
-    plan.n_pairs = (p.nq + kPairRows - 1) / kPairRows;
+void plan_attn_bf16(const AttnProblem &p, int sms, int cg, AttnPlan &plan) {
+    plan.cg = (cg == 2 && p.head_dim == 128) ? 2 : 1;
+    plan.unit_rows = kPairRows * plan.cg;
+    plan.n_pairs = (p.nq + plan.unit_rows - 1) / plan.unit_rows;
     plan.n_units = plan.n_pairs * p.heads;
-    const int G = std::max(1, std::min(sms, kMaxGrid));
+    const int G = std::max(1, std::min(sms / plan.cg, kMaxGrid));   // clusters
     plan.full_rounds = plan.n_units / G;
     std::vector<int> pt(plan.n_pairs);
     int tmin = 1 << 30, tmax = 0;
     for (int pr = 0; pr < plan.n_pairs; ++pr) {
-        pt[pr] = host_pair_tiles(p, pr);
+        pt[pr] = host_pair_tiles(p, pr, plan.unit_rows);
         tmin = std::min(tmin, pt[pr]);
         tmax = std::max(tmax, pt[pr]);
     }
@@ -807,7 +902,8 @@ void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan) {
         if (U + T > plan.rem_lo[c + 1]) plan.has_split = true;
         U += T;
     }
-    plan.scratch_bytes = (size_t)plan.grid * 2 * ((size_t)kPairRows * p.head_dim * 4 + (size_t)kPairRows * 8);
+    plan.scratch_bytes =
+        (size_t)plan.cg * plan.grid * 2 * ((size_t)kPairRows * p.head_dim * 4 + (size_t)kPairRows * 8);
 }
 
 namespace {
@@ -819,7 +915,8 @@ void inject_wait_timeouts(int device, int launches) {
 }
 
 cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const CUtensorMap *tm_k0,
-                             const CUtensorMap *tm_v0, unsigned *status, void *scratch, cudaStream_t s) {
+                             const CUtensorMap *tm_k0h, const CUtensorMap *tm_v0, unsigned *status, void *scratch,
+                             cudaStream_t s) {
     TcParams tp;
     memset(&tp, 0, sizeof(tp));
     int dev = 0;
@@ -835,21 +932,28 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
     if (have1) {
         if (!make_tmap_bf16(&tp.tm_k1, p.k1, D, p.heads, p.rows1, 1, kBN)) return cudaErrorInvalidValue;
         if (!make_tmap_bf16(&tp.tm_v1, p.v1, D, p.heads, p.rows1, 1, kBN)) return cudaErrorInvalidValue;
+        if (plan.cg == 2 && !make_tmap_bf16(&tp.tm_k1h, p.k1, D, p.heads, p.rows1, 1, kBN / 2))
+            return cudaErrorInvalidValue;
     } else {
         tp.tm_k1 = tp.tm_q;   // never read; any valid map
         tp.tm_v1 = tp.tm_q;
     }
+    if (plan.cg != 2 || !have1) tp.tm_k1h = tp.tm_k1;
     if (have0) {
         tp.tm_k0 = *tm_k0;
         tp.tm_v0 = *tm_v0;
+        if (plan.cg == 2 && !tm_k0h) return cudaErrorInvalidValue;
+        tp.tm_k0h = tm_k0h ? *tm_k0h : *tm_k0;
     } else {
         tp.tm_k0 = tp.tm_q;
         tp.tm_v0 = tp.tm_q;
+        tp.tm_k0h = tp.tm_q;
     }
     tp.nq = p.nq;
     tp.heads = p.heads;
     tp.kpf = p.kpf;
     tp.nseg = p.nseg;
+    tp.unit_rows = plan.unit_rows;
     for (int i = 0; i < p.nseg; ++i) tp.seg[i] = p.seg[i];
     tp.scale_log2 = p.scale * 1.4426950408889634f;
     tp.status = status;
@@ -862,12 +966,13 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
     for (int c = 0; c <= plan.grid; ++c) tp.rem_lo[c] = plan.rem_lo[c];
     if (plan.rem_U.size() > (size_t)kMaxGrid) return cudaErrorInvalidValue;
     for (size_t i = 0; i < plan.rem_U.size(); ++i) tp.rem_U[i] = plan.rem_U[i];
-    const size_t part_o_bytes = (size_t)plan.grid * 2 * kPairRows * p.head_dim * 4;
+    const size_t part_o_bytes = (size_t)plan.cg * plan.grid * 2 * kPairRows * p.head_dim * 4;
     tp.part_o = static_cast<float4 *>(scratch);
     tp.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(scratch) + part_o_bytes);
     tp.out = static_cast<__nv_bfloat16 *>(p.o);
-    if (p.head_dim == 128) return launch_tc<128>(tp, plan.has_split, s);
-    if (p.head_dim == 64) return launch_tc<64>(tp, plan.has_split, s);
+    if (p.head_dim == 128)
+        return plan.cg == 2 ? launch_tc<128, 2>(tp, plan.has_split, s) : launch_tc<128, 1>(tp, plan.has_split, s);
+    if (p.head_dim == 64) return launch_tc<64, 1>(tp, plan.has_split, s);
     return cudaErrorInvalidValue;
 }
 

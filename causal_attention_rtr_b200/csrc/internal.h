@@ -49,18 +49,25 @@ struct AttnProblem {
 // remaining units' key tiles are cut into per-CTA ranges that even out the
 // CTAs' totals.
 struct AttnPlan {
-    int n_pairs, n_units, grid, full_rounds, head_major;
+    int cg;                    // CTAs per cluster sharing each MMA (1, or 2 for the CTA pair)
+    int unit_rows;             // query rows per unit: 256 per CTA of the cluster
+    int n_pairs, n_units, grid, full_rounds, head_major;   // grid: clusters
     std::vector<int> rem_lo;   // grid + 1 boundaries of the per-CTA remainder ranges
     std::vector<int> rem_U;    // key-tile offset of each remainder unit
     bool has_split;            // some unit is shared by two CTAs (combine kernel runs)
     size_t scratch_bytes;      // partial results of split units
 };
 
-void plan_attn_bf16(const AttnProblem &p, int sms, AttnPlan &plan);
+void plan_attn_bf16(const AttnProblem &p, int sms, int cg, AttnPlan &plan);
+
+// CTAs per cluster for the tensor-core attention: 1, or 2 (CTA-pair MMA) when
+// the environment variable RTR_CTA_GROUP says 2.
+int attn_cta_group();
 
 // Kernel launchers; return cudaSuccess or the launch error.
 cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const CUtensorMap *tm_k0,
-                             const CUtensorMap *tm_v0, unsigned *status, void *scratch, cudaStream_t s);
+                             const CUtensorMap *tm_k0h, const CUtensorMap *tm_v0, unsigned *status, void *scratch,
+                             cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnProblem &p, cudaStream_t s);
 
 // Copy n_tok rows of [n_tok][heads][d] into a head-major buffer
@@ -82,6 +89,9 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, 
                     uint32_t box_mid, uint32_t box_outer);
 
 unsigned *device_status_ptr(int device);
+
+// Count of kernels this library has launched (all devices, since load).
+void count_launch(int n = 1);
 
 // Test hook: the next `launches` tensor-core attention launches on `device`
 // issue no loads, so their bounded waits expire and latch RTR_E_TIMEOUT.

@@ -115,7 +115,9 @@ cudaError_t launch_kv_scatter(const ScatterArgs &a, cudaStream_t s) {
     const unsigned long long per_block = (unsigned long long)kBlock * kUnroll;
     const unsigned long long blocks = (2 * per_tensor + per_block - 1) / per_block;
     kv_scatter<<<(unsigned)blocks, kBlock, 0, s>>>(d);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launch();
+    return e;
 }
 
 }  // namespace rtr

@@ -97,13 +97,13 @@ extern "C" rtr_status rtr_attn_block_causal_prefill_noalloc(const void *q, const
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0)
             return RTR_E_CUDA;
         AttnPlan plan;
-        plan_attn_bf16(pb, sms, plan);
+        plan_attn_bf16(pb, sms, attn_cta_group(), plan);
         // The scratch this launch needs must fit in the static array.
         if (plan.scratch_bytes > (size_t)RTR_NOALLOC_SCRATCH_BYTES) return RTR_E_INVAL;
         void *scratch = noalloc_scratch_ptr(device);
         unsigned *status = device_status_ptr(device);
         if (!scratch || !status) return RTR_E_CUDA;
-        e = launch_attn_bf16(pb, plan, nullptr, nullptr, status, scratch, (cudaStream_t)stream);
+        e = launch_attn_bf16(pb, plan, nullptr, nullptr, nullptr, status, scratch, (cudaStream_t)stream);
     } else {
         e = launch_attn_f32(pb, (cudaStream_t)stream);   // the fp32 kernel uses no scratch
     }

@@ -54,6 +54,7 @@ _SIGNATURES = [
     ("rtr_attn_cross", _i, [_vp, _i, _vp, _i, _vp, _f, _vp]),
     ("rtr_get_device_status", _i, [_i, _vp]),
     ("rtr_test_inject_wait_timeout", _i, [_i, _i]),
+    ("rtr_kernel_launches", ctypes.c_ulonglong, []),
 ]
 
 for _name, _res, _args in _SIGNATURES:
@@ -226,3 +227,8 @@ def rtr_test_inject_wait_timeout(device, launches):
     issue no loads, so their bounded waits expire and RTR_E_TIMEOUT is
     latched (see include/rtr.h)."""
     return _check(_lib.rtr_test_inject_wait_timeout(device, launches), "rtr_test_inject_wait_timeout")
+
+
+def rtr_kernel_launches():
+    """Kernels this library has launched since it was loaded."""
+    return int(_lib.rtr_kernel_launches())

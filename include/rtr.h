@@ -231,6 +231,11 @@ rtr_status rtr_get_device_status(int device, rtr_stream_t stream);
  * normally.  launches == 0 cancels.  For tests only. */
 rtr_status rtr_test_inject_wait_timeout(int device, int launches);
 
+/* Number of kernels this library has launched since it was loaded (all
+ * devices and streams).  Diagnostic: lets a caller count the launches of a
+ * region of its own code. */
+unsigned long long rtr_kernel_launches(void);
+
 /* Library build information (static string). */
 const char *rtr_build_info(void);
 
