@@ -55,7 +55,7 @@
 #include "ptx.cuh"
 
 #ifndef RTR_REGS_LOW
-#define RTR_REGS_LOW 88      // producer / MMA warpgroup after setmaxnreg
+#define RTR_REGS_LOW 120     // producer / MMA warpgroup after setmaxnreg
 #endif
 #define RTR_REGS_HIGH (168 + (168 - RTR_REGS_LOW) / 2)   // each softmax warpgroup
 #ifndef RTR_UNIT_ORDER_RATIO
@@ -239,28 +239,23 @@ __device__ __forceinline__ void locate_tile(const TcParams &p, int q0, int t, in
     tt = t;
 }
 
-// P = exp2(s * scale_log2 - m) for one row of 128 scores, packed to bf16
-// pairs and stored over the row's first 64 TMEM columns; row sums into acc.
-// The scale-and-shift and the sums use packed f32x2 instructions.
+// P = exp2(s * scale_log2 - m) for 32 scores of a row, packed to 16 bf16
+// pairs and stored at TMEM column `tP`; row sums into acc.  The scale-and-
+// shift and the sums use packed f32x2 instructions.
 template <bool POLY>
-__device__ __forceinline__ void softmax_probs(const uint32_t (&sr)[128], float sl2, float neg_m, uint32_t tS,
+__device__ __forceinline__ void softmax_chunk(const uint32_t (&sr)[32], float sl2, float neg_m, uint32_t tP,
                                               float2 (&acc)[4]) {
     const float2 sl2x2 = make_float2(sl2, sl2), negm2 = make_float2(neg_m, neg_m);
+    uint32_t pk[16];
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int c = 32 * q4 + 2 * e;
-            const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
-            const bool poly = POLY && (e % 4) < (RTR_EXP2_POLY_PER8 / 2);
-            const float2 pr = make_float2(poly ? exp2_poly(x.x) : fast_exp2(x.x),
-                                          poly ? exp2_poly(x.y) : fast_exp2(x.y));
-            acc[e & 3] = fadd2(acc[e & 3], pr);
-            pk[e] = pack_bf16x2(pr.x, pr.y);
-        }
-        tmem_st16(tS + 16 * q4, pk);
+    for (int e = 0; e < 16; ++e) {
+        const float2 x = ffma2(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2x2, negm2);
+        const bool poly = POLY && (e % 4) < (RTR_EXP2_POLY_PER8 / 2);
+        const float2 pr = make_float2(poly ? exp2_poly(x.x) : fast_exp2(x.x), poly ? exp2_poly(x.y) : fast_exp2(x.y));
+        acc[e & 3] = fadd2(acc[e & 3], pr);
+        pk[e] = pack_bf16x2(pr.x, pr.y);
     }
+    tmem_st16(tP, pk);
 }
 
 template <int D, int CG>
@@ -560,33 +555,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 w = __all_sync(0xffffffffu, w);
                 if (!w) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sr[128];
-                tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-                tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-                tmem_wait_ld();
-                // Warp-uniform: the code below holds tcgen05.st.sync.aligned,
-                // which every lane of the warp must execute together.
+                // Pass 1: row max, 64 columns per TMEM round trip (the row is read
+                // again in pass 2 instead of being held in registers).
+                // Warp-uniform: the code below holds tcgen05 .sync.aligned
+                // instructions, which every lane of the warp must execute together.
                 const bool masked = __any_sync(0xffffffffu, lim < kBN);
-                if (masked) {
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < kBN; ++c)
-                        if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
-                }
-#define SV(c) __uint_as_float(sr[c])
-                float mx0 = max3f(SV(0), SV(1), SV(2)), mx1 = max3f(SV(3), SV(4), SV(5));
-                float mx2 = max3f(SV(6), SV(7), SV(8)), mx3 = max3f(SV(9), SV(10), SV(11));
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32(tS + 64 * h, ra);
+                    tmem_ld32(tS + 64 * h + 32, rb);
+                    tmem_wait_ld();
+                    if (masked) {
 #pragma unroll
-                for (int c = 12; c < 124; c += 8) {
-                    mx0 = max3f(mx0, SV(c + 0), SV(c + 1));
-                    mx1 = max3f(mx1, SV(c + 2), SV(c + 3));
-                    mx2 = max3f(mx2, SV(c + 4), SV(c + 5));
-                    mx3 = max3f(mx3, SV(c + 6), SV(c + 7));
+                        for (int e = 0; e < 32; ++e) {
+                            if (64 * h + e >= lim) ra[e] = __float_as_uint(-INFINITY);
+                            if (64 * h + 32 + e >= lim) rb[e] = __float_as_uint(-INFINITY);
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        mx0 = max3f(mx0, __uint_as_float(ra[e + 0]), __uint_as_float(ra[e + 1]));
+                        mx1 = max3f(mx1, __uint_as_float(ra[e + 2]), __uint_as_float(ra[e + 3]));
+                        mx2 = max3f(mx2, __uint_as_float(ra[e + 4]), __uint_as_float(ra[e + 5]));
+                        mx3 = max3f(mx3, __uint_as_float(ra[e + 6]), __uint_as_float(ra[e + 7]));
+                        mx0 = max3f(mx0, __uint_as_float(rb[e + 0]), __uint_as_float(rb[e + 1]));
+                        mx1 = max3f(mx1, __uint_as_float(rb[e + 2]), __uint_as_float(rb[e + 3]));
+                        mx2 = max3f(mx2, __uint_as_float(rb[e + 4]), __uint_as_float(rb[e + 5]));
+                        mx3 = max3f(mx3, __uint_as_float(rb[e + 6]), __uint_as_float(rb[e + 7]));
+                    }
                 }
-                mx0 = max3f(mx0, SV(124), SV(125));
-                mx1 = max3f(mx1, SV(126), SV(127));
-#undef SV
                 const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
                 const float m_new = fmaxf(m_run, mx * sl2);
                 const bool upd = m_new > m_run + 8.0f;
@@ -610,12 +609,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
                 float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                                  make_float2(0.f, 0.f)};
-                // The polynomial exp2 runs only on tiles without masked
-                // entries (every input finite); ex2 maps -inf to exactly 0.
-                if (masked)
-                    softmax_probs<false>(sr, sl2, neg_m, tS, acc);
-                else
-                    softmax_probs<true>(sr, sl2, neg_m, tS, acc);
+                // Pass 2: P for 32 columns per step, the next 32 loading while
+                // these are computed; P (bf16 pairs) goes over the row's first
+                // 64 columns, behind the scores already read.  The polynomial
+                // exp2 runs only on tiles without masked entries (every input
+                // finite); ex2 maps -inf to exactly 0.
+                {
+                    uint32_t buf[2][32];
+                    tmem_ld32(tS, buf[0]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        if (q4 < 3) tmem_ld32(tS + 32 * (q4 + 1), buf[(q4 + 1) & 1]);
+                        if (masked) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (32 * q4 + e >= lim) buf[q4 & 1][e] = __float_as_uint(-INFINITY);
+                            softmax_chunk<false>(buf[q4 & 1], sl2, neg_m, tS + 16 * q4, acc);
+                        } else {
+                            softmax_chunk<true>(buf[q4 & 1], sl2, neg_m, tS + 16 * q4, acc);
+                        }
+                        if (q4 < 3) tmem_wait_ld();
+                    }
+                }
                 const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
                 const float2 a4 = fadd2(a01, a23);
                 l_run += a4.x + a4.y;
