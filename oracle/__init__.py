@@ -18,13 +18,18 @@ Streaming Video Stylization with Autoregressive Diffusion Transformer"):
   keeps the most recent frame.
 * Method > Key Designs 1 -- the reference latent is one extra latent frame in
   front of the first frame; TV2V has no reference (c = {empty, c_text}).
+* Method > Key Designs 3 -- training (Self Forcing, DMD) runs gradient descent
+  through the block-causal attention; ``backward.py`` holds its plain
+  derivative.
 
-Every function here is the plain definition; see ``attention.py`` and
-``cache.py``.  Parity pins live in ``tests/test_oracle_*.py``.
+Every function here is the plain definition; see ``attention.py``,
+``cache.py`` and ``backward.py``.  Parity pins live in ``tests/test_oracle_*.py``.
 """
 from .attention import (attention, prefill, visible, decode, max_threads,
                         library_path)
 from .cache import ReferenceCache, CrossCache
+from .backward import prefill_lse, prefill_backward, prefill_backward_key_rows
 
 __all__ = ["attention", "prefill", "visible", "decode", "max_threads",
-           "library_path", "ReferenceCache", "CrossCache"]
+           "library_path", "ReferenceCache", "CrossCache", "prefill_lse",
+           "prefill_backward", "prefill_backward_key_rows"]
