@@ -49,7 +49,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--workload", default="wan13_layer",
-                    choices=["wan13_layer", "prefill_22", "long_stream", "switch_14b", "tiny_f32"],
+                    choices=["wan13_layer", "prefill_22", "prefill_22_bwd", "long_stream", "switch_14b", "tiny_f32"],
                     help="wan13_layer is the headline step; the others print one line each for reference")
     return ap.parse_args()
 
@@ -347,6 +347,29 @@ def run_ours(args, rank, world, local_rank):
     if status != rtr.RTR_OK:
         raise RuntimeError(f"device status {rtr.rtr_status_string(status)}")
 
+    # ---- the same step with the chunk written by the attention launch
+    # (rtr_attn_frame_causal_commit on a cache with commit room for the chunk)
+    cf = rtr.rtr_kvcache_create_ex(1, w.heads, w.head_dim, w.k, w.ref_frames, w.window_frames, C, "bf16", dev_id)
+    rtr.rtr_kvcache_set_reference(cf, 0, dev(x.ref_k), dev(x.ref_v))
+    for fk, fv in zip(x.window_k, x.window_v):
+        rtr.rtr_kvcache_append_frame(cf, 0, dev(fk), dev(fv), 1)
+    for _ in range(max(3, args.warmup)):
+        rtr.rtr_attn_frame_causal_commit(cf, 0, q, kc, vc, C, out, 0.0, sh)
+    evf = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(K):
+        flush.zero_()
+        evf[s][0].record(stream)
+        rtr.rtr_attn_frame_causal_commit(cf, 0, q, kc, vc, C, out, 0.0, sh)
+        evf[s][1].record(stream)
+    torch.cuda.synchronize()
+    fused_ms = [e[0].elapsed_time(e[1]) for e in evf]
+    if rtr.rtr_get_device_status(dev_id, sh) != rtr.RTR_OK:
+        raise RuntimeError("device status not OK after the fused-commit steps")
+    rtr.rtr_kvcache_destroy(cf)
+
     # ---- end to end through the C ABI with host buffers (pinned), copies inside
     # the timed region: every step uploads its Q, K, V from pinned host memory
     # and reads its output back.  Two device buffer sets and a copy stream let
@@ -398,9 +421,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = [e_start.elapsed_time(e_end) / Ke]
 
-    step_mean, attn_mean, app_mean, e2e_mean = max_over_ranks(
-        [statistics.mean(step_ms), statistics.mean(attn_ms), statistics.mean(app_ms), statistics.mean(e2e_ms)],
-        world, "cuda")
+    step_mean, attn_mean, app_mean, e2e_mean, fused_mean = max_over_ranks(
+        [statistics.mean(step_ms), statistics.mean(attn_ms), statistics.mean(app_ms), statistics.mean(e2e_ms),
+         statistics.mean(fused_ms)], world, "cuda")
 
     rtr.rtr_kvcache_destroy(c)
     if rank != 0:
@@ -437,6 +460,10 @@ def run_ours(args, rank, world, local_rank):
                 "ms_per_step": e2e_mean,
                 "how": "pinned host Q/K/V uploaded and output read back every step; copies of neighbouring "
                        "steps overlap the kernels (copy stream, two buffer sets)"},
+        "fused_commit": {"entry": "rtr_attn_frame_causal_commit", "ms_per_step": fused_mean,
+                         "value": job_throughput(flops, fused_mean, world), "unit": "TFLOP/s",
+                         "how": "the same step (attention of the chunk + commit of its 3 frames) with the K/V "
+                                "write done by the attention launch; cache created with commit room 3"},
         "gpu_launches": launches_timed,
         "clocks": clk,
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
@@ -497,6 +524,37 @@ def run_other(args):
         ms = statistics.mean(ts)
         line.update({"config": w.name, "ms_per_call": ms, "tflop_per_call": flops / 1e12,
                      "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc})
+    elif args.workload == "prefill_22_bwd":
+        # backward of the same prefill: algorithmic work 5 matmuls per visible
+        # (query, key) pair = 10 * d flops (2.5x the forward's 4 * d)
+        w = synth.PREFILL_22
+        n, H, d = w.chunk_frames * w.k, w.heads, w.head_dim
+        q, k, v, do = (rnd((n, H, d)) for _ in range(4))
+        out = torch.empty_like(q)
+        lse = torch.empty((H, n), dtype=torch.float32, device="cuda")
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        vis = sum(min(n, (i // w.k + 1) * w.k) for i in range(0, n, 1))
+        flops = 10.0 * d * H * vis
+        rtr.rtr_attn_block_causal_prefill_lse(q, k, v, n, H, d, w.k, "bf16", out, lse, 0.0, 0, sh)
+        for _ in range(3):
+            rtr.rtr_attn_block_causal_backward(q, k, v, out, do, lse, n, H, d, w.k, "bf16", dq, dk, dv, 0.0, 0, sh)
+        ts = []
+        for _ in range(max(1, args.steps)):
+            flush.zero_()
+            a, b = _events(2)
+            a.record()
+            rtr.rtr_attn_block_causal_backward(q, k, v, out, do, lse, n, H, d, w.k, "bf16", dq, dk, dv, 0.0, 0, sh)
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.mean(ts)
+        if rtr.rtr_get_device_status(0, sh) != rtr.RTR_OK:
+            raise RuntimeError("device status not OK after the backward")
+        line.update({"config": w.name + ", backward (dQ, dK, dV)", "ms_per_call": ms,
+                     "tflop_per_call": flops / 1e12, "tflops": flops / ms / 1e9,
+                     "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
+                     "kernels": "bwd_prep + bwd_dkdv (S^T, dP^T, dV, dK) + bwd_dq (S, dP, dQ): 7 tile MMAs per "
+                                "visible tile pair for 5 of algorithmic work"})
     elif args.workload == "long_stream":
         w = synth.LONG_STREAM
         L, H, d, k, C, W = w.layers, w.heads, w.head_dim, w.k, w.chunk_frames, w.window_frames

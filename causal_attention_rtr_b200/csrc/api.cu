@@ -103,9 +103,10 @@ using namespace rtr;
 // ------------------------------------------------------------------ handles
 struct rtr_kvcache {
     int layers, heads, head_dim, k, R, W;
+    int S;                   // physical window slots: W + commit room
     rtr_dtype dt;
     int device;
-    long long rows;          // (R + W) * k rows per head
+    long long rows;          // (R + S) * k rows per head
     size_t layer_bytes;      // heads * rows * head_dim * elt
     char *kbuf = nullptr, *vbuf = nullptr;
     std::vector<int> ref_valid, count;
@@ -183,7 +184,8 @@ rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0
         unsigned *st = device_status_ptr(device);
         if (!st) return RTR_E_CUDA;
         AttnPlan plan;
-        plan_attn_bf16(pb, sm_count(device), attn_cta_group(), plan);
+        // The chunk write (commit) is implemented for one CTA per MMA.
+        plan_attn_bf16(pb, sm_count(device), pb.commit_k ? 1 : attn_cta_group(), plan);
         void *scratch = stream_workspace(device, s, plan.scratch_bytes);
         if (!scratch) return RTR_E_NOMEM;
         e = launch_attn_bf16(pb, plan, tm_k0, tm_k0h, tm_v0, st, scratch, s);
@@ -217,19 +219,25 @@ const char *rtr_build_info(void) {
 
 rtr_status rtr_kvcache_create(int layers, int heads, int head_dim, int k, int ref_frames, int window_frames,
                               rtr_dtype dt, int device, rtr_kvcache **out) {
+    return rtr_kvcache_create_ex(layers, heads, head_dim, k, ref_frames, window_frames, 0, dt, device, out);
+}
+
+rtr_status rtr_kvcache_create_ex(int layers, int heads, int head_dim, int k, int ref_frames, int window_frames,
+                                 int commit_frames, rtr_dtype dt, int device, rtr_kvcache **out) {
     if (!out) return RTR_E_INVAL;
     *out = nullptr;
     if (layers < 1 || !shape_ok(heads, head_dim) || k < 1 || ref_frames < 0 || window_frames < 1 ||
-        (dt != RTR_BF16 && dt != RTR_F32) || device < 0)
+        commit_frames < 0 || commit_frames > window_frames || (dt != RTR_BF16 && dt != RTR_F32) || device < 0)
         return RTR_E_INVAL;
-    const long long rows = (long long)(ref_frames + window_frames) * k;
+    const long long rows = (long long)(ref_frames + window_frames + commit_frames) * k;
     if (rows > (1ll << 30) || (long long)heads * rows * head_dim >= (1ll << 40)) return RTR_E_INVAL;
     DeviceGuard dg(device);
     if (!dg.ok) return RTR_E_INVAL;
     rtr_kvcache *c = new (std::nothrow) rtr_kvcache();
     if (!c) return RTR_E_NOMEM;
     c->layers = layers; c->heads = heads; c->head_dim = head_dim; c->k = k;
-    c->R = ref_frames; c->W = window_frames; c->dt = dt; c->device = device;
+    c->R = ref_frames; c->W = window_frames; c->S = window_frames + commit_frames;
+    c->dt = dt; c->device = device;
     c->rows = rows;
     c->layer_bytes = (size_t)heads * rows * head_dim * elt_size(dt);
     const size_t total = c->layer_bytes * layers;
@@ -310,7 +318,7 @@ rtr_status rtr_kvcache_append_frame(rtr_kvcache *c, int layer, const void *k_new
     a.dst_k = c->kbuf + layer * c->layer_bytes;
     a.dst_v = c->vbuf + layer * c->layer_bytes;
     a.n_tok = n_frames * c->k; a.heads = c->heads; a.row_bytes = c->head_dim * (int)elt_size(c->dt);
-    a.k_frame = c->k; a.first_slot = (int)(c->g[layer] % c->W); a.slot_mod = c->W; a.slot_off = c->R;
+    a.k_frame = c->k; a.first_slot = (int)(c->g[layer] % c->S); a.slot_mod = c->S; a.slot_off = c->R;
     a.rows_per_head = c->rows;
     rtr_status st = cuda_status(launch_kv_scatter(a, (cudaStream_t)stream));
     if (st == RTR_OK) {
@@ -333,8 +341,8 @@ rtr_status rtr_kvcache_get_index_map(const rtr_kvcache *c, int layer, int32_t *s
     const long long g = c->g[layer];
     const int cnt = c->count[layer];
     if (slot_frame) {
-        for (int s = 0; s < c->W; ++s) slot_frame[s] = -1;
-        for (long long f = g - cnt; f < g; ++f) slot_frame[f % c->W] = (int32_t)f;
+        for (int s = 0; s < c->S; ++s) slot_frame[s] = -1;
+        for (long long f = g - cnt; f < g; ++f) slot_frame[f % c->S] = (int32_t)f;
     }
     if (ref_valid) *ref_valid = c->ref_valid[layer];
     if (frames_appended) *frames_appended = g;
@@ -349,8 +357,12 @@ rtr_status rtr_kvcache_device_ptrs(const rtr_kvcache *c, int layer, void **k, vo
     return RTR_OK;
 }
 
-rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q, const void *k_cur,
-                                 const void *v_cur, int n_cur_frames, void *out, float scale, rtr_stream_t stream) {
+namespace {
+
+// The stream attention problem of one layer: key runs for the reference and
+// the held window frames (physical order), then the chunk itself.
+rtr_status stream_problem(const rtr_kvcache *c, int layer, const void *q, const void *k_cur, const void *v_cur,
+                          int n_cur_frames, void *out, float scale, AttnProblem &pb) {
     if (!c || layer < 0 || layer >= c->layers || n_cur_frames < 1) return RTR_E_INVAL;
     if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out)) return RTR_E_INVAL;
     const long long nq = (long long)n_cur_frames * c->k;
@@ -362,7 +374,7 @@ rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q,
     if (c->ref_valid[layer] && c->R > 0) iv.push_back({0, (long long)c->R * c->k});
     const long long g = c->g[layer];
     for (long long f = g - c->count[layer]; f < g; ++f) {
-        const long long s = f % c->W;
+        const long long s = f % c->S;
         iv.push_back({(c->R + s) * c->k, (c->R + s + 1) * c->k});
     }
     std::sort(iv.begin(), iv.end());
@@ -374,7 +386,6 @@ rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q,
             merged.push_back(x);
     }
     if (merged.size() > (size_t)kMaxSegs - 1) return RTR_E_UNSUPPORTED;   // cannot happen: <= 3 runs
-    AttnProblem pb;
     memset(&pb, 0, sizeof(pb));
     pb.nq = (int)nq; pb.heads = c->heads; pb.head_dim = c->head_dim; pb.kpf = c->k;
     for (auto &x : merged) pb.seg[pb.nseg++] = KvSeg{0, (int)x.first, (int)(x.second - x.first), 0};
@@ -383,11 +394,50 @@ rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q,
     pb.q = q; pb.o = out;
     pb.k0 = c->kbuf + layer * c->layer_bytes; pb.v0 = c->vbuf + layer * c->layer_bytes; pb.rows0 = c->rows;
     pb.k1 = k_cur; pb.v1 = v_cur; pb.rows1 = nq;
+    return RTR_OK;
+}
+
+}  // namespace
+
+rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q, const void *k_cur,
+                                 const void *v_cur, int n_cur_frames, void *out, float scale, rtr_stream_t stream) {
+    AttnProblem pb;
+    const rtr_status st = stream_problem(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale, pb);
+    if (st != RTR_OK) return st;
     DeviceGuard dg(c->device);
     const CUtensorMap *tk = c->dt == RTR_BF16 ? &c->tmk[layer] : nullptr;
     const CUtensorMap *tkh = c->dt == RTR_BF16 ? &c->tmk64[layer] : nullptr;
     const CUtensorMap *tv = c->dt == RTR_BF16 ? &c->tmv[layer] : nullptr;
     return run_attention(pb, c->dt, tk, tkh, tv, c->device, (cudaStream_t)stream);
+}
+
+rtr_status rtr_attn_frame_causal_commit(rtr_kvcache *c, int layer, const void *q, const void *k_cur,
+                                        const void *v_cur, int n_cur_frames, void *out, float scale,
+                                        rtr_stream_t stream) {
+    AttnProblem pb;
+    const rtr_status st = stream_problem(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale, pb);
+    if (st != RTR_OK) return st;
+    // The chunk's frames go to slots the held window does not use.
+    if (n_cur_frames > c->S - c->W) return RTR_E_INVAL;
+    DeviceGuard dg(c->device);
+    if (c->dt != RTR_BF16) {
+        // fp32 storage: the attention kernel, then the scatter kernel.
+        rtr_status r = run_attention(pb, c->dt, nullptr, nullptr, nullptr, c->device, (cudaStream_t)stream);
+        if (r != RTR_OK) return r;
+        return rtr_kvcache_append_frame(c, layer, k_cur, v_cur, n_cur_frames, stream);
+    }
+    pb.commit_k = c->kbuf + layer * c->layer_bytes;
+    pb.commit_v = c->vbuf + layer * c->layer_bytes;
+    pb.commit_first_slot = (int)(c->g[layer] % c->S);
+    pb.commit_slots = c->S;
+    pb.commit_row0 = c->R * c->k;
+    const rtr_status r = run_attention(pb, c->dt, &c->tmk[layer], &c->tmk64[layer], &c->tmv[layer], c->device,
+                                       (cudaStream_t)stream);
+    if (r == RTR_OK) {
+        c->g[layer] += n_cur_frames;
+        c->count[layer] = std::min(c->W, c->count[layer] + n_cur_frames);
+    }
+    return r;
 }
 
 rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k, const void *v, int n_tokens, int heads,
@@ -409,6 +459,55 @@ rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k, const voi
     DeviceGuard dg(device);
     if (!dg.ok) return RTR_E_INVAL;
     return run_attention(pb, dt, nullptr, nullptr, nullptr, device, (cudaStream_t)stream);
+}
+
+rtr_status rtr_attn_block_causal_prefill_lse(const void *q, const void *k, const void *v, int n_tokens, int heads,
+                                             int head_dim, int k_per_frame, rtr_dtype dt, void *out, float *lse,
+                                             float scale, int device, rtr_stream_t stream) {
+    if (n_tokens < 0 || !shape_ok(heads, head_dim) || k_per_frame < 1 || (dt != RTR_BF16 && dt != RTR_F32) ||
+        device < 0)
+        return RTR_E_INVAL;
+    if (dt != RTR_BF16) return RTR_E_UNSUPPORTED;
+    if (n_tokens == 0) return RTR_OK;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !lse) return RTR_E_INVAL;
+    if (n_tokens > (1 << 30)) return RTR_E_INVAL;
+    AttnProblem pb;
+    memset(&pb, 0, sizeof(pb));
+    pb.nq = n_tokens; pb.heads = heads; pb.head_dim = head_dim; pb.kpf = k_per_frame;
+    pb.nseg = 1;
+    pb.seg[0] = KvSeg{1, 0, n_tokens, 1};
+    pb.scale = resolve_scale(scale, head_dim);
+    pb.q = q; pb.o = out; pb.k1 = k; pb.v1 = v; pb.rows1 = n_tokens;
+    pb.lse = lse;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    return run_attention(pb, dt, nullptr, nullptr, nullptr, device, (cudaStream_t)stream);
+}
+
+rtr_status rtr_attn_block_causal_backward(const void *q, const void *k, const void *v, const void *out,
+                                          const void *dout, const float *lse, int n_tokens, int heads,
+                                          int head_dim, int k_per_frame, rtr_dtype dt, void *dq, void *dk,
+                                          void *dv, float scale, int device, rtr_stream_t stream) {
+    if (n_tokens < 0 || !shape_ok(heads, head_dim) || k_per_frame < 1 || (dt != RTR_BF16 && dt != RTR_F32) ||
+        device < 0)
+        return RTR_E_INVAL;
+    if (dt != RTR_BF16) return RTR_E_UNSUPPORTED;
+    if (n_tokens == 0) return RTR_OK;
+    for (const void *ptr : {q, k, v, out, dout, (const void *)dq, (const void *)dk, (const void *)dv})
+        if (!aligned16(ptr)) return RTR_E_INVAL;
+    if (!lse || n_tokens > (1 << 30)) return RTR_E_INVAL;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    unsigned *st = device_status_ptr(device);
+    if (!st) return RTR_E_CUDA;
+    void *scratch = stream_workspace(device, (cudaStream_t)stream, bwd_scratch_bytes(n_tokens, heads));
+    if (!scratch) return RTR_E_NOMEM;
+    BwdProblem pb;
+    pb.q = q; pb.k = k; pb.v = v; pb.o = out; pb.dout = dout; pb.lse = lse;
+    pb.dq = dq; pb.dk = dk; pb.dv = dv;
+    pb.n = n_tokens; pb.heads = heads; pb.head_dim = head_dim; pb.kpf = k_per_frame;
+    pb.scale = resolve_scale(scale, head_dim);
+    return cuda_status(launch_attn_bwd(pb, st, scratch, (cudaStream_t)stream));
 }
 
 rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_text, rtr_dtype dt, int device,

@@ -26,6 +26,9 @@
 //   warp 1      tcgen05 issuer (one thread): S_i = Q_i K_j^T into TMEM,
 //               O_i += P_i V_j with P_i read from TMEM (the "A in tensor
 //               memory" form), commits to mbarriers
+//   warps 2-3   chunk write (rtr_attn_frame_causal_commit): copy the chunk's
+//               key / value tiles from the ring slots to their cache rows;
+//               idle otherwise
 //   warps 4-7   softmax for Q0, warps 8-11 softmax for Q1: one thread per
 //               query row reads its S row from TMEM, online softmax in fp32
 //               (exp2 domain; O is rescaled only when the running max grows
@@ -101,6 +104,12 @@ struct TcParams {
     float4 *part_o;     // [CTAs][2][D/4][256]
     float2 *part_ml;    // [CTAs][2][256]: running max (log2 units), row sum
     __nv_bfloat16 *out; // token-major output (combine kernel)
+    // chunk write: the src-1 run's rows into the ring of the head-major
+    // buffers (null commit_k: none); see AttnProblem
+    __nv_bfloat16 *commit_k, *commit_v;
+    long long commit_rows_per_head;
+    int commit_first_slot, commit_slots, commit_row0;
+    float *lse;         // [heads][nq] natural-log row log-sum-exp, or null
 };
 
 // CG = CTAs per cluster working one MMA: 1, or 2 for the CTA-pair MMA
@@ -114,8 +123,9 @@ struct Layout {
     static constexpr int kQ = 0;                            // Q0, Q1
     static constexpr int kKV = 2 * kTileBytes;              // ring slots
     static constexpr int kBars = kKV + kSlots * kSlotBytes; // mbarriers
-    static constexpr int bQ = 0, bQfree = 1, bFull = 2, bEmpty = bFull + kSlots, bS = bEmpty + kSlots,
-                         bP = bS + 2, bO = bP + 2, bEpi = bO + 2, bDrain = bEpi + 2, kNumBars = bDrain + 1;
+    static constexpr int bQ = 0, bQfree = 1, bFull = 2, bEmpty = bFull + kSlots, bCopied = bEmpty + kSlots,
+                         bGo = bCopied + kSlots, bS = bGo + kSlots, bP = bS + 2, bO = bP + 2, bEpi = bO + 2, bDrain = bEpi + 2,
+                         kNumBars = bDrain + 1;
     static constexpr int kMisc = kBars + kNumBars * 8;      // tmem holder, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1 KB alignment
@@ -251,11 +261,47 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&sr)[32], float sl
     for (int e = 0; e < 16; ++e) {
         const float2 x = ffma2(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2x2, negm2);
         const bool poly = POLY && (e % 4) < (RTR_EXP2_POLY_PER8 / 2);
-        const float2 pr = make_float2(poly ? exp2_poly(x.x) : fast_exp2(x.x), poly ? exp2_poly(x.y) : fast_exp2(x.y));
+        const float2 pr = poly ? exp2_poly_x2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
         acc[e & 3] = fadd2(acc[e & 3], pr);
         pk[e] = pack_bf16x2(pr.x, pr.y);
     }
     tmem_st16(tP, pk);
+}
+
+// Chunk write: rows [64*part, 64*part+64) of chunk key (or value) tile tt,
+// held in shared memory at `src` in the TMA layout (D/64 boxes of 128 rows x
+// 128 bytes, 128-byte swizzle), stored to their ring rows.  Lanes cover
+// consecutive 16-byte pieces of a row, so each row is one contiguous store.
+template <int D>
+__device__ __forceinline__ void commit_tile_rows(const TcParams &p, uint32_t src, __nv_bfloat16 *dst, int head,
+                                                 int tt, int part, int lane) {
+    constexpr int kPieces = D / 8;          // 16-byte pieces per row
+    constexpr int kRowsPerStep = 32 / kPieces;
+    const int piece = lane % kPieces, sub = lane / kPieces;
+    const int box = piece / 8, c16 = piece % 8;
+    // Ring row of chunk row r in frame f: commit_row0 + slot(f) * kpf + r - f * kpf.
+    auto ring_row = [&](int r, int f) {
+        int slot = p.commit_first_slot + f;           // < 2 * commit_slots
+        if (slot >= p.commit_slots) slot -= p.commit_slots;
+        return p.commit_row0 + (long long)slot * p.kpf + (r - f * p.kpf);
+    };
+    const int rbase = tt * kBN + 64 * part;
+    const int f0 = rbase / p.kpf;                     // frame of the first row
+    const int r_next = (f0 + 1) * p.kpf;              // first row of the next frame
+    const long long off0 = ring_row(rbase, f0) - rbase;
+#pragma unroll 4
+    for (int r0 = 0; r0 < 64; r0 += kRowsPerStep) {
+        const int row = 64 * part + r0 + sub;         // row within the tile
+        const int r = tt * kBN + row;                 // chunk row
+        if (r < p.nq) {
+            const long long drow = r < r_next ? off0 + r : ring_row(r, r / p.kpf);
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(src + box * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4)));
+            *reinterpret_cast<uint4 *>(dst + ((long long)head * p.commit_rows_per_head + drow) * D + piece * 8) = v;
+        }
+    }
 }
 
 template <int D, int CG>
@@ -285,9 +331,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
     if (threadIdx.x == 0) {
         mbar_init(bar(L::bQ), 1);
         mbar_init(bar(L::bQfree), 2);          // one arrive per softmax group
+        // A slot is free once its MMAs completed (bEmpty) and, if it held a
+        // chunk tile this CTA writes out, once both chunk-write warps have
+        // copied it (bCopied).  bGo tells the chunk-write warps that such a
+        // tile has landed: its phases advance only with copied loads, so a
+        // parity wait on it always names the right load.
         for (int i = 0; i < L::kSlots; ++i) {
             mbar_init(bar(L::bFull + i), 1);
             mbar_init(bar(L::bEmpty + i), 1);
+            mbar_init(bar(L::bCopied + i), 2);
+            mbar_init(bar(L::bGo + i), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(L::bS + i), 1);
@@ -332,6 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             Sched sc;
             Item it;
             int n = 0, k = 0;
+            unsigned copy_pending = 0;     // slots whose last load the chunk-write warps copy out
+            unsigned copy_phase = 0;       // per slot (bit), parity of its next bCopied phase
             bool ok = true;
             while (ok && sched_next<CG>(p, sc, it)) {
                 int unit_row, head;
@@ -363,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     }
                     const KvSeg g = p.seg[s];
                     const int row = g.row0 + tt * kBN;
+                    const bool copied = p.commit_k != nullptr && g.src == 1 && (tt >> 1) == unit_row;
                     for (int kv = 0; kv < 2; ++kv, ++n) {
                         const int slot = n % L::kSlots, use = n / L::kSlots;
                         if (*abort_flag) { ok = false; break; }
@@ -371,6 +427,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                             ok = false;
                             break;
                         }
+                        if (copy_pending & (1u << slot)) {
+                            if (!mbar_wait(bar(L::bCopied + slot), (copy_phase >> slot) & 1, kWaitNs)) {
+                                raise_timeout(p, abort_flag);
+                                ok = false;
+                                break;
+                            }
+                            copy_phase ^= 1u << slot;
+                        }
+                        copy_pending = copied ? (copy_pending | (1u << slot)) : (copy_pending & ~(1u << slot));
                         const uint32_t dst = sKV + slot * L::kSlotBytes;
                         if (rank == 0) mbar_arrive_tx(bar(L::bFull + slot), CG * L::kSlotBytes);
                         if (CG == 1) {
@@ -456,11 +521,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             bool ok = true;
             while (ok && sched_next<CG>(p, sc, it)) {
                 const int T = it.t1 - it.t0;
+                // Unit tiles t >= copy_lo are the chunk's; those with chunk tile
+                // (t - copy_lo) / 2 == the unit's pair index are copied out.
+                int copy_lo = 1 << 30, copy_pair = 0;
+                if (p.commit_k != nullptr) {
+                    int head_m;
+                    unit_coords(p, it.unit, copy_pair, head_m);
+                    copy_lo = pair_tiles(p, copy_pair) - seg_tiles(p, p.nseg - 1, copy_pair * p.unit_rows);
+                }
+                auto go = [&](int t, int slot_) {
+                    if (t >= copy_lo && ((t - copy_lo) >> 1) == copy_pair) mbar_arrive(bar(L::bGo + slot_));
+                };
                 ok = wait(bar(L::bQ), k & 1) && !*abort_flag;
                 if (!ok) break;
                 int slot = n % L::kSlots;
                 ok = wait(bar(L::bFull + slot), (n / L::kSlots) & 1);
                 if (!ok) break;
+                go(it.t0, slot);
                 tc_fence_after();
                 int kslot = slot;
                 issue_s(0, kslot);
@@ -473,6 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     const int vs = n % L::kSlots;
                     ok = wait(bar(L::bFull + vs), (n / L::kSlots) & 1);
                     if (!ok) break;
+                    go(it.t0 + j, vs);
                     ++n;
                     const int vslot = vs;
                     ok = wait(bar(L::bP + 0), jj & 1) && !*abort_flag;
@@ -485,6 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                         ks = n % L::kSlots;
                         ok = wait(bar(L::bFull + ks), (n / L::kSlots) & 1);
                         if (!ok) break;
+                        go(it.t0 + j + 1, ks);
                         tc_fence_after();
                         kslot = ks;
                         issue_s(0, kslot);
@@ -515,6 +594,51 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             mbar_wait(bar(L::bDrain), 0, kWaitNs);
         }
         __syncwarp();
+    } else if (warp >= 2 && p.commit_k != nullptr) {
+        // ------------------------------------------------------------ chunk write
+        // Walks the producer's load sequence and waits (on bGo) only for the
+        // loads it copies.  Chunk key tile tt belongs to the unit of query tiles 2u,
+        // 2u+1 with u = tt / 2 (that unit always loads it), so every chunk
+        // tile is written by exactly one CTA.  The producer refills such a
+        // slot only after both warps arrived on its bCopied barrier.
+        const int part = warp - 2;
+        Sched sc;
+        Item it;
+        int n = 0;
+        unsigned go_phase = 0;         // per slot (bit), parity of its next bGo phase
+        bool ok = true;
+        while (ok && sched_next<CG>(p, sc, it)) {
+            int unit_row, head;
+            unit_coords(p, it.unit, unit_row, head);
+            const int q0 = unit_row * p.unit_rows;
+            int s, tt;
+            locate_tile(p, q0, it.t0, s, tt);
+            int ntile = seg_tiles(p, s, q0);
+            for (int t = it.t0; t < it.t1 && ok; ++t, ++tt) {
+                while (tt >= ntile) {
+                    ++s;
+                    tt = 0;
+                    ntile = seg_tiles(p, s, q0);
+                }
+                const bool mine = p.seg[s].src == 1 && (tt >> 1) == unit_row;
+                if (!mine) {
+                    n += 2;
+                    continue;
+                }
+                for (int kv = 0; kv < 2; ++kv, ++n) {
+                    const int slot = n % L::kSlots;
+                    bool w = !*abort_flag && mbar_wait(bar(L::bGo + slot), (go_phase >> slot) & 1, kWaitNs);
+                    w = __all_sync(0xffffffffu, w);
+                    if (!w) { ok = false; break; }
+                    go_phase ^= 1u << slot;
+                    commit_tile_rows<D>(p, sKV + slot * L::kSlotBytes, kv ? p.commit_v : p.commit_k, head, tt, part,
+                                        lane);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(L::bCopied + slot));
+                }
+            }
+        }
+        if (!ok) raise_timeout(p, abort_flag);
     }
     } else {
         set_max_regs_inc<RTR_REGS_HIGH>();
@@ -652,6 +776,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             const int prow = i * kBM + row_local;       // row within the pair
             if (it.slot < 0) {
                 const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                if (p.lse != nullptr && q_row < p.nq)
+                    p.lse[(size_t)head * p.nq + q_row] =
+                        l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
@@ -774,6 +901,8 @@ __global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcPa
         }
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
+    if (p.lse != nullptr && quarter == 0)
+        p.lse[(size_t)head * p.nq + q] = l > 0.f ? (M + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)q * p.heads + head) * D + quarter * (D / 4));
 #pragma unroll
     for (int e = 0; e < NV / 2; ++e) {
@@ -986,6 +1115,20 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
     tp.part_o = static_cast<float4 *>(scratch);
     tp.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(scratch) + part_o_bytes);
     tp.out = static_cast<__nv_bfloat16 *>(p.o);
+    tp.lse = p.lse;
+    if (p.commit_k) {
+        // the chunk write is implemented for one CTA per MMA and needs the
+        // chunk as the token-major run
+        if (plan.cg != 1 || !p.commit_v || p.commit_slots < 1 || p.commit_first_slot < 0 ||
+            p.commit_first_slot >= p.commit_slots || !have1)
+            return cudaErrorInvalidValue;
+        tp.commit_k = static_cast<__nv_bfloat16 *>(p.commit_k);
+        tp.commit_v = static_cast<__nv_bfloat16 *>(p.commit_v);
+        tp.commit_rows_per_head = p.rows0;
+        tp.commit_first_slot = p.commit_first_slot;
+        tp.commit_slots = p.commit_slots;
+        tp.commit_row0 = p.commit_row0;
+    }
     if (p.head_dim == 128)
         return plan.cg == 2 ? launch_tc<128, 2>(tp, plan.has_split, s) : launch_tc<128, 1>(tp, plan.has_split, s);
     if (p.head_dim == 64) return launch_tc<64, 1>(tp, plan.has_split, s);

@@ -11,6 +11,8 @@
 // are clamped (their result, < 2^-125, is negligible next to the row sum).
 #pragma once
 
+#include "ptx.cuh"   // ffma2, fadd2
+
 #define RTR_EXP2_C0 0.9999280571937561f
 #define RTR_EXP2_C1 0.6932609677314758f
 #define RTR_EXP2_C2 0.2426111251115799f
@@ -27,6 +29,24 @@ __device__ __forceinline__ float exp2_poly(float x) {
     p = fmaf(p, f, RTR_EXP2_C1);
     p = fmaf(p, f, RTR_EXP2_C0);
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// The same evaluation for two inputs at once: the reduction and the Horner
+// steps as packed f32x2 instructions (half the FMA-pipe issue of two scalar
+// calls), the clamp and the exponent insertion per element.  Results are
+// identical to exp2_poly on each element.
+__device__ __forceinline__ float2 exp2_poly_x2(float2 x) {
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);
+    const float2 t = fadd2(x, magic);
+    const float2 n = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+    float2 p = ffma2(make_float2(RTR_EXP2_C3, RTR_EXP2_C3), f, make_float2(RTR_EXP2_C2, RTR_EXP2_C2));
+    p = ffma2(p, f, make_float2(RTR_EXP2_C1, RTR_EXP2_C1));
+    p = ffma2(p, f, make_float2(RTR_EXP2_C0, RTR_EXP2_C0));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 }  // namespace rtr

@@ -42,6 +42,17 @@ struct AttnProblem {
     long long rows0;       // rows per head of the head-major source
     const void *k1, *v1;   // token-major source
     long long rows1;       // rows of the token-major source
+    // Optional write of the token-major source (the chunk) into the
+    // head-major buffers commit_k / commit_v ([heads][rows0][d]) by the same
+    // launch: row r of chunk frame c = r / kpf goes to row commit_row0 +
+    // ((commit_first_slot + c) mod commit_slots) * kpf + r mod kpf.  Null
+    // commit_k: no write.  The rows written must be disjoint from every key
+    // run the launch reads.
+    void *commit_k, *commit_v;
+    int commit_first_slot, commit_slots, commit_row0;
+    // Optional row statistics: lse[h * nq + i] = log sum_j exp(scale q_i.k_j)
+    // over the keys row i sees (natural log, fp32).  Null: not written.
+    float *lse;
 };
 
 // Schedule of the persistent tensor-core kernel for one problem: units are
@@ -59,6 +70,19 @@ struct AttnPlan {
 };
 
 void plan_attn_bf16(const AttnProblem &p, int sms, int cg, AttnPlan &plan);
+
+// Backward pass of the block-causal attention over one sequence (bf16).
+// Token-major [n][heads][head_dim] tensors; lse [heads][n] natural-log row
+// log-sum-exp from the forward.
+struct BwdProblem {
+    const void *q, *k, *v, *o, *dout;
+    const float *lse;
+    void *dq, *dk, *dv;
+    int n, heads, head_dim, kpf;
+    float scale;
+};
+size_t bwd_scratch_bytes(int n, int heads);
+cudaError_t launch_attn_bwd(const BwdProblem &p, unsigned *status, void *scratch, cudaStream_t s);
 
 // CTAs per cluster for the tensor-core attention: 1, or 2 (CTA-pair MMA) when
 // the environment variable RTR_CTA_GROUP says 2.

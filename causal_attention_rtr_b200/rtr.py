@@ -35,6 +35,7 @@ _SIGNATURES = [
     ("rtr_status_string", ctypes.c_char_p, [_i]),
     ("rtr_build_info", ctypes.c_char_p, []),
     ("rtr_kvcache_create", _i, [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
+    ("rtr_kvcache_create_ex", _i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
     ("rtr_kvcache_destroy", None, [_vp]),
     ("rtr_kvcache_set_reference", _i, [_vp, _i, _vp, _vp, _vp]),
     ("rtr_kvcache_clear_reference", _i, [_vp, _i]),
@@ -45,8 +46,12 @@ _SIGNATURES = [
                                        ctypes.POINTER(ctypes.c_int32)]),
     ("rtr_kvcache_device_ptrs", _i, [_vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
     ("rtr_attn_frame_causal", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
+    ("rtr_attn_frame_causal_commit", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
     ("rtr_attn_block_causal_prefill", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     ("rtr_attn_block_causal_prefill_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
+    ("rtr_attn_block_causal_prefill_lse", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _i, _vp]),
+    ("rtr_attn_block_causal_backward", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f,
+                                            _i, _vp]),
     ("rtr_crossattn_create", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
     ("rtr_crossattn_destroy", None, [_vp]),
     ("rtr_crossattn_set_text", _i, [_vp, _i, _vp, _vp, _i, _vp]),
@@ -123,6 +128,13 @@ def rtr_kvcache_create(layers, heads, head_dim, k, ref_frames, window_frames, dt
     return h.value
 
 
+def rtr_kvcache_create_ex(layers, heads, head_dim, k, ref_frames, window_frames, commit_frames, dt, device):
+    h = _vp()
+    _check(_lib.rtr_kvcache_create_ex(layers, heads, head_dim, k, ref_frames, window_frames, commit_frames,
+                                      _dtype(dt), device, ctypes.byref(h)), "rtr_kvcache_create_ex")
+    return h.value
+
+
 def rtr_kvcache_destroy(c):
     _lib.rtr_kvcache_destroy(c)
 
@@ -145,9 +157,10 @@ def rtr_kvcache_retain_last(c, layer, n_frames):
     return _check(_lib.rtr_kvcache_retain_last(c, layer, n_frames), "rtr_kvcache_retain_last")
 
 
-def rtr_kvcache_get_index_map(c, layer, window_frames):
-    """Returns (slot_frame list, ref_valid, frames_appended, count)."""
-    slots = (ctypes.c_int32 * window_frames)()
+def rtr_kvcache_get_index_map(c, layer, n_slots):
+    """Returns (slot_frame list, ref_valid, frames_appended, count).  n_slots:
+    the cache's physical window slots (window_frames + commit_frames)."""
+    slots = (ctypes.c_int32 * n_slots)()
     ref = ctypes.c_int32()
     g = ctypes.c_int64()
     cnt = ctypes.c_int32()
@@ -165,6 +178,28 @@ def rtr_kvcache_device_ptrs(c, layer):
 def rtr_attn_frame_causal(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale=0.0, stream=None):
     return _check(_lib.rtr_attn_frame_causal(c, layer, _ptr(q), _ptr(k_cur), _ptr(v_cur), n_cur_frames,
                                              _ptr(out), float(scale), _stream(stream)), "rtr_attn_frame_causal")
+
+
+def rtr_attn_frame_causal_commit(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale=0.0, stream=None):
+    return _check(_lib.rtr_attn_frame_causal_commit(c, layer, _ptr(q), _ptr(k_cur), _ptr(v_cur), n_cur_frames,
+                                                    _ptr(out), float(scale), _stream(stream)),
+                  "rtr_attn_frame_causal_commit")
+
+
+def rtr_attn_block_causal_prefill_lse(q, k, v, n_tokens, heads, head_dim, k_per_frame, dt, out, lse, scale=0.0,
+                                      device=0, stream=None):
+    return _check(_lib.rtr_attn_block_causal_prefill_lse(_ptr(q), _ptr(k), _ptr(v), n_tokens, heads, head_dim,
+                                                         k_per_frame, _dtype(dt), _ptr(out), _ptr(lse),
+                                                         float(scale), device, _stream(stream)),
+                  "rtr_attn_block_causal_prefill_lse")
+
+
+def rtr_attn_block_causal_backward(q, k, v, out, dout, lse, n_tokens, heads, head_dim, k_per_frame, dt, dq, dk, dv,
+                                   scale=0.0, device=0, stream=None):
+    return _check(_lib.rtr_attn_block_causal_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                                                      n_tokens, heads, head_dim, k_per_frame, _dtype(dt), _ptr(dq),
+                                                      _ptr(dk), _ptr(dv), float(scale), device, _stream(stream)),
+                  "rtr_attn_block_causal_backward")
 
 
 def rtr_attn_block_causal_prefill(q, k, v, n_tokens, heads, head_dim, k_per_frame, dt, out, scale=0.0,

@@ -75,12 +75,13 @@ const char *rtr_status_string(rtr_status s);
  * Reference-preserving rolling KV cache (Key Designs 4; reference frame from
  * Key Designs 1).
  *
- * Per layer the cache holds K and V, each [heads][(ref_frames +
- * window_frames) * k][head_dim]: rows [0, ref_frames*k) are the anchored
- * reference slot, window slot s occupies rows (ref_frames+s)*k ... +k-1.
- * Frame f (counted from creation) lives in slot f mod window_frames.  All
- * slots start empty and the reference starts invalid.  Buffers are zeroed at
- * creation.
+ * Per layer the cache holds K and V, each [heads][(ref_frames + S) *
+ * k][head_dim], with S = window_frames physical window slots
+ * (window_frames + commit_frames for rtr_kvcache_create_ex): rows
+ * [0, ref_frames*k) are the anchored reference slot, window slot s occupies
+ * rows (ref_frames+s)*k ... +k-1.  Frame f (counted from creation) lives in
+ * slot f mod S; at most window_frames frames are held.  All slots start
+ * empty and the reference starts invalid.  Buffers are zeroed at creation.
  *
  * rtr_kvcache_create: layers >= 1, heads >= 1, head_dim in {64, 128}, k >= 1,
  *   ref_frames >= 0, window_frames >= 1, dt RTR_BF16 or RTR_F32, device a
@@ -90,6 +91,19 @@ const char *rtr_status_string(rtr_status s);
 rtr_status rtr_kvcache_create(int layers, int heads, int head_dim, int k,
                               int ref_frames, int window_frames, rtr_dtype dt,
                               int device, rtr_kvcache **out);
+
+/* rtr_kvcache_create with commit room: the ring gets commit_frames physical
+ * slots beyond the window_frames it holds (0 <= commit_frames <=
+ * window_frames; 0 is rtr_kvcache_create).  The spare slots let
+ * rtr_attn_frame_causal_commit write a chunk of up to commit_frames frames
+ * while the frames that chunk attends to stay in place.  Memory per layer
+ * grows by 2 * heads * commit_frames * k * head_dim elements.  This is a
+ * layout choice of the library; the held frames, and so every attention
+ * result, are the same as with rtr_kvcache_create. */
+rtr_status rtr_kvcache_create_ex(int layers, int heads, int head_dim, int k,
+                                 int ref_frames, int window_frames,
+                                 int commit_frames, rtr_dtype dt, int device,
+                                 rtr_kvcache **out);
 
 /* Frees the buffers after synchronising the device.  NULL is ignored. */
 void rtr_kvcache_destroy(rtr_kvcache *c);
@@ -108,8 +122,9 @@ rtr_status rtr_kvcache_clear_reference(rtr_kvcache *c, int layer);
 
 /* Append n_frames latent frames to layer `layer`: k_new / v_new are
  * [n_frames*k][heads][head_dim].  Frame f = frames_appended + i goes to slot
- * f mod window_frames, overwriting (evicting) the oldest frame once the
- * window is full; the reference slot is never written.  Then
+ * f mod S; once the window is full the oldest frames drop out of it
+ * (eviction; with S == window_frames the new frame overwrites the evicted
+ * one's slot); the reference slot is never written.  Then
  * frames_appended += n_frames and count = min(window_frames, count +
  * n_frames).  1 <= n_frames <= window_frames, else RTR_E_INVAL. */
 rtr_status rtr_kvcache_append_frame(rtr_kvcache *c, int layer,
@@ -121,8 +136,8 @@ rtr_status rtr_kvcache_append_frame(rtr_kvcache *c, int layer,
  * page keeps one frame as the bridge (n_frames = 1).  Index-map work only. */
 rtr_status rtr_kvcache_retain_last(rtr_kvcache *c, int layer, int n_frames);
 
-/* Host copy of layer `layer`'s index map.  slot_frame (window_frames
- * entries, may be NULL): frame index held by each slot, -1 if empty.
+/* Host copy of layer `layer`'s index map.  slot_frame (S entries: window_frames
+ * + commit_frames; may be NULL): frame index held by each slot, -1 if empty.
  * ref_valid (may be NULL): 1 if a reference is anchored.  frames_appended
  * (may be NULL): frames appended since creation.  count (may be NULL): frames
  * currently held. */
@@ -155,6 +170,27 @@ rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer,
                                  const void *v_cur, int n_cur_frames,
                                  void *out, float scale, rtr_stream_t stream);
 
+/* rtr_attn_frame_causal followed by the commit of the chunk, as in
+ * rtr_kvcache_append_frame(c, layer, k_cur, v_cur, n_cur_frames), with the
+ * chunk written by the attention launch itself (Key Designs 4: the chunk's
+ * K/V enter the rolling cache once it is generated).  The kernel already
+ * holds each chunk key / value tile in shared memory to attend to it, so the
+ * separate append's re-read of k_cur / v_cur and its launch go away.
+ *
+ * Call it for the last denoising step of a chunk; earlier steps use
+ * rtr_attn_frame_causal.  Requires a cache from rtr_kvcache_create_ex with
+ * commit_frames >= n_cur_frames (else RTR_E_INVAL): frames g..g+n-1 (g =
+ * frames_appended) go to slots (g+i) mod S, which the held frames do not
+ * occupy, so no key this call reads is overwritten.  On success the index
+ * map advances exactly as after rtr_kvcache_append_frame; outputs and cache
+ * bytes are those of the two separate calls.  For fp32 storage the commit
+ * runs as a second kernel. */
+rtr_status rtr_attn_frame_causal_commit(rtr_kvcache *c, int layer,
+                                        const void *q, const void *k_cur,
+                                        const void *v_cur, int n_cur_frames,
+                                        void *out, float scale,
+                                        rtr_stream_t stream);
+
 /* Block-causal attention over one whole sequence (Key Designs 2: training
  * sees all frames at once under M).  q, k, v, out: [n_tokens][heads]
  * [head_dim]; token i belongs to frame floor(i / k_per_frame).  scale <= 0
@@ -165,6 +201,39 @@ rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k,
                                          int k_per_frame, rtr_dtype dt,
                                          void *out, float scale,
                                          int device, rtr_stream_t stream);
+
+/* rtr_attn_block_causal_prefill that also returns each row's log-sum-exp,
+ * the statistic the backward pass needs: lse[h * n_tokens + i] = log
+ * sum_{j visible to i} exp(scale * q_i . k_j) (natural log), fp32
+ * [heads][n_tokens], caller-owned device memory.  bf16 only
+ * (RTR_E_UNSUPPORTED for RTR_F32). */
+rtr_status rtr_attn_block_causal_prefill_lse(const void *q, const void *k,
+                                             const void *v, int n_tokens,
+                                             int heads, int head_dim,
+                                             int k_per_frame, rtr_dtype dt,
+                                             void *out, float *lse,
+                                             float scale, int device,
+                                             rtr_stream_t stream);
+
+/* Backward pass of the block-causal attention (Key Designs 2 and 3: the
+ * causal student is trained with Self Forcing and DMD, whose gradients flow
+ * through this attention).  Given the forward's inputs q, k, v, its output
+ * out and row log-sum-exp lse (from rtr_attn_block_causal_prefill_lse, same
+ * scale), and the upstream gradient dout, writes dq, dk, dv: the gradients
+ * of sum(dout * out) with respect to q, k and v.  All tensors
+ * [n_tokens][heads][head_dim] bf16 (lse fp32 [heads][n_tokens]); outputs
+ * are computed in fp32 and rounded once to bf16.  Caller-owned device
+ * memory, 16-byte aligned; the library uses a per-stream scratch buffer of
+ * 8 * heads * n_tokens bytes (rounded up to 128-row tiles).  bf16 only
+ * (RTR_E_UNSUPPORTED for RTR_F32); n_tokens == 0 is a no-op. */
+rtr_status rtr_attn_block_causal_backward(const void *q, const void *k,
+                                          const void *v, const void *out,
+                                          const void *dout, const float *lse,
+                                          int n_tokens, int heads,
+                                          int head_dim, int k_per_frame,
+                                          rtr_dtype dt, void *dq, void *dk,
+                                          void *dv, float scale, int device,
+                                          rtr_stream_t stream);
 
 /* Block-causal prefill that allocates no device memory.  The paper has no
  * counterpart: this is a library addition for callers that cannot let a

@@ -28,8 +28,10 @@ Every function here is the plain definition; see ``attention.py``,
 from .attention import (attention, prefill, visible, decode, max_threads,
                         library_path)
 from .cache import ReferenceCache, CrossCache
-from .backward import prefill_lse, prefill_backward, prefill_backward_key_rows
+from .backward import (prefill_lse, prefill_backward, prefill_backward_key_rows,
+                       prefill_backward_query_rows)
 
 __all__ = ["attention", "prefill", "visible", "decode", "max_threads",
            "library_path", "ReferenceCache", "CrossCache", "prefill_lse",
-           "prefill_backward", "prefill_backward_key_rows"]
+           "prefill_backward", "prefill_backward_key_rows",
+           "prefill_backward_query_rows"]

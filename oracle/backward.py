@@ -107,3 +107,22 @@ def prefill_backward_key_rows(q, k, v, do, k_per_frame, key_rows, scale=None, bl
             dk[:, h] += scale * (ds.T @ qh[rows])
             dv[:, h] += ps.T @ doh[rows]
     return dk, dv
+
+
+def prefill_backward_query_rows(q, k, v, do, k_per_frame, rows, scale=None):
+    """dQ of selected query rows only: each row's dQ needs only its own row of
+    P and dP.  Returns [len(rows), H, d] float64."""
+    q, k, v, do = (np.asarray(a, np.float64) for a in (q, k, v, do))
+    n, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rows = np.asarray(rows, np.int64)
+    dq = np.empty((rows.size, H, d))
+    for h in range(H):
+        qh, kh, vh, doh = q[:, h], k[:, h], v[:, h], do[:, h]
+        s = _scores(qh, kh, rows, k_per_frame, scale)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        dp = doh[rows] @ vh.T
+        ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+        dq[:, h] = scale * (ds @ kh)
+    return dq

@@ -23,6 +23,12 @@ Readings where the pages are silent (each listed in the design doc):
 * eviction is by whole latent frames, oldest first;
 * without a reference (TV2V) the reference span is simply absent.
 
+Physical placement (a layout choice of this library, not of the pages): the
+window ring may have more physical slots than the W frames it holds
+(``slots`` >= W).  Frame f lives in slot f mod slots; which frames are held,
+and so the attention, does not depend on ``slots``.  The extra slots are
+where a chunk can be written while the W frames it attends to stay intact.
+
 Stored data are the caller's raw bits (uint16 bfloat16 patterns or float32),
 copied exactly.  A slot holds the bytes last written to it; the bytes of an
 invalid slot are unspecified and never compared.
@@ -36,23 +42,25 @@ class ReferenceCache:
     """One layer of the 3D-attention cache.
 
     State: ``ref_valid``; ``g`` = frames appended since creation; ``count`` =
-    frames currently held (<= W); ``slots[s]`` = data of the frame f with
-    f mod W == s.  Slot s holds a valid frame f iff g - count <= f < g.
-    Every tensor is [tokens, H, d].
+    frames currently held (<= W); ``slots_k/v[s]`` = data of the frame f with
+    f mod S == s, S = ``slots`` physical slots (W unless given).  Slot s holds
+    a valid frame f iff g - count <= f < g.  Every tensor is [tokens, H, d].
     """
 
-    def __init__(self, heads, head_dim, k, ref_frames, window_frames, dtype):
-        if min(heads, head_dim, k, window_frames) <= 0 or ref_frames < 0:
+    def __init__(self, heads, head_dim, k, ref_frames, window_frames, dtype, slots=None):
+        slots = window_frames if slots is None else slots
+        if min(heads, head_dim, k, window_frames) <= 0 or ref_frames < 0 or slots < window_frames:
             raise ValueError("bad cache shape")
         self.H, self.d, self.k = heads, head_dim, k
         self.R, self.W = ref_frames, window_frames
+        self.S = slots
         self.dtype = dtype
         raw = np.uint16 if dtype == "bf16" else np.float32
         self._raw = raw
         self.ref_k = np.zeros((ref_frames * k, heads, head_dim), raw)
         self.ref_v = np.zeros_like(self.ref_k)
-        self.slots_k = [np.zeros((k, heads, head_dim), raw) for _ in range(window_frames)]
-        self.slots_v = [np.zeros((k, heads, head_dim), raw) for _ in range(window_frames)]
+        self.slots_k = [np.zeros((k, heads, head_dim), raw) for _ in range(slots)]
+        self.slots_v = [np.zeros((k, heads, head_dim), raw) for _ in range(slots)]
         self.ref_valid = False
         self.g = 0
         self.count = 0
@@ -74,15 +82,16 @@ class ReferenceCache:
         self.ref_valid = False
 
     def append(self, k_new, v_new, n_frames):
-        """Append n frames: frame f goes to slot f mod W, overwriting (=
-        evicting) the oldest frame once the window is full."""
+        """Append n frames: frame f goes to slot f mod S; once the window is
+        full the oldest frames drop out of it (= eviction; with S == W the
+        new frame overwrites the evicted one's slot)."""
         if not 1 <= n_frames <= self.W:
             raise ValueError("n_frames must be in [1, W]")
         k_new = np.asarray(k_new, self._raw).reshape(n_frames, self.k, self.H, self.d)
         v_new = np.asarray(v_new, self._raw).reshape(n_frames, self.k, self.H, self.d)
         for i in range(n_frames):
             f = self.g + i
-            s = f % self.W
+            s = f % self.S
             self.slots_k[s] = k_new[i].copy()
             self.slots_v[s] = v_new[i].copy()
         self.g += n_frames
@@ -101,10 +110,10 @@ class ReferenceCache:
         return list(range(self.g - self.count, self.g))
 
     def index_map(self):
-        """(slot_frame[W] with -1 for empty, ref_valid, g)."""
-        slot_frame = [-1] * self.W
+        """(slot_frame[S] with -1 for empty, ref_valid, g)."""
+        slot_frame = [-1] * self.S
         for f in self.window_frames():
-            slot_frame[f % self.W] = f
+            slot_frame[f % self.S] = f
         return slot_frame, int(self.ref_valid), self.g
 
     def logical_kv(self):
@@ -115,8 +124,8 @@ class ReferenceCache:
             ks.append(self.ref_k)
             vs.append(self.ref_v)
         for f in self.window_frames():
-            ks.append(self.slots_k[f % self.W])
-            vs.append(self.slots_v[f % self.W])
+            ks.append(self.slots_k[f % self.S])
+            vs.append(self.slots_v[f % self.S])
         empty = np.zeros((0, self.H, self.d), self._raw)
         K = np.concatenate(ks, axis=0) if ks else empty
         V = np.concatenate(vs, axis=0) if vs else empty

@@ -36,10 +36,10 @@ def gpu_view(c, layer, H, rows, d, dtype, which):
 
 def compare_cache(c, ref: oracle.ReferenceCache, layer=0):
     from causal_attention_rtr_b200 import rtr
-    slots, ref_valid, g, count = rtr.rtr_kvcache_get_index_map(c, layer, ref.W)
+    slots, ref_valid, g, count = rtr.rtr_kvcache_get_index_map(c, layer, ref.S)
     want_slots, want_ref, want_g = ref.index_map()
     assert (slots, ref_valid, g, count) == (want_slots, want_ref, want_g, ref.count)
-    rows = (ref.R + ref.W) * ref.k
+    rows = (ref.R + ref.S) * ref.k
     for which in ("k", "v"):
         buf = gpu_view(c, layer, ref.H, rows, ref.d, ref.dtype, which)
         if ref.ref_valid:

@@ -76,6 +76,13 @@ def test_validation_before_device_work(lib):
         assert st == rtr.RTR_E_INVAL, args
         assert h.value is None
     assert rtr.raw_status("rtr_kvcache_create", 1, 2, 128, 16, 1, 4, 0, 0, None) == rtr.RTR_E_INVAL
+    # commit room: 0 <= commit_frames <= window_frames
+    for commit in (-1, 5):
+        st = rtr.raw_status("rtr_kvcache_create_ex", 1, 2, 128, 16, 1, 4, commit, 0, 0, ctypes.byref(h))
+        assert st == rtr.RTR_E_INVAL, commit
+        assert h.value is None
+    assert rtr.raw_status("rtr_attn_frame_causal_commit", None, 0, None, None, None, 1, None, 0.0,
+                          None) == rtr.RTR_E_INVAL
     # null handles
     assert rtr.raw_status("rtr_kvcache_append_frame", None, 0, None, None, 1, None) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_attn_frame_causal", None, 0, None, None, None, 1, None, 0.0, None) == rtr.RTR_E_INVAL

@@ -93,8 +93,8 @@ def test_softmax_jacobian_invariants():
 
 
 def test_blocking_and_key_row_selection_agree():
-    """The query-row blocking does not change the result, and the key-row
-    variant returns the same dK, dV rows."""
+    """The query-row blocking does not change the result, and the key-row and
+    query-row variants return the same dK, dV and dQ rows."""
     n, k, H, d = 50, 6, 2, 8
     q, kk, v, do = inputs(n, H, d, 12)
     a = oracle.prefill_backward(q, kk, v, do, k, block=512)
@@ -105,6 +105,8 @@ def test_blocking_and_key_row_selection_agree():
     dk, dv = oracle.prefill_backward_key_rows(q, kk, v, do, k, rows, block=11)
     assert np.allclose(dk, a[1][rows], rtol=1e-12, atol=1e-13)
     assert np.allclose(dv, a[2][rows], rtol=1e-12, atol=1e-13)
+    dq = oracle.prefill_backward_query_rows(q, kk, v, do, k, rows)
+    assert np.allclose(dq, a[0][rows], rtol=1e-12, atol=1e-13)
 
 
 def test_lse_definition():

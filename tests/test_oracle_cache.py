@@ -214,3 +214,62 @@ def test_cross_cache_reset_and_set():
     x.reset()
     with pytest.raises(RuntimeError):
         x.attention(q)
+
+
+@pytest.mark.parametrize("W,extra", [(1, 1), (3, 2), (5, 3), (21, 3)])
+def test_closed_form_eviction_with_spare_slots(W, extra):
+    """With S = W + extra physical slots and no trims, the map is
+    {f mod S -> f, f in [g-min(g,W), g)}: W frames held, S slots addressed."""
+    S = W + extra
+    rng = np.random.default_rng(100 + W)
+    c = oracle.ReferenceCache(1, 2, 1, 1, W, "f32", slots=S)
+    g = 0
+    for _ in range(60):
+        n = int(rng.integers(1, W + 1))
+        c.append(np.zeros((n, 1, 2), np.float32), np.zeros((n, 1, 2), np.float32), n)
+        g += n
+        want = [-1] * S
+        for f in range(g - min(g, W), g):
+            want[f % S] = f
+        assert c.index_map() == (want, 0, g)
+
+
+def test_spare_slots_change_nothing_but_placement():
+    """Two caches fed the same random operations, one with S = W and one with
+    S = W + 3 slots, hold the same logical sequence and give bit-identical
+    attention; every held frame sits at f mod S in its own cache."""
+    H, d, k, W, C = 2, 8, 3, 4, 2
+    rng = np.random.default_rng(77)
+    a = oracle.ReferenceCache(H, d, k, 1, W, "bf16")
+    b = oracle.ReferenceCache(H, d, k, 1, W, "bf16", slots=W + 3)
+    frames = {}
+    g = 0
+    for step in range(40):
+        op = int(rng.integers(0, 6))
+        if op == 0:
+            rk, rv = (synth.normal(rng, (k, H, d), 1.0, "bf16") for _ in range(2))
+            a.set_reference(rk, rv); b.set_reference(rk, rv)
+        elif op == 1:
+            r = int(rng.integers(0, 3))
+            a.retain_last(r); b.retain_last(r)
+        else:
+            n = int(rng.integers(1, W + 1))
+            x, y = (synth.normal(rng, (n * k, H, d), 1.0, "bf16") for _ in range(2))
+            a.append(x, y, n); b.append(x, y, n)
+            for i in range(n):
+                frames[g + i] = x[i * k:(i + 1) * k]
+            g += n
+        Ka, Va = a.logical_kv()
+        Kb, Vb = b.logical_kv()
+        assert np.array_equal(Ka, Kb) and np.array_equal(Va, Vb)
+        assert a.window_frames() == b.window_frames()
+        for f in b.window_frames():
+            assert np.array_equal(b.slots_k[f % (W + 3)], frames[f])
+        if step % 8 == 7:
+            q, kc, vc = (synth.normal(rng, (C * k, H, d), 1.0, "bf16") for _ in range(3))
+            assert np.array_equal(a.stream_attention(q, kc, vc, C), b.stream_attention(q, kc, vc, C))
+
+
+def test_spare_slots_must_cover_window():
+    with pytest.raises(ValueError):
+        oracle.ReferenceCache(1, 2, 1, 1, 4, "f32", slots=3)
