@@ -16,13 +16,18 @@
 //               L +inf, so padded query rows carry exactly zero probability).
 //   bwd_dkdv    key-stationary: one CTA per (head, 128-key tile); streams the
 //               query tiles that see it (frame-causal: query frames >= the
-//               key tile's first frame).  Per query tile: S^T = K Q^T and
-//               dP^T = V dO^T into TMEM, the softmax warps turn them into P^T
-//               and dS^T (bf16, back into TMEM), then dV += P^T dO and
-//               dK += dS^T Q with the "A in tensor memory" form.
+//               key tile's first frame), each as two halves of 64 queries.
+//               Per half: S^T = K Q^T and dP^T = V dO^T into one of two TMEM
+//               buffers, the softmax warps turn them into P^T and dS^T (bf16,
+//               back into TMEM), then dV += P^T dO and dK += dS^T Q with the
+//               "A in tensor memory" form; the tensor core runs the other
+//               buffer's MMAs meanwhile.
 //   bwd_dq      query-stationary: one CTA per (head, 128-query tile); streams
 //               the key tiles it sees.  S = Q K^T and dP = dO V^T into TMEM,
-//               dS (bf16) back into TMEM, dQ += dS K.
+//               dS (bf16) back into TMEM, dQ += dS K.  (The two-buffer scheme
+//               of bwd_dkdv measured 14 % slower here: its 64-wide S and dP
+//               MMAs re-read Q and dO per half, and each half pays the
+//               softmax hand-off again.)
 // Splitting dQ from dK/dV recomputes S and dP once more (7 tile MMAs per
 // (query tile, key tile) instead of 5) but needs no atomic accumulation of
 // dQ across CTAs: every output tile is written once, in bf16, by TMA.
@@ -37,6 +42,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -76,7 +82,7 @@ struct BwdLayout {
     static constexpr int kStage = 2 * kTile + 1024;      // B0, B1, row stats
     static constexpr int kB = 2 * kTile;                 // stage s at kB + s * kStage
     static constexpr int kBars = kB + 2 * kStage;
-    static constexpr int bA = 0, bFull = 1, bEmpty = 3, bS = 5, bP = 6, bO = 7, bEpi = 8, kNumBars = 9;
+    static constexpr int bA = 0, bFull = 1, bEmpty = 3, bS = 5, bP = 7, bO = 9, bEpi = 10, kNumBars = 11;
     static constexpr int kMisc = kBars + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -94,8 +100,8 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap *map, 
     for (int b = 0; b < D / 64; ++b) tma_load_3d(dst + b * 16384, map, bar, b * 64, head, row0);
 }
 
-// SS MMA chain over d: C[128 x 128] = A[128 x D] B[128 x D]^T, both K-major
-// tiles in the TMA layout.
+// SS MMA chain over d: C[128 x N] = A[128 x D] B[N x D]^T, both K-major
+// tiles in the TMA layout (B may start at a row offset inside its tile).
 template <int D>
 __device__ __forceinline__ void mma_tile_ss(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
 #pragma unroll
@@ -105,16 +111,18 @@ __device__ __forceinline__ void mma_tile_ss(uint32_t d_tmem, uint64_t a0, uint64
     }
 }
 
-// TS MMA chain over 128 rows: C[128 x D] (+)= A[128 x 128] B[128 x D] with A
-// packed bf16 pairs in TMEM at a_tmem (8 columns per 16 rows of B) and B the
-// tile in the TMA layout read as MN-major.
-template <int D>
+// TS MMA chain over KR rows of B: C[128 x D] (+)= A[128 x KR] B[KR x D] with
+// A packed bf16 pairs in TMEM at a_tmem (8 columns per 16 rows of B) and B
+// read as MN-major from the TMA layout (16 rows = 2048 bytes per step).
+template <int D, int KR>
 __device__ __forceinline__ void mma_tile_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
                                             bool acc) {
 #pragma unroll
-    for (int kk = 0; kk < kBT / 16; ++kk)
+    for (int kk = 0; kk < KR / 16; ++kk)
         mma_ts(d_tmem, a_tmem + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc, (acc || kk > 0) ? 1u : 0u);
 }
+
+constexpr int kHalf = 64;     // rows of the streamed half tile (MMA N of S / dP)
 
 // Epilogue: 128 x D fp32 accumulator rows (this thread's TMEM lane) times
 // `mul`, to bf16 in the swizzled TMA layout at `dst`.
@@ -154,11 +162,14 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16 *o, const __
     const int h = (int)(warp / n_pad), r = (int)(warp % n_pad);
     float acc = 0.f;
     if (r < n) {
-        constexpr int E = D / 32;     // 2 or 4 elements per lane
-        const __nv_bfloat16 *po = o + ((size_t)r * heads + h) * D + lane * E;
-        const __nv_bfloat16 *pd = dout + ((size_t)r * heads + h) * D + lane * E;
+        constexpr int E = D / 32;     // 2 or 4 elements per lane, one 4- or 8-byte load
+        using Vec = typename std::conditional<E == 4, uint2, uint32_t>::type;
+        const Vec vo = *reinterpret_cast<const Vec *>(o + ((size_t)r * heads + h) * D + lane * E);
+        const Vec vd = *reinterpret_cast<const Vec *>(dout + ((size_t)r * heads + h) * D + lane * E);
+        const __nv_bfloat16 *eo = reinterpret_cast<const __nv_bfloat16 *>(&vo);
+        const __nv_bfloat16 *ed = reinterpret_cast<const __nv_bfloat16 *>(&vd);
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(po[e]), __bfloat162float(pd[e]), acc);
+        for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(eo[e]), __bfloat162float(ed[e]), acc);
     }
 #pragma unroll
     for (int w = 16; w > 0; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
@@ -212,8 +223,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
             mbar_init(bar(L::bFull + s), 1);
             mbar_init(bar(L::bEmpty + s), 1);
         }
-        mbar_init(bar(L::bS), 1);
-        mbar_init(bar(L::bP), 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(L::bS + b), 1);
+            mbar_init(bar(L::bP + b), 4);
+        }
         mbar_init(bar(L::bO), 1);
         mbar_init(bar(L::bEpi), kBT);
         *abort_flag = 0;
@@ -227,7 +240,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    // TMEM: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,256+D), dK [256+D,256+2D)
+    // TMEM: S^T / P^T buffers [0,64), [64,128); dP^T / dS^T buffers [128,192),
+    // [192,256); dV [256,256+D); dK [256+D,256+2D).  Each streamed query tile
+    // is taken as two halves of 64 queries (step t: tile t/2, half t%2,
+    // buffer t%2): while the softmax works on step t the tensor core runs
+    // dV/dK of step t-1 and S^T/dP^T of step t+1.
 
     if (warp == 0) {
         if (lane == 0) {
@@ -254,27 +271,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, 0, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBT, D, 0, 1);
             const uint64_t descK = smem_desc_sw128(sK, 16, 1024), descV = smem_desc_sw128(sV, 16, 1024);
+            constexpr uint32_t idesc_h = idesc_bf16_f32(kBT, kHalf, 0, 0);
             bool ok = mbar_wait(bar(L::bA), 0, kBwdWaitNs);
-            for (int t = 0; ok && t < T; ++t) {
-                const int st = t & 1;
-                const uint32_t sb = stage_b(st);
-                ok = mbar_wait(bar(L::bFull + st), (t >> 1) & 1, kBwdWaitNs) && !*abort_flag;
-                if (!ok) break;
-                tc_fence_after();
-                mma_tile_ss<D>(tmem + 0, descK, smem_desc_sw128(sb, 16, 1024), idesc_s);               // S^T
-                mma_tile_ss<D>(tmem + 128, descV, smem_desc_sw128(sb + L::kTile, 16, 1024), idesc_s);  // dP^T
-                tc_commit(bar(L::bS));
-                ok = mbar_wait(bar(L::bP), t & 1, kBwdWaitNs) && !*abort_flag;
-                if (!ok) break;
-                tc_fence_after();
-                mma_tile_ts<D>(tmem + 256, tmem + 0, smem_desc_sw128(sb + L::kTile, 16384, 1024), idesc_o,
-                               t > 0);                                                              // dV += P^T dO
-                mma_tile_ts<D>(tmem + 256 + D, tmem + 128, smem_desc_sw128(sb, 16384, 1024), idesc_o,
-                               t > 0);                                                              // dK += dS^T Q
-                tc_commit(bar(L::bEmpty + st));
+            for (int t = 0; ok && t <= 2 * T; ++t) {
+                if (t < 2 * T) {
+                    const int ti = t >> 1, h = t & 1, b = t & 1;
+                    const uint32_t sb = stage_b(ti & 1);
+                    if (h == 0) {
+                        ok = mbar_wait(bar(L::bFull + (ti & 1)), (ti >> 1) & 1, kBwdWaitNs) && !*abort_flag;
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
+                    const uint32_t hoff = (uint32_t)(h * kHalf * 128);
+                    mma_tile_ss<D>(tmem + 64 * b, descK, smem_desc_sw128(sb + hoff, 16, 1024), idesc_h);   // S^T
+                    mma_tile_ss<D>(tmem + 128 + 64 * b, descV, smem_desc_sw128(sb + L::kTile + hoff, 16, 1024),
+                                   idesc_h);                                                           // dP^T
+                    tc_commit(bar(L::bS + b));
+                }
+                if (t >= 1) {
+                    const int tp = t - 1, ti = tp >> 1, h = tp & 1, b = tp & 1;
+                    const uint32_t sb = stage_b(ti & 1);
+                    ok = mbar_wait(bar(L::bP + b), (tp >> 1) & 1, kBwdWaitNs) && !*abort_flag;
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t hoff = (uint32_t)(h * kHalf * 128);
+                    mma_tile_ts<D, kHalf>(tmem + 256, tmem + 64 * b, smem_desc_sw128(sb + L::kTile + hoff, 16384, 1024),
+                                          idesc_o, tp > 0);                                    // dV += P^T dO
+                    mma_tile_ts<D, kHalf>(tmem + 256 + D, tmem + 128 + 64 * b, smem_desc_sw128(sb + hoff, 16384, 1024),
+                                          idesc_o, tp > 0);                                    // dK += dS^T Q
+                    if (h == 1) tc_commit(bar(L::bEmpty + (ti & 1)));
+                }
             }
             if (!ok) bwd_timeout(p, abort_flag);
             tc_commit(bar(L::bO));   // all MMAs above done (also on the error path)
@@ -284,21 +312,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const uint32_t lane_bits = (uint32_t)(sub * 32) << 16;
-        const uint32_t tS = tmem + lane_bits, tdP = tS + 128;
         const int kr = kt * kBT + row;                     // key row
         const int q_lo = (kr / p.kpf) * p.kpf;             // first query row that sees it
         bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int i = i_first + t;
-            const float *l2s = reinterpret_cast<const float *>(smem + L::kB + (t & 1) * L::kStage + 2 * L::kTile);
+        for (int t = 0; t < 2 * T; ++t) {
+            const int ti = t >> 1, h = t & 1, b = t & 1;
+            const int i = i_first + ti;
+            const float *l2s =
+                reinterpret_cast<const float *>(smem + L::kB + (ti & 1) * L::kStage + 2 * L::kTile) + h * kHalf;
             const float *dls = l2s + 128;
-            bool w = !*abort_flag && mbar_wait(bar(L::bS), t & 1, kBwdWaitNs);
+            const uint32_t tS = tmem + lane_bits + 64 * b, tdP = tS + 128;
+            bool w = !*abort_flag && mbar_wait(bar(L::bS + b), (t >> 1) & 1, kBwdWaitNs);
             w = __all_sync(0xffffffffu, w);
             if (!w) { ok = false; break; }
             tc_fence_after();
-            const int lo = q_lo - i * kBT;                 // columns below lo are hidden from this key
+            const int lo = q_lo - i * kBT - h * kHalf;     // columns below lo are hidden from this key
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t s[32], dp[32], pk[16], dk[16];
                 float l2[32], dl[32];
                 tmem_ld32(tS + 32 * c, s);
@@ -306,9 +336,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     const float4 a = *reinterpret_cast<const float4 *>(l2s + 32 * c + e);
-                    const float4 b = *reinterpret_cast<const float4 *>(dls + 32 * c + e);
+                    const float4 bq = *reinterpret_cast<const float4 *>(dls + 32 * c + e);
                     l2[e] = a.x; l2[e + 1] = a.y; l2[e + 2] = a.z; l2[e + 3] = a.w;
-                    dl[e] = b.x; dl[e + 1] = b.y; dl[e + 2] = b.z; dl[e + 3] = b.w;
+                    dl[e] = bq.x; dl[e + 1] = bq.y; dl[e + 2] = bq.z; dl[e + 3] = bq.w;
                 }
                 tmem_wait_ld();
                 p_ds_chunk(s, dp, l2, dl, p.scale_log2, lo - 32 * c, 32, pk, dk);
@@ -318,7 +348,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::bP));
+            if (lane == 0) mbar_arrive(bar(L::bP + b));
         }
         // epilogue: dV -> V's tile, dK * scale -> K's tile, then TMA stores
         bool w = ok && !*abort_flag && mbar_wait(bar(L::bO), 0, kBwdWaitNs);
@@ -379,7 +409,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
             mbar_init(bar(L::bFull + s), 1);
             mbar_init(bar(L::bEmpty + s), 1);
         }
-        mbar_init(bar(L::bS), 1);
+        mbar_init(bar(L::bS), 1);   // one S / dP buffer: bS + 0, bP + 0
         mbar_init(bar(L::bP), 4);
         mbar_init(bar(L::bO), 1);
         mbar_init(bar(L::bEpi), kBT);
@@ -433,7 +463,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
                 ok = mbar_wait(bar(L::bP), t & 1, kBwdWaitNs) && !*abort_flag;
                 if (!ok) break;
                 tc_fence_after();
-                mma_tile_ts<D>(tmem + 256, tmem + 128, smem_desc_sw128(sb, 16384, 1024), idesc_o, t > 0);  // dQ += dS K
+                mma_tile_ts<D, kBT>(tmem + 256, tmem + 128, smem_desc_sw128(sb, 16384, 1024), idesc_o, t > 0);  // dQ += dS K
                 tc_commit(bar(L::bEmpty + st));
             }
             if (!ok) bwd_timeout(p, abort_flag);
