@@ -592,8 +592,31 @@ def run_other(args):
         b.record()
         torch.cuda.synchronize()
         ms = a.elapsed_time(b)
+        # the 30 layers' appends of one chunk back to back (1.73 GB moved), each
+        # from its own source, after an L2 flush: the append kernel's HBM
+        # asymptote, labelled as such
+        peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        batch_bytes = L * 4.0 * C * k * H * d * 2
+        srcs = [(rnd((C * k, H, d)), rnd((C * k, H, d))) for _ in range(L)]
+        bts = []
+        for _ in range(5):
+            flush.zero_()
+            a2, b2 = _events(2)
+            a2.record()
+            for l in range(L):
+                rtr.rtr_kvcache_append_frame(c, l, srcs[l][0], srcs[l][1], C, sh)
+            b2.record()
+            torch.cuda.synchronize()
+            bts.append(a2.elapsed_time(b2))
+        bms = statistics.mean(bts[1:])
         st = rtr.rtr_get_device_status(0, sh)
         rtr.rtr_kvcache_destroy(c)
+        line["append_batch_30_layers"] = {
+            "what": "30 rtr_kvcache_append_frame calls (one per layer, 3 frames each, distinct sources) back to "
+                    "back after an L2 flush: the append kernel's asymptote, not a step of the stream",
+            "bytes": batch_bytes, "ms": bms,
+            "achieved_gbs": batch_bytes / bms / 1e6, "peak_gbs": peak_hbm,
+            "frac": batch_bytes / bms / 1e6 / peak_hbm}
         line.update({"config": w.name, "total_ms": ms, "attention_tflop": flops / 1e12,
                      "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
                      "latent_frames_per_s_per_layer": w.frames_total / (ms / 1e3 / L),

@@ -130,3 +130,36 @@ def test_full_prefill_backward_sampled():
     assert np.linalg.norm(gdv - gdo) <= 2e-2 * np.linalg.norm(gdo)
     gdk = dk.float().sum(dim=0).cpu().numpy()
     assert np.linalg.norm(gdk) <= 2e-2 * np.linalg.norm(dk.float().abs().sum(dim=0).cpu().numpy())
+
+
+def test_backward_custom_scale():
+    """A softmax scale other than 1/sqrt(d) reaches both the forward's row
+    log-sum-exp and every gradient (dQ and dK carry it, dV through P)."""
+    rtr = _rtr()
+    n, H, d, kpf, scale = 333, 2, 128, 70, 0.05
+    q, k, v, do = bf16_inputs(n, H, d, 99)
+    tq, tk, tv, tdo = dev(q), dev(k), dev(v), dev(do)
+    out = torch.empty_like(tq)
+    lse = torch.empty((H, n), dtype=torch.float32, device="cuda")
+    rtr.rtr_attn_block_causal_prefill_lse(tq, tk, tv, n, H, d, kpf, "bf16", out, lse, scale)
+    dq, dk, dv = torch.empty_like(tq), torch.empty_like(tq), torch.empty_like(tq)
+    rtr.rtr_attn_block_causal_backward(tq, tk, tv, out, tdo, lse, n, H, d, kpf, "bf16", dq, dk, dv, scale)
+    torch.cuda.synchronize()
+    Q, K, V, dO = (oracle.decode(a, "bf16") for a in (q, k, v, do))
+    assert np.max(np.abs(lse.cpu().numpy().T - oracle.prefill_lse(Q, K, kpf, scale=scale))) <= LSE_ABS
+    wq, wk, wv = oracle.prefill_backward(Q, K, V, dO, kpf, scale=scale)
+    assert_grad_close(host_f64(dq), wq, "dQ")
+    assert_grad_close(host_f64(dk), wk, "dK")
+    assert_grad_close(host_f64(dv), wv, "dV")
+
+
+def test_backward_is_deterministic():
+    """Every output tile is written once by one CTA (no atomics): two calls
+    give bit-identical gradients."""
+    rtr = _rtr()
+    n, H, d, kpf = 500, 2, 128, 100
+    q, k, v, do = bf16_inputs(n, H, d, 7)
+    a = run_gpu(q, k, v, do, n, H, d, kpf)
+    b = run_gpu(q, k, v, do, n, H, d, kpf)
+    for x, y in zip(a[2:], b[2:]):
+        assert torch.equal(x.view(torch.int16), y.view(torch.int16))
