@@ -89,6 +89,63 @@ std::atomic<unsigned long long> g_launches{0};
 
 void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
+// Device allocations of the library go through lib_malloc, so that a test can
+// make chosen ones fail (rtr_test_fail_allocs) and check the RTR_E_NOMEM paths.
+namespace {
+std::mutex g_alloc_mu;
+int g_alloc_skip = 0, g_alloc_fail = 0;
+}
+
+cudaError_t lib_malloc(void **p, size_t bytes) {
+    {
+        std::lock_guard<std::mutex> lock(g_alloc_mu);
+        if (g_alloc_skip > 0) {
+            --g_alloc_skip;
+        } else if (g_alloc_fail > 0) {
+            --g_alloc_fail;
+            *p = nullptr;
+            return cudaErrorMemoryAllocation;
+        }
+    }
+    return cudaMalloc(p, bytes);
+}
+
+// Cache buffers carry guard bands of a known byte on both sides; a kernel
+// that writes outside its buffer changes them (rtr_*_check_guards).
+constexpr size_t kGuardBytes = 64u << 10;
+constexpr int kGuardByte = 0xA5;
+
+char *guarded_alloc(size_t bytes) {
+    void *raw = nullptr;
+    if (lib_malloc(&raw, bytes + 2 * kGuardBytes) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    char *p = static_cast<char *>(raw) + kGuardBytes;
+    if (cudaMemset(raw, kGuardByte, kGuardBytes) != cudaSuccess ||
+        cudaMemset(p + bytes, kGuardByte, kGuardBytes) != cudaSuccess) {
+        cudaFree(raw);
+        return nullptr;
+    }
+    return p;
+}
+
+void guarded_free(char *p) {
+    if (p) cudaFree(p - kGuardBytes);
+}
+
+// RTR_OK if both guard bands still hold kGuardByte (synchronises the device).
+rtr_status guards_status(const char *p, size_t bytes) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return RTR_E_CUDA;
+    std::vector<unsigned char> h(kGuardBytes);
+    for (const char *g : {p - kGuardBytes, p + bytes}) {
+        if (cudaMemcpy(h.data(), g, kGuardBytes, cudaMemcpyDeviceToHost) != cudaSuccess) return RTR_E_CUDA;
+        for (unsigned char b : h)
+            if (b != (unsigned char)kGuardByte) return RTR_E_STATE;
+    }
+    return RTR_OK;
+}
+
 int attn_cta_group() {
     const char *e = std::getenv("RTR_CTA_GROUP");
     if (e && e[0] == '1') return 1;
@@ -162,7 +219,7 @@ void *stream_workspace(int device, cudaStream_t s, size_t bytes) {
         if (w.first) cudaFree(w.first);
         w.first = nullptr;
         w.second = 0;
-        if (cudaMalloc(&w.first, bytes) != cudaSuccess) {
+        if (lib_malloc(&w.first, bytes) != cudaSuccess) {
             cudaGetLastError();
             w.first = nullptr;
             return nullptr;
@@ -241,14 +298,15 @@ rtr_status rtr_kvcache_create_ex(int layers, int heads, int head_dim, int k, int
     c->rows = rows;
     c->layer_bytes = (size_t)heads * rows * head_dim * elt_size(dt);
     const size_t total = c->layer_bytes * layers;
-    if (cudaMalloc(&c->kbuf, total) != cudaSuccess || cudaMalloc(&c->vbuf, total) != cudaSuccess) {
-        cudaGetLastError();
-        if (c->kbuf) cudaFree(c->kbuf);
+    c->kbuf = guarded_alloc(total);
+    c->vbuf = c->kbuf ? guarded_alloc(total) : nullptr;
+    if (!c->kbuf || !c->vbuf) {
+        guarded_free(c->kbuf);
         delete c;
         return RTR_E_NOMEM;
     }
     if (cudaMemset(c->kbuf, 0, total) != cudaSuccess || cudaMemset(c->vbuf, 0, total) != cudaSuccess) {
-        cudaFree(c->kbuf); cudaFree(c->vbuf); delete c;
+        guarded_free(c->kbuf); guarded_free(c->vbuf); delete c;
         return RTR_E_CUDA;
     }
     c->ref_valid.assign(layers, 0);
@@ -262,13 +320,13 @@ rtr_status rtr_kvcache_create_ex(int layers, int heads, int head_dim, int k, int
             if (!make_tmap_bf16(&c->tmk[l], c->kbuf + l * c->layer_bytes, head_dim, rows, heads, 128, 1) ||
                 !make_tmap_bf16(&c->tmk64[l], c->kbuf + l * c->layer_bytes, head_dim, rows, heads, 64, 1) ||
                 !make_tmap_bf16(&c->tmv[l], c->vbuf + l * c->layer_bytes, head_dim, rows, heads, 128, 1)) {
-                cudaFree(c->kbuf); cudaFree(c->vbuf); delete c;
+                guarded_free(c->kbuf); guarded_free(c->vbuf); delete c;
                 return RTR_E_CUDA;
             }
         }
     }
     if (cudaDeviceSynchronize() != cudaSuccess) {
-        cudaFree(c->kbuf); cudaFree(c->vbuf); delete c;
+        guarded_free(c->kbuf); guarded_free(c->vbuf); delete c;
         return RTR_E_CUDA;
     }
     *out = c;
@@ -279,8 +337,8 @@ void rtr_kvcache_destroy(rtr_kvcache *c) {
     if (!c) return;
     DeviceGuard dg(c->device);
     cudaDeviceSynchronize();
-    cudaFree(c->kbuf);
-    cudaFree(c->vbuf);
+    guarded_free(c->kbuf);
+    guarded_free(c->vbuf);
     delete c;
 }
 
@@ -348,6 +406,25 @@ rtr_status rtr_kvcache_get_index_map(const rtr_kvcache *c, int layer, int32_t *s
     if (frames_appended) *frames_appended = g;
     if (count) *count = cnt;
     return RTR_OK;
+}
+
+rtr_status rtr_kvcache_set_index_map(rtr_kvcache *c, int layer, int64_t frames_appended, int32_t count,
+                                     int32_t ref_valid) {
+    if (!c || layer < 0 || layer >= c->layers || frames_appended < 0 || count < 0 || count > c->W ||
+        (int64_t)count > frames_appended || (ref_valid != 0 && ref_valid != 1) || (ref_valid && c->R == 0))
+        return RTR_E_INVAL;
+    c->g[layer] = frames_appended;
+    c->count[layer] = count;
+    c->ref_valid[layer] = ref_valid;
+    return RTR_OK;
+}
+
+rtr_status rtr_kvcache_check_guards(const rtr_kvcache *c) {
+    if (!c) return RTR_E_INVAL;
+    DeviceGuard dg(c->device);
+    const size_t total = c->layer_bytes * c->layers;
+    const rtr_status a = guards_status(c->kbuf, total);
+    return a != RTR_OK ? a : guards_status(c->vbuf, total);
 }
 
 rtr_status rtr_kvcache_device_ptrs(const rtr_kvcache *c, int layer, void **k, void **v) {
@@ -525,14 +602,15 @@ rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_tex
     x->dt = dt; x->device = device;
     x->layer_bytes = (size_t)heads * max_text * head_dim * elt_size(dt);
     const size_t total = x->layer_bytes * layers;
-    if (cudaMalloc(&x->kbuf, total) != cudaSuccess || cudaMalloc(&x->vbuf, total) != cudaSuccess) {
-        cudaGetLastError();
-        if (x->kbuf) cudaFree(x->kbuf);
+    x->kbuf = guarded_alloc(total);
+    x->vbuf = x->kbuf ? guarded_alloc(total) : nullptr;
+    if (!x->kbuf || !x->vbuf) {
+        guarded_free(x->kbuf);
         delete x;
         return RTR_E_NOMEM;
     }
     if (cudaMemset(x->kbuf, 0, total) != cudaSuccess || cudaMemset(x->vbuf, 0, total) != cudaSuccess) {
-        cudaFree(x->kbuf); cudaFree(x->vbuf); delete x;
+        guarded_free(x->kbuf); guarded_free(x->vbuf); delete x;
         return RTR_E_CUDA;
     }
     x->n_text.assign(layers, 0);
@@ -544,13 +622,13 @@ rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_tex
             if (!make_tmap_bf16(&x->tmk[l], x->kbuf + l * x->layer_bytes, head_dim, max_text, heads, 128, 1) ||
                 !make_tmap_bf16(&x->tmk64[l], x->kbuf + l * x->layer_bytes, head_dim, max_text, heads, 64, 1) ||
                 !make_tmap_bf16(&x->tmv[l], x->vbuf + l * x->layer_bytes, head_dim, max_text, heads, 128, 1)) {
-                cudaFree(x->kbuf); cudaFree(x->vbuf); delete x;
+                guarded_free(x->kbuf); guarded_free(x->vbuf); delete x;
                 return RTR_E_CUDA;
             }
         }
     }
     if (cudaDeviceSynchronize() != cudaSuccess) {
-        cudaFree(x->kbuf); cudaFree(x->vbuf); delete x;
+        guarded_free(x->kbuf); guarded_free(x->vbuf); delete x;
         return RTR_E_CUDA;
     }
     *out = x;
@@ -561,8 +639,8 @@ void rtr_crossattn_destroy(rtr_xattn *x) {
     if (!x) return;
     DeviceGuard dg(x->device);
     cudaDeviceSynchronize();
-    cudaFree(x->kbuf);
-    cudaFree(x->vbuf);
+    guarded_free(x->kbuf);
+    guarded_free(x->vbuf);
     delete x;
 }
 
@@ -586,6 +664,22 @@ rtr_status rtr_crossattn_set_text(rtr_xattn *x, int layer, const void *k_text, c
 rtr_status rtr_crossattn_reset(rtr_xattn *x) {
     if (!x) return RTR_E_INVAL;
     std::fill(x->n_text.begin(), x->n_text.end(), 0);
+    return RTR_OK;
+}
+
+rtr_status rtr_crossattn_check_guards(const rtr_xattn *x) {
+    if (!x) return RTR_E_INVAL;
+    DeviceGuard dg(x->device);
+    const size_t total = x->layer_bytes * x->layers;
+    const rtr_status a = guards_status(x->kbuf, total);
+    return a != RTR_OK ? a : guards_status(x->vbuf, total);
+}
+
+rtr_status rtr_test_fail_allocs(int after, int n) {
+    if (after < 0 || n < 0) return RTR_E_INVAL;
+    std::lock_guard<std::mutex> lock(g_alloc_mu);
+    g_alloc_skip = after;
+    g_alloc_fail = n;
     return RTR_OK;
 }
 

@@ -45,6 +45,10 @@ _SIGNATURES = [
                                        ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64),
                                        ctypes.POINTER(ctypes.c_int32)]),
     ("rtr_kvcache_device_ptrs", _i, [_vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
+    ("rtr_kvcache_set_index_map", _i, [_vp, _i, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32]),
+    ("rtr_kvcache_check_guards", _i, [_vp]),
+    ("rtr_crossattn_check_guards", _i, [_vp]),
+    ("rtr_test_fail_allocs", _i, [_i, _i]),
     ("rtr_attn_frame_causal", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
     ("rtr_attn_frame_causal_commit", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
     ("rtr_attn_block_causal_prefill", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
@@ -167,6 +171,23 @@ def rtr_kvcache_get_index_map(c, layer, n_slots):
     _check(_lib.rtr_kvcache_get_index_map(c, layer, slots, ctypes.byref(ref), ctypes.byref(g),
                                           ctypes.byref(cnt)), "rtr_kvcache_get_index_map")
     return list(slots), ref.value, g.value, cnt.value
+
+
+def rtr_kvcache_set_index_map(c, layer, frames_appended, count, ref_valid):
+    return _check(_lib.rtr_kvcache_set_index_map(c, layer, int(frames_appended), int(count), int(ref_valid)),
+                  "rtr_kvcache_set_index_map")
+
+
+def rtr_kvcache_check_guards(c):
+    return _check(_lib.rtr_kvcache_check_guards(c), "rtr_kvcache_check_guards")
+
+
+def rtr_crossattn_check_guards(x):
+    return _check(_lib.rtr_crossattn_check_guards(x), "rtr_crossattn_check_guards")
+
+
+def rtr_test_fail_allocs(after, n):
+    return _check(_lib.rtr_test_fail_allocs(int(after), int(n)), "rtr_test_fail_allocs")
 
 
 def rtr_kvcache_device_ptrs(c, layer):

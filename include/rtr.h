@@ -145,6 +145,25 @@ rtr_status rtr_kvcache_get_index_map(const rtr_kvcache *c, int layer,
                                      int32_t *slot_frame, int32_t *ref_valid,
                                      int64_t *frames_appended, int32_t *count);
 
+/* Restore the index map of `layer`, e.g. after copying a snapshot's K / V
+ * bytes back in through rtr_kvcache_device_ptrs: a stream saved with
+ * rtr_kvcache_get_index_map and a device-to-host copy of the buffers resumes
+ * from the same state (the pages' stream state is exactly this cache).
+ * Requires 0 <= count <= min(window_frames, frames_appended), ref_valid 0 or
+ * 1 (1 only with ref_frames > 0); else RTR_E_INVAL and nothing changes.  No
+ * data moves: the caller restores the bytes of the slots the map names, at
+ * the same physical slots (frame f in slot f mod S). */
+rtr_status rtr_kvcache_set_index_map(rtr_kvcache *c, int layer,
+                                     int64_t frames_appended, int32_t count,
+                                     int32_t ref_valid);
+
+/* Guard bands: every K / V buffer of a cache (and of a cross-attention cache)
+ * is allocated with 64 KB on each side holding a fixed byte pattern.  These
+ * synchronise the device and return RTR_OK if all bands are intact,
+ * RTR_E_STATE if any byte changed (a kernel wrote outside its buffer), or
+ * RTR_E_CUDA. */
+rtr_status rtr_kvcache_check_guards(const rtr_kvcache *c);
+
 /* Device pointers of layer `layer`'s K and V buffers (layout above), for
  * inspection and snapshotting.  The library keeps ownership. */
 rtr_status rtr_kvcache_device_ptrs(const rtr_kvcache *c, int layer,
@@ -190,6 +209,15 @@ rtr_status rtr_attn_frame_causal_commit(rtr_kvcache *c, int layer,
                                         const void *v_cur, int n_cur_frames,
                                         void *out, float scale,
                                         rtr_stream_t stream);
+
+/* See rtr_kvcache_check_guards. */
+rtr_status rtr_crossattn_check_guards(const rtr_xattn *x);
+
+/* Test hook: of the library's next device allocations (cache buffers,
+ * scratch), let `after` succeed and make the `n` that follow fail as if the
+ * device were out of memory, so that tests can reach every RTR_E_NOMEM path.
+ * (0, 0) clears it.  Negative arguments: RTR_E_INVAL. */
+rtr_status rtr_test_fail_allocs(int after, int n);
 
 /* Block-causal attention over one whole sequence (Key Designs 2: training
  * sees all frames at once under M).  q, k, v, out: [n_tokens][heads]

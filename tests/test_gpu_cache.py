@@ -36,6 +36,7 @@ def gpu_view(c, layer, H, rows, d, dtype, which):
 
 def compare_cache(c, ref: oracle.ReferenceCache, layer=0):
     from causal_attention_rtr_b200 import rtr
+    rtr.rtr_kvcache_check_guards(c)                   # no kernel wrote outside the buffers
     slots, ref_valid, g, count = rtr.rtr_kvcache_get_index_map(c, layer, ref.S)
     want_slots, want_ref, want_g = ref.index_map()
     assert (slots, ref_valid, g, count) == (want_slots, want_ref, want_g, ref.count)
@@ -154,3 +155,119 @@ def test_argument_errors_leave_state_unchanged():
         assert rtr.rtr_kvcache_get_index_map(c, 0, W) == ([-1] * W, 0, 0, 0)
     finally:
         rtr.rtr_kvcache_destroy(c)
+
+
+def _raw_view(ptr, nbytes):
+    """uint8 device tensor over library-owned memory (no copy)."""
+    return torch.as_tensor(_DevArray(ptr, nbytes, "|u1"), device="cuda")
+
+
+def test_guard_bands_intact_after_every_kind_of_update():
+    """Appends through eviction and wrap, reference overwrites, fused commits
+    and text set/reset leave the 64 KB guard bands around every buffer
+    untouched (no kernel writes outside its buffer)."""
+    from causal_attention_rtr_b200 import rtr
+    H, d, k, W, C = 3, 128, 200, 4, 2
+    rng = np.random.default_rng(8)
+    c = rtr.rtr_kvcache_create_ex(2, H, d, k, 1, W, C, "bf16", 0)
+    x = rtr.rtr_crossattn_create(2, H, d, 64, "bf16", 0)
+    try:
+        for layer in range(2):
+            kr, vr = (synth.normal(rng, (k, H, d), 1.0, "bf16") for _ in range(2))
+            rtr.rtr_kvcache_set_reference(c, layer, dev(kr), dev(vr))
+            for i in range(7):
+                n = 1 + i % C
+                q, kk, vv = (synth.normal(rng, (n * k, H, d), 1.0, "bf16") for _ in range(3))
+                out = torch.empty((n * k, H, d), dtype=torch.bfloat16, device="cuda")
+                if i % 2:
+                    rtr.rtr_attn_frame_causal_commit(c, layer, dev(q), dev(kk), dev(vv), n, out)
+                else:
+                    rtr.rtr_kvcache_append_frame(c, layer, dev(kk), dev(vv), n)
+            kt, vt = (synth.normal(rng, (64, H, d), 1.0, "bf16") for _ in range(2))
+            rtr.rtr_crossattn_set_text(x, layer, dev(kt), dev(vt), 64)
+        rtr.rtr_crossattn_reset(x)
+        rtr.rtr_kvcache_check_guards(c)
+        rtr.rtr_crossattn_check_guards(x)
+    finally:
+        rtr.rtr_kvcache_destroy(c)
+        rtr.rtr_crossattn_destroy(x)
+
+
+def test_allocation_failures_return_nomem():
+    """Injected device-allocation failures: cache and text-cache creation and
+    the attention scratch of a new stream return RTR_E_NOMEM, leave nothing
+    behind, and the library works normally once the hook is cleared."""
+    from causal_attention_rtr_b200 import rtr
+    try:
+        for after in (0, 1):
+            rtr.rtr_test_fail_allocs(after, 1)
+            with pytest.raises(rtr.RtrError) as e:
+                rtr.rtr_kvcache_create(1, 2, 128, 16, 1, 4, "bf16", 0)
+            assert e.value.status == rtr.RTR_E_NOMEM
+            rtr.rtr_test_fail_allocs(after, 1)
+            with pytest.raises(rtr.RtrError) as e:
+                rtr.rtr_crossattn_create(1, 2, 128, 16, "bf16", 0)
+            assert e.value.status == rtr.RTR_E_NOMEM
+        rtr.rtr_test_fail_allocs(0, 0)
+        c = rtr.rtr_kvcache_create(1, 2, 128, 16, 1, 4, "bf16", 0)
+        try:
+            q = torch.zeros((16, 2, 128), dtype=torch.bfloat16, device="cuda")
+            out = torch.empty_like(q)
+            torch.cuda.synchronize()
+            s = torch.cuda.Stream()
+            rtr.rtr_test_fail_allocs(0, 1)
+            with pytest.raises(rtr.RtrError) as e:
+                rtr.rtr_attn_frame_causal(c, 0, q, q, q, 1, out, 0.0, s)
+            assert e.value.status == rtr.RTR_E_NOMEM
+            rtr.rtr_test_fail_allocs(0, 0)
+            rtr.rtr_attn_frame_causal(c, 0, q, q, q, 1, out, 0.0, s)
+            s.synchronize()
+            assert rtr.rtr_kvcache_get_index_map(c, 0, 4) == ([-1] * 4, 0, 0, 0)
+        finally:
+            rtr.rtr_kvcache_destroy(c)
+    finally:
+        rtr.rtr_test_fail_allocs(0, 0)
+
+
+def test_snapshot_and_restore_resume_the_stream():
+    """A cache saved (index map + a copy of its buffers) and restored into a
+    new cache (bytes copied back, rtr_kvcache_set_index_map) continues the
+    stream exactly: bit-identical attention and the same index maps."""
+    from causal_attention_rtr_b200 import rtr
+    H, d, k, R, W = 2, 128, 150, 1, 4
+    rng = np.random.default_rng(21)
+    a = rtr.rtr_kvcache_create(1, H, d, k, R, W, "bf16", 0)
+    b = rtr.rtr_kvcache_create(1, H, d, k, R, W, "bf16", 0)
+    nbytes = H * (R + W) * k * d * 2
+    try:
+        kr, vr = (synth.normal(rng, (k, H, d), 1.0, "bf16") for _ in range(2))
+        rtr.rtr_kvcache_set_reference(a, 0, dev(kr), dev(vr))
+        for _ in range(6):
+            kk, vv = (synth.normal(rng, (k, H, d), 1.0, "bf16") for _ in range(2))
+            rtr.rtr_kvcache_append_frame(a, 0, dev(kk), dev(vv), 1)
+        torch.cuda.synchronize()
+        slots, ref_valid, g, count = rtr.rtr_kvcache_get_index_map(a, 0, W)
+        ka, va = rtr.rtr_kvcache_device_ptrs(a, 0)
+        snap = [_raw_view(p, nbytes).clone() for p in (ka, va)]          # the saved state
+        kb, vb = rtr.rtr_kvcache_device_ptrs(b, 0)
+        for p, saved in zip((kb, vb), snap):
+            _raw_view(p, nbytes).copy_(saved)
+        rtr.rtr_kvcache_set_index_map(b, 0, g, count, ref_valid)
+        assert rtr.rtr_kvcache_get_index_map(b, 0, W) == (slots, ref_valid, g, count)
+        for step in range(3):
+            q, kk, vv = (synth.normal(rng, (2 * k, H, d), 1.0, "bf16") for _ in range(3))
+            oa, ob = (torch.empty((2 * k, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2))
+            rtr.rtr_attn_frame_causal(a, 0, dev(q), dev(kk), dev(vv), 2, oa)
+            rtr.rtr_attn_frame_causal(b, 0, dev(q), dev(kk), dev(vv), 2, ob)
+            torch.cuda.synchronize()
+            assert torch.equal(oa.view(torch.int16), ob.view(torch.int16)), f"step {step}"
+            rtr.rtr_kvcache_append_frame(a, 0, dev(kk), dev(vv), 2)
+            rtr.rtr_kvcache_append_frame(b, 0, dev(kk), dev(vv), 2)
+            assert rtr.rtr_kvcache_get_index_map(a, 0, W) == rtr.rtr_kvcache_get_index_map(b, 0, W)
+        with pytest.raises(rtr.RtrError):
+            rtr.rtr_kvcache_set_index_map(b, 0, 3, 4, 1)                 # count > frames appended
+        with pytest.raises(rtr.RtrError):
+            rtr.rtr_kvcache_set_index_map(b, 0, 30, W + 1, 1)            # count > window
+    finally:
+        rtr.rtr_kvcache_destroy(a)
+        rtr.rtr_kvcache_destroy(b)
