@@ -24,10 +24,12 @@
 //               buffer's MMAs meanwhile.
 //   bwd_dq      query-stationary: one CTA per (head, 128-query tile); streams
 //               the key tiles it sees.  S = Q K^T and dP = dO V^T into TMEM,
-//               dS (bf16) back into TMEM, dQ += dS K.  (The two-buffer scheme
-//               of bwd_dkdv measured 14 % slower here: its 64-wide S and dP
-//               MMAs re-read Q and dO per half, and each half pays the
-//               softmax hand-off again.)
+//               dS (bf16) back into TMEM, dQ += dS K.  S has two TMEM
+//               buffers, so S of the next key tile runs during this tile's
+//               softmax; dP has one (dS lives in it until dQ has read it).
+//               (bwd_dkdv's half-tile scheme measured 14 % slower here: its
+//               64-wide S and dP MMAs re-read Q and dO per half, and each
+//               half pays the softmax hand-off again.)
 // Splitting dQ from dK/dV recomputes S and dP once more (7 tile MMAs per
 // (query tile, key tile) instead of 5) but needs no atomic accumulation of
 // dQ across CTAs: every output tile is written once, in bf16, by TMA.
@@ -424,7 +426,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    // TMEM: S [0,128), dP / dS [128,256), dQ [256,256+D)
+    // TMEM: S buffers [0,128), [128,256) (tile t in buffer t % 2); dP / dS
+    // [256,384); dQ [384,384+D).
 
     if (warp == 0) {
         if (lane == 0) {
@@ -450,21 +453,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, 0, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBT, D, 0, 1);
             const uint64_t descQ = smem_desc_sw128(sQ, 16, 1024), descdO = smem_desc_sw128(sdO, 16, 1024);
-            bool ok = mbar_wait(bar(L::bA), 0, kBwdWaitNs);
-            for (int t = 0; ok && t < T; ++t) {
-                const int st = t & 1;
-                const uint32_t sb = stage_b(st);
-                ok = mbar_wait(bar(L::bFull + st), (t >> 1) & 1, kBwdWaitNs) && !*abort_flag;
-                if (!ok) break;
+            // S(t+1) goes into the other S buffer while the softmax works on
+            // tile t; dP(t+1) follows dQ(t), which reads dS(t) from dP's columns.
+            bool ok = mbar_wait(bar(L::bA), 0, kBwdWaitNs) &&
+                      mbar_wait(bar(L::bFull + 0), 0, kBwdWaitNs) && !*abort_flag;
+            if (ok) {
                 tc_fence_after();
-                mma_tile_ss<D>(tmem + 0, descQ, smem_desc_sw128(sb, 16, 1024), idesc_s);                 // S
-                mma_tile_ss<D>(tmem + 128, descdO, smem_desc_sw128(sb + L::kTile, 16, 1024), idesc_s);   // dP
+                mma_tile_ss<D>(tmem + 0, descQ, smem_desc_sw128(stage_b(0), 16, 1024), idesc_s);                  // S(0)
+                mma_tile_ss<D>(tmem + 256, descdO, smem_desc_sw128(stage_b(0) + L::kTile, 16, 1024), idesc_s);   // dP(0)
                 tc_commit(bar(L::bS));
+            }
+            for (int t = 0; ok && t < T; ++t) {
+                const int st = t & 1, stn = st ^ 1;
+                const uint32_t sb = stage_b(st), sbn = stage_b(stn);
+                if (t + 1 < T) {
+                    ok = mbar_wait(bar(L::bFull + stn), ((t + 1) >> 1) & 1, kBwdWaitNs) && !*abort_flag;
+                    if (!ok) break;
+                    tc_fence_after();
+                    mma_tile_ss<D>(tmem + 128 * ((t + 1) & 1), descQ, smem_desc_sw128(sbn, 16, 1024), idesc_s);  // S(t+1)
+                }
                 ok = mbar_wait(bar(L::bP), t & 1, kBwdWaitNs) && !*abort_flag;
                 if (!ok) break;
                 tc_fence_after();
-                mma_tile_ts<D, kBT>(tmem + 256, tmem + 128, smem_desc_sw128(sb, 16384, 1024), idesc_o, t > 0);  // dQ += dS K
+                mma_tile_ts<D, kBT>(tmem + 384, tmem + 256, smem_desc_sw128(sb, 16384, 1024), idesc_o, t > 0);  // dQ += dS K
                 tc_commit(bar(L::bEmpty + st));
+                if (t + 1 < T) {
+                    mma_tile_ss<D>(tmem + 256, descdO, smem_desc_sw128(sbn + L::kTile, 16, 1024), idesc_s);      // dP(t+1)
+                    tc_commit(bar(L::bS));
+                }
             }
             if (!ok) bwd_timeout(p, abort_flag);
             tc_commit(bar(L::bO));
@@ -474,7 +490,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const uint32_t lane_bits = (uint32_t)(sub * 32) << 16;
-        const uint32_t tS = tmem + lane_bits, tdP = tS + 128;
+        const uint32_t tdP = tmem + lane_bits + 256;
         const int qr = qt * kBT + row;                                  // query row
         const int row_end = min(p.n, (qr / p.kpf + 1) * p.kpf);        // keys it sees: [0, row_end)
         const float l2v = p.lse2[(size_t)head * p.n_pad + qr];          // +inf past n: P = 0
@@ -491,6 +507,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
             w = __all_sync(0xffffffffu, w);
             if (!w) { ok = false; break; }
             tc_fence_after();
+            const uint32_t tS = tmem + lane_bits + 128 * (t & 1);
             const int hi = row_end - t * kBT;                           // columns at and past hi are hidden
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
@@ -510,7 +527,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
         w = __all_sync(0xffffffffu, w);
         if (w) {
             tc_fence_after();
-            acc_to_smem<D>(tmem + lane_bits + 256, p.scale, sQ, row);   // Q's tile is free after the last MMA
+            acc_to_smem<D>(tmem + lane_bits + 384, p.scale, sQ, row);   // Q's tile is free after the last MMA
             fence_proxy_async_smem();
         }
         mbar_arrive(bar(L::bEpi));
