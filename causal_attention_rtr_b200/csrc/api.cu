@@ -83,6 +83,20 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, 
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_bf16_strided(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, uint64_t outer,
+                            uint64_t stride_outer, uint32_t box_mid, uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || !aligned16(base)) return false;
+    cuuint64_t dims[3] = {d, mid, outer};
+    cuuint64_t strides[2] = {d * 2, stride_outer};
+    cuuint32_t box[3] = {64, box_mid, box_outer};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 std::atomic<unsigned long long> g_launches{0};
 }
@@ -170,6 +184,9 @@ struct rtr_kvcache {
     std::vector<long long> g;
     std::vector<CUtensorMap> tmk, tmv;
     std::vector<CUtensorMap> tmk64;   // K maps with 64-row boxes (CTA-pair attention)
+    // Chunk-write maps of the fused commit, device array [layer][S][K, V][128-row, 8-row box]
+    // (bf16 caches with commit room and k a multiple of 8), else null.
+    CUtensorMap *cmaps = nullptr;
 };
 
 struct rtr_xattn {
@@ -325,7 +342,29 @@ rtr_status rtr_kvcache_create_ex(int layers, int heads, int head_dim, int k, int
             }
         }
     }
+    if (dt == RTR_BF16 && commit_frames > 0 && k % 8 == 0) {
+        std::vector<CUtensorMap> maps((size_t)layers * c->S * 4);
+        bool ok = true;
+        const uint64_t row_bytes = (uint64_t)head_dim * 2;
+        for (int l = 0; l < layers && ok; ++l)
+            for (int sl = 0; sl < c->S && ok; ++sl)
+                for (int kv = 0; kv < 2 && ok; ++kv) {
+                    const char *base = (kv ? c->vbuf : c->kbuf) + l * c->layer_bytes + (size_t)(c->R + sl) * k * row_bytes;
+                    CUtensorMap *m = &maps[(((size_t)l * c->S + sl) * 2 + kv) * 2];
+                    ok = make_tmap_bf16_strided(m, base, head_dim, k, heads, (uint64_t)rows * row_bytes, 128, 1) &&
+                         make_tmap_bf16_strided(m + 1, base, head_dim, k, heads, (uint64_t)rows * row_bytes, 8, 1);
+                }
+        if (!ok || lib_malloc(reinterpret_cast<void **>(&c->cmaps), maps.size() * sizeof(CUtensorMap)) != cudaSuccess ||
+            cudaMemcpy(c->cmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            if (c->cmaps) cudaFree(c->cmaps);
+            guarded_free(c->kbuf); guarded_free(c->vbuf); delete c;
+            return ok ? RTR_E_NOMEM : RTR_E_CUDA;
+        }
+    }
     if (cudaDeviceSynchronize() != cudaSuccess) {
+        if (c->cmaps) cudaFree(c->cmaps);
         guarded_free(c->kbuf); guarded_free(c->vbuf); delete c;
         return RTR_E_CUDA;
     }
@@ -337,6 +376,7 @@ void rtr_kvcache_destroy(rtr_kvcache *c) {
     if (!c) return;
     DeviceGuard dg(c->device);
     cudaDeviceSynchronize();
+    if (c->cmaps) cudaFree(c->cmaps);
     guarded_free(c->kbuf);
     guarded_free(c->vbuf);
     delete c;
@@ -465,6 +505,10 @@ rtr_status stream_problem(const rtr_kvcache *c, int layer, const void *q, const 
     if (merged.size() > (size_t)kMaxSegs - 1) return RTR_E_UNSUPPORTED;   // cannot happen: <= 3 runs
     memset(&pb, 0, sizeof(pb));
     pb.nq = (int)nq; pb.heads = c->heads; pb.head_dim = c->head_dim; pb.kpf = c->k;
+    // The chunk's run goes last, so that every unit of a head sweeps the
+    // cached keys in step with the others (they share them through L2).  The
+    // fused commit uses the same order, so its outputs are bit-identical to
+    // attention + append on the same cache.
     for (auto &x : merged) pb.seg[pb.nseg++] = KvSeg{0, (int)x.first, (int)(x.second - x.first), 0};
     pb.seg[pb.nseg++] = KvSeg{1, 0, (int)nq, 1};
     pb.scale = resolve_scale(scale, c->head_dim);
@@ -508,6 +552,7 @@ rtr_status rtr_attn_frame_causal_commit(rtr_kvcache *c, int layer, const void *q
     pb.commit_first_slot = (int)(c->g[layer] % c->S);
     pb.commit_slots = c->S;
     pb.commit_row0 = c->R * c->k;
+    pb.commit_maps = c->cmaps ? c->cmaps + (size_t)layer * c->S * 4 : nullptr;
     const rtr_status r = run_attention(pb, c->dt, &c->tmk[layer], &c->tmk64[layer], &c->tmv[layer], c->device,
                                        (cudaStream_t)stream);
     if (r == RTR_OK) {

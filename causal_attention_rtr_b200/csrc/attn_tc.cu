@@ -109,6 +109,7 @@ struct TcParams {
     __nv_bfloat16 *commit_k, *commit_v;
     long long commit_rows_per_head;
     int commit_first_slot, commit_slots, commit_row0;
+    const CUtensorMap *commit_maps;   // per-slot store maps (see AttnProblem) or null
     float *lse;         // [heads][nq] natural-log row log-sum-exp, or null
 };
 
@@ -304,6 +305,38 @@ __device__ __forceinline__ void commit_tile_rows(const TcParams &p, uint32_t src
     }
 }
 
+// Chunk write by TMA: the 128 rows of chunk key (or value) tile tt, held in
+// shared memory at `src` in the TMA layout, stored to their ring slots by one
+// thread.  A tile inside one frame is one 128-row box per 64 columns; the
+// pieces of a tile that straddles frames (or ends the chunk) go out as 8-row
+// boxes, all starting on a 1024-byte swizzle atom (frame boundaries are
+// multiples of 8 rows).  Returns after the stores have read shared memory.
+template <int D>
+__device__ __forceinline__ void commit_tile_tma(const TcParams &p, uint32_t src, int kv, int head, int tt) {
+    const int r0 = tt * kBN, r_end = min(r0 + kBN, p.nq);
+    fence_proxy_async_smem();
+    for (int r = r0; r < r_end;) {
+        const int f = r / p.kpf;
+        const int seg_end = min(r_end, (f + 1) * p.kpf);
+        int slot = p.commit_first_slot + f;               // < 2 * commit_slots
+        if (slot >= p.commit_slots) slot -= p.commit_slots;
+        const CUtensorMap *m128 = p.commit_maps + (slot * 2 + kv) * 2;
+        const int y = r - f * p.kpf, a = r - r0, len = seg_end - r;
+        if (a == 0 && len == kBN) {
+#pragma unroll
+            for (int b = 0; b < D / 64; ++b) tma_store_3d(m128, src + b * 16384, b * 64, y, head);
+        } else {
+            for (int i = 0; i < len; i += 8)
+#pragma unroll
+                for (int b = 0; b < D / 64; ++b)
+                    tma_store_3d(m128 + 1, src + b * 16384 + (a + i) * 128, b * 64, y + i, head);
+        }
+        r = seg_end;
+    }
+    bulk_commit();
+    bulk_wait_read0();
+}
+
 template <int D, int CG>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant__ TcParams p) {
     using L = Layout<D, CG>;
@@ -339,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
         for (int i = 0; i < L::kSlots; ++i) {
             mbar_init(bar(L::bFull + i), 1);
             mbar_init(bar(L::bEmpty + i), 1);
-            mbar_init(bar(L::bCopied + i), 2);
+            mbar_init(bar(L::bCopied + i), p.commit_maps ? 1 : 2);   // TMA: one thread; else both warps
             mbar_init(bar(L::bGo + i), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -521,16 +554,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             bool ok = true;
             while (ok && sched_next<CG>(p, sc, it)) {
                 const int T = it.t1 - it.t0;
-                // Unit tiles t >= copy_lo are the chunk's; those with chunk tile
-                // (t - copy_lo) / 2 == the unit's pair index are copied out.
-                int copy_lo = 1 << 30, copy_pair = 0;
+                // Unit tiles from copy_lo on are the chunk's; those with chunk
+                // tile (t - copy_lo) / 2 == the unit's pair index are copied out.
+                int copy_lo = 1 << 30, copy_hi = 0, copy_pair = 0;
                 if (p.commit_k != nullptr) {
                     int head_m;
                     unit_coords(p, it.unit, copy_pair, head_m);
-                    copy_lo = pair_tiles(p, copy_pair) - seg_tiles(p, p.nseg - 1, copy_pair * p.unit_rows);
+                    const int q0m = copy_pair * p.unit_rows;
+                    copy_lo = 0;                               // tiles of the runs before the chunk's
+                    int s = 0;
+                    for (; s < p.nseg && p.seg[s].src != 1; ++s) copy_lo += seg_tiles(p, s, q0m);
+                    copy_hi = s < p.nseg ? copy_lo + seg_tiles(p, s, q0m) : copy_lo;
                 }
+                // [copy_lo, copy_hi) bounds the chunk's tiles: with an odd
+                // tile count the tile after the chunk would otherwise match.
                 auto go = [&](int t, int slot_) {
-                    if (t >= copy_lo && ((t - copy_lo) >> 1) == copy_pair) mbar_arrive(bar(L::bGo + slot_));
+                    if (t >= copy_lo && t < copy_hi && ((t - copy_lo) >> 1) == copy_pair)
+                        mbar_arrive(bar(L::bGo + slot_));
                 };
                 ok = wait(bar(L::bQ), k & 1) && !*abort_flag;
                 if (!ok) break;
@@ -594,13 +634,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             mbar_wait(bar(L::bDrain), 0, kWaitNs);
         }
         __syncwarp();
-    } else if (warp >= 2 && p.commit_k != nullptr) {
+    } else if (warp >= 2 && p.commit_k != nullptr && (p.commit_maps == nullptr || (warp == 2 && lane == 0))) {
         // ------------------------------------------------------------ chunk write
         // Walks the producer's load sequence and waits (on bGo) only for the
         // loads it copies.  Chunk key tile tt belongs to the unit of query tiles 2u,
         // 2u+1 with u = tt / 2 (that unit always loads it), so every chunk
         // tile is written by exactly one CTA.  The producer refills such a
         // slot only after both warps arrived on its bCopied barrier.
+        // With store maps, lane 0 of warp 2 alone issues TMA stores;
+        // otherwise both warps copy half of each tile's rows.
+        const bool tma = p.commit_maps != nullptr;
         const int part = warp - 2;
         Sched sc;
         Item it;
@@ -628,13 +671,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 for (int kv = 0; kv < 2; ++kv, ++n) {
                     const int slot = n % L::kSlots;
                     bool w = !*abort_flag && mbar_wait(bar(L::bGo + slot), (go_phase >> slot) & 1, kWaitNs);
-                    w = __all_sync(0xffffffffu, w);
+                    if (!tma) w = __all_sync(0xffffffffu, w);
                     if (!w) { ok = false; break; }
                     go_phase ^= 1u << slot;
-                    commit_tile_rows<D>(p, sKV + slot * L::kSlotBytes, kv ? p.commit_v : p.commit_k, head, tt, part,
-                                        lane);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(L::bCopied + slot));
+                    if (tma) {
+                        commit_tile_tma<D>(p, sKV + slot * L::kSlotBytes, kv, head, tt);
+                        mbar_arrive(bar(L::bCopied + slot));
+                    } else {
+                        commit_tile_rows<D>(p, sKV + slot * L::kSlotBytes, kv ? p.commit_v : p.commit_k, head, tt,
+                                            part, lane);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(L::bCopied + slot));
+                    }
                 }
             }
         }
@@ -1128,6 +1176,7 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
         tp.commit_first_slot = p.commit_first_slot;
         tp.commit_slots = p.commit_slots;
         tp.commit_row0 = p.commit_row0;
+        tp.commit_maps = p.commit_maps;
     }
     if (p.head_dim == 128)
         return plan.cg == 2 ? launch_tc<128, 2>(tp, plan.has_split, s) : launch_tc<128, 1>(tp, plan.has_split, s);

@@ -50,6 +50,11 @@ struct AttnProblem {
     // run the launch reads.
     void *commit_k, *commit_v;
     int commit_first_slot, commit_slots, commit_row0;
+    // Optional device array of tensor maps, [commit_slots][K, V][128-row box,
+    // 8-row box], each over one ring slot's k rows (128-byte swizzle): the
+    // chunk write is then a few TMA stores issued by one thread.  Null: the
+    // chunk-write warps copy rows themselves.
+    const CUtensorMap *commit_maps;
     // Optional row statistics: lse[h * nq + i] = log sum_j exp(scale q_i.k_j)
     // over the keys row i sees (natural log, fp32).  Null: not written.
     float *lse;
@@ -111,6 +116,9 @@ cudaError_t launch_kv_scatter(const ScatterArgs &a, cudaStream_t s);
 // (64, box_mid, box_outer) elements and 128-byte swizzle.
 bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, uint64_t outer,
                     uint32_t box_mid, uint32_t box_outer);
+// The same with an explicit byte stride between `outer` entries.
+bool make_tmap_bf16_strided(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, uint64_t outer,
+                            uint64_t stride_outer, uint32_t box_mid, uint32_t box_outer);
 
 unsigned *device_status_ptr(int device);
 

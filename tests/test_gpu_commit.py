@@ -13,7 +13,7 @@ import oracle
 from causal_attention_rtr_b200 import synth
 
 from gpu_util import assert_close, dev, host_f64
-from test_gpu_cache import compare_cache
+from test_gpu_cache import _raw_view, compare_cache
 
 pytestmark = pytest.mark.gpu
 
@@ -151,3 +151,40 @@ def test_full_layer_commit_sampled():
         assert rtr.rtr_get_device_status(0) == rtr.RTR_OK
     finally:
         rtr.rtr_kvcache_destroy(c)
+
+
+@pytest.mark.parametrize("k", [200, 77])
+def test_commit_equals_attention_then_append_bitwise(k):
+    """On two caches with the same commit room and history, the fused call
+    and attention followed by append give bit-identical outputs, rings and
+    index maps (TMA chunk write for k a multiple of 8, warp copy otherwise)."""
+    rtr = _rtr()
+    H, d, W, C = 2, 128, 4, 3
+    rng = np.random.default_rng(k)
+    a = rtr.rtr_kvcache_create_ex(1, H, d, k, 1, W, C, "bf16", 0)
+    b = rtr.rtr_kvcache_create_ex(1, H, d, k, 1, W, C, "bf16", 0)
+    nbytes = H * (1 + W + C) * k * d * 2
+    try:
+        kr, vr = (synth.normal(rng, (k, H, d), 0.5, "bf16") for _ in range(2))
+        for c in (a, b):
+            rtr.rtr_kvcache_set_reference(c, 0, dev(kr), dev(vr))
+        for step in range(6):
+            n = 1 + step % C
+            q, kc, vc = (synth.normal(rng, (n * k, H, d), 0.5, "bf16") for _ in range(3))
+            oa, ob = (torch.empty((n * k, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2))
+            rtr.rtr_attn_frame_causal_commit(a, 0, dev(q), dev(kc), dev(vc), n, oa)
+            rtr.rtr_attn_frame_causal(b, 0, dev(q), dev(kc), dev(vc), n, ob)
+            rtr.rtr_kvcache_append_frame(b, 0, dev(kc), dev(vc), n)
+            torch.cuda.synchronize()
+            assert torch.equal(oa.view(torch.int16), ob.view(torch.int16)), f"step {step}"
+            assert rtr.rtr_kvcache_get_index_map(a, 0, W + C) == rtr.rtr_kvcache_get_index_map(b, 0, W + C)
+        slots = rtr.rtr_kvcache_get_index_map(a, 0, W + C)[0]
+        for pa, pb in zip(rtr.rtr_kvcache_device_ptrs(a, 0), rtr.rtr_kvcache_device_ptrs(b, 0)):
+            ta = _raw_view(pa, nbytes).view(H, 1 + W + C, k * d * 2)
+            tb = _raw_view(pb, nbytes).view(H, 1 + W + C, k * d * 2)
+            for s_, f in enumerate(slots):
+                if f >= 0:
+                    assert torch.equal(ta[:, 1 + s_], tb[:, 1 + s_]), f"slot {s_}"
+    finally:
+        rtr.rtr_kvcache_destroy(a)
+        rtr.rtr_kvcache_destroy(b)
