@@ -57,7 +57,7 @@ typedef enum {
     RTR_E_STATE = 3,        /* call not valid in the handle's current state */
     RTR_E_CUDA = 4,         /* a CUDA runtime/driver call failed */
     RTR_E_TIMEOUT = 5,      /* a kernel's bounded wait expired (device status) */
-    RTR_E_UNSUPPORTED = 6   /* valid request this build does not implement */
+    RTR_E_UNSUPPORTED = 6   /* valid request this library does not implement */
 } rtr_status;
 
 typedef enum { RTR_BF16 = 0, RTR_F32 = 1 } rtr_dtype;

@@ -15,7 +15,7 @@ Designs 4, and Key Designs 1 for the reference frame:
 * The reference latent counts as one latent frame placed before the first
   frame; TV2V carries no reference.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 * the window W counts past frames only; the chunk being generated attends to
   [reference | window | chunk] and is appended afterwards;
 * "keeps the most recent frame" is ``retain_last(1)``: the window shrinks to
