@@ -213,19 +213,31 @@ def oracle_sample_flops(w, rows):
     return sum(4.0 * w.head_dim * w.heads * (cached + (r // w.k + 1) * w.k) for r in rows)
 
 
-def time_oracle(w, x, o, seconds_target):
-    """Time the oracle on sampled query rows (all heads) of the chunk,
-    growing the sample until it takes about ``seconds_target``.  Returns
-    (flops, seconds, rows)."""
-    import numpy as np
+def oracle_operands(w, x):
+    """The oracle's decoded operands of the chunk's stream attention (queries,
+    their logical positions, logical keys and values), assembled once so that
+    the timed calls are the attention itself."""
+    return oracle_cache_for(w, x).stream_operands(x.q, x.k_cur, x.v_cur, w.chunk_frames)
+
+
+def oracle_rows(w, ops, rows, nthreads=0):
     import oracle
+    Q, pos, K, V = ops
+    return oracle.attention(Q[rows], pos[rows], K, V, w.k, True, None, nthreads)
+
+
+def time_oracle(w, ops, seconds_target, nthreads=0):
+    """Time the oracle on sampled query rows (all heads) of the chunk,
+    growing the sample until it takes about ``seconds_target``, on
+    ``nthreads`` threads (0: all).  Returns (flops, seconds, rows)."""
+    import numpy as np
     nq = w.chunk_frames * w.k
     rng = np.random.default_rng(123)
     n = 2
     while True:
         rows = np.sort(rng.choice(nq, size=min(n, nq), replace=False))
         t0 = time.perf_counter()
-        o.stream_attention(x.q, x.k_cur, x.v_cur, w.chunk_frames, rows=rows)
+        oracle_rows(w, ops, rows, nthreads)
         dt = time.perf_counter() - t0
         if dt >= 0.5 * seconds_target or n >= nq:
             return oracle_sample_flops(w, rows), dt, rows
@@ -258,14 +270,14 @@ def run_reference(args, rank, world):
     from causal_attention_rtr_b200 import synth
     w = workload()
     x = synth.stream_layer_inputs(w)
-    o = oracle_cache_for(w, x)
+    ops = oracle_operands(w, x)
     per_step = max(0.05, 150.0 / max(1, args.steps + args.warmup))
-    flops, dt, rows = time_oracle(w, x, o, per_step)
+    flops, dt, rows = time_oracle(w, ops, per_step)
     for _ in range(args.warmup):
-        o.stream_attention(x.q, x.k_cur, x.v_cur, w.chunk_frames, rows=rows)
+        oracle_rows(w, ops, rows)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        o.stream_attention(x.q, x.k_cur, x.v_cur, w.chunk_frames, rows=rows)
+        oracle_rows(w, ops, rows)
     total = time.perf_counter() - t0
     value = flops * args.steps / total / 1e12
     cb = cpu_baseline_entry(flops * args.steps, total, rows, w)
@@ -480,9 +492,13 @@ def run_ours(args, rank, world, local_rank):
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        o = oracle_cache_for(w, x)
-        fl, dt, rows = time_oracle(w, x, o, 12.0)
+        ops = oracle_operands(w, x)
+        fl, dt, rows = time_oracle(w, ops, 12.0)
         line["cpu_baseline"] = cpu_baseline_entry(fl, dt, rows, w)
+        fl1, dt1, rows1 = time_oracle(w, ops, 4.0, nthreads=1)
+        line["cpu_baseline"]["single_core"] = {
+            "value": fl1 / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+            "sample": f"{len(rows1)} query rows x {w.heads} heads, {fl1 / 1e9:.1f} GFLOP in {dt1:.2f} s"}
     print(json.dumps(line), flush=True)
 
 

@@ -147,6 +147,14 @@ class ReferenceCache:
         chunk frames see chunk frames up to their own.  ``rows`` selects query
         rows.  Returns fp64 [len(rows), H, d].
         """
+        Q, pos, K, V = self.stream_operands(q, k_cur, v_cur, n_cur_frames)
+        rows = np.arange(Q.shape[0], dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+        return attention(Q[rows], pos[rows], K, V, self.k, True, scale, nthreads)
+
+    def stream_operands(self, q, k_cur, v_cur, n_cur_frames):
+        """The decoded operands of ``stream_attention``: queries [nc, H, d],
+        their logical positions [nc], and the logical keys and values
+        [reference | window | chunk], all fp64."""
         nc = n_cur_frames * self.k
         shape = (nc, self.H, self.d)
         q = np.asarray(q).reshape(shape)
@@ -155,10 +163,8 @@ class ReferenceCache:
         Kc, Vc = self.logical_kv()
         K = decode(np.concatenate([Kc, k_cur], axis=0), self.dtype)
         V = decode(np.concatenate([Vc, v_cur], axis=0), self.dtype)
-        rows = np.arange(nc, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
-        base = self.chunk_first_frame() * self.k
-        return attention(decode(q[rows], self.dtype), base + rows, K, V,
-                         self.k, True, scale, nthreads)
+        pos = self.chunk_first_frame() * self.k + np.arange(nc, dtype=np.int64)
+        return decode(q, self.dtype), pos, K, V
 
 
 class CrossCache:

@@ -63,12 +63,13 @@ void rtr_oracle_attention(const double *q, const int64_t *q_pos, int64_t nq,
                           int causal, double scale, double *out, int nthreads)
 {
 #ifdef _OPENMP
-    if (nthreads > 0) omp_set_num_threads(nthreads);
+    /* the thread count applies to this call only */
+    const int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
 #else
     (void)nthreads;
 #endif
     int64_t npairs = nq * heads;
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
     for (int64_t pr = 0; pr < npairs; ++pr) {
         int64_t r = pr / heads, h = pr % heads;
         const double *qi = q + (r * heads + h) * d;
