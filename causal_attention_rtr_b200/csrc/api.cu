@@ -38,16 +38,18 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                    CUtensorMapFloatOOBfill);
 
+EncodeTiledFn lookup_encode_fn() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+}
+
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+    static const EncodeTiledFn fn = lookup_encode_fn();   // initialised once, thread-safe
     return fn;
 }
 
@@ -213,14 +215,14 @@ rtr_status cuda_status(cudaError_t e) {
 float resolve_scale(float scale, int head_dim) { return scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim); }
 
 int sm_count(int device) {
-    static int cache[64] = {};
+    static std::atomic<int> cache[64] = {};
     if (device < 0 || device >= 64) return 148;
-    if (!cache[device]) {
-        int n = 0;
+    int n = cache[device].load(std::memory_order_relaxed);
+    if (!n) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) n = 148;
-        cache[device] = n;
+        cache[device].store(n, std::memory_order_relaxed);
     }
-    return cache[device];
+    return n;
 }
 
 // Scratch for the partial results of split attention units, one buffer per

@@ -42,6 +42,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <type_traits>
@@ -553,15 +554,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
 template <int D>
 cudaError_t launch_bwd_t(const BwdParams &bp, const BwdProblem &pb, cudaStream_t s) {
     using L = BwdLayout<D>;
-    static int configured_mask = 0;
+    static std::atomic<unsigned long long> configured{0};   // one bit per device (0..63)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!(configured_mask & (1 << dev))) {
+    const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
         cudaError_t e = cudaFuncSetAttribute(bwd_dkdv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(bwd_dq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
         if (e != cudaSuccess) return e;
-        configured_mask |= 1 << dev;
+        configured.fetch_or(bit, std::memory_order_release);
     }
     const long long prep_warps = (long long)bp.n_pad * bp.heads;
     bwd_prep<D><<<(unsigned)((prep_warps * 32 + 255) / 256), 256, 0, s>>>(
