@@ -119,6 +119,50 @@ def test_prefill_empty_is_noop():
     rtr().rtr_attn_block_causal_prefill(None, None, None, 0, 2, 128, 4, "bf16", None)
 
 
+def _growing_score_qkv(n, H, d, jumps, step_log2, seed):
+    """Q, K, V (bf16 bits, [n, H, d]) whose scaled scores rise by about
+    ``step_log2`` (log2 units) at every key position in ``jumps``:
+    Q ~ 1 + 0.05 N(0,1), K_j ~ a_j + 0.05 N(0,1) with a_j stepping up by
+    step_log2 / (log2(e) sqrt(d)) at each jump, V ~ N(0,1)."""
+    rng = np.random.default_rng(seed)
+    da = step_log2 / (np.log2(np.e) * np.sqrt(d))
+    a = da * np.searchsorted(np.sort(np.asarray(jumps)), np.arange(n), side="right")
+    q = 1.0 + 0.05 * rng.standard_normal((n, H, d))
+    k = a[:, None, None] + 0.05 * rng.standard_normal((n, H, d))
+    v = rng.standard_normal((n, H, d))
+    return tuple(synth.f32_to_bf16_bits(x.astype(np.float32)) for x in (q, k, v))
+
+
+GROWTH_CASES = [
+    # d, n, k_per_frame, key positions where every row's score jumps
+    (128, 700, 1000, [5, 128, 296, 454, 639, 690]),   # all keys visible; a jump in each 32-column chunk
+    (128, 700, 150, [5, 128, 296, 454, 639, 690]),    # frame-causal: rows see different prefixes
+    (64, 520, 520, [0, 160, 200, 383, 500]),          # head_dim 64, jump at a tile's first and last column
+]
+
+
+@pytest.mark.parametrize("case", GROWTH_CASES, ids=lambda c: f"d{c[0]}-n{c[1]}-k{c[2]}")
+def test_prefill_parity_scores_growing_along_keys(case):
+    """Row maxima that grow by about 10 (log2 units) part-way through key
+    tiles, at each of the four 32-column positions and in the ragged last tile:
+    the kernel's running max, the rescale of O, of the row sum and of the P
+    already formed for the tile stay exact, so outputs and the row log-sum-exp
+    match the oracle.  (With N(0,1) inputs the max rarely grows this much after
+    the first tile.)"""
+    d, n, kpf, jumps = case
+    H = 2
+    q, k, v = _growing_score_qkv(n, H, d, jumps, 10.0, seed=n + d + kpf)
+    out = torch.empty((n, H, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((H, n), dtype=torch.float32, device="cuda")
+    rtr().rtr_attn_block_causal_prefill_lse(dev(q), dev(k), dev(v), n, H, d, kpf, "bf16", out, lse)
+    torch.cuda.synchronize()
+    Q, K, V = (oracle.decode(x, "bf16") for x in (q, k, v))
+    assert_close(host_f64(out), oracle.prefill(Q, K, V, kpf), str(case))
+    want_lse = oracle.prefill_lse(Q, K, kpf)
+    assert np.max(np.abs(lse.cpu().numpy().T.astype(np.float64) - want_lse)) <= 2e-3 * max(1.0, np.max(np.abs(want_lse)))
+    assert rtr().rtr_get_device_status(0) == rtr().RTR_OK
+
+
 @pytest.mark.parametrize("T,nq,H", [(512, 300, 4), (77, 129, 2), (1, 5, 1)])
 def test_cross_attention_parity(T, nq, H):
     lib = rtr()
