@@ -393,15 +393,16 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside
     # the timed region: every step uploads its Q, K, V from pinned host memory
-    # and reads its output back.  Two device buffer sets and a copy stream let
-    # step s+1's uploads and step s-1's download overlap step s's kernels.
+    # and reads its output back.  Two device buffer sets and one stream per copy
+    # direction let step s+1's uploads and step s-1's download overlap step s's
+    # kernels and each other (PCIe carries both directions at once).
     hq = torch.from_numpy(x.q.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
     hk = torch.from_numpy(x.k_cur.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
     hv = torch.from_numpy(x.v_cur.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
     Ke = min(K, 100)
     ho = [torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     bufs = [(torch.empty_like(q), torch.empty_like(kc), torch.empty_like(vc), torch.empty_like(out)) for _ in range(2)]
-    copy_stream = torch.cuda.Stream()
+    up_stream, down_stream = torch.cuda.Stream(), torch.cuda.Stream()
     up_done = [torch.cuda.Event() for _ in range(Ke)]
     comp_done = [torch.cuda.Event() for _ in range(Ke)]
     down_done = [torch.cuda.Event() for _ in range(Ke)]
@@ -409,19 +410,20 @@ def run_ours(args, rank, world, local_rank):
 
     def upload(s_):
         bq, bk, bv, _ = bufs[s_ % 2]
-        with torch.cuda.stream(copy_stream):
+        with torch.cuda.stream(up_stream):
             if s_ >= 2:
-                copy_stream.wait_event(comp_done[s_ - 2])      # buffer set free again
+                up_stream.wait_event(comp_done[s_ - 2])        # buffer set free again
             bq.copy_(hq, non_blocking=True)
             bk.copy_(hk, non_blocking=True)
             bv.copy_(hv, non_blocking=True)
-            up_done[s_].record(copy_stream)
+            up_done[s_].record(up_stream)
 
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e_start.record(stream)
-    copy_stream.wait_stream(stream)
+    up_stream.wait_stream(stream)
+    down_stream.wait_stream(stream)
     upload(0)
     for s in range(Ke):
         if s + 1 < Ke:
@@ -433,10 +435,10 @@ def run_ours(args, rank, world, local_rank):
         rtr.rtr_attn_frame_causal(c, 0, bq, bk, bv, C, bo, 0.0, sh)
         rtr.rtr_kvcache_append_frame(c, 0, bk, bv, C, sh)
         comp_done[s].record(stream)
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(comp_done[s])
+        with torch.cuda.stream(down_stream):
+            down_stream.wait_event(comp_done[s])
             ho[s % 2].copy_(bo, non_blocking=True)
-            down_done[s].record(copy_stream)
+            down_done[s].record(down_stream)
     stream.wait_event(down_done[Ke - 1])
     e_end.record(stream)
     torch.cuda.synchronize()
@@ -480,7 +482,7 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int(3 * hq.numel() * 2), "d2h_bytes_per_step": int(ho[0].numel() * 2),
                 "ms_per_step": e2e_mean,
                 "how": "pinned host Q/K/V uploaded and output read back every step; copies of neighbouring "
-                       "steps overlap the kernels (copy stream, two buffer sets)"},
+                       "steps overlap the kernels (one stream per copy direction, two buffer sets)"},
         "fused_commit": {"entry": "rtr_attn_frame_causal_commit", "ms_per_step": fused_mean,
                          "separate_ms_per_step": sep_mean, "steps": Kf,
                          "value": job_throughput(flops, fused_mean, world), "unit": "TFLOP/s",
@@ -593,6 +595,8 @@ def run_other(args):
         out = torch.empty_like(chunks[0][0])
         n_chunks = w.frames_total // C
         flops = 0.0
+        for _ in range(3):                               # warm-up: attention leaves the cache unchanged
+            rtr.rtr_attn_frame_causal(c, 0, chunks[0][0], chunks[0][1], chunks[0][2], C, out, 0.0, sh)
         torch.cuda.synchronize()
         a, b = _events(2)
         a.record()
@@ -642,58 +646,74 @@ def run_other(args):
     elif args.workload == "switch_14b":
         w = synth.SWITCH_14B
         H, d, k, W, T = w.heads, w.head_dim, w.k, w.window_frames, w.text_tokens
-        c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "bf16", 0)
-        x = rtr.rtr_crossattn_create(1, H, d, T, "bf16", 0)
         ref, kt, vt = rnd((k, H, d)), rnd((T, H, d)), rnd((T, H, d))
         frames = [tuple(rnd((k, H, d)) for _ in range(3)) for _ in range(2)]
         out = torch.empty_like(frames[0][0])
         xout = torch.empty_like(out)
-        rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
-        rtr.rtr_crossattn_set_text(x, 0, kt, vt, T, sh)
-        torch.cuda.synchronize()
-        flops = 0.0
-        count = 0
-        a, b = _events(2)
-        sw_ev = []
-        a.record()
-        for f in range(w.frames_total):
-            if f > 0 and f % w.switch_every == 0:
-                e0, e1 = _events(2)
-                e0.record()
-                rtr.rtr_crossattn_reset(x)
-                rtr.rtr_crossattn_set_text(x, 0, vt, kt, T, sh)
-                rtr.rtr_kvcache_retain_last(c, 0, 1)
-                count = min(count, 1)
-                rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
-                e1.record()
-                sw_ev.append((e0, e1))
-            q, kk, vv = frames[f % 2]
-            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, 1, out, 0.0, sh)
-            rtr.rtr_attn_cross(x, 0, q, k, xout, 0.0, sh)
-            rtr.rtr_kvcache_append_frame(c, 0, kk, vv, 1, sh)
-            flops += stream_flops(H, d, k, 1 + count, 1) + 4.0 * d * H * k * T
-            count = min(W, count + 1)
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
-        sw_ms = [e0.elapsed_time(e1) for e0, e1 in sw_ev]
-        rtr.rtr_kvcache_destroy(c)
-        rtr.rtr_crossattn_destroy(x)
+
+        def run_stream(timed):
+            """The 64-frame stream with its three switches on fresh caches;
+            returns (ms, flops, switch ms) when ``timed``."""
+            c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "bf16", 0)
+            x = rtr.rtr_crossattn_create(1, H, d, T, "bf16", 0)
+            rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
+            rtr.rtr_crossattn_set_text(x, 0, kt, vt, T, sh)
+            torch.cuda.synchronize()
+            flops = 0.0
+            count = 0
+            a, b = _events(2)
+            sw_ev = []
+            a.record()
+            for f in range(w.frames_total):
+                if f > 0 and f % w.switch_every == 0:
+                    e0, e1 = _events(2)
+                    e0.record()
+                    rtr.rtr_crossattn_reset(x)
+                    rtr.rtr_crossattn_set_text(x, 0, vt, kt, T, sh)
+                    rtr.rtr_kvcache_retain_last(c, 0, 1)
+                    count = min(count, 1)
+                    rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
+                    e1.record()
+                    sw_ev.append((e0, e1))
+                q, kk, vv = frames[f % 2]
+                rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, 1, out, 0.0, sh)
+                rtr.rtr_attn_cross(x, 0, q, k, xout, 0.0, sh)
+                rtr.rtr_kvcache_append_frame(c, 0, kk, vv, 1, sh)
+                flops += stream_flops(H, d, k, 1 + count, 1) + 4.0 * d * H * k * T
+                count = min(W, count + 1)
+            b.record()
+            torch.cuda.synchronize()
+            res = (a.elapsed_time(b), flops, [e0.elapsed_time(e1) for e0, e1 in sw_ev]) if timed else None
+            rtr.rtr_kvcache_destroy(c)
+            rtr.rtr_crossattn_destroy(x)
+            return res
+
+        run_stream(False)                                # warm-up: first launches, scratch growth
+        ms, flops, sw_ms = run_stream(True)
         line.update({"config": w.name, "total_ms": ms, "ms_per_frame": ms / w.frames_total,
                      "attention_tflop": flops / 1e12, "tflops": flops / ms / 1e9,
                      "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
                      "latent_frames_per_s": w.frames_total / (ms / 1e3),
                      "switch_ms": sw_ms,
                      "note": "per frame: self-attention (ref + window + frame), cross-attention to 512 text "
-                             "tokens, append; switches at frames 16/32/48 reset+set text, retain 1, set ref"})
+                             "tokens, append; switches at frames 16/32/48 reset+set text, retain 1, set ref; "
+                             "one untimed pass of the whole stream first"})
     elif args.workload == "tiny_f32":
         w = synth.TINY_F32
         H, d, k, W = w.heads, w.head_dim, w.k, w.window_frames
-        c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "f32", 0)
         ref = rnd((k, H, d), torch.float32, 1.0)
-        rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
         fr = [tuple(rnd((k, H, d), torch.float32, 1.0) for _ in range(3)) for _ in range(w.frames_total)]
         out = torch.empty_like(fr[0][0])
+        for _ in range(max(3, args.warmup)):          # warm-up streams on throwaway caches
+            cw = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "f32", 0)
+            rtr.rtr_kvcache_set_reference(cw, 0, ref, ref, sh)
+            for q, kk, vv in fr:
+                rtr.rtr_attn_frame_causal(cw, 0, q, kk, vv, 1, out, 0.0, sh)
+                rtr.rtr_kvcache_append_frame(cw, 0, kk, vv, 1, sh)
+            torch.cuda.synchronize()
+            rtr.rtr_kvcache_destroy(cw)
+        c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "f32", 0)
+        rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
         torch.cuda.synchronize()
         a, b = _events(2)
         a.record()
