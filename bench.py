@@ -551,8 +551,36 @@ def run_other(args):
             torch.cuda.synchronize()
             ts.append(a.elapsed_time(b))
         ms = statistics.mean(ts)
+        # the same prefill filling a cache (reference + 21-frame window) in the
+        # same launch, alternated call by call with the plain prefill
+        F = w.chunk_frames
+        c = rtr.rtr_kvcache_create(1, w.heads, w.head_dim, w.k, 1, F - 1, "bf16", 0)
+        for _ in range(3):
+            rtr.rtr_attn_block_causal_prefill_cache(c, 0, q, k, v, F, True, out, 0.0, sh)
+        tf, tp = [], []
+        for _ in range(min(max(1, args.steps), 50)):
+            for fill, acc in ((True, tf), (False, tp)):
+                flush.zero_()
+                a, b = _events(2)
+                a.record()
+                if fill:
+                    rtr.rtr_attn_block_causal_prefill_cache(c, 0, q, k, v, F, True, out, 0.0, sh)
+                else:
+                    rtr.rtr_attn_block_causal_prefill(q, k, v, n, w.heads, w.head_dim, w.k, "bf16", out, 0.0, 0, sh)
+                b.record()
+                torch.cuda.synchronize()
+                acc.append(a.elapsed_time(b))
+        if rtr.rtr_get_device_status(0, sh) != rtr.RTR_OK:
+            raise RuntimeError("device status not OK after the prefill into the cache")
+        rtr.rtr_kvcache_destroy(c)
         line.update({"config": w.name, "ms_per_call": ms, "tflop_per_call": flops / 1e12,
-                     "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc})
+                     "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
+                     "with_cache_fill": {
+                         "entry": "rtr_attn_block_causal_prefill_cache (reference + 21 window frames written "
+                                  "by the attention launch)",
+                         "ms_per_call": statistics.mean(tf), "plain_ms_per_call": statistics.mean(tp),
+                         "bytes_written": 2.0 * n * w.heads * w.head_dim * 2,
+                         "how": "alternated call by call with the plain prefill, L2 flushed before each"}})
     elif args.workload == "prefill_22_bwd":
         # backward of the same prefill: algorithmic work 5 matmuls per visible
         # (query, key) pair = 10 * d flops (2.5x the forward's 4 * d)

@@ -186,8 +186,9 @@ struct rtr_kvcache {
     std::vector<long long> g;
     std::vector<CUtensorMap> tmk, tmv;
     std::vector<CUtensorMap> tmk64;   // K maps with 64-row boxes (CTA-pair attention)
-    // Chunk-write maps of the fused commit, device array [layer][S][K, V][128-row, 8-row box]
-    // (bf16 caches with commit room and k a multiple of 8), else null.
+    // Store maps of the fused cache writes, device array [layer][R + S][K, V][128-row, 8-row box]:
+    // entry j covers row block j of a head (the reference frames, then the ring slots); bf16
+    // caches with k a multiple of 8, else null.
     CUtensorMap *cmaps = nullptr;
 };
 
@@ -344,15 +345,16 @@ rtr_status rtr_kvcache_create_ex(int layers, int heads, int head_dim, int k, int
             }
         }
     }
-    if (dt == RTR_BF16 && commit_frames > 0 && k % 8 == 0) {
-        std::vector<CUtensorMap> maps((size_t)layers * c->S * 4);
+    if (dt == RTR_BF16 && k % 8 == 0) {
+        const int blocks = c->R + c->S;
+        std::vector<CUtensorMap> maps((size_t)layers * blocks * 4);
         bool ok = true;
         const uint64_t row_bytes = (uint64_t)head_dim * 2;
         for (int l = 0; l < layers && ok; ++l)
-            for (int sl = 0; sl < c->S && ok; ++sl)
+            for (int j = 0; j < blocks && ok; ++j)
                 for (int kv = 0; kv < 2 && ok; ++kv) {
-                    const char *base = (kv ? c->vbuf : c->kbuf) + l * c->layer_bytes + (size_t)(c->R + sl) * k * row_bytes;
-                    CUtensorMap *m = &maps[(((size_t)l * c->S + sl) * 2 + kv) * 2];
+                    const char *base = (kv ? c->vbuf : c->kbuf) + l * c->layer_bytes + (size_t)j * k * row_bytes;
+                    CUtensorMap *m = &maps[(((size_t)l * blocks + j) * 2 + kv) * 2];
                     ok = make_tmap_bf16_strided(m, base, head_dim, k, heads, (uint64_t)rows * row_bytes, 128, 1) &&
                          make_tmap_bf16_strided(m + 1, base, head_dim, k, heads, (uint64_t)rows * row_bytes, 8, 1);
                 }
@@ -554,7 +556,7 @@ rtr_status rtr_attn_frame_causal_commit(rtr_kvcache *c, int layer, const void *q
     pb.commit_first_slot = (int)(c->g[layer] % c->S);
     pb.commit_slots = c->S;
     pb.commit_row0 = c->R * c->k;
-    pb.commit_maps = c->cmaps ? c->cmaps + (size_t)layer * c->S * 4 : nullptr;
+    pb.commit_maps = c->cmaps ? c->cmaps + ((size_t)layer * (c->R + c->S) + c->R) * 4 : nullptr;
     const rtr_status r = run_attention(pb, c->dt, &c->tmk[layer], &c->tmk64[layer], &c->tmv[layer], c->device,
                                        (cudaStream_t)stream);
     if (r == RTR_OK) {
@@ -606,6 +608,71 @@ rtr_status rtr_attn_block_causal_prefill_lse(const void *q, const void *k, const
     DeviceGuard dg(device);
     if (!dg.ok) return RTR_E_INVAL;
     return run_attention(pb, dt, nullptr, nullptr, nullptr, device, (cudaStream_t)stream);
+}
+
+rtr_status rtr_attn_block_causal_prefill_cache(rtr_kvcache *c, int layer, const void *q, const void *k,
+                                               const void *v, int n_frames, int with_reference, void *out,
+                                               float scale, rtr_stream_t stream) {
+    if (!c || layer < 0 || layer >= c->layers || n_frames < 1 || (with_reference != 0 && with_reference != 1))
+        return RTR_E_INVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return RTR_E_INVAL;
+    if (with_reference && c->R == 0) return RTR_E_STATE;
+    const int nref = with_reference ? c->R : 0;
+    const int nwin = n_frames - nref;
+    if (nwin < 0 || nwin > c->W) return RTR_E_INVAL;
+    const long long n = (long long)n_frames * c->k;
+    if (n > (1ll << 30)) return RTR_E_INVAL;
+    DeviceGuard dg(c->device);
+    AttnProblem pb;
+    memset(&pb, 0, sizeof(pb));
+    pb.nq = (int)n; pb.heads = c->heads; pb.head_dim = c->head_dim; pb.kpf = c->k;
+    pb.nseg = 1;
+    pb.seg[0] = KvSeg{1, 0, (int)n, 1};
+    pb.scale = resolve_scale(scale, c->head_dim);
+    pb.q = q; pb.o = out; pb.k1 = k; pb.v1 = v; pb.rows1 = n;
+    pb.rows0 = c->rows;
+    const long long g = c->g[layer];
+    // One launch writes the sequence's K/V while it attends when every frame's
+    // rows follow from one slot rule: without a reference part the frames are
+    // appended to the ring (slot (g + i) mod S); with one, the reference frames
+    // and the ring slots form one run of row blocks when g is a multiple of S.
+    if (c->dt == RTR_BF16 && (nref == 0 || g % c->S == 0)) {
+        pb.commit_k = c->kbuf + layer * c->layer_bytes;
+        pb.commit_v = c->vbuf + layer * c->layer_bytes;
+        const size_t maps0 = (size_t)layer * (c->R + c->S);
+        if (nref > 0) {
+            pb.commit_row0 = 0;
+            pb.commit_slots = c->R + c->S;
+            pb.commit_first_slot = 0;
+            pb.commit_maps = c->cmaps ? c->cmaps + maps0 * 4 : nullptr;
+        } else {
+            pb.commit_row0 = c->R * c->k;
+            pb.commit_slots = c->S;
+            pb.commit_first_slot = (int)(g % c->S);
+            pb.commit_maps = c->cmaps ? c->cmaps + (maps0 + c->R) * 4 : nullptr;
+        }
+        const rtr_status r = run_attention(pb, c->dt, nullptr, nullptr, nullptr, c->device, (cudaStream_t)stream);
+        if (r != RTR_OK) return r;
+        if (nref > 0) c->ref_valid[layer] = 1;
+        if (nwin > 0) {
+            c->g[layer] += nwin;
+            c->count[layer] = std::min(c->W, c->count[layer] + nwin);
+        }
+        return RTR_OK;
+    }
+    // Otherwise (fp32 storage, or a reference part with g not a multiple of
+    // S): the attention, then the copy kernels of set_reference and append.
+    rtr_status r = run_attention(pb, c->dt, nullptr, nullptr, nullptr, c->device, (cudaStream_t)stream);
+    if (r != RTR_OK) return r;
+    const size_t frame_bytes = (size_t)c->k * c->heads * c->head_dim * elt_size(c->dt);
+    if (nref > 0) {
+        r = rtr_kvcache_set_reference(c, layer, k, v, stream);
+        if (r != RTR_OK) return r;
+    }
+    if (nwin > 0)
+        r = rtr_kvcache_append_frame(c, layer, static_cast<const char *>(k) + nref * frame_bytes,
+                                     static_cast<const char *>(v) + nref * frame_bytes, nwin, stream);
+    return r;
 }
 
 rtr_status rtr_attn_block_causal_backward(const void *q, const void *k, const void *v, const void *out,

@@ -54,6 +54,7 @@ _SIGNATURES = [
     ("rtr_attn_block_causal_prefill", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     ("rtr_attn_block_causal_prefill_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     ("rtr_attn_block_causal_prefill_lse", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _i, _vp]),
+    ("rtr_attn_block_causal_prefill_cache", _i, [_vp, _i, _vp, _vp, _vp, _i, _i, _vp, _f, _vp]),
     ("rtr_attn_block_causal_backward", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f,
                                             _i, _vp]),
     ("rtr_crossattn_create", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
@@ -213,6 +214,13 @@ def rtr_attn_block_causal_prefill_lse(q, k, v, n_tokens, heads, head_dim, k_per_
                                                          k_per_frame, _dtype(dt), _ptr(out), _ptr(lse),
                                                          float(scale), device, _stream(stream)),
                   "rtr_attn_block_causal_prefill_lse")
+
+
+def rtr_attn_block_causal_prefill_cache(c, layer, q, k, v, n_frames, with_reference, out, scale=0.0, stream=None):
+    return _check(_lib.rtr_attn_block_causal_prefill_cache(c, layer, _ptr(q), _ptr(k), _ptr(v), n_frames,
+                                                           1 if with_reference else 0, _ptr(out), float(scale),
+                                                           _stream(stream)),
+                  "rtr_attn_block_causal_prefill_cache")
 
 
 def rtr_attn_block_causal_backward(q, k, v, out, dout, lse, n_tokens, heads, head_dim, k_per_frame, dt, dq, dk, dv,

@@ -245,6 +245,34 @@ rtr_status rtr_attn_block_causal_prefill_lse(const void *q, const void *k,
                                              float scale, int device,
                                              rtr_stream_t stream);
 
+/* Block-causal prefill that also fills layer `layer` of cache c with the
+ * sequence's K/V (papernotes.org note "DiT as Real-Time Rerenderer", Key
+ * Designs 2 and 4: a context attended once under M becomes the cache that
+ * streaming continues from).  q, k, v, out: [n_frames * k][heads][head_dim]
+ * in the cache's element type, k, heads and head_dim; out is exactly what
+ * rtr_attn_block_causal_prefill(q, k, v, n_frames * k, ..., k_per_frame = k)
+ * returns.  The attention reads only this sequence, never the cache.
+ *
+ * with_reference = 1: the first R (ref_frames) frames are the reference.
+ * They are written to the resident slot, which becomes valid; that needs
+ * R >= 1, else RTR_E_STATE.  The remaining n_frames - R frames are appended
+ * to the window as by rtr_kvcache_append_frame.  with_reference = 0: all
+ * n_frames frames are appended and the reference slot is left as it is.
+ * The appended count must be <= window_frames (else RTR_E_INVAL).  The
+ * index map then reads as after rtr_kvcache_set_reference (when
+ * with_reference = 1) followed by rtr_kvcache_append_frame.
+ *
+ * One launch attends and writes for bf16 caches, when with_reference = 0
+ * or when frames_appended is a multiple of the ring's slot count (a fresh
+ * cache, for instance).  Otherwise the copy kernels run after the
+ * attention.  Pointers are caller-owned device memory, 16-byte aligned. */
+rtr_status rtr_attn_block_causal_prefill_cache(rtr_kvcache *c, int layer,
+                                               const void *q, const void *k,
+                                               const void *v, int n_frames,
+                                               int with_reference, void *out,
+                                               float scale,
+                                               rtr_stream_t stream);
+
 /* Backward pass of the block-causal attention (Key Designs 2 and 3: the
  * causal student is trained with Self Forcing and DMD, whose gradients flow
  * through this attention).  Given the forward's inputs q, k, v, its output

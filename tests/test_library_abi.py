@@ -83,6 +83,8 @@ def test_validation_before_device_work(lib):
         assert h.value is None
     assert rtr.raw_status("rtr_attn_frame_causal_commit", None, 0, None, None, None, 1, None, 0.0,
                           None) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_attn_block_causal_prefill_cache", None, 0, None, None, None, 1, 1, None, 0.0,
+                          None) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_kvcache_set_index_map", None, 0, 0, 0, 0) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_kvcache_check_guards", None) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_crossattn_check_guards", None) == rtr.RTR_E_INVAL
