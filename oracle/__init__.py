@@ -21,6 +21,10 @@ Streaming Video Stylization with Autoregressive Diffusion Transformer"):
 * Method > Key Designs 3 -- training (Self Forcing, DMD) runs gradient descent
   through the block-causal attention; ``backward.py`` holds its plain
   derivative.
+* Method > Overall Architecture and Key Designs 1 -- the DiT block around the
+  attention (``dit_block.py``: modulated layer norms, projections, 3D rotary
+  encoding, cross attention to the text, feed-forward), with the readings the
+  pages leave open stated there.
 
 Every function here is the plain definition; see ``attention.py``,
 ``cache.py`` and ``backward.py``.  Parity pins live in ``tests/test_oracle_*.py``.
@@ -30,8 +34,9 @@ from .attention import (attention, prefill, visible, decode, max_threads,
 from .cache import ReferenceCache, CrossCache
 from .backward import (prefill_lse, prefill_backward, prefill_backward_key_rows,
                        prefill_backward_query_rows)
+from . import dit_block
 
 __all__ = ["attention", "prefill", "visible", "decode", "max_threads",
            "library_path", "ReferenceCache", "CrossCache", "prefill_lse",
            "prefill_backward", "prefill_backward_key_rows",
-           "prefill_backward_query_rows"]
+           "prefill_backward_query_rows", "dit_block"]
