@@ -49,7 +49,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--workload", default="wan13_layer",
-                    choices=["wan13_layer", "prefill_22", "prefill_22_bwd", "long_stream", "switch_14b", "tiny_f32"],
+                    choices=["wan13_layer", "prefill_22", "prefill_22_bwd", "long_stream", "switch_14b", "tiny_f32",
+                             "dit_block_13b"],
                     help="wan13_layer is the headline step; the others print one line each for reference")
     return ap.parse_args()
 
@@ -726,6 +727,68 @@ def run_other(args):
                      "note": "per frame: self-attention (ref + window + frame), cross-attention to 512 text "
                              "tokens, append; switches at frames 16/32/48 reset+set text, retain 1, set ref; "
                              "one untimed pass of the whole stream first"})
+    elif args.workload == "dit_block_13b":
+        # one Wan-1.3B-shaped DiT block on the 3-frame chunk: 12 heads x 128,
+        # 30 x 52 tokens per frame, 1 reference + 21 window frames, 512 text
+        # tokens, feed-forward 8960; random bf16 weights
+        w = synth.WAN13_LAYER
+        H, d, k, W, C, F, T = w.heads, w.head_dim, w.k, w.window_frames, w.chunk_frames, 8960, 512
+        D, n = H * d, C * k
+        c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "bf16", 0)
+        x = rtr.rtr_crossattn_create(1, H, d, T, "bf16", 0)
+        rtr.rtr_kvcache_set_reference(c, 0, rnd((k, H, d)), rnd((k, H, d)), sh)
+        for _ in range(W):
+            rtr.rtr_kvcache_append_frame(c, 0, rnd((k, H, d)), rnd((k, H, d)), 1, sh)
+        rtr.rtr_crossattn_set_text(x, 0, rnd((T, H, d)), rnd((T, H, d)), T, sh)
+        shapes = {"wqkv": (D, 3 * D), "bqkv": (3 * D,), "wo": (D, D), "bo": (D,), "wq2": (D, D), "bq2": (D,),
+                  "wo2": (D, D), "bo2": (D,), "w1": (D, F), "b1": (F,), "w2": (F, D), "b2": (D,)}
+        wts = {name: (torch.randn(shp, device="cuda") * (0.1 if name[0] == "b" else shp[0] ** -0.5)).to(torch.bfloat16)
+               for name, shp in shapes.items()}
+        wts["d_ffn"] = F
+        dw = rtr.dit_weights(wts, F)
+        mod = (torch.randn((6, D), device="cuda") * 0.2).to(torch.bfloat16)
+        hid0 = torch.randn((n, D), device="cuda").to(torch.bfloat16)
+        hid = hid0.clone()
+        q, kk, vv = rnd((n, H, d)), rnd((n, H, d)), rnd((n, H, d))
+        out = torch.empty_like(q)
+        for _ in range(3):
+            hid.copy_(hid0)
+            rtr.rtr_dit_block_forward(c, x, 0, dw, mod, hid, C, 30, 52, 22, False, sh)
+            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, C, out, 0.0, sh)
+        tb, ta = [], []
+        for _ in range(min(max(1, args.steps), 50)):
+            hid.copy_(hid0)
+            flush.zero_()
+            a, b = _events(2)
+            a.record()
+            rtr.rtr_dit_block_forward(c, x, 0, dw, mod, hid, C, 30, 52, 22, False, sh)
+            b.record()
+            flush.zero_()
+            a2, b2 = _events(2)
+            a2.record()
+            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, C, out, 0.0, sh)
+            b2.record()
+            torch.cuda.synchronize()
+            tb.append(a.elapsed_time(b))
+            ta.append(a2.elapsed_time(b2))
+        if rtr.rtr_get_device_status(0, sh) != rtr.RTR_OK:
+            raise RuntimeError("device status not OK after the DiT block")
+        rtr.rtr_kvcache_destroy(c)
+        rtr.rtr_crossattn_destroy(x)
+        ms, ams = statistics.mean(tb), statistics.mean(ta)
+        attn_flops = stream_flops(H, d, k, 1 + W, C)
+        cross_flops = 4.0 * d * H * n * T
+        mm_flops = 2.0 * n * (6.0 * D * D + 2.0 * D * F)
+        total = attn_flops + cross_flops + mm_flops
+        line.update({"config": "Wan-1.3B-shaped DiT block: H=12 d=128 k=1560 (30x52), chunk of 3 frames vs ref 1 "
+                               "+ window 21, text 512, FFN 8960, random bf16 weights",
+                     "ms_per_block": ms, "latent_frames_per_s_per_block": C / (ms / 1e3),
+                     "tflop_per_block": total / 1e12, "tflops": total / ms / 1e9,
+                     "frac_of_bf16_peak": total / ms / 1e9 / peak_tc,
+                     "self_attention_tflop": attn_flops / 1e12, "projection_tflop": mm_flops / 1e12,
+                     "attention_alone_ms": ams, "attention_share": ams / ms,
+                     "how": "block calls alternated with the attention alone on the same cache, L2 flushed "
+                            "before each; GEMMs through cuBLAS, the rest in the library's kernels"})
     elif args.workload == "tiny_f32":
         w = synth.TINY_F32
         H, d, k, W = w.heads, w.head_dim, w.k, w.window_frames

@@ -18,9 +18,11 @@
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <tuple>
 #include <utility>
 #include <vector>
 
+#include "dit_internal.h"
 #include "internal.h"
 #include "rtr.h"
 
@@ -226,15 +228,16 @@ int sm_count(int device) {
     return n;
 }
 
-// Scratch for the partial results of split attention units, one buffer per
-// (device, stream) so that calls on different streams never share it.  Grown
-// on demand (cudaFree synchronises the device, so no kernel still uses the old
-// buffer) and kept until the process exits.
-void *stream_workspace(int device, cudaStream_t s, size_t bytes) {
+// Scratch buffers, one per (device, stream, slot) so that calls on different
+// streams never share one: slot 0 holds the partial results of split
+// attention units, slot 1 the DiT block's activations.  Grown on demand
+// (cudaFree synchronises the device, so no kernel still uses the old buffer)
+// and kept until the process exits.
+void *stream_workspace(int device, cudaStream_t s, size_t bytes, int slot = 0) {
     static std::mutex mu;
-    static std::map<std::pair<int, cudaStream_t>, std::pair<void *, size_t>> ws;
+    static std::map<std::tuple<int, cudaStream_t, int>, std::pair<void *, size_t>> ws;
     std::lock_guard<std::mutex> lock(mu);
-    auto &w = ws[{device, s}];
+    auto &w = ws[std::make_tuple(device, s, slot)];
     if (w.second < bytes) {
         if (w.first) cudaFree(w.first);
         w.first = nullptr;
@@ -699,6 +702,78 @@ rtr_status rtr_attn_block_causal_backward(const void *q, const void *k, const vo
     pb.n = n_tokens; pb.heads = heads; pb.head_dim = head_dim; pb.kpf = k_per_frame;
     pb.scale = resolve_scale(scale, head_dim);
     return cuda_status(launch_attn_bwd(pb, st, scratch, (cudaStream_t)stream));
+}
+
+rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer, const rtr_dit_weights *w,
+                                 const void *modulation, void *hidden, int n_cur_frames, int grid_h, int grid_w,
+                                 int t0, int commit, rtr_stream_t stream) {
+    if (!c || !x || !w || layer < 0 || layer >= c->layers || layer >= x->layers || n_cur_frames < 1 ||
+        grid_h < 1 || grid_w < 1 || t0 < 0 || (commit != 0 && commit != 1))
+        return RTR_E_INVAL;
+    if (c->dt != RTR_BF16 || x->dt != RTR_BF16 || x->heads != c->heads || x->head_dim != c->head_dim ||
+        x->device != c->device || (long long)grid_h * grid_w != c->k)
+        return RTR_E_INVAL;
+    const int H = c->heads, d = c->head_dim, D = H * d, F = w->d_ffn;
+    if (F < 8 || F % 8 != 0 || (commit && n_cur_frames > c->W)) return RTR_E_INVAL;
+    for (const void *ptr : {modulation, (const void *)hidden, w->wqkv, w->bqkv, w->wo, w->bo, w->wq2, w->bq2,
+                            w->wo2, w->bo2, w->w1, w->b1, w->w2, w->b2})
+        if (!aligned16(ptr)) return RTR_E_INVAL;
+    const long long n = (long long)n_cur_frames * c->k;
+    if (n > (1 << 24)) return RTR_E_INVAL;
+    if (x->n_text[layer] == 0) return RTR_E_STATE;
+    DeviceGuard dg(c->device);
+    const cudaStream_t s = (cudaStream_t)stream;
+    // activations: h, q, k, v, o (bf16 [n][D]), the GELU output (bf16 [n][F])
+    // and the fp32 projection output ([n][max(3D, F)])
+    auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
+    const size_t nd = up((size_t)n * D * 2), nf = up((size_t)n * F * 2);
+    const size_t n32 = up((size_t)n * std::max(3 * D, F) * 4);
+    char *ws = static_cast<char *>(stream_workspace(c->device, s, 5 * nd + nf + n32, 1));
+    if (!ws) return RTR_E_NOMEM;
+    void *h = ws, *q = ws + nd, *k = ws + 2 * nd, *v = ws + 3 * nd, *o = ws + 4 * nd, *f = ws + 5 * nd;
+    float *g32 = reinterpret_cast<float *>(ws + 5 * nd + nf);
+    const char *mod = static_cast<const char *>(modulation);
+    const size_t mrow = (size_t)D * 2;   // one modulation vector, bytes
+    const int ni = (int)n;
+    const float eps = 1e-6f;
+    cudaError_t e = cudaSuccess;
+    rtr_status st = RTR_OK;
+#define RTR_TRY(call)                                   \
+    do {                                                \
+        if ((e = (call)) != cudaSuccess) return cuda_status(e); \
+    } while (0)
+#define RTR_TRY_ST(call)                                \
+    do {                                                \
+        if ((st = (call)) != RTR_OK) return st;         \
+    } while (0)
+    // self attention branch
+    RTR_TRY(launch_ln_modulate(hidden, mod, mod + mrow, h, ni, D, eps, s));
+    RTR_TRY(gemm_bf16_f32(c->device, s, h, w->wqkv, g32, ni, 3 * D, D));
+    RTR_TRY(launch_rope_qkv(g32, w->bqkv, q, k, v, ni, H, d, c->k, grid_w, t0, s));
+    if (commit && c->S - c->W >= n_cur_frames) {
+        RTR_TRY_ST(rtr_attn_frame_causal_commit(c, layer, q, k, v, n_cur_frames, o, 0.f, stream));
+    } else {
+        RTR_TRY_ST(rtr_attn_frame_causal(c, layer, q, k, v, n_cur_frames, o, 0.f, stream));
+        if (commit) RTR_TRY_ST(rtr_kvcache_append_frame(c, layer, k, v, n_cur_frames, stream));
+    }
+    RTR_TRY(gemm_bf16_f32(c->device, s, o, w->wo, g32, ni, D, D));
+    RTR_TRY(launch_gated_residual(g32, w->bo, mod + 2 * mrow, hidden, ni, D, s));
+    // cross attention branch
+    RTR_TRY(launch_ln_modulate(hidden, nullptr, nullptr, h, ni, D, eps, s));
+    RTR_TRY(gemm_bf16_f32(c->device, s, h, w->wq2, g32, ni, D, D));
+    RTR_TRY(launch_bias_act(g32, w->bq2, q, ni, D, 0, s));
+    RTR_TRY_ST(rtr_attn_cross(x, layer, q, ni, o, 0.f, stream));
+    RTR_TRY(gemm_bf16_f32(c->device, s, o, w->wo2, g32, ni, D, D));
+    RTR_TRY(launch_gated_residual(g32, w->bo2, nullptr, hidden, ni, D, s));
+    // feed-forward branch
+    RTR_TRY(launch_ln_modulate(hidden, mod + 3 * mrow, mod + 4 * mrow, h, ni, D, eps, s));
+    RTR_TRY(gemm_bf16_f32(c->device, s, h, w->w1, g32, ni, F, D));
+    RTR_TRY(launch_bias_act(g32, w->b1, f, ni, F, 1, s));
+    RTR_TRY(gemm_bf16_f32(c->device, s, f, w->w2, g32, ni, D, F));
+    RTR_TRY(launch_gated_residual(g32, w->b2, mod + 5 * mrow, hidden, ni, D, s));
+#undef RTR_TRY
+#undef RTR_TRY_ST
+    return RTR_OK;
 }
 
 rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_text, rtr_dtype dt, int device,

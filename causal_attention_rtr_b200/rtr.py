@@ -30,6 +30,14 @@ _vp = ctypes.c_void_p
 _i = ctypes.c_int
 _f = ctypes.c_float
 
+class DitWeights(ctypes.Structure):
+    """rtr_dit_weights of include/rtr.h: device pointers of one block's bf16
+    weights ([in][out] row-major) and biases, and the feed-forward width."""
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("wqkv", "bqkv", "wo", "bo", "wq2", "bq2", "wo2", "bo2", "w1", "b1", "w2", "b2")] + \
+               [("d_ffn", ctypes.c_int)]
+
+
 # (name, restype, argtypes) for every symbol of include/rtr.h
 _SIGNATURES = [
     ("rtr_status_string", ctypes.c_char_p, [_i]),
@@ -54,6 +62,7 @@ _SIGNATURES = [
     ("rtr_attn_block_causal_prefill", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     ("rtr_attn_block_causal_prefill_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     ("rtr_attn_block_causal_prefill_lse", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _i, _vp]),
+    ("rtr_dit_block_forward", _i, [_vp, _vp, _i, ctypes.POINTER(DitWeights), _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     ("rtr_attn_block_causal_prefill_cache", _i, [_vp, _i, _vp, _vp, _vp, _i, _i, _vp, _f, _vp]),
     ("rtr_attn_block_causal_backward", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f,
                                             _i, _vp]),
@@ -221,6 +230,22 @@ def rtr_attn_block_causal_prefill_cache(c, layer, q, k, v, n_frames, with_refere
                                                            1 if with_reference else 0, _ptr(out), float(scale),
                                                            _stream(stream)),
                   "rtr_attn_block_causal_prefill_cache")
+
+
+def dit_weights(weights, d_ffn):
+    """DitWeights from a mapping of the twelve names to device buffers."""
+    return DitWeights(*[_ptr(weights[f[0]]) for f in DitWeights._fields_[:-1]], int(d_ffn))
+
+
+def rtr_dit_block_forward(c, x, layer, weights, modulation, hidden, n_cur_frames, grid_h, grid_w, t0, commit=False,
+                          stream=None):
+    """``weights``: a DitWeights, or a mapping of its twelve names to device
+    buffers plus "d_ffn"."""
+    w = weights if isinstance(weights, DitWeights) else dit_weights(weights, weights["d_ffn"])
+    return _check(_lib.rtr_dit_block_forward(c, x, layer, ctypes.byref(w), _ptr(modulation), _ptr(hidden),
+                                             n_cur_frames, grid_h, grid_w, t0, 1 if commit else 0,
+                                             _stream(stream)),
+                  "rtr_dit_block_forward")
 
 
 def rtr_attn_block_causal_backward(q, k, v, out, dout, lse, n_tokens, heads, head_dim, k_per_frame, dt, dq, dk, dv,

@@ -273,6 +273,57 @@ rtr_status rtr_attn_block_causal_prefill_cache(rtr_kvcache *c, int layer,
                                                float scale,
                                                rtr_stream_t stream);
 
+/* Weights of one DiT block (see rtr_dit_block_forward): bf16, row-major,
+ * [in][out] so that y = x W + b; D = heads * head_dim of the cache, F =
+ * d_ffn.  wqkv [D][3D] holds the q, k and v projections side by side (q in
+ * columns [0, D), k in [D, 2D), v in [2D, 3D)); bqkv [3D]; wo, wq2, wo2 [D][D]
+ * with biases bo, bq2, bo2 [D]; w1 [D][F], b1 [F]; w2 [F][D], b2 [D].  Every
+ * pointer is caller-owned device memory, 16-byte aligned. */
+typedef struct rtr_dit_weights {
+    const void *wqkv, *bqkv;
+    const void *wo, *bo;
+    const void *wq2, *bq2;
+    const void *wo2, *bo2;
+    const void *w1, *b1;
+    const void *w2, *b2;
+    int d_ffn;
+} rtr_dit_weights;
+
+/* One DiT block on the current chunk of n_cur_frames latent frames
+ * (papernotes.org note "DiT as Real-Time Rerenderer", Method > Overall
+ * Architecture: the patchified tokens go through DiT blocks whose 3D
+ * attention carries the temporal causal mask; Key Designs 1: text enters
+ * through cross attention; Key Designs 4: the rolling caches).  hidden: the
+ * chunk's tokens [n][D] bf16, n = n_cur_frames * k, updated in place to
+ *
+ *   h  = LN(x)(1 + scale1) + shift1;   q, k, v = h Wqkv + bqkv
+ *   q, k rotated by the 3D rotary encoding of (frame t0 + i / k,
+ *        row (i % k) / grid_w, column i % grid_w), grid_h * grid_w = k
+ *   x1 = x + gate1 (A Wo + bo),  A = rtr_attn_frame_causal on cache c
+ *   x2 = x1 + (A2 Wo2 + bo2),    A2 = rtr_attn_cross on x of (LN(x1) Wq2 + bq2)
+ *   x3 = x2 + gate2 (GELU(h3 W1 + b1) W2 + b2),  h3 = LN(x2)(1 + scale2) + shift2
+ *
+ * LN: no affine, eps 1e-6.  GELU: tanh form.  Rotary encoding: each head's
+ * d channels split into (frame, row, column) parts of d - 2P, P, P channels,
+ * P = 2 floor(d / 6); pair (2j, 2j+1) of a part of size S turns by
+ * pos * 10000^(-2j/S).  modulation: bf16 [6][D] = shift1, scale1, gate1,
+ * shift2, scale2, gate2 (from the timestep, computed by the caller).  Every
+ * tensor a later step consumes is stored in bf16; accumulation is fp32
+ * (GEMMs through cuBLAS, the rest in this library's kernels).
+ *
+ * commit = 1 appends the chunk's rotated keys and values to the cache after
+ * its attention, as rtr_kvcache_append_frame would (n_cur_frames <= W), in
+ * the attention launch itself when the cache has that much commit room.
+ * Requires bf16 caches of equal heads and head_dim on one device, text set
+ * in x for this layer (else RTR_E_STATE), d_ffn a multiple of 8.  The
+ * library keeps a per-stream activation buffer of about
+ * n * (10 D + 2 F + 4 max(3D, F)) bytes. */
+rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer,
+                                 const rtr_dit_weights *w,
+                                 const void *modulation, void *hidden,
+                                 int n_cur_frames, int grid_h, int grid_w,
+                                 int t0, int commit, rtr_stream_t stream);
+
 /* Backward pass of the block-causal attention (Key Designs 2 and 3: the
  * causal student is trained with Self Forcing and DMD, whose gradients flow
  * through this attention).  Given the forward's inputs q, k, v, its output

@@ -110,7 +110,7 @@ def rope3d(x, t, y, xc, base=ROPE_BASE):
     return out
 
 
-def dit_block(x, mod, w, cache, xcache, n_cur_frames, grid_h, grid_w, t0, eps=EPS):
+def dit_block(x, mod, w, cache, xcache, n_cur_frames, grid_h, grid_w, t0, eps=EPS, rows=None):
     """One block on the current chunk.
 
     x: bf16 bits [n, D] (n = n_cur_frames * grid_h * grid_w, D = H d); mod:
@@ -121,7 +121,10 @@ def dit_block(x, mod, w, cache, xcache, n_cur_frames, grid_h, grid_w, t0, eps=EP
     (keys already rotary-encoded); xcache: oracle.CrossCache with the text
     keys and values.  Returns a dict with "out" (fp64 values of the bf16
     result [n, D]) and "k", "v" (bf16 bits [n, H, d], the chunk's rotated
-    keys and values, which a commit appends to the cache)."""
+    keys and values, which a commit appends to the cache).  ``rows``
+    selects output rows: every token's keys and values are still formed (the
+    attention needs them), the rest only for those rows, so "out" then has
+    one row per selected token."""
     H, d = cache.H, cache.d
     X = decode(x, "bf16")
     n, D = X.shape
@@ -129,17 +132,21 @@ def dit_block(x, mod, w, cache, xcache, n_cur_frames, grid_h, grid_w, t0, eps=EP
     W = {name: decode(a, "bf16") for name, a in w.items()}
     r = round_bf16
 
+    rows = np.arange(n, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    m = rows.size
     h = r(layer_norm(X, eps) * (1.0 + M[1]) + M[0])
     qkv = h @ W["wqkv"] + W["bqkv"]
     q, k, v = (qkv[:, i * D:(i + 1) * D].reshape(n, H, d) for i in range(3))
     t, yy, xx = token_positions(n_cur_frames, grid_h, grid_w, t0)
-    qb = bf16_bits(r(rope3d(q, t, yy, xx)))
+    qb = np.zeros((n, H, d), np.uint16)
+    qb[rows] = bf16_bits(r(rope3d(q[rows], t[rows], yy[rows], xx[rows])))
     kb = bf16_bits(r(rope3d(k, t, yy, xx)))
     vb = bf16_bits(r(v))
-    o = r(cache.stream_attention(qb, kb, vb, n_cur_frames)).reshape(n, D)
+    o = r(cache.stream_attention(qb, kb, vb, n_cur_frames, rows=rows)).reshape(m, D)
+    X = X[rows]
     x1 = r(X + M[2] * (o @ W["wo"] + W["bo"]))
     q2 = r(r(layer_norm(x1, eps)) @ W["wq2"] + W["bq2"])
-    o2 = r(xcache.attention(bf16_bits(q2).reshape(n, H, d))).reshape(n, D)
+    o2 = r(xcache.attention(bf16_bits(q2).reshape(m, H, d))).reshape(m, D)
     x2 = r(x1 + (o2 @ W["wo2"] + W["bo2"]))
     h3 = r(layer_norm(x2, eps) * (1.0 + M[4]) + M[3])
     f = r(gelu_tanh(h3 @ W["w1"] + W["b1"]))

@@ -260,3 +260,12 @@ def test_planted_block_mistakes_fail_a_pin(slip, monkeypatch):
     want, want_k = _torch_block(x, mod, w, cache, xc, with_keys=True)
     got_k = oracle.decode(r["k"], "bf16")
     assert _rel(r["out"], want) > 1e-2 or _rel(got_k, want_k) > 1e-2
+
+
+def test_block_sampled_rows_equal_the_full_block():
+    x, mod, w, cache, xc = _setup(11)
+    full = _run(x, mod, w, cache, xc)
+    rows = np.array([0, 5, 11, 12, 23])
+    part = db.dit_block(x, mod, w, cache, xc, C, GH, GW, 5, rows=rows)
+    assert np.array_equal(part["out"], full["out"][rows])
+    assert np.array_equal(part["k"], full["k"]) and np.array_equal(part["v"], full["v"])
