@@ -19,6 +19,10 @@
  *   - Method > Key Designs 1: the reference latent is one extra latent frame
  *     placed before the first frame; text enters through cross-attention;
  *     TV2V runs without a reference.
+ *   - Method > Overall Architecture and Key Designs 3: the tokens pass through
+ *     DiT blocks (rtr_dit_block_forward runs one block around the attention),
+ *     and training runs gradient descent through the block-causal attention
+ *     (rtr_attn_block_causal_backward).
  *
  * Conventions shared by every call
  *   - Device tensors are row-major.  Q, K, V and outputs use the layout
