@@ -101,6 +101,42 @@ __global__ void __launch_bounds__(256) ln_modulate(const __nv_bfloat16 *x, const
     }
 }
 
+// One CTA per row with one 8-channel vector per thread held in registers
+// (D <= 8192): the row is read once; mean and variance around it by two block
+// sums; the normalised, modulated row in one rounding.
+__global__ void __launch_bounds__(1024) ln_modulate_reg(const __nv_bfloat16 *x, const __nv_bfloat16 *shift,
+                                                        const __nv_bfloat16 *scale, __nv_bfloat16 *out, int D,
+                                                        float eps) {
+    __shared__ float red[32];
+    const size_t row = blockIdx.x;
+    const int nv = D / 8, i = threadIdx.x;
+    float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (i < nv) unpack8(reinterpret_cast<const uint4 *>(x + row * D)[i], f);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s += f[e];
+    const float mean = block_sum(s, red) / (float)D;
+    float q = 0.f;
+    if (i < nv) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q += (f[e] - mean) * (f[e] - mean);
+    }
+    const float rstd = 1.0f / sqrtf(block_sum(q, red) / (float)D + eps);
+    if (i >= nv) return;
+    if (scale != nullptr) {
+        float sc[8], sh[8];
+        unpack8(reinterpret_cast<const uint4 *>(scale)[i], sc);
+        unpack8(reinterpret_cast<const uint4 *>(shift)[i], sh);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = (f[e] - mean) * rstd * (1.0f + sc[e]) + sh[e];
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = (f[e] - mean) * rstd;
+    }
+    reinterpret_cast<uint4 *>(out + row * D)[i] =
+        make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
+
 // One thread per (token, head, channel pair): bias, rotation of the q and k
 // pairs by the pair's angle, v copied; outputs rounded once to bf16.
 __global__ void __launch_bounds__(256) rope_qkv(const float *qkv, const __nv_bfloat16 *bias, __nv_bfloat16 *q,
@@ -199,6 +235,13 @@ cudaError_t launch_ln_modulate(const void *x, const void *shift, const void *sca
                                float eps, cudaStream_t s) {
     if (n <= 0) return cudaSuccess;
     if (D % 8 != 0 || (scale == nullptr) != (shift == nullptr)) return cudaErrorInvalidValue;
+    if (D / 8 <= 1024) {
+        const int threads = (D / 8 + 31) / 32 * 32;
+        ln_modulate_reg<<<n, threads, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(shift),
+            static_cast<const __nv_bfloat16 *>(scale), static_cast<__nv_bfloat16 *>(out), D, eps);
+        return launched();
+    }
     ln_modulate<<<n, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(shift),
                                   static_cast<const __nv_bfloat16 *>(scale), static_cast<__nv_bfloat16 *>(out), D,
                                   eps);
