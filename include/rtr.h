@@ -269,7 +269,8 @@ rtr_status rtr_attn_block_causal_prefill_lse(const void *q, const void *k,
  * One launch attends and writes for bf16 caches, when with_reference = 0
  * or when frames_appended is a multiple of the ring's slot count (a fresh
  * cache, for instance).  Otherwise the copy kernels run after the
- * attention.  Pointers are caller-owned device memory, 16-byte aligned. */
+ * attention; if the second of those fails, the reference part stays
+ * written.  Pointers are caller-owned device memory, 16-byte aligned. */
 rtr_status rtr_attn_block_causal_prefill_cache(rtr_kvcache *c, int layer,
                                                const void *q, const void *k,
                                                const void *v, int n_frames,
@@ -321,7 +322,9 @@ typedef struct rtr_dit_weights {
  * Requires bf16 caches of equal heads and head_dim on one device, text set
  * in x for this layer (else RTR_E_STATE), d_ffn a multiple of 8.  The
  * library keeps a per-stream activation buffer of about
- * n * (10 D + 2 F + 4 max(3D, F)) bytes. */
+ * n * (10 D + 2 F + 4 max(3D, F)) bytes.  Argument errors leave everything
+ * unchanged; a CUDA error in a step after the commit returns RTR_E_CUDA with
+ * the commit already applied to the index map. */
 rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer,
                                  const rtr_dit_weights *w,
                                  const void *modulation, void *hidden,
