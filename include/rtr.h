@@ -101,11 +101,12 @@ rtr_status rtr_kvcache_create(int layers, int heads, int head_dim, int k,
  * window_frames; 0 is rtr_kvcache_create).  The spare slots let
  * rtr_attn_frame_causal_commit write a chunk of up to commit_frames frames
  * while the frames that chunk attends to stay in place.  Memory per layer
- * grows by 2 * heads * commit_frames * k * head_dim elements (plus 512 bytes
- * of TMA store descriptors per ring slot for bf16 caches with k a multiple
- * of 8, whose chunk write is then done by TMA).  This is a layout choice of
- * the library; the held frames, and so every attention result, are the same
- * as with rtr_kvcache_create. */
+ * grows by 2 * heads * commit_frames * k * head_dim elements.  (Every bf16
+ * cache with k a multiple of 8 also holds 512 bytes of TMA store descriptors
+ * per reference frame and ring slot, through which the fused writes of
+ * rtr_attn_frame_causal_commit and rtr_attn_block_causal_prefill_cache go.)
+ * This is a layout choice of the library; the held frames, and so every
+ * attention result, are the same as with rtr_kvcache_create. */
 rtr_status rtr_kvcache_create_ex(int layers, int heads, int head_dim, int k,
                                  int ref_frames, int window_frames,
                                  int commit_frames, rtr_dtype dt, int device,
