@@ -85,6 +85,8 @@ def test_validation_before_device_work(lib):
                           None) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_attn_block_causal_prefill_cache", None, 0, None, None, None, 1, 1, None, 0.0,
                           None) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_dit_block_forward", None, None, 0, None, None, None, 1, 1, 1, 0, 0,
+                          None) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_kvcache_set_index_map", None, 0, 0, 0, 0) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_kvcache_check_guards", None) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_crossattn_check_guards", None) == rtr.RTR_E_INVAL
