@@ -39,6 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 PROFILE = os.path.join(ROOT, "profiles", "fc_attn_fwd_tc__wan13_layer.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "causal_attention_rtr_b200", "csrc", f)
                   for f in ("attn_tc.cu", "ptx.cuh", "exp2_poly.h", "internal.h")]
+APPEND_PROFILE = os.path.join(ROOT, "profiles", "kv_scatter__wan13_append.md")
+APPEND_SOURCES = [os.path.join(ROOT, "causal_attention_rtr_b200", "csrc", f) for f in ("kv_copy.cu", "internal.h")]
 
 
 def parse_args():
@@ -48,9 +50,11 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-extra-legs", action="store_true",
+                    help="skip the prefill, backward and switching legs of the headline line")
     ap.add_argument("--workload", default="wan13_layer",
                     choices=["wan13_layer", "prefill_22", "prefill_22_bwd", "long_stream", "switch_14b", "tiny_f32",
-                             "dit_block_13b"],
+                             "dit_block_13b", "append_13b"],
                     help="wan13_layer is the headline step; the others print one line each for reference")
     return ap.parse_args()
 
@@ -100,18 +104,18 @@ def measured_peaks():
     return dict(FALLBACK_PEAKS)
 
 
-def profiled_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel source (else None)."""
-    if not os.path.exists(PROFILE):
+def profiled_traffic(profile=PROFILE, sources=KERNEL_SOURCES):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    if not os.path.exists(profile):
         return None
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in sources:
         with open(p, "rb") as f:
             h.update(f.read())
     digest = h.hexdigest()
     vals = {}
-    with open(PROFILE) as f:
+    with open(profile) as f:
         for line in f:
             if ":" in line:
                 k, v = line.split(":", 1)
@@ -197,6 +201,15 @@ class ClockSampler:
         reasons = sorted({n for r in loaded for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(loaded[0][2]),
                 "reasons": reasons, "samples": len(loaded), "power_w_max": pmax}
+
+
+def device_bus_id(torch, dev_id):
+    """PCI bus id of a device, for nvidia-smi -i."""
+    props = torch.cuda.get_device_properties(dev_id)
+    try:
+        return f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    except AttributeError:
+        return os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0]
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -330,11 +343,8 @@ def run_ours(args, rank, world, local_rank):
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    props = torch.cuda.get_device_properties(dev_id)
-    try:
-        bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
-    except AttributeError:
-        bus = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0]
+    bus = device_bus_id(torch, dev_id)
+    sms = torch.cuda.get_device_properties(dev_id).multi_processor_count
     clocks = ClockSampler(bus)
     if world > 1:
         dist.barrier()
@@ -359,6 +369,18 @@ def run_ours(args, rank, world, local_rank):
     status = rtr.rtr_get_device_status(dev_id, sh)
     if status != rtr.RTR_OK:
         raise RuntimeError(f"device status {rtr.rtr_status_string(status)}")
+
+    # ---- the append alone from a cold source: the flush write (256 MiB, twice
+    # L2) evicts the chunk's K/V, so the copy reads them from DRAM
+    Kc = min(K, 50)
+    evc = [_events(2) for _ in range(Kc)]
+    for a, b in evc:
+        flush.zero_()
+        a.record(stream)
+        rtr.rtr_kvcache_append_frame(c, 0, kc, vc, C, sh)
+        b.record(stream)
+    torch.cuda.synchronize()
+    cold_ms = [a.elapsed_time(b) for a, b in evc]
 
     # ---- the same step with the chunk written by the attention launch
     # (rtr_attn_frame_causal_commit on a cache with commit room for the chunk),
@@ -445,9 +467,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = [e_start.elapsed_time(e_end) / Ke]
 
-    step_mean, attn_mean, app_mean, e2e_mean, fused_mean, sep_mean = max_over_ranks(
+    step_mean, attn_mean, app_mean, e2e_mean, fused_mean, sep_mean, cold_mean = max_over_ranks(
         [statistics.mean(step_ms), statistics.mean(attn_ms), statistics.mean(app_ms), statistics.mean(e2e_ms),
-         statistics.mean(fused_ms), statistics.mean(sep_ms)], world, "cuda")
+         statistics.mean(fused_ms), statistics.mean(sep_ms), statistics.mean(cold_ms)], world, "cuda")
 
     rtr.rtr_kvcache_destroy(c)
     if rank != 0:
@@ -461,6 +483,9 @@ def run_ours(args, rank, world, local_rank):
     attn_tflops = flops / (attn_mean * 1e-3) / 1e12
     app_gbs = append_bytes(w) / (app_mean * 1e-3) / 1e9
     traffic = profiled_traffic()
+    app_traffic = profiled_traffic(APPEND_PROFILE, APPEND_SOURCES)
+    per_clock = per_clock_peak_tflops(sms, clk.get("sm_mhz"))
+    cold_gbs = append_bytes(w) / (cold_mean * 1e-3) / 1e9
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
@@ -475,10 +500,18 @@ def run_ours(args, rank, world, local_rank):
                      "frac": attn_tflops / peak_tc, "traffic": traffic,
                      "kernel": "attn_fwd_tc<128> (rtr_attn_frame_causal)",
                      "peak_source": f"{peaks.get('source')} bf16_tflops (burst cuBLAS)",
-                     "flops_per_launch": flops, "ms_per_launch": attn_mean},
+                     "flops_per_launch": flops, "ms_per_launch": attn_mean,
+                     "per_clock_peak": per_clock,
+                     "frac_per_clock": attn_tflops / per_clock if per_clock else None,
+                     "per_clock_how": "sms x 8192 flop/clk x median sampled SM clock"},
         "cache_update": {"kernel": "kv_scatter (rtr_kvcache_append_frame)", "bytes_per_launch": append_bytes(w),
                          "ms_per_launch": app_mean, "achieved_gbs": app_gbs, "peak_gbs": peak_hbm,
-                         "frac": app_gbs / peak_hbm, "peak_source": f"{peaks.get('source')} hbm_gbs"},
+                         "frac": app_gbs / peak_hbm, "peak_source": f"{peaks.get('source')} hbm_gbs",
+                         "traffic": app_traffic,
+                         "source": "warm: in the step, right after the attention read the chunk's K/V",
+                         "cold": {"ms_per_launch": cold_mean, "achieved_gbs": cold_gbs, "frac": cold_gbs / peak_hbm,
+                                  "launches": Kc,
+                                  "source": "cold: the append alone right after a 256 MiB L2 flush"}},
         "e2e": {"value": world * flops / (e2e_mean * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(3 * hq.numel() * 2), "d2h_bytes_per_step": int(ho[0].numel() * 2),
                 "ms_per_step": e2e_mean,
@@ -494,6 +527,14 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
     }
+    if world == 1 and not args.no_extra_legs:
+        # the block-causal prefill, its backward and the 40-head switching
+        # stream, each with its own clock record (single GPU only)
+        cx = LegContext()
+        line["prefill_22"] = clocked(cx, bus, leg_prefill_22, 100, False)
+        line["prefill_22_bwd"] = clocked(cx, bus, leg_prefill_22_bwd, 40)
+        line["switch_14b"] = clocked(cx, bus, leg_switch_14b, 8)
+        del cx
     if world == 1 and not args.no_cpu_baseline:
         ops = oracle_operands(w, x)
         fl, dt, rows = time_oracle(w, ops, 12.0)
@@ -511,312 +552,419 @@ def _events(n):
     return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
 
 
-def run_other(args):
-    """One JSON line per workload other than the headline one (single GPU)."""
-    import numpy as np
-    import torch
+class LegContext:
+    """What the timing legs of the non-headline workloads share (one GPU):
+    the library, the stream, an L2 flush buffer, a seeded device generator
+    (inputs drawn on the device as torch.randn * 0.5: values do not change
+    the time) and the roofline denominators."""
 
-    from causal_attention_rtr_b200 import rtr, synth
+    def __init__(self):
+        import torch
 
-    torch.cuda.set_device(0)
-    sh = torch.cuda.current_stream().cuda_stream
-    peaks = measured_peaks()
-    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    gen = torch.Generator(device="cuda").manual_seed(0)
+        from causal_attention_rtr_b200 import rtr, synth
+        self.torch, self.rtr, self.synth = torch, rtr, synth
+        torch.cuda.set_device(0)
+        self.sh = torch.cuda.current_stream().cuda_stream
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        self.gen = torch.Generator(device="cuda").manual_seed(0)
+        peaks = measured_peaks()
+        self.peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        self.peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        self.sms = torch.cuda.get_device_properties(0).multi_processor_count
 
-    def rnd(shape, dtype=torch.bfloat16, scale=0.5):
-        return (torch.randn(shape, generator=gen, device="cuda", dtype=torch.float32) * scale).to(dtype)
+    def rnd(self, shape, dtype=None, scale=0.5):
+        torch = self.torch
+        dtype = torch.bfloat16 if dtype is None else dtype
+        return (torch.randn(shape, generator=self.gen, device="cuda", dtype=torch.float32) * scale).to(dtype)
 
-    def stream_flops(H, d, k, cached_frames, C):
-        nq = C * k
-        return 4.0 * d * H * (nq * cached_frames * k + sum(k * (c + 1) * k for c in range(C)))
+    def check(self, what):
+        if self.rtr.rtr_get_device_status(0, self.sh) != self.rtr.RTR_OK:
+            raise RuntimeError(f"device status not OK after {what}")
 
-    line = {"workload": args.workload, "n_gpus": 1, "dtype": "bf16", "data": "synthetic (torch.randn * 0.5 on device)"}
-    if args.workload == "prefill_22":
-        w = synth.PREFILL_22
-        n = w.chunk_frames * w.k
-        q, k, v = rnd((n, w.heads, w.head_dim)), rnd((n, w.heads, w.head_dim)), rnd((n, w.heads, w.head_dim))
-        out = torch.empty_like(q)
-        vis = sum(min(n, (i // w.k + 1) * w.k) for i in range(0, n, 1))
-        flops = 4.0 * w.head_dim * w.heads * vis
-        for _ in range(3):
-            rtr.rtr_attn_block_causal_prefill(q, k, v, n, w.heads, w.head_dim, w.k, "bf16", out, 0.0, 0, sh)
-        ts = []
-        for _ in range(max(1, args.steps)):
-            flush.zero_()
-            a, b = _events(2)
-            a.record()
-            rtr.rtr_attn_block_causal_prefill(q, k, v, n, w.heads, w.head_dim, w.k, "bf16", out, 0.0, 0, sh)
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        ms = statistics.mean(ts)
-        # the same prefill filling a cache (reference + 21-frame window) in the
-        # same launch, alternated call by call with the plain prefill
+
+def per_clock_peak_tflops(sms, sm_mhz):
+    """Dense bf16 tensor peak at the sampled SM clock: 8192 flop per clock per
+    SM (148 SMs x 8192 x 1.856 GHz = the nominal 2.25 PFLOP/s)."""
+    return sms * 8192.0 * sm_mhz * 1e-6 if sm_mhz else None
+
+
+def stream_flops(H, d, k, cached_frames, C):
+    nq = C * k
+    return 4.0 * d * H * (nq * cached_frames * k + sum(k * (c + 1) * k for c in range(C)))
+
+
+def prefill_visible_pairs(n, k):
+    return sum(min(n, (i // k + 1) * k) for i in range(n))
+
+
+def leg_prefill_22(cx, calls, with_fill=True):
+    """The 22-frame block-causal prefill (34,320 tokens, 12 heads), L2
+    flushed before each call; optionally the prefill into a cache alternated
+    call by call with the plain one."""
+    rtr, w = cx.rtr, cx.synth.PREFILL_22
+    n, H, d = w.chunk_frames * w.k, w.heads, w.head_dim
+    q, k, v = (cx.rnd((n, H, d)) for _ in range(3))
+    out = cx.torch.empty_like(q)
+    flops = 4.0 * d * H * prefill_visible_pairs(n, w.k)
+    for _ in range(3):
+        rtr.rtr_attn_block_causal_prefill(q, k, v, n, H, d, w.k, "bf16", out, 0.0, 0, cx.sh)
+    evs = [_events(2) for _ in range(calls)]
+    for a, b in evs:
+        cx.flush.zero_()
+        a.record()
+        rtr.rtr_attn_block_causal_prefill(q, k, v, n, H, d, w.k, "bf16", out, 0.0, 0, cx.sh)
+        b.record()
+    cx.torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    cx.check("the prefill")
+    res = {"config": w.name, "ms_per_call": ms, "tflop_per_call": flops / 1e12, "tflops": flops / ms / 1e9,
+           "frac_of_bf16_peak": flops / ms / 1e9 / cx.peak_tc, "calls": calls}
+    if with_fill:
         F = w.chunk_frames
-        c = rtr.rtr_kvcache_create(1, w.heads, w.head_dim, w.k, 1, F - 1, "bf16", 0)
+        c = rtr.rtr_kvcache_create(1, H, d, w.k, 1, F - 1, "bf16", 0)
         for _ in range(3):
-            rtr.rtr_attn_block_causal_prefill_cache(c, 0, q, k, v, F, True, out, 0.0, sh)
+            rtr.rtr_attn_block_causal_prefill_cache(c, 0, q, k, v, F, True, out, 0.0, cx.sh)
         tf, tp = [], []
-        for _ in range(min(max(1, args.steps), 50)):
+        for _ in range(min(calls, 50)):
             for fill, acc in ((True, tf), (False, tp)):
-                flush.zero_()
+                cx.flush.zero_()
                 a, b = _events(2)
                 a.record()
                 if fill:
-                    rtr.rtr_attn_block_causal_prefill_cache(c, 0, q, k, v, F, True, out, 0.0, sh)
+                    rtr.rtr_attn_block_causal_prefill_cache(c, 0, q, k, v, F, True, out, 0.0, cx.sh)
                 else:
-                    rtr.rtr_attn_block_causal_prefill(q, k, v, n, w.heads, w.head_dim, w.k, "bf16", out, 0.0, 0, sh)
+                    rtr.rtr_attn_block_causal_prefill(q, k, v, n, H, d, w.k, "bf16", out, 0.0, 0, cx.sh)
                 b.record()
-                torch.cuda.synchronize()
-                acc.append(a.elapsed_time(b))
-        if rtr.rtr_get_device_status(0, sh) != rtr.RTR_OK:
-            raise RuntimeError("device status not OK after the prefill into the cache")
+                acc.append((a, b))
+        cx.torch.cuda.synchronize()
+        cx.check("the prefill into the cache")
         rtr.rtr_kvcache_destroy(c)
-        line.update({"config": w.name, "ms_per_call": ms, "tflop_per_call": flops / 1e12,
-                     "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
-                     "with_cache_fill": {
-                         "entry": "rtr_attn_block_causal_prefill_cache (reference + 21 window frames written "
-                                  "by the attention launch)",
-                         "ms_per_call": statistics.mean(tf), "plain_ms_per_call": statistics.mean(tp),
-                         "bytes_written": 2.0 * n * w.heads * w.head_dim * 2,
-                         "how": "alternated call by call with the plain prefill, L2 flushed before each"}})
-    elif args.workload == "prefill_22_bwd":
-        # backward of the same prefill: algorithmic work 5 matmuls per visible
-        # (query, key) pair = 10 * d flops (2.5x the forward's 4 * d)
-        w = synth.PREFILL_22
-        n, H, d = w.chunk_frames * w.k, w.heads, w.head_dim
-        q, k, v, do = (rnd((n, H, d)) for _ in range(4))
-        out = torch.empty_like(q)
-        lse = torch.empty((H, n), dtype=torch.float32, device="cuda")
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-        vis = sum(min(n, (i // w.k + 1) * w.k) for i in range(0, n, 1))
-        flops = 10.0 * d * H * vis
-        rtr.rtr_attn_block_causal_prefill_lse(q, k, v, n, H, d, w.k, "bf16", out, lse, 0.0, 0, sh)
-        for _ in range(3):
-            rtr.rtr_attn_block_causal_backward(q, k, v, out, do, lse, n, H, d, w.k, "bf16", dq, dk, dv, 0.0, 0, sh)
-        ts = []
-        for _ in range(max(1, args.steps)):
-            flush.zero_()
-            a, b = _events(2)
-            a.record()
-            rtr.rtr_attn_block_causal_backward(q, k, v, out, do, lse, n, H, d, w.k, "bf16", dq, dk, dv, 0.0, 0, sh)
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        ms = statistics.mean(ts)
-        if rtr.rtr_get_device_status(0, sh) != rtr.RTR_OK:
-            raise RuntimeError("device status not OK after the backward")
-        line.update({"config": w.name + ", backward (dQ, dK, dV)", "ms_per_call": ms,
-                     "tflop_per_call": flops / 1e12, "tflops": flops / ms / 1e9,
-                     "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
-                     "kernels": "bwd_prep + bwd_dkdv (S^T, dP^T, dV, dK) + bwd_dq (S, dP, dQ): 7 tile MMAs per "
-                                "visible tile pair for 5 of algorithmic work"})
-    elif args.workload == "long_stream":
-        w = synth.LONG_STREAM
-        L, H, d, k, C, W = w.layers, w.heads, w.head_dim, w.k, w.chunk_frames, w.window_frames
-        c = rtr.rtr_kvcache_create(L, H, d, k, 1, W, "bf16", 0)
-        ref = rnd((k, H, d))
-        for l in range(L):
-            rtr.rtr_kvcache_set_reference(c, l, ref, ref, sh)
-        chunks = [tuple(rnd((C * k, H, d)) for _ in range(3)) for _ in range(2)]  # reused inputs
-        out = torch.empty_like(chunks[0][0])
-        n_chunks = w.frames_total // C
-        flops = 0.0
-        for _ in range(3):                               # warm-up: attention leaves the cache unchanged
-            rtr.rtr_attn_frame_causal(c, 0, chunks[0][0], chunks[0][1], chunks[0][2], C, out, 0.0, sh)
-        torch.cuda.synchronize()
-        a, b = _events(2)
+        res["with_cache_fill"] = {
+            "entry": "rtr_attn_block_causal_prefill_cache (reference + 21 window frames written by the attention "
+                     "launch)",
+            "ms_per_call": statistics.mean(a.elapsed_time(b) for a, b in tf),
+            "plain_ms_per_call": statistics.mean(a.elapsed_time(b) for a, b in tp),
+            "bytes_written": 2.0 * n * H * d * 2,
+            "how": "alternated call by call with the plain prefill, L2 flushed before each"}
+    return res
+
+
+def leg_prefill_22_bwd(cx, calls):
+    """Backward of the 22-frame prefill: algorithmic work 5 matmuls per
+    visible (query, key) pair = 10 * d flops (2.5x the forward's 4 * d)."""
+    rtr, w = cx.rtr, cx.synth.PREFILL_22
+    n, H, d = w.chunk_frames * w.k, w.heads, w.head_dim
+    q, k, v, do = (cx.rnd((n, H, d)) for _ in range(4))
+    out = cx.torch.empty_like(q)
+    lse = cx.torch.empty((H, n), dtype=cx.torch.float32, device="cuda")
+    dq, dk, dv = (cx.torch.empty_like(q) for _ in range(3))
+    flops = 10.0 * d * H * prefill_visible_pairs(n, w.k)
+    rtr.rtr_attn_block_causal_prefill_lse(q, k, v, n, H, d, w.k, "bf16", out, lse, 0.0, 0, cx.sh)
+    for _ in range(3):
+        rtr.rtr_attn_block_causal_backward(q, k, v, out, do, lse, n, H, d, w.k, "bf16", dq, dk, dv, 0.0, 0, cx.sh)
+    evs = [_events(2) for _ in range(calls)]
+    for a, b in evs:
+        cx.flush.zero_()
         a.record()
-        for ch in range(n_chunks):
-            cached = 1 + min(W, ch * C)
-            for step_ in range(w.steps_per_chunk):
-                q, kk, vv = chunks[(ch + step_) % 2]
-                for l in range(L):
-                    rtr.rtr_attn_frame_causal(c, l, q, kk, vv, C, out, 0.0, sh)
-                    flops += stream_flops(H, d, k, cached, C)
-            for l in range(L):
-                rtr.rtr_kvcache_append_frame(c, l, kk, vv, C, sh)
+        rtr.rtr_attn_block_causal_backward(q, k, v, out, do, lse, n, H, d, w.k, "bf16", dq, dk, dv, 0.0, 0, cx.sh)
         b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
-        # the 30 layers' appends of one chunk back to back (1.73 GB moved), each
-        # from its own source, after an L2 flush: the append kernel's HBM
-        # asymptote, labelled as such
-        peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        batch_bytes = L * 4.0 * C * k * H * d * 2
-        srcs = [(rnd((C * k, H, d)), rnd((C * k, H, d))) for _ in range(L)]
-        bts = []
-        for _ in range(5):
-            flush.zero_()
-            a2, b2 = _events(2)
-            a2.record()
-            for l in range(L):
-                rtr.rtr_kvcache_append_frame(c, l, srcs[l][0], srcs[l][1], C, sh)
-            b2.record()
-            torch.cuda.synchronize()
-            bts.append(a2.elapsed_time(b2))
-        bms = statistics.mean(bts[1:])
-        st = rtr.rtr_get_device_status(0, sh)
-        rtr.rtr_kvcache_destroy(c)
-        line["append_batch_30_layers"] = {
-            "what": "30 rtr_kvcache_append_frame calls (one per layer, 3 frames each, distinct sources) back to "
-                    "back after an L2 flush: the append kernel's asymptote, not a step of the stream",
-            "bytes": batch_bytes, "ms": bms,
-            "achieved_gbs": batch_bytes / bms / 1e6, "peak_gbs": peak_hbm,
-            "frac": batch_bytes / bms / 1e6 / peak_hbm}
-        line.update({"config": w.name, "total_ms": ms, "attention_tflop": flops / 1e12,
-                     "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
-                     "latent_frames_per_s_per_layer": w.frames_total / (ms / 1e3 / L),
-                     "latent_frames_per_s_all_layers": w.frames_total / (ms / 1e3),
-                     "device_status": rtr.rtr_status_string(st),
-                     "note": "attention calls + appends of 30 layers x 40 chunks x 2 steps, one stream"})
-    elif args.workload == "switch_14b":
-        w = synth.SWITCH_14B
-        H, d, k, W, T = w.heads, w.head_dim, w.k, w.window_frames, w.text_tokens
-        ref, kt, vt = rnd((k, H, d)), rnd((T, H, d)), rnd((T, H, d))
-        frames = [tuple(rnd((k, H, d)) for _ in range(3)) for _ in range(2)]
-        out = torch.empty_like(frames[0][0])
-        xout = torch.empty_like(out)
+    cx.torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    cx.check("the backward")
+    return {"config": w.name + ", backward (dQ, dK, dV)", "ms_per_call": ms, "tflop_per_call": flops / 1e12,
+            "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / cx.peak_tc, "calls": calls,
+            "kernels": "bwd_prep + bwd_dkdv (S^T, dP^T, dV, dK) + bwd_dq (S, dP, dQ): 7 tile MMAs per visible "
+                       "tile pair for 5 of algorithmic work"}
 
-        def run_stream(timed):
-            """The 64-frame stream with its three switches on fresh caches;
-            returns (ms, flops, switch ms) when ``timed``."""
-            c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "bf16", 0)
-            x = rtr.rtr_crossattn_create(1, H, d, T, "bf16", 0)
-            rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
-            rtr.rtr_crossattn_set_text(x, 0, kt, vt, T, sh)
-            torch.cuda.synchronize()
-            flops = 0.0
-            count = 0
-            a, b = _events(2)
-            sw_ev = []
-            a.record()
-            for f in range(w.frames_total):
-                if f > 0 and f % w.switch_every == 0:
-                    e0, e1 = _events(2)
-                    e0.record()
-                    rtr.rtr_crossattn_reset(x)
-                    rtr.rtr_crossattn_set_text(x, 0, vt, kt, T, sh)
-                    rtr.rtr_kvcache_retain_last(c, 0, 1)
-                    count = min(count, 1)
-                    rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
-                    e1.record()
-                    sw_ev.append((e0, e1))
-                q, kk, vv = frames[f % 2]
-                rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, 1, out, 0.0, sh)
-                rtr.rtr_attn_cross(x, 0, q, k, xout, 0.0, sh)
-                rtr.rtr_kvcache_append_frame(c, 0, kk, vv, 1, sh)
-                flops += stream_flops(H, d, k, 1 + count, 1) + 4.0 * d * H * k * T
-                count = min(W, count + 1)
-            b.record()
-            torch.cuda.synchronize()
-            res = (a.elapsed_time(b), flops, [e0.elapsed_time(e1) for e0, e1 in sw_ev]) if timed else None
-            rtr.rtr_kvcache_destroy(c)
-            rtr.rtr_crossattn_destroy(x)
-            return res
 
-        run_stream(False)                                # warm-up: first launches, scratch growth
-        ms, flops, sw_ms = run_stream(True)
-        line.update({"config": w.name, "total_ms": ms, "ms_per_frame": ms / w.frames_total,
-                     "attention_tflop": flops / 1e12, "tflops": flops / ms / 1e9,
-                     "frac_of_bf16_peak": flops / ms / 1e9 / peak_tc,
-                     "latent_frames_per_s": w.frames_total / (ms / 1e3),
-                     "switch_ms": sw_ms,
-                     "note": "per frame: self-attention (ref + window + frame), cross-attention to 512 text "
-                             "tokens, append; switches at frames 16/32/48 reset+set text, retain 1, set ref; "
-                             "one untimed pass of the whole stream first"})
-    elif args.workload == "dit_block_13b":
-        # one Wan-1.3B-shaped DiT block on the 3-frame chunk: 12 heads x 128,
-        # 30 x 52 tokens per frame, 1 reference + 21 window frames, 512 text
-        # tokens, feed-forward 8960; random bf16 weights
-        w = synth.WAN13_LAYER
-        H, d, k, W, C, F, T = w.heads, w.head_dim, w.k, w.window_frames, w.chunk_frames, 8960, 512
-        D, n = H * d, C * k
+def leg_switch_14b(cx, passes):
+    """The 64-frame, 40-head stream with its three switches, frame by frame:
+    self-attention (reference + window + frame), cross-attention to 512 text
+    tokens, append; at frames 16/32/48 the text cache is reset and refilled,
+    the window cut to its newest frame and the reference overwritten.  Each
+    part is timed with its own events; ``passes`` passes on fresh caches
+    after one untimed pass."""
+    rtr, torch, w = cx.rtr, cx.torch, cx.synth.SWITCH_14B
+    H, d, k, W, T = w.heads, w.head_dim, w.k, w.window_frames, w.text_tokens
+    ref, kt, vt = cx.rnd((k, H, d)), cx.rnd((T, H, d)), cx.rnd((T, H, d))
+    frames = [tuple(cx.rnd((k, H, d)) for _ in range(3)) for _ in range(2)]
+    out = torch.empty_like(frames[0][0])
+    xout = torch.empty_like(out)
+    self_flops = cross_flops = 0.0
+    count = 0
+    for f in range(w.frames_total):
+        if f > 0 and f % w.switch_every == 0:
+            count = min(count, 1)
+        self_flops += stream_flops(H, d, k, 1 + count, 1)
+        cross_flops += 4.0 * d * H * k * T
+        count = min(W, count + 1)
+
+    def one_pass():
         c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "bf16", 0)
         x = rtr.rtr_crossattn_create(1, H, d, T, "bf16", 0)
-        rtr.rtr_kvcache_set_reference(c, 0, rnd((k, H, d)), rnd((k, H, d)), sh)
-        for _ in range(W):
-            rtr.rtr_kvcache_append_frame(c, 0, rnd((k, H, d)), rnd((k, H, d)), 1, sh)
-        rtr.rtr_crossattn_set_text(x, 0, rnd((T, H, d)), rnd((T, H, d)), T, sh)
-        shapes = {"wqkv": (D, 3 * D), "bqkv": (3 * D,), "wo": (D, D), "bo": (D,), "wq2": (D, D), "bq2": (D,),
-                  "wo2": (D, D), "bo2": (D,), "w1": (D, F), "b1": (F,), "w2": (F, D), "b2": (D,)}
-        wts = {name: (torch.randn(shp, device="cuda") * (0.1 if name[0] == "b" else shp[0] ** -0.5)).to(torch.bfloat16)
-               for name, shp in shapes.items()}
-        wts["d_ffn"] = F
-        dw = rtr.dit_weights(wts, F)
-        mod = (torch.randn((6, D), device="cuda") * 0.2).to(torch.bfloat16)
-        hid0 = torch.randn((n, D), device="cuda").to(torch.bfloat16)
-        hid = hid0.clone()
-        q, kk, vv = rnd((n, H, d)), rnd((n, H, d)), rnd((n, H, d))
-        out = torch.empty_like(q)
-        for _ in range(3):
-            hid.copy_(hid0)
-            rtr.rtr_dit_block_forward(c, x, 0, dw, mod, hid, C, 30, 52, 22, False, sh)
-            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, C, out, 0.0, sh)
-        tb, ta = [], []
-        for _ in range(min(max(1, args.steps), 50)):
-            hid.copy_(hid0)
-            flush.zero_()
-            a, b = _events(2)
-            a.record()
-            rtr.rtr_dit_block_forward(c, x, 0, dw, mod, hid, C, 30, 52, 22, False, sh)
-            b.record()
-            flush.zero_()
-            a2, b2 = _events(2)
-            a2.record()
-            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, C, out, 0.0, sh)
-            b2.record()
-            torch.cuda.synchronize()
-            tb.append(a.elapsed_time(b))
-            ta.append(a2.elapsed_time(b2))
-        if rtr.rtr_get_device_status(0, sh) != rtr.RTR_OK:
-            raise RuntimeError("device status not OK after the DiT block")
-        rtr.rtr_kvcache_destroy(c)
-        rtr.rtr_crossattn_destroy(x)
-        ms, ams = statistics.mean(tb), statistics.mean(ta)
-        attn_flops = stream_flops(H, d, k, 1 + W, C)
-        cross_flops = 4.0 * d * H * n * T
-        mm_flops = 2.0 * n * (6.0 * D * D + 2.0 * D * F)
-        total = attn_flops + cross_flops + mm_flops
-        line.update({"config": "Wan-1.3B-shaped DiT block: H=12 d=128 k=1560 (30x52), chunk of 3 frames vs ref 1 "
-                               "+ window 21, text 512, FFN 8960, random bf16 weights",
-                     "ms_per_block": ms, "latent_frames_per_s_per_block": C / (ms / 1e3),
-                     "tflop_per_block": total / 1e12, "tflops": total / ms / 1e9,
-                     "frac_of_bf16_peak": total / ms / 1e9 / peak_tc,
-                     "self_attention_tflop": attn_flops / 1e12, "projection_tflop": mm_flops / 1e12,
-                     "attention_alone_ms": ams, "attention_share": ams / ms,
-                     "how": "block calls alternated with the attention alone on the same cache, L2 flushed "
-                            "before each; GEMMs through cuBLAS, the rest in the library's kernels"})
-    elif args.workload == "tiny_f32":
-        w = synth.TINY_F32
-        H, d, k, W = w.heads, w.head_dim, w.k, w.window_frames
-        ref = rnd((k, H, d), torch.float32, 1.0)
-        fr = [tuple(rnd((k, H, d), torch.float32, 1.0) for _ in range(3)) for _ in range(w.frames_total)]
-        out = torch.empty_like(fr[0][0])
-        for _ in range(max(3, args.warmup)):          # warm-up streams on throwaway caches
-            cw = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "f32", 0)
-            rtr.rtr_kvcache_set_reference(cw, 0, ref, ref, sh)
-            for q, kk, vv in fr:
-                rtr.rtr_attn_frame_causal(cw, 0, q, kk, vv, 1, out, 0.0, sh)
-                rtr.rtr_kvcache_append_frame(cw, 0, kk, vv, 1, sh)
-            torch.cuda.synchronize()
-            rtr.rtr_kvcache_destroy(cw)
-        c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "f32", 0)
-        rtr.rtr_kvcache_set_reference(c, 0, ref, ref, sh)
+        rtr.rtr_kvcache_set_reference(c, 0, ref, ref, cx.sh)
+        rtr.rtr_crossattn_set_text(x, 0, kt, vt, T, cx.sh)
         torch.cuda.synchronize()
+        ev = []
         a, b = _events(2)
         a.record()
-        for q, kk, vv in fr:
-            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, 1, out, 0.0, sh)
-            rtr.rtr_kvcache_append_frame(c, 0, kk, vv, 1, sh)
+        for f in range(w.frames_total):
+            e = _events(5)
+            e[0].record()
+            if f > 0 and f % w.switch_every == 0:
+                rtr.rtr_crossattn_reset(x)
+                rtr.rtr_crossattn_set_text(x, 0, vt, kt, T, cx.sh)
+                rtr.rtr_kvcache_retain_last(c, 0, 1)
+                rtr.rtr_kvcache_set_reference(c, 0, ref, ref, cx.sh)
+            e[1].record()
+            q, kk, vv = frames[f % 2]
+            rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, 1, out, 0.0, cx.sh)
+            e[2].record()
+            rtr.rtr_attn_cross(x, 0, q, k, xout, 0.0, cx.sh)
+            e[3].record()
+            rtr.rtr_kvcache_append_frame(c, 0, kk, vv, 1, cx.sh)
+            e[4].record()
+            ev.append(e)
         b.record()
         torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
+        parts = [sum(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(4)]
         rtr.rtr_kvcache_destroy(c)
-        line.update({"config": w.name, "dtype": "f32", "total_ms": ms, "ms_per_frame": ms / w.frames_total,
-                     "note": "correctness workload; time is launch-bound"})
+        rtr.rtr_crossattn_destroy(x)
+        return a.elapsed_time(b), parts
+
+    one_pass()
+    runs = [one_pass() for _ in range(passes)]
+    cx.check("the switching stream")
+    ms = statistics.mean(r[0] for r in runs)
+    sw, self_ms, cross_ms, app_ms = (statistics.mean(r[1][i] for r in runs) for i in range(4))
+    flops = self_flops + cross_flops
+    frame_bytes = 4.0 * k * H * d * 2
+    return {"config": w.name, "total_ms": ms, "ms_per_frame": ms / w.frames_total,
+            "attention_tflop": flops / 1e12, "tflops": flops / ms / 1e9,
+            "frac_of_bf16_peak": flops / ms / 1e9 / cx.peak_tc,
+            "latent_frames_per_s": w.frames_total / (ms / 1e3),
+            "self_attention": {"ms": self_ms, "tflop": self_flops / 1e12, "tflops": self_flops / self_ms / 1e9,
+                               "frac_of_bf16_peak": self_flops / self_ms / 1e9 / cx.peak_tc},
+            "cross_attention": {"ms": cross_ms, "tflop": cross_flops / 1e12, "tflops": cross_flops / cross_ms / 1e9,
+                                "frac_of_bf16_peak": cross_flops / cross_ms / 1e9 / cx.peak_tc},
+            "append": {"ms": app_ms, "bytes": frame_bytes * w.frames_total,
+                       "achieved_gbs": frame_bytes * w.frames_total / app_ms / 1e6},
+            "switch_ms": sw, "passes": passes,
+            "note": "parts timed with events around each call of every frame (sums over the 64 frames); "
+                    "one untimed pass of the whole stream first"}
+
+
+def leg_long_stream(cx):
+    """The 30-layer, 120-frame stream (chunks of 3, 2 denoising steps), one
+    stream; plus the 30 layers' appends of one chunk back to back after an L2
+    flush (the append kernel's asymptote, labelled as such)."""
+    rtr, torch, w = cx.rtr, cx.torch, cx.synth.LONG_STREAM
+    L, H, d, k, C, W = w.layers, w.heads, w.head_dim, w.k, w.chunk_frames, w.window_frames
+    c = rtr.rtr_kvcache_create(L, H, d, k, 1, W, "bf16", 0)
+    ref = cx.rnd((k, H, d))
+    for l in range(L):
+        rtr.rtr_kvcache_set_reference(c, l, ref, ref, cx.sh)
+    chunks = [tuple(cx.rnd((C * k, H, d)) for _ in range(3)) for _ in range(2)]  # reused inputs
+    out = torch.empty_like(chunks[0][0])
+    n_chunks = w.frames_total // C
+    flops = 0.0
+    for _ in range(3):                               # warm-up: attention leaves the cache unchanged
+        rtr.rtr_attn_frame_causal(c, 0, chunks[0][0], chunks[0][1], chunks[0][2], C, out, 0.0, cx.sh)
+    torch.cuda.synchronize()
+    a, b = _events(2)
+    a.record()
+    for ch in range(n_chunks):
+        cached = 1 + min(W, ch * C)
+        for step_ in range(w.steps_per_chunk):
+            q, kk, vv = chunks[(ch + step_) % 2]
+            for l in range(L):
+                rtr.rtr_attn_frame_causal(c, l, q, kk, vv, C, out, 0.0, cx.sh)
+                flops += stream_flops(H, d, k, cached, C)
+        for l in range(L):
+            rtr.rtr_kvcache_append_frame(c, l, kk, vv, C, cx.sh)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    batch_bytes = L * 4.0 * C * k * H * d * 2
+    srcs = [(cx.rnd((C * k, H, d)), cx.rnd((C * k, H, d))) for _ in range(L)]
+    bts = []
+    for _ in range(5):
+        cx.flush.zero_()
+        a2, b2 = _events(2)
+        a2.record()
+        for l in range(L):
+            rtr.rtr_kvcache_append_frame(c, l, srcs[l][0], srcs[l][1], C, cx.sh)
+        b2.record()
+        torch.cuda.synchronize()
+        bts.append(a2.elapsed_time(b2))
+    bms = statistics.mean(bts[1:])
+    st = rtr.rtr_get_device_status(0, cx.sh)
+    rtr.rtr_kvcache_destroy(c)
+    return {"config": w.name, "total_ms": ms, "attention_tflop": flops / 1e12,
+            "tflops": flops / ms / 1e9, "frac_of_bf16_peak": flops / ms / 1e9 / cx.peak_tc,
+            "latent_frames_per_s_per_layer": w.frames_total / (ms / 1e3 / L),
+            "latent_frames_per_s_all_layers": w.frames_total / (ms / 1e3),
+            "device_status": rtr.rtr_status_string(st),
+            "append_batch_30_layers": {
+                "what": "30 rtr_kvcache_append_frame calls (one per layer, 3 frames each, distinct sources) back "
+                        "to back after an L2 flush: the append kernel's asymptote, not a step of the stream",
+                "bytes": batch_bytes, "ms": bms, "achieved_gbs": batch_bytes / bms / 1e6, "peak_gbs": cx.peak_hbm,
+                "frac": batch_bytes / bms / 1e6 / cx.peak_hbm},
+            "note": "attention calls + appends of 30 layers x 40 chunks x 2 steps, one stream"}
+
+
+def leg_dit_block_13b(cx, calls):
+    """One Wan-1.3B-shaped DiT block on the 3-frame chunk (12 heads x 128,
+    30 x 52 tokens per frame, 1 reference + 21 window frames, 512 text
+    tokens, feed-forward 8960, random bf16 weights), alternated with the
+    attention alone on the same cache, L2 flushed before each."""
+    rtr, torch, w = cx.rtr, cx.torch, cx.synth.WAN13_LAYER
+    H, d, k, W, C, F, T = w.heads, w.head_dim, w.k, w.window_frames, w.chunk_frames, 8960, 512
+    D, n = H * d, C * k
+    c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "bf16", 0)
+    x = rtr.rtr_crossattn_create(1, H, d, T, "bf16", 0)
+    rtr.rtr_kvcache_set_reference(c, 0, cx.rnd((k, H, d)), cx.rnd((k, H, d)), cx.sh)
+    for _ in range(W):
+        rtr.rtr_kvcache_append_frame(c, 0, cx.rnd((k, H, d)), cx.rnd((k, H, d)), 1, cx.sh)
+    rtr.rtr_crossattn_set_text(x, 0, cx.rnd((T, H, d)), cx.rnd((T, H, d)), T, cx.sh)
+    shapes = {"wqkv": (D, 3 * D), "bqkv": (3 * D,), "wo": (D, D), "bo": (D,), "wq2": (D, D), "bq2": (D,),
+              "wo2": (D, D), "bo2": (D,), "w1": (D, F), "b1": (F,), "w2": (F, D), "b2": (D,)}
+    wts = {name: cx.rnd(shp, scale=(0.1 if name[0] == "b" else shp[0] ** -0.5)) for name, shp in shapes.items()}
+    dw = rtr.dit_weights(wts, F)
+    mod = cx.rnd((6, D), scale=0.2)
+    hid0 = cx.rnd((n, D), scale=1.0)
+    hid = hid0.clone()
+    q, kk, vv = cx.rnd((n, H, d)), cx.rnd((n, H, d)), cx.rnd((n, H, d))
+    out = torch.empty_like(q)
+    for _ in range(3):
+        hid.copy_(hid0)
+        rtr.rtr_dit_block_forward(c, x, 0, dw, mod, hid, C, 30, 52, 22, False, cx.sh)
+        rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, C, out, 0.0, cx.sh)
+    tb, ta = [], []
+    for _ in range(calls):
+        hid.copy_(hid0)
+        cx.flush.zero_()
+        a, b = _events(2)
+        a.record()
+        rtr.rtr_dit_block_forward(c, x, 0, dw, mod, hid, C, 30, 52, 22, False, cx.sh)
+        b.record()
+        cx.flush.zero_()
+        a2, b2 = _events(2)
+        a2.record()
+        rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, C, out, 0.0, cx.sh)
+        b2.record()
+        tb.append((a, b))
+        ta.append((a2, b2))
+    torch.cuda.synchronize()
+    cx.check("the DiT block")
+    rtr.rtr_kvcache_destroy(c)
+    rtr.rtr_crossattn_destroy(x)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in tb)
+    ams = statistics.mean(a.elapsed_time(b) for a, b in ta)
+    attn = stream_flops(H, d, k, 1 + W, C)
+    cross = 4.0 * d * H * n * T
+    mm = 2.0 * n * (6.0 * D * D + 2.0 * D * F)
+    total = attn + cross + mm
+    return {"config": "Wan-1.3B-shaped DiT block: H=12 d=128 k=1560 (30x52), chunk of 3 frames vs ref 1 + window "
+                      "21, text 512, FFN 8960, random bf16 weights",
+            "ms_per_block": ms, "latent_frames_per_s_per_block": C / (ms / 1e3),
+            "tflop_per_block": total / 1e12, "tflops": total / ms / 1e9,
+            "frac_of_bf16_peak": total / ms / 1e9 / cx.peak_tc,
+            "self_attention_tflop": attn / 1e12, "projection_tflop": mm / 1e12,
+            "attention_alone_ms": ams, "attention_share": ams / ms,
+            "rest_ms": ms - ams, "rest_tflops": (total - attn) / (ms - ams) / 1e9,
+            "how": "block calls alternated with the attention alone on the same cache, L2 flushed before each"}
+
+
+def leg_append_13b(cx, calls):
+    """The headline step's cache update alone: rtr_kvcache_append_frame of a
+    3-frame Wan-1.3B chunk (12 heads x 128, k = 1560) into a full 21-frame
+    window (every call evicts 3 frames), each call right after a 256 MiB L2
+    flush, so its source is read from DRAM."""
+    rtr, torch, w = cx.rtr, cx.torch, cx.synth.WAN13_LAYER
+    H, d, k, W, C = w.heads, w.head_dim, w.k, w.window_frames, w.chunk_frames
+    c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "bf16", 0)
+    rtr.rtr_kvcache_set_reference(c, 0, cx.rnd((k, H, d)), cx.rnd((k, H, d)), cx.sh)
+    for _ in range(W):
+        rtr.rtr_kvcache_append_frame(c, 0, cx.rnd((k, H, d)), cx.rnd((k, H, d)), 1, cx.sh)
+    kc, vc = cx.rnd((C * k, H, d)), cx.rnd((C * k, H, d))
+    for _ in range(3):
+        rtr.rtr_kvcache_append_frame(c, 0, kc, vc, C, cx.sh)
+    evs = [_events(2) for _ in range(calls)]
+    for a, b in evs:
+        cx.flush.zero_()
+        a.record()
+        rtr.rtr_kvcache_append_frame(c, 0, kc, vc, C, cx.sh)
+        b.record()
+    torch.cuda.synchronize()
+    cx.check("the appends")
+    rtr.rtr_kvcache_destroy(c)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    nbytes = 4.0 * C * k * H * d * 2
+    return {"config": w.name + ", append of the 3-frame chunk (cold source)", "ms_per_call": ms,
+            "bytes_per_call": nbytes, "achieved_gbs": nbytes / ms / 1e6, "peak_gbs": cx.peak_hbm,
+            "frac": nbytes / ms / 1e6 / cx.peak_hbm, "calls": calls}
+
+
+def leg_tiny_f32(cx, warmup):
+    """The fp32 correctness stream (10 frames, one at a time): launch-bound."""
+    rtr, torch, w = cx.rtr, cx.torch, cx.synth.TINY_F32
+    H, d, k, W = w.heads, w.head_dim, w.k, w.window_frames
+    ref = cx.rnd((k, H, d), torch.float32, 1.0)
+    fr = [tuple(cx.rnd((k, H, d), torch.float32, 1.0) for _ in range(3)) for _ in range(w.frames_total)]
+    out = torch.empty_like(fr[0][0])
+    for _ in range(max(3, warmup)):               # warm-up streams on throwaway caches
+        cw = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "f32", 0)
+        rtr.rtr_kvcache_set_reference(cw, 0, ref, ref, cx.sh)
+        for q, kk, vv in fr:
+            rtr.rtr_attn_frame_causal(cw, 0, q, kk, vv, 1, out, 0.0, cx.sh)
+            rtr.rtr_kvcache_append_frame(cw, 0, kk, vv, 1, cx.sh)
+        torch.cuda.synchronize()
+        rtr.rtr_kvcache_destroy(cw)
+    c = rtr.rtr_kvcache_create(1, H, d, k, 1, W, "f32", 0)
+    rtr.rtr_kvcache_set_reference(c, 0, ref, ref, cx.sh)
+    torch.cuda.synchronize()
+    a, b = _events(2)
+    a.record()
+    for q, kk, vv in fr:
+        rtr.rtr_attn_frame_causal(c, 0, q, kk, vv, 1, out, 0.0, cx.sh)
+        rtr.rtr_kvcache_append_frame(c, 0, kk, vv, 1, cx.sh)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    rtr.rtr_kvcache_destroy(c)
+    return {"config": w.name, "dtype": "f32", "total_ms": ms, "ms_per_frame": ms / w.frames_total,
+            "note": "correctness workload; time is launch-bound"}
+
+
+def clocked(cx, bus, fn, *args):
+    """Run one leg with its own clock record; adds the fraction of the
+    per-clock tensor peak where the leg reports TFLOP/s."""
+    sampler = ClockSampler(bus)
+    sampler.start()
+    res = fn(cx, *args)
+    res["clocks"] = sampler.stop()
+    pc = per_clock_peak_tflops(cx.sms, res["clocks"].get("sm_mhz"))
+    if pc and "tflops" in res:
+        res["frac_per_clock"] = res["tflops"] / pc
+    return res
+
+
+def run_other(args):
+    """One JSON line for a workload other than the headline one (single GPU)."""
+    cx = LegContext()
+    bus = device_bus_id(cx.torch, 0)
+    legs = {"prefill_22": (leg_prefill_22, max(1, args.steps)),
+            "prefill_22_bwd": (leg_prefill_22_bwd, max(1, args.steps)),
+            "long_stream": (leg_long_stream,),
+            "switch_14b": (leg_switch_14b, 3),
+            "dit_block_13b": (leg_dit_block_13b, min(max(1, args.steps), 50)),
+            "tiny_f32": (leg_tiny_f32, args.warmup),
+            "append_13b": (leg_append_13b, max(1, args.steps))}
+    fn, *rest = legs[args.workload]
+    line = {"workload": args.workload, "n_gpus": 1, "dtype": "bf16",
+            "data": "synthetic (torch.randn * 0.5 on device)"}
+    line.update(clocked(cx, bus, fn, *rest))
     print(json.dumps(line), flush=True)
 
 

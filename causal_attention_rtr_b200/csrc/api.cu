@@ -26,10 +26,6 @@
 #include "internal.h"
 #include "rtr.h"
 
-#ifndef RTR_DEFAULT_CTA_GROUP
-#define RTR_DEFAULT_CTA_GROUP 1   // the CTA-pair kernel (2) measured slower on every workload
-#endif
-
 namespace rtr {
 
 // ------------------------------------------------------------------ tensor maps
@@ -164,11 +160,22 @@ rtr_status guards_status(const char *p, size_t bytes) {
     return RTR_OK;
 }
 
-int attn_cta_group() {
-    const char *e = std::getenv("RTR_CTA_GROUP");
-    if (e && e[0] == '1') return 1;
-    if (e && e[0] == '2') return 2;
-    return RTR_DEFAULT_CTA_GROUP;
+bool shape_ok(int heads, int head_dim) { return heads >= 1 && (head_dim == 64 || head_dim == 128); }
+
+float resolve_scale(float scale, int head_dim) { return scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim); }
+
+int sm_count(int device) {
+    static std::atomic<int> cache[64] = {};
+    if (device < 0 || device >= 64) return 148;
+    int n = cache[device].load(std::memory_order_relaxed);
+    if (!n) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        cache[device].store(n, std::memory_order_relaxed);
+    }
+    return n;
 }
 
 }  // namespace rtr
@@ -207,54 +214,96 @@ struct rtr_xattn {
 
 namespace {
 
-bool shape_ok(int heads, int head_dim) { return heads >= 1 && (head_dim == 64 || head_dim == 128); }
-
 rtr_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return RTR_OK;
     if (e == cudaErrorMemoryAllocation) return RTR_E_NOMEM;
     return RTR_E_CUDA;
 }
 
-float resolve_scale(float scale, int head_dim) { return scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim); }
-
-int sm_count(int device) {
-    static std::atomic<int> cache[64] = {};
-    if (device < 0 || device >= 64) return 148;
-    int n = cache[device].load(std::memory_order_relaxed);
-    if (!n) {
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) n = 148;
-        cache[device].store(n, std::memory_order_relaxed);
-    }
-    return n;
-}
-
 // Scratch buffers, one per (device, stream, slot) so that calls on different
 // streams never share one: slot 0 holds the partial results of split
 // attention units, slot 1 the DiT block's activations.  Grown on demand
-// (cudaFree synchronises the device, so no kernel still uses the old buffer)
-// and kept until the process exits.
+// (cudaFree synchronises the device, so no kernel still uses the old buffer).
+// A device keeps the buffers of its kMaxWorkspaceStreams most recently used
+// (stream, slot) pairs: a caller that cycles through short-lived streams
+// does not accumulate one buffer per stream.  The least recently used one is
+// freed after a device synchronisation, so no kernel still reads it.
+// rtr_release_workspaces frees a device's buffers on request.
+constexpr size_t kMaxWorkspaceStreams = 8;
+
+struct Workspace {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+    unsigned long long last_use = 0;
+};
+
+std::mutex g_ws_mu;
+std::map<std::tuple<int, cudaStream_t, int>, Workspace> g_ws;
+unsigned long long g_ws_clock = 0;
+
 void *stream_workspace(int device, cudaStream_t s, size_t bytes, int slot = 0) {
-    static std::mutex mu;
-    static std::map<std::tuple<int, cudaStream_t, int>, std::pair<void *, size_t>> ws;
-    std::lock_guard<std::mutex> lock(mu);
-    auto &w = ws[std::make_tuple(device, s, slot)];
-    if (w.second < bytes) {
-        if (w.first) cudaFree(w.first);
-        w.first = nullptr;
-        w.second = 0;
-        if (lib_malloc(&w.first, bytes) != cudaSuccess) {
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    const auto key = std::make_tuple(device, s, slot);
+    auto it = g_ws.find(key);
+    if (it == g_ws.end()) {
+        size_t on_device = 0;
+        auto lru = g_ws.end();
+        for (auto j = g_ws.begin(); j != g_ws.end(); ++j) {
+            if (std::get<0>(j->first) != device) continue;
+            ++on_device;
+            if (lru == g_ws.end() || j->second.last_use < lru->second.last_use) lru = j;
+        }
+        if (on_device >= kMaxWorkspaceStreams && lru != g_ws.end()) {
+            if (cudaDeviceSynchronize() != cudaSuccess) return nullptr;
+            if (lru->second.ptr) cudaFree(lru->second.ptr);
+            g_ws.erase(lru);
+        }
+        it = g_ws.emplace(key, Workspace()).first;
+    }
+    Workspace &w = it->second;
+    w.last_use = ++g_ws_clock;
+    if (w.bytes < bytes) {
+        if (w.ptr) cudaFree(w.ptr);
+        w.ptr = nullptr;
+        w.bytes = 0;
+        if (lib_malloc(&w.ptr, bytes) != cudaSuccess) {
             cudaGetLastError();
-            w.first = nullptr;
+            w.ptr = nullptr;
             return nullptr;
         }
-        w.second = bytes;
+        w.bytes = bytes;
     }
-    return w.first;
+    return w.ptr;
+}
+
+// Frees every scratch buffer of `device` (the device is current).
+rtr_status release_workspaces(int device) {
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    if (cudaDeviceSynchronize() != cudaSuccess) return RTR_E_CUDA;
+    for (auto j = g_ws.begin(); j != g_ws.end();) {
+        if (std::get<0>(j->first) == device) {
+            if (j->second.ptr) cudaFree(j->second.ptr);
+            j = g_ws.erase(j);
+        } else {
+            ++j;
+        }
+    }
+    return RTR_OK;
+}
+
+size_t workspace_count(int device) {
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    size_t n = 0;
+    for (auto &x : g_ws)
+        if (std::get<0>(x.first) == device) ++n;
+    return n;
 }
 
 // Launch the attention for a problem; picks the kernel for the element type.
+// cta_group: 1 (one CTA per MMA, the default everywhere) or 2 (the CTA-pair
+// kernel, reached only through rtr_attn_block_causal_prefill_ex).
 rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0, const CUtensorMap *tm_k0h,
-                         const CUtensorMap *tm_v0, int device, cudaStream_t s) {
+                         const CUtensorMap *tm_v0, int device, cudaStream_t s, int cta_group = 1) {
     if (pb.nq == 0) return RTR_OK;
     for (int i = 0; i < pb.nseg; ++i)
         if (pb.seg[i].len <= 0) return RTR_E_INVAL;
@@ -265,7 +314,7 @@ rtr_status run_attention(AttnProblem &pb, rtr_dtype dt, const CUtensorMap *tm_k0
         if (!st) return RTR_E_CUDA;
         AttnPlan plan;
         // The chunk write (commit) is implemented for one CTA per MMA.
-        plan_attn_bf16(pb, sm_count(device), pb.commit_k ? 1 : attn_cta_group(), plan);
+        plan_attn_bf16(pb, sm_count(device), pb.commit_k ? 1 : cta_group, plan);
         void *scratch = stream_workspace(device, s, plan.scratch_bytes);
         if (!scratch) return RTR_E_NOMEM;
         e = launch_attn_bf16(pb, plan, tm_k0, tm_k0h, tm_v0, st, scratch, s);
@@ -529,6 +578,13 @@ rtr_status stream_problem(const rtr_kvcache *c, int layer, const void *q, const 
 
 rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q, const void *k_cur,
                                  const void *v_cur, int n_cur_frames, void *out, float scale, rtr_stream_t stream) {
+    return rtr_attn_frame_causal_ex(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale, 1, stream);
+}
+
+rtr_status rtr_attn_frame_causal_ex(const rtr_kvcache *c, int layer, const void *q, const void *k_cur,
+                                    const void *v_cur, int n_cur_frames, void *out, float scale, int cta_group,
+                                    rtr_stream_t stream) {
+    if (cta_group != 1 && cta_group != 2) return RTR_E_INVAL;
     AttnProblem pb;
     const rtr_status st = stream_problem(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale, pb);
     if (st != RTR_OK) return st;
@@ -536,7 +592,7 @@ rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer, const void *q,
     const CUtensorMap *tk = c->dt == RTR_BF16 ? &c->tmk[layer] : nullptr;
     const CUtensorMap *tkh = c->dt == RTR_BF16 ? &c->tmk64[layer] : nullptr;
     const CUtensorMap *tv = c->dt == RTR_BF16 ? &c->tmv[layer] : nullptr;
-    return run_attention(pb, c->dt, tk, tkh, tv, c->device, (cudaStream_t)stream);
+    return run_attention(pb, c->dt, tk, tkh, tv, c->device, (cudaStream_t)stream, cta_group);
 }
 
 rtr_status rtr_attn_frame_causal_commit(rtr_kvcache *c, int layer, const void *q, const void *k_cur,
@@ -572,8 +628,15 @@ rtr_status rtr_attn_frame_causal_commit(rtr_kvcache *c, int layer, const void *q
 rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k, const void *v, int n_tokens, int heads,
                                          int head_dim, int k_per_frame, rtr_dtype dt, void *out, float scale,
                                          int device, rtr_stream_t stream) {
+    return rtr_attn_block_causal_prefill_ex(q, k, v, n_tokens, heads, head_dim, k_per_frame, dt, out, scale, 1,
+                                            device, stream);
+}
+
+rtr_status rtr_attn_block_causal_prefill_ex(const void *q, const void *k, const void *v, int n_tokens, int heads,
+                                            int head_dim, int k_per_frame, rtr_dtype dt, void *out, float scale,
+                                            int cta_group, int device, rtr_stream_t stream) {
     if (n_tokens < 0 || !shape_ok(heads, head_dim) || k_per_frame < 1 || (dt != RTR_BF16 && dt != RTR_F32) ||
-        device < 0)
+        device < 0 || (cta_group != 1 && cta_group != 2))
         return RTR_E_INVAL;
     if (n_tokens == 0) return RTR_OK;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return RTR_E_INVAL;
@@ -587,7 +650,7 @@ rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k, const voi
     pb.q = q; pb.o = out; pb.k1 = k; pb.v1 = v; pb.rows1 = n_tokens;
     DeviceGuard dg(device);
     if (!dg.ok) return RTR_E_INVAL;
-    return run_attention(pb, dt, nullptr, nullptr, nullptr, device, (cudaStream_t)stream);
+    return run_attention(pb, dt, nullptr, nullptr, nullptr, device, (cudaStream_t)stream, cta_group);
 }
 
 rtr_status rtr_attn_block_causal_prefill_lse(const void *q, const void *k, const void *v, int n_tokens, int heads,
@@ -723,21 +786,34 @@ rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer, 
     if (x->n_text[layer] == 0) return RTR_E_STATE;
     DeviceGuard dg(c->device);
     const cudaStream_t s = (cudaStream_t)stream;
-    // activations: h, q, k, v, o (bf16 [n][D]), the GELU output (bf16 [n][F])
-    // and the fp32 projection output ([n][max(3D, F)])
+    unsigned *status = device_status_ptr(c->device);
+    if (!status) return RTR_E_CUDA;
+    const int sms = sm_count(c->device);
+    // activations: h, q, k, v, o (bf16 [n][D]) and the GELU output (bf16 [n][F])
     auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
     const size_t nd = up((size_t)n * D * 2), nf = up((size_t)n * F * 2);
-    const size_t n32 = up((size_t)n * std::max(3 * D, F) * 4);
-    char *ws = static_cast<char *>(stream_workspace(c->device, s, 5 * nd + nf + n32, 1));
+    char *ws = static_cast<char *>(stream_workspace(c->device, s, 5 * nd + nf, 1));
     if (!ws) return RTR_E_NOMEM;
     void *h = ws, *q = ws + nd, *k = ws + 2 * nd, *v = ws + 3 * nd, *o = ws + 4 * nd, *f = ws + 5 * nd;
-    float *g32 = reinterpret_cast<float *>(ws + 5 * nd + nf);
     const char *mod = static_cast<const char *>(modulation);
     const size_t mrow = (size_t)D * 2;   // one modulation vector, bytes
     const int ni = (int)n;
     const float eps = 1e-6f;
     cudaError_t e = cudaSuccess;
     rtr_status st = RTR_OK;
+    // One projection with its epilogue: a = activations [n][in], w = [in][out].
+    auto gemm = [&](const void *a, const void *wt, int n_out, int n_in, int epi, const void *bias, const void *gate,
+                    void *out) {
+        GemmArgs g;
+        memset(&g, 0, sizeof(g));
+        g.a = a; g.w = wt; g.m = ni; g.n = n_out; g.k = n_in; g.epi = epi;
+        g.bias = bias; g.gate = gate; g.out = out;
+        if (epi == kEpiQkvRope) {
+            g.q = q; g.k_out = k; g.v = v;
+            g.head_dim = d; g.kpf = c->k; g.grid_w = grid_w; g.t0 = t0;
+        }
+        return launch_gemm_bf16(g, status, sms, s);
+    };
 #define RTR_TRY(call)                                   \
     do {                                                \
         if ((e = (call)) != cudaSuccess) return cuda_status(e); \
@@ -748,32 +824,68 @@ rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer, 
     } while (0)
     // self attention branch
     RTR_TRY(launch_ln_modulate(hidden, mod, mod + mrow, h, ni, D, eps, s));
-    RTR_TRY(gemm_bf16_f32(c->device, s, h, w->wqkv, g32, ni, 3 * D, D));
-    RTR_TRY(launch_rope_qkv(g32, w->bqkv, q, k, v, ni, H, d, c->k, grid_w, t0, s));
+    RTR_TRY(gemm(h, w->wqkv, 3 * D, D, kEpiQkvRope, w->bqkv, nullptr, nullptr));
     if (commit && c->S - c->W >= n_cur_frames) {
         RTR_TRY_ST(rtr_attn_frame_causal_commit(c, layer, q, k, v, n_cur_frames, o, 0.f, stream));
     } else {
         RTR_TRY_ST(rtr_attn_frame_causal(c, layer, q, k, v, n_cur_frames, o, 0.f, stream));
         if (commit) RTR_TRY_ST(rtr_kvcache_append_frame(c, layer, k, v, n_cur_frames, stream));
     }
-    RTR_TRY(gemm_bf16_f32(c->device, s, o, w->wo, g32, ni, D, D));
-    RTR_TRY(launch_gated_residual(g32, w->bo, mod + 2 * mrow, hidden, ni, D, s));
+    RTR_TRY(gemm(o, w->wo, D, D, kEpiGatedResidual, w->bo, mod + 2 * mrow, hidden));
     // cross attention branch
     RTR_TRY(launch_ln_modulate(hidden, nullptr, nullptr, h, ni, D, eps, s));
-    RTR_TRY(gemm_bf16_f32(c->device, s, h, w->wq2, g32, ni, D, D));
-    RTR_TRY(launch_bias_act(g32, w->bq2, q, ni, D, 0, s));
+    RTR_TRY(gemm(h, w->wq2, D, D, kEpiBias, w->bq2, nullptr, q));
     RTR_TRY_ST(rtr_attn_cross(x, layer, q, ni, o, 0.f, stream));
-    RTR_TRY(gemm_bf16_f32(c->device, s, o, w->wo2, g32, ni, D, D));
-    RTR_TRY(launch_gated_residual(g32, w->bo2, nullptr, hidden, ni, D, s));
+    RTR_TRY(gemm(o, w->wo2, D, D, kEpiGatedResidual, w->bo2, nullptr, hidden));
     // feed-forward branch
     RTR_TRY(launch_ln_modulate(hidden, mod + 3 * mrow, mod + 4 * mrow, h, ni, D, eps, s));
-    RTR_TRY(gemm_bf16_f32(c->device, s, h, w->w1, g32, ni, F, D));
-    RTR_TRY(launch_bias_act(g32, w->b1, f, ni, F, 1, s));
-    RTR_TRY(gemm_bf16_f32(c->device, s, f, w->w2, g32, ni, D, F));
-    RTR_TRY(launch_gated_residual(g32, w->b2, mod + 5 * mrow, hidden, ni, D, s));
+    RTR_TRY(gemm(h, w->w1, F, D, kEpiBiasGelu, w->b1, nullptr, f));
+    RTR_TRY(gemm(f, w->w2, D, F, kEpiGatedResidual, w->b2, mod + 5 * mrow, hidden));
 #undef RTR_TRY
 #undef RTR_TRY_ST
     return RTR_OK;
+}
+
+rtr_status rtr_dit_linear(const void *a, const void *w, int m, int n, int k, rtr_epilogue epilogue, const void *bias,
+                          const void *gate, void *out, int device, rtr_stream_t stream) {
+    if (m < 0 || n < 8 || k < 8 || n % 8 != 0 || k % 8 != 0 || device < 0 ||
+        (epilogue != RTR_EPI_BIAS && epilogue != RTR_EPI_BIAS_GELU && epilogue != RTR_EPI_GATED_RESIDUAL))
+        return RTR_E_INVAL;
+    if (m == 0) return RTR_OK;
+    if (!aligned16(a) || !aligned16(w) || !aligned16(bias) || !aligned16(out) || (gate && !aligned16(gate)) ||
+        (gate && epilogue != RTR_EPI_GATED_RESIDUAL))
+        return RTR_E_INVAL;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    unsigned *status = device_status_ptr(device);
+    if (!status) return RTR_E_CUDA;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.a = a; g.w = w; g.m = m; g.n = n; g.k = k;
+    g.epi = epilogue == RTR_EPI_BIAS ? kEpiBias : epilogue == RTR_EPI_BIAS_GELU ? kEpiBiasGelu : kEpiGatedResidual;
+    g.bias = bias; g.gate = gate; g.out = out;
+    return cuda_status(launch_gemm_bf16(g, status, sm_count(device), (cudaStream_t)stream));
+}
+
+rtr_status rtr_dit_qkv_rope(const void *a, const void *wqkv, const void *bqkv, int m, int d_in, int heads,
+                            int head_dim, int k_per_frame, int grid_w, int t0, void *q, void *k, void *v, int device,
+                            rtr_stream_t stream) {
+    if (m < 0 || d_in < 8 || d_in % 8 != 0 || !shape_ok(heads, head_dim) || k_per_frame < 1 || grid_w < 1 ||
+        t0 < 0 || device < 0)
+        return RTR_E_INVAL;
+    if (m == 0) return RTR_OK;
+    for (const void *ptr : {a, wqkv, bqkv, (const void *)q, (const void *)k, (const void *)v})
+        if (!aligned16(ptr)) return RTR_E_INVAL;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    unsigned *status = device_status_ptr(device);
+    if (!status) return RTR_E_CUDA;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.a = a; g.w = wqkv; g.m = m; g.n = 3 * heads * head_dim; g.k = d_in; g.epi = kEpiQkvRope;
+    g.bias = bqkv; g.q = q; g.k_out = k; g.v = v;
+    g.head_dim = head_dim; g.kpf = k_per_frame; g.grid_w = grid_w; g.t0 = t0;
+    return cuda_status(launch_gemm_bf16(g, status, sm_count(device), (cudaStream_t)stream));
 }
 
 rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_text, rtr_dtype dt, int device,
@@ -894,6 +1006,14 @@ rtr_status rtr_attn_cross(const rtr_xattn *x, int layer, const void *q, int n_q,
 }
 
 unsigned long long rtr_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+rtr_status rtr_release_workspaces(int device, int *held_before) {
+    if (device < 0) return RTR_E_INVAL;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    if (held_before) *held_before = (int)workspace_count(device);
+    return release_workspaces(device);
+}
 
 rtr_status rtr_test_inject_wait_timeout(int device, int launches) {
     if (device < 0 || device >= 64 || launches < 0) return RTR_E_INVAL;

@@ -51,6 +51,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "exp2_poly.h"
@@ -1023,12 +1024,20 @@ int host_pair_tiles(const AttnProblem &p, int idx, int unit_rows) {
 
 }  // namespace
 
+// Device address of g_device_status on `device` (which must be current),
+// looked up once per device under a lock: two host threads making their
+// first call at the same time both get the same address.
 unsigned *device_status_ptr(int device) {
+    static std::mutex mu;
     static unsigned *ptrs[64] = {};
     if (device < 0 || device >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
     if (!ptrs[device]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
         ptrs[device] = static_cast<unsigned *>(p);
     }
     return ptrs[device];

@@ -11,22 +11,33 @@ namespace rtr {
 cudaError_t launch_ln_modulate(const void *x, const void *shift, const void *scale, void *out, int n, int D,
                                float eps, cudaStream_t s);
 
-// q, k, v ([n][heads][d] = [n][D]) from the fp32 projection qkv ([n][3D]) and
-// its bias ([3D]): q and k rotated by the 3D rotary encoding of token i of a
-// chunk (frame t0 + i / kpf, row (i % kpf) / grid_w, column i % grid_w).
-cudaError_t launch_rope_qkv(const float *qkv, const void *bias, void *q, void *k, void *v, int n, int heads, int d,
-                            int kpf, int grid_w, int t0, cudaStream_t s);
 
-// out = in + bias, or GELU(in + bias) (tanh form) when gelu != 0; in fp32
-// [n][N], bias and out bf16; N a multiple of 4.
-cudaError_t launch_bias_act(const float *in, const void *bias, void *out, int n, int N, int gelu, cudaStream_t s);
+// Epilogues of the tensor-core projection (gemm_tc.cu), applied to the fp32
+// product C = A W before anything is stored; every output is rounded once to
+// bf16:
+//   kEpiBias           out[m][n] = C + bias
+//   kEpiBiasGelu       out[m][n] = GELU_tanh(C + bias)
+//   kEpiGatedResidual  out[m][n] += gate * (C + bias) in place (gate null: 1)
+//   kEpiQkvRope        n = 3D: q, k, v [m][D] = thirds of C + bias, q and k
+//                      turned by the 3D rotary encoding of token i (frame t0 +
+//                      i / kpf, row (i % kpf) / grid_w, column i % grid_w) over
+//                      heads of head_dim channels
+enum { kEpiBias = 0, kEpiBiasGelu = 1, kEpiGatedResidual = 2, kEpiQkvRope = 3 };
 
-// x += gate * (in + bias) in place (gate null: 1); in fp32 [n][D], x bf16.
-cudaError_t launch_gated_residual(const float *in, const void *bias, const void *gate, void *x, int n, int D,
-                                  cudaStream_t s);
+struct GemmArgs {
+    const void *a;        // bf16 [m][k], 16-byte aligned
+    const void *w;        // bf16 [k][n] ([in][out]), 16-byte aligned
+    int m, n, k;          // n and k multiples of 8
+    int epi;
+    const void *bias;     // bf16 [n]
+    const void *gate;     // bf16 [n] or null (kEpiGatedResidual)
+    void *out;            // bf16 [m][n] (kEpiBias, kEpiBiasGelu, kEpiGatedResidual)
+    void *q, *k_out, *v;  // bf16 [m][n / 3] each (kEpiQkvRope)
+    int head_dim, kpf, grid_w, t0;   // kEpiQkvRope
+};
 
-// c = a w with a bf16 [m][k], w bf16 [k][n], c fp32 [m][n], fp32 accumulation
-// (cuBLAS GEMM on the given device and stream).
-cudaError_t gemm_bf16_f32(int device, cudaStream_t s, const void *a, const void *w, float *c, int m, int n, int k);
+// C = A W on the tensor cores with the epilogue fused (persistent, up to
+// `sms` CTAs); a bounded wait that expires latches RTR_E_TIMEOUT in *status.
+cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaStream_t s);
 
 }  // namespace rtr

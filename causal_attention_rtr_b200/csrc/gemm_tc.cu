@@ -1,0 +1,430 @@
+// gemm_tc.cu -- the projections of the DiT block on the 5th-generation
+// tensor cores (sm_100a), each with its elementwise epilogue fused into the
+// output stage.
+//
+// C = A W with A bf16 [m][k] (token-major activations) and W bf16 [k][n]
+// (weights stored [in][out]), fp32 accumulation in tensor memory, then one
+// of four epilogues applied to the fp32 tile before anything reaches global
+// memory:
+//   bias            out = bf16(C + b)
+//   bias + GELU     out = bf16(GELU_tanh(C + b))
+//   gated residual  x   = bf16(x + g (C + b))   (x updated in place; g = 1 if null)
+//   QKV + rotary    q, k, v = bf16 of (C + b) split in thirds, q and k turned
+//                   by the 3D rotary encoding of each token
+// Every stored value is rounded once, from the same fp32 quantities a
+// separate epilogue kernel would read back (papernotes.org note "DiT as
+// Real-Time Rerenderer", Method > Overall Architecture: the DiT blocks around
+// the frame-causal attention; the rotary form is RoFormer's, eq. 13-15, split
+// over (frame, row, column) channel parts).
+//
+// Persistent kernel, one CTA per SM, 320 threads:
+//   warp 0      TMA producer: per 64-wide K block, the A tile (128 rows x 64)
+//               and the W tile (64 x BN, BN/64 boxes) into a ring of stages
+//   warp 1      TMEM allocation and the tcgen05.mma issuer (one thread):
+//               D[128 x BN] += A[128 x 16] W[16 x BN], A K-major and W
+//               MN-major from 128-byte-swizzled shared memory
+//   warps 2-9   epilogue: two warps per TMEM lane quarter (one thread per
+//               row), each taking alternate 32-column chunks of the tile
+// Two accumulators of up to 256 columns live in TMEM, so the epilogue of
+// one tile overlaps the MMAs of the next.  Tiles are numbered with N
+// fastest and dealt round-robin; the host picks BN in {128, 192, 256} so
+// that the tile count fills the SMs in as few, evenly loaded rounds as it
+// can.  Every wait is bounded (1 s); a timeout latches RTR_E_TIMEOUT in the
+// device status word and every role stops.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "dit_internal.h"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace rtr {
+namespace {
+
+constexpr int kBM = 128;               // rows per tile
+constexpr int kBK = 64;                // K per stage (one 128-byte swizzle row of bf16)
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr int kATileBytes = kBM * kBK * 2;          // 16 KB
+constexpr int kBBoxBytes = kBK * 64 * 2;            // 8 KB: 64 K rows x 64 N columns
+constexpr int kMaxSmem = 200 * 1024;                // stages share this
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr float kLog2RopeBase = 13.287712379549449f;   // log2(10000)
+
+struct GemmParams {
+    CUtensorMap tm_a;   // A [m][k]: dims (k, m, 1), box (64, 128, 1)
+    CUtensorMap tm_w;   // W [k][n]: dims (n, k, 1), box (64, 64, 1)
+    int m, n, k;
+    int bn, n_tiles_n, n_tiles, k_blocks, stages;
+    const __nv_bfloat16 *bias, *gate;
+    __nv_bfloat16 *out;                 // bias / GELU: [m][n]; gated residual: [m][n] in place
+    __nv_bfloat16 *q, *kk, *v;          // QKV: [m][D] each, D = n / 3
+    int D, head_dim, kpf, grid_w, t0, rope_dt, rope_dp;
+    unsigned *status;
+};
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&b);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
+
+__device__ __forceinline__ float gelu_tanh(float x) {
+    const float kS = 0.7978845608028654f;   // sqrt(2 / pi)
+    return 0.5f * x * (1.0f + tanhf(kS * (x + 0.044715f * x * x * x)));
+}
+
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitNs) return false;
+    }
+}
+
+__device__ __forceinline__ void raise_timeout(const GemmParams &p, volatile int *abort_flag) {
+    *abort_flag = 1;
+    atomicExch(p.status, (unsigned)RTR_E_TIMEOUT);
+}
+
+// The epilogue of 32 consecutive accumulator columns [col, col + 32) of one
+// row (nvalid of them inside the matrix, a multiple of 8).
+template <int EPI>
+__device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&acc)[32], long long row, int col,
+                                          int nvalid, int f_pos, int y_pos, int x_pos) {
+    if (EPI == kEpiQkvRope) {
+        const int part = col / p.D, cc = col - part * p.D;
+        __nv_bfloat16 *dst = (part == 0 ? p.q : part == 1 ? p.kk : p.v) + row * p.D + cc;
+        const int c0 = cc % p.head_dim;                 // channel of the first column within its head
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            if (8 * g >= nvalid) break;
+            float b[8], r[8];
+            unpack8(*reinterpret_cast<const uint4 *>(p.bias + col + 8 * g), b);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[e] = __uint_as_float(acc[8 * g + e]) + b[e];
+            if (part < 2) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const int c = c0 + 8 * g + e;       // even channel of the pair
+                    int j, size, pos;
+                    if (c < p.rope_dt) {
+                        j = c / 2; size = p.rope_dt; pos = f_pos;
+                    } else if (c < p.rope_dt + p.rope_dp) {
+                        j = (c - p.rope_dt) / 2; size = p.rope_dp; pos = y_pos;
+                    } else {
+                        j = (c - p.rope_dt - p.rope_dp) / 2; size = p.rope_dp; pos = x_pos;
+                    }
+                    const float theta = exp2f(-(float)(2 * j) / (float)size * kLog2RopeBase);
+                    float sn, cs;
+                    sincosf((float)pos * theta, &sn, &cs);
+                    const float a0 = r[e], a1 = r[e + 1];
+                    r[e] = a0 * cs - a1 * sn;
+                    r[e + 1] = a0 * sn + a1 * cs;
+                }
+            }
+            *reinterpret_cast<uint4 *>(dst + 8 * g) = pack8(r);
+        }
+    } else if (EPI == kEpiGatedResidual) {
+        __nv_bfloat16 *x = p.out + row * p.n + col;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            if (8 * g >= nvalid) break;
+            float b[8], xv[8], gt[8], r[8];
+            unpack8(*reinterpret_cast<const uint4 *>(p.bias + col + 8 * g), b);
+            unpack8(*reinterpret_cast<const uint4 *>(x + 8 * g), xv);
+            if (p.gate != nullptr) {
+                unpack8(*reinterpret_cast<const uint4 *>(p.gate + col + 8 * g), gt);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gt[e] = 1.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[e] = xv[e] + gt[e] * (__uint_as_float(acc[8 * g + e]) + b[e]);
+            *reinterpret_cast<uint4 *>(x + 8 * g) = pack8(r);
+        }
+    } else {
+        __nv_bfloat16 *o = p.out + row * p.n + col;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            if (8 * g >= nvalid) break;
+            float b[8], r[8];
+            unpack8(*reinterpret_cast<const uint4 *>(p.bias + col + 8 * g), b);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                r[e] = __uint_as_float(acc[8 * g + e]) + b[e];
+                if (EPI == kEpiBiasGelu) r[e] = gelu_tanh(r[e]);
+            }
+            *reinterpret_cast<uint4 *>(o + 8 * g) = pack8(r);
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t s_base = smem_u32(smem);
+    const int S = p.stages;
+    const int stage_bytes = kATileBytes + (p.bn / 64) * kBBoxBytes;
+    const uint32_t bars = s_base + (uint32_t)(S * stage_bytes);
+    // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
+    auto full = [&](int s) { return bars + 8u * (uint32_t)s; };
+    auto empty = [&](int s) { return bars + 8u * (uint32_t)(S + s); };
+    auto accf = [&](int b) { return bars + 8u * (uint32_t)(2 * S + b); };
+    auto acce = [&](int b) { return bars + 8u * (uint32_t)(2 * S + 2 + b); };
+    const uint32_t drain = bars + 8u * (uint32_t)(2 * S + 4);
+    uint8_t *misc = smem + S * stage_bytes + 8 * (2 * S + 5);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf(b), 1);
+            mbar_init(acce(b), kEpiWarps);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&p.tm_a);
+        prefetch_tmap(&p.tm_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            int it = 0;                                  // stage loads issued
+            bool ok = true;
+            const uint32_t tx = (uint32_t)stage_bytes;
+            for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+                const int m0 = (t / p.n_tiles_n) * kBM, n0 = (t % p.n_tiles_n) * p.bn;
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int s = it % S, use = it / S;
+                    if (use > 0 && !wait_bar(empty(s), (use - 1) & 1, abort_flag)) {
+                        raise_timeout(p, abort_flag);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = s_base + (uint32_t)(s * stage_bytes);
+                    mbar_arrive_tx(full(s), tx);
+                    tma_load_3d(sa, &p.tm_a, full(s), kb * kBK, m0, 0);
+                    for (int j = 0; j < p.bn / 64; ++j)
+                        tma_load_3d(sa + kATileBytes + j * kBBoxBytes, &p.tm_w, full(s), n0 + 64 * j, kb * kBK, 0);
+                }
+            }
+            // Loads still in flight land before the CTA can exit: wait for
+            // the last load of every stage (bounded).
+            for (int s = 0; s < S && s < it; ++s) {
+                const int last = ((it - 1 - s) / S) * S + s;   // last load index that used stage s
+                mbar_wait(full(s), (last / S) & 1, kWaitNs);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(kBM, p.bn, 0, 1);
+            int it = 0, tc = 0;                          // stages consumed, tiles done
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++tc) {
+                const int b = tc & 1, use_b = tc >> 1;
+                if (use_b > 0 && !wait_bar(acce(b), (use_b - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(b * 256);
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int s = it % S;
+                    if (!wait_bar(full(s), (it / S) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = s_base + (uint32_t)(s * stage_bytes);
+                    const uint64_t da = smem_desc_sw128(sa, 16, 1024);
+                    const uint64_t dw = smem_desc_sw128(sa + kATileBytes, kBBoxBytes, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_ss(d_tmem, da + (uint64_t)((kk * 32) >> 4), dw + (uint64_t)((kk * 2048) >> 4), idesc,
+                               (kb > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(empty(s));
+                }
+                if (!ok) break;
+                tc_commit(accf(b));
+            }
+            if (!ok) raise_timeout(p, abort_flag);
+            // every MMA issued above completes before TMEM is freed
+            tc_commit(drain);
+            mbar_wait(drain, 0, kWaitNs);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int quarter = warp & 3, half = (warp - 2) >> 2;
+        const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
+        int tc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++tc) {
+            const int b = tc & 1, use_b = tc >> 1;
+            const int m0 = (t / p.n_tiles_n) * kBM, n0 = (t % p.n_tiles_n) * p.bn;
+            bool w = wait_bar(accf(b), use_b & 1, abort_flag);
+            w = __all_sync(0xffffffffu, w);
+            if (!w) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const long long row = (long long)m0 + quarter * 32 + lane;
+            const bool row_ok = row < p.m;
+            int f_pos = 0, y_pos = 0, x_pos = 0;
+            if (EPI == kEpiQkvRope) {
+                const int f = (int)(row / p.kpf), r = (int)(row - (long long)f * p.kpf);
+                f_pos = p.t0 + f;
+                y_pos = r / p.grid_w;
+                x_pos = r - y_pos * p.grid_w;
+            }
+            for (int c = half; c < p.bn / 32; c += 2) {
+                const int col = n0 + 32 * c;
+                if (col >= p.n) break;                   // warp-uniform
+                uint32_t acc[32];
+                tmem_ld32(tmem + lane_bits + (uint32_t)(b * 256 + 32 * c), acc);
+                tmem_wait_ld();
+                if (row_ok) epi_chunk<EPI>(p, acc, row, col, min(32, p.n - col), f_pos, y_pos, x_pos);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce(b));
+        }
+        if (!ok) raise_timeout(p, abort_flag);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int EPI>
+cudaError_t set_smem_attr_once() {
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        err = cudaFuncSetAttribute(gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem + 2048);
+    });
+    return err;
+}
+
+// Tile width: the candidate whose rounds of `grid` tiles take the least
+// time, counting a tile's time as proportional to BN plus a fixed 32-column
+// cost of its prologue and epilogue hand-off; ties go to the wider tile.
+int pick_bn(int m, int n, int sms) {
+    const int m_tiles = (m + kBM - 1) / kBM;
+    int best = 256;
+    long long best_cost = -1;
+    for (int bn : {256, 192, 128}) {
+        const long long tiles = (long long)m_tiles * ((n + bn - 1) / bn);
+        const long long rounds = (tiles + sms - 1) / sms;
+        const long long cost = rounds * (bn + 32);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+template <int EPI>
+cudaError_t launch_epi(const GemmParams &p, int grid, int smem, cudaStream_t s) {
+    const cudaError_t e = set_smem_attr_once<EPI>();
+    if (e != cudaSuccess) return e;
+    gemm_tc<EPI><<<grid, kThreads, smem, s>>>(p);
+    const cudaError_t le = cudaGetLastError();
+    if (le == cudaSuccess) count_launch();
+    return le;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaStream_t s) {
+    if (g.m <= 0) return cudaSuccess;
+    if (g.n < 8 || g.k < 8 || g.n % 8 != 0 || g.k % 8 != 0 || g.epi < 0 || g.epi > kEpiQkvRope)
+        return cudaErrorInvalidValue;
+    if (g.epi == kEpiQkvRope && (g.n % 3 != 0 || (g.n / 3) % g.head_dim != 0 || g.head_dim % 32 != 0 ||
+                                 g.kpf < 1 || g.grid_w < 1))
+        return cudaErrorInvalidValue;
+    if (!status || sms < 1) return cudaErrorInvalidValue;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    if (!make_tmap_bf16(&p.tm_a, g.a, (uint64_t)g.k, (uint64_t)g.m, 1, kBM, 1) ||
+        !make_tmap_bf16(&p.tm_w, g.w, (uint64_t)g.n, (uint64_t)g.k, 1, kBK, 1))
+        return cudaErrorInvalidValue;
+    p.m = g.m; p.n = g.n; p.k = g.k;
+    p.bn = pick_bn(g.m, g.n, sms);
+    p.n_tiles_n = (g.n + p.bn - 1) / p.bn;
+    p.n_tiles = ((g.m + kBM - 1) / kBM) * p.n_tiles_n;
+    p.k_blocks = (g.k + kBK - 1) / kBK;
+    const int stage_bytes = kATileBytes + (p.bn / 64) * kBBoxBytes;
+    p.stages = kMaxSmem / stage_bytes;
+    if (p.stages > 8) p.stages = 8;
+    p.bias = static_cast<const __nv_bfloat16 *>(g.bias);
+    p.gate = static_cast<const __nv_bfloat16 *>(g.gate);
+    p.out = static_cast<__nv_bfloat16 *>(g.out);
+    p.q = static_cast<__nv_bfloat16 *>(g.q);
+    p.kk = static_cast<__nv_bfloat16 *>(g.k_out);
+    p.v = static_cast<__nv_bfloat16 *>(g.v);
+    p.D = g.epi == kEpiQkvRope ? g.n / 3 : g.n;
+    p.head_dim = g.head_dim;
+    p.kpf = g.kpf;
+    p.grid_w = g.grid_w;
+    p.t0 = g.t0;
+    p.rope_dp = g.head_dim > 0 ? 2 * (g.head_dim / 6) : 0;
+    p.rope_dt = g.head_dim - 2 * p.rope_dp;
+    p.status = status;
+    const int grid = p.n_tiles < sms ? p.n_tiles : sms;
+    // stages, barriers (2S + 5), the TMEM holder and the abort flag, plus
+    // slack for the 1 KB alignment of the stage ring
+    const int smem = p.stages * stage_bytes + 8 * (2 * p.stages + 5) + 16 + 1024;
+    switch (g.epi) {
+        case kEpiBias: return launch_epi<kEpiBias>(p, grid, smem, s);
+        case kEpiBiasGelu: return launch_epi<kEpiBiasGelu>(p, grid, smem, s);
+        case kEpiGatedResidual: return launch_epi<kEpiGatedResidual>(p, grid, smem, s);
+        default: return launch_epi<kEpiQkvRope>(p, grid, smem, s);
+    }
+}
+
+}  // namespace rtr

@@ -89,9 +89,10 @@ struct BwdProblem {
 size_t bwd_scratch_bytes(int n, int heads);
 cudaError_t launch_attn_bwd(const BwdProblem &p, unsigned *status, void *scratch, cudaStream_t s);
 
-// CTAs per cluster for the tensor-core attention: 1, or 2 (CTA-pair MMA) when
-// the environment variable RTR_CTA_GROUP says 2.
-int attn_cta_group();
+// Argument checks and defaults shared by every entry point.
+bool shape_ok(int heads, int head_dim);                 // heads >= 1, head_dim 64 or 128
+float resolve_scale(float scale, int head_dim);         // scale > 0 ? scale : 1 / sqrt(head_dim)
+int sm_count(int device);                               // SMs of `device` (cached; 148 if unknown)
 
 // Kernel launchers; return cudaSuccess or the launch error.
 cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const CUtensorMap *tm_k0,

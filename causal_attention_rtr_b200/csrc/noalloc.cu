@@ -58,8 +58,10 @@ extern "C" rtr_status rtr_attn_block_causal_prefill_noalloc(const void *q, const
                                                             int n_tokens, int heads, int head_dim,
                                                             int k_per_frame, rtr_dtype dt, void *out, float scale,
                                                             int device, rtr_stream_t stream) {
-    if (n_tokens < 0 || heads < 1 || (head_dim != 64 && head_dim != 128) || k_per_frame < 1 ||
-        (dt != RTR_BF16 && dt != RTR_F32) || device < 0)
+    // The same checks, scale, SM count and schedule as rtr_attn_block_causal_prefill, so
+    // that both entry points run identical launches.
+    if (n_tokens < 0 || !shape_ok(heads, head_dim) || k_per_frame < 1 || (dt != RTR_BF16 && dt != RTR_F32) ||
+        device < 0)
         return RTR_E_INVAL;
     if (n_tokens == 0) return RTR_OK;
     auto aligned16 = [](const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
@@ -84,7 +86,7 @@ extern "C" rtr_status rtr_attn_block_causal_prefill_noalloc(const void *q, const
     pb.kpf = k_per_frame;
     pb.nseg = 1;
     pb.seg[0] = KvSeg{1, 0, n_tokens, 1};
-    pb.scale = scale > 0.f ? scale : 1.f / sqrtf((float)head_dim);
+    pb.scale = resolve_scale(scale, head_dim);
     pb.q = q;
     pb.o = out;
     pb.k1 = k;
@@ -93,11 +95,8 @@ extern "C" rtr_status rtr_attn_block_causal_prefill_noalloc(const void *q, const
 
     cudaError_t e;
     if (dt == RTR_BF16) {
-        int sms = 0;
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0)
-            return RTR_E_CUDA;
         AttnPlan plan;
-        plan_attn_bf16(pb, sms, attn_cta_group(), plan);
+        plan_attn_bf16(pb, sm_count(device), 1, plan);
         // The scratch this launch needs must fit in the static array.
         if (plan.scratch_bytes > (size_t)RTR_NOALLOC_SCRATCH_BYTES) return RTR_E_INVAL;
         void *scratch = noalloc_scratch_ptr(device);

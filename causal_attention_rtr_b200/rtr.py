@@ -25,6 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 RTR_OK, RTR_E_INVAL, RTR_E_NOMEM, RTR_E_STATE, RTR_E_CUDA, RTR_E_TIMEOUT, RTR_E_UNSUPPORTED = range(7)
 RTR_BF16, RTR_F32 = 0, 1
+RTR_EPI_BIAS, RTR_EPI_BIAS_GELU, RTR_EPI_GATED_RESIDUAL = 0, 1, 2
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -58,12 +59,16 @@ _SIGNATURES = [
     ("rtr_crossattn_check_guards", _i, [_vp]),
     ("rtr_test_fail_allocs", _i, [_i, _i]),
     ("rtr_attn_frame_causal", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
+    ("rtr_attn_frame_causal_ex", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _i, _vp]),
     ("rtr_attn_frame_causal_commit", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
     ("rtr_attn_block_causal_prefill", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
+    ("rtr_attn_block_causal_prefill_ex", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _i, _vp]),
     ("rtr_attn_block_causal_prefill_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     ("rtr_attn_block_causal_prefill_lse", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _i, _vp]),
     ("rtr_dit_block_forward", _i, [_vp, _vp, _i, ctypes.POINTER(DitWeights), _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     ("rtr_attn_block_causal_prefill_cache", _i, [_vp, _i, _vp, _vp, _vp, _i, _i, _vp, _f, _vp]),
+    ("rtr_dit_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
+    ("rtr_dit_qkv_rope", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
     ("rtr_attn_block_causal_backward", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f,
                                             _i, _vp]),
     ("rtr_crossattn_create", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
@@ -74,6 +79,7 @@ _SIGNATURES = [
     ("rtr_get_device_status", _i, [_i, _vp]),
     ("rtr_test_inject_wait_timeout", _i, [_i, _i]),
     ("rtr_kernel_launches", ctypes.c_ulonglong, []),
+    ("rtr_release_workspaces", _i, [_i, ctypes.POINTER(_i)]),
 ]
 
 for _name, _res, _args in _SIGNATURES:
@@ -211,6 +217,12 @@ def rtr_attn_frame_causal(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale=0.
                                              _ptr(out), float(scale), _stream(stream)), "rtr_attn_frame_causal")
 
 
+def rtr_attn_frame_causal_ex(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale=0.0, cta_group=1, stream=None):
+    return _check(_lib.rtr_attn_frame_causal_ex(c, layer, _ptr(q), _ptr(k_cur), _ptr(v_cur), n_cur_frames,
+                                                _ptr(out), float(scale), cta_group, _stream(stream)),
+                  "rtr_attn_frame_causal_ex")
+
+
 def rtr_attn_frame_causal_commit(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale=0.0, stream=None):
     return _check(_lib.rtr_attn_frame_causal_commit(c, layer, _ptr(q), _ptr(k_cur), _ptr(v_cur), n_cur_frames,
                                                     _ptr(out), float(scale), _stream(stream)),
@@ -248,6 +260,22 @@ def rtr_dit_block_forward(c, x, layer, weights, modulation, hidden, n_cur_frames
                   "rtr_dit_block_forward")
 
 
+def rtr_dit_linear(a, w, m, n, k, epilogue, bias, gate, out, device=0, stream=None):
+    """out = epilogue(a w + bias) on the tensor cores (see include/rtr.h)."""
+    epi = {"bias": RTR_EPI_BIAS, "gelu": RTR_EPI_BIAS_GELU, "gated_residual": RTR_EPI_GATED_RESIDUAL}.get(epilogue,
+                                                                                                       epilogue)
+    return _check(_lib.rtr_dit_linear(_ptr(a), _ptr(w), m, n, k, int(epi), _ptr(bias), _ptr(gate), _ptr(out),
+                                      device, _stream(stream)), "rtr_dit_linear")
+
+
+def rtr_dit_qkv_rope(a, wqkv, bqkv, m, d_in, heads, head_dim, k_per_frame, grid_w, t0, q, k, v, device=0,
+                     stream=None):
+    """q, k, v = thirds of a wqkv + bqkv, q and k rotary-encoded (see include/rtr.h)."""
+    return _check(_lib.rtr_dit_qkv_rope(_ptr(a), _ptr(wqkv), _ptr(bqkv), m, d_in, heads, head_dim, k_per_frame,
+                                        grid_w, t0, _ptr(q), _ptr(k), _ptr(v), device, _stream(stream)),
+                  "rtr_dit_qkv_rope")
+
+
 def rtr_attn_block_causal_backward(q, k, v, out, dout, lse, n_tokens, heads, head_dim, k_per_frame, dt, dq, dk, dv,
                                    scale=0.0, device=0, stream=None):
     return _check(_lib.rtr_attn_block_causal_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
@@ -262,6 +290,14 @@ def rtr_attn_block_causal_prefill(q, k, v, n_tokens, heads, head_dim, k_per_fram
                                                      k_per_frame, _dtype(dt), _ptr(out), float(scale),
                                                      device, _stream(stream)),
                   "rtr_attn_block_causal_prefill")
+
+
+def rtr_attn_block_causal_prefill_ex(q, k, v, n_tokens, heads, head_dim, k_per_frame, dt, out, scale=0.0,
+                                     cta_group=1, device=0, stream=None):
+    return _check(_lib.rtr_attn_block_causal_prefill_ex(_ptr(q), _ptr(k), _ptr(v), n_tokens, heads, head_dim,
+                                                        k_per_frame, _dtype(dt), _ptr(out), float(scale),
+                                                        cta_group, device, _stream(stream)),
+                  "rtr_attn_block_causal_prefill_ex")
 
 
 def rtr_attn_block_causal_prefill_noalloc(q, k, v, n_tokens, heads, head_dim, k_per_frame, dt, out, scale=0.0,
@@ -321,3 +357,11 @@ def rtr_test_inject_wait_timeout(device, launches):
 def rtr_kernel_launches():
     """Kernels this library has launched since it was loaded."""
     return int(_lib.rtr_kernel_launches())
+
+
+def rtr_release_workspaces(device=0):
+    """Free the library's per-stream scratch buffers of `device`; returns
+    how many it held."""
+    n = _i(0)
+    _check(_lib.rtr_release_workspaces(device, ctypes.byref(n)), "rtr_release_workspaces")
+    return n.value

@@ -196,6 +196,15 @@ rtr_status rtr_attn_frame_causal(const rtr_kvcache *c, int layer,
                                  const void *v_cur, int n_cur_frames,
                                  void *out, float scale, rtr_stream_t stream);
 
+/* rtr_attn_frame_causal with the MMA form chosen explicitly, as in
+ * rtr_attn_block_causal_prefill_ex: cta_group 1 (the default kernel) or 2
+ * (the CTA-pair kernel); other values RTR_E_INVAL. */
+rtr_status rtr_attn_frame_causal_ex(const rtr_kvcache *c, int layer,
+                                    const void *q, const void *k_cur,
+                                    const void *v_cur, int n_cur_frames,
+                                    void *out, float scale, int cta_group,
+                                    rtr_stream_t stream);
+
 /* rtr_attn_frame_causal followed by the commit of the chunk, as in
  * rtr_kvcache_append_frame(c, layer, k_cur, v_cur, n_cur_frames), with the
  * chunk written by the attention launch itself (Key Designs 4: the chunk's
@@ -236,6 +245,21 @@ rtr_status rtr_attn_block_causal_prefill(const void *q, const void *k,
                                          int k_per_frame, rtr_dtype dt,
                                          void *out, float scale,
                                          int device, rtr_stream_t stream);
+
+/* rtr_attn_block_causal_prefill with the tensor-core kernel's MMA form
+ * chosen explicitly: cta_group = 1 is the default kernel (one CTA per
+ * 128-row MMA); cta_group = 2 runs the CTA-pair kernel (tcgen05
+ * cta_group::2: one MMA covers 256 query rows on two SMs, each SM holding
+ * half of every key / value tile).  Both return the same attention within
+ * rounding; the CTA pair was measured slower and is kept for comparison.
+ * Other values: RTR_E_INVAL.  fp32 ignores cta_group. */
+rtr_status rtr_attn_block_causal_prefill_ex(const void *q, const void *k,
+                                            const void *v, int n_tokens,
+                                            int heads, int head_dim,
+                                            int k_per_frame, rtr_dtype dt,
+                                            void *out, float scale,
+                                            int cta_group, int device,
+                                            rtr_stream_t stream);
 
 /* rtr_attn_block_causal_prefill that also returns each row's log-sum-exp,
  * the statistic the backward pass needs: lse[h * n_tokens + i] = log
@@ -314,23 +338,61 @@ typedef struct rtr_dit_weights {
  * P = 2 floor(d / 6); pair (2j, 2j+1) of a part of size S turns by
  * pos * 10000^(-2j/S).  modulation: bf16 [6][D] = shift1, scale1, gate1,
  * shift2, scale2, gate2 (from the timestep, computed by the caller).  Every
- * tensor a later step consumes is stored in bf16; accumulation is fp32
- * (GEMMs through cuBLAS, the rest in this library's kernels).
+ * tensor a later step consumes is stored in bf16; accumulation is fp32.
+ * The six projections are this library's tensor-core GEMM with the bias,
+ * rotary, GELU and gated-residual steps fused into its output stage (as
+ * rtr_dit_qkv_rope and rtr_dit_linear).
  *
  * commit = 1 appends the chunk's rotated keys and values to the cache after
  * its attention, as rtr_kvcache_append_frame would (n_cur_frames <= W), in
  * the attention launch itself when the cache has that much commit room.
  * Requires bf16 caches of equal heads and head_dim on one device, text set
  * in x for this layer (else RTR_E_STATE), d_ffn a multiple of 8.  The
- * library keeps a per-stream activation buffer of about
- * n * (10 D + 2 F + 4 max(3D, F)) bytes.  Argument errors leave everything
- * unchanged; a CUDA error in a step after the commit returns RTR_E_CUDA with
- * the commit already applied to the index map. */
+ * library keeps a per-stream activation buffer of about n * (10 D + 2 F)
+ * bytes.  Argument errors leave everything unchanged; a CUDA error in a
+ * step after the commit returns RTR_E_CUDA with the commit already applied
+ * to the index map. */
 rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer,
                                  const rtr_dit_weights *w,
                                  const void *modulation, void *hidden,
                                  int n_cur_frames, int grid_h, int grid_w,
                                  int t0, int commit, rtr_stream_t stream);
+
+/* The projections of the DiT block, for callers that assemble their own
+ * blocks: out = epilogue(a w + bias) on the tensor cores, with the epilogue
+ * applied to the fp32 product before anything is stored and each output
+ * rounded once to bf16 (papernotes.org note "DiT as Real-Time Rerenderer",
+ * Method > Overall Architecture).  a: bf16 [m][k] activations; w: bf16
+ * [k][n] weights ([in][out], y = x w + b); bias: bf16 [n]; n and k
+ * multiples of 8.
+ *   RTR_EPI_BIAS            out[m][n] = a w + bias
+ *   RTR_EPI_BIAS_GELU       out[m][n] = GELU_tanh(a w + bias)
+ *   RTR_EPI_GATED_RESIDUAL  out[m][n] += gate * (a w + bias), in place;
+ *                           gate bf16 [n], or null for 1
+ * gate must be null for the other two.  Caller-owned device memory,
+ * 16-byte aligned; out must not overlap a or w.  m == 0 is a no-op. */
+typedef enum {
+    RTR_EPI_BIAS = 0,
+    RTR_EPI_BIAS_GELU = 1,
+    RTR_EPI_GATED_RESIDUAL = 2
+} rtr_epilogue;
+rtr_status rtr_dit_linear(const void *a, const void *w, int m, int n, int k,
+                          rtr_epilogue epilogue, const void *bias,
+                          const void *gate, void *out, int device,
+                          rtr_stream_t stream);
+
+/* The block's QKV projection with the 3D rotary encoding fused: for the m
+ * tokens of a chunk (a: bf16 [m][d_in]), the product with wqkv ([d_in][3D],
+ * D = heads * head_dim; q, k and v side by side) plus bqkv ([3D]) is split
+ * into q, k, v ([m][heads][head_dim] bf16 each), and q and k are turned by
+ * the rotary encoding of token i at (frame t0 + i / k_per_frame, row
+ * (i % k_per_frame) / grid_w, column i % grid_w), as rtr_dit_block_forward
+ * describes.  head_dim 64 or 128; d_in a multiple of 8; 16-byte aligned
+ * caller-owned device memory. */
+rtr_status rtr_dit_qkv_rope(const void *a, const void *wqkv, const void *bqkv,
+                            int m, int d_in, int heads, int head_dim,
+                            int k_per_frame, int grid_w, int t0, void *q,
+                            void *k, void *v, int device, rtr_stream_t stream);
 
 /* Backward pass of the block-causal attention (Key Designs 2 and 3: the
  * causal student is trained with Self Forcing and DMD, whose gradients flow
@@ -407,6 +469,19 @@ rtr_status rtr_attn_cross(const rtr_xattn *x, int layer, const void *q,
  * status of `device` (RTR_OK or RTR_E_TIMEOUT) and clears it.
  */
 rtr_status rtr_get_device_status(int device, rtr_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Scratch memory.  Calls that need scratch (split attention units, the
+ * backward's row statistics, the DiT block's activations) keep one
+ * library-owned device buffer per (stream, use), grown on demand and reused
+ * by later calls on that stream.  A device keeps the buffers of its 8 most
+ * recently used streams; the least recently used is freed (after a device
+ * synchronisation) when a ninth stream needs one, so short-lived streams do
+ * not accumulate buffers.  rtr_release_workspaces synchronises `device` and
+ * frees all of its buffers now; *held_before (if not null) receives how many
+ * there were.  Later calls allocate again as needed.
+ */
+rtr_status rtr_release_workspaces(int device, int *held_before);
 
 /* Test hook for the failure path: the next `launches` bf16 attention
  * launches on `device` (any of the attention calls) deliberately issue no

@@ -33,7 +33,7 @@ def _load():
         lib.rtr_oracle_visible.restype = ctypes.c_int
         lib.rtr_oracle_visible.argtypes = [ctypes.c_int64] * 3
         p = ctypes.c_void_p
-        lib.rtr_oracle_attention.restype = None
+        lib.rtr_oracle_attention.restype = ctypes.c_int
         lib.rtr_oracle_attention.argtypes = [
             p, p, ctypes.c_int64, p, p, ctypes.c_int64, ctypes.c_int64,
             ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_double, p,
@@ -93,9 +93,11 @@ def attention(q, q_pos, k, v, k_per_frame, causal=True, scale=None,
     if nq == 0:
         return out
     ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
-    _load().rtr_oracle_attention(ptr(q), ptr(q_pos), nq, ptr(k), ptr(v), nk,
-                                 H, d, int(k_per_frame), 1 if causal else 0,
-                                 float(scale), ptr(out), int(nthreads))
+    failed = _load().rtr_oracle_attention(ptr(q), ptr(q_pos), nq, ptr(k), ptr(v), nk,
+                                          H, d, int(k_per_frame), 1 if causal else 0,
+                                          float(scale), ptr(out), int(nthreads))
+    if failed:
+        raise MemoryError("oracle attention: row buffers could not be allocated")
     return out
 
 

@@ -52,12 +52,15 @@ int rtr_oracle_visible(int64_t i, int64_t j, int64_t k)
  *   scale                   multiplies q.k (1/sqrt(d) in the equation)
  *   out    [nq][heads][d]
  *
+ * Returns 0, or 1 if a row's work buffers could not be allocated (that row's
+ * output is then left as NaN and the caller must treat the result as
+ * failed).
  * Per (row, head):  s_j = scale * sum_t q_t key_jt over visible j,
  * m = max_j s_j, p_j = exp(s_j - m), out = sum_j p_j val_j / sum_j p_j.
  * Subtracting m is the usual exact rewrite of softmax (it cancels in the
  * ratio) and keeps exp() finite.  A row that sees no key returns zeros.
  */
-void rtr_oracle_attention(const double *q, const int64_t *q_pos, int64_t nq,
+int rtr_oracle_attention(const double *q, const int64_t *q_pos, int64_t nq,
                           const double *key, const double *val, int64_t nk,
                           int64_t heads, int64_t d, int64_t k_per_frame,
                           int causal, double scale, double *out, int nthreads)
@@ -69,6 +72,7 @@ void rtr_oracle_attention(const double *q, const int64_t *q_pos, int64_t nq,
     (void)nthreads;
 #endif
     int64_t npairs = nq * heads;
+    int failed = 0;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
     for (int64_t pr = 0; pr < npairs; ++pr) {
         int64_t r = pr / heads, h = pr % heads;
@@ -76,6 +80,14 @@ void rtr_oracle_attention(const double *q, const int64_t *q_pos, int64_t nq,
         double *oi = out + (r * heads + h) * d;
         double *s = (double *)malloc((size_t)(nk > 0 ? nk : 1) * sizeof(double));
         unsigned char *vis = (unsigned char *)malloc((size_t)(nk > 0 ? nk : 1));
+        if (!s || !vis) {
+            free(s);
+            free(vis);
+            for (int64_t t = 0; t < d; ++t) oi[t] = NAN;
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
         double m = -INFINITY;
         for (int64_t j = 0; j < nk; ++j) {
             vis[j] = causal ? (unsigned char)rtr_oracle_visible(q_pos[r], j, k_per_frame) : 1;
@@ -100,6 +112,7 @@ void rtr_oracle_attention(const double *q, const int64_t *q_pos, int64_t nq,
         free(s);
         free(vis);
     }
+    return failed;
 }
 
 /* Number of threads OpenMP would use (reported next to CPU timings). */

@@ -4,14 +4,14 @@ bits (papernotes.org note "DiT as Real-Time Rerenderer", Method > Key
 Designs 2: the attention and its mask; Key Designs 3: training runs
 gradient descent through it).
 
-Tolerance of the gradients, per tensor: relative L2 error <= 1e-2 and max
-|gpu - oracle| <= 2e-2 * max |oracle|.  Derivation: P and dS enter the
-tensor cores as bf16 (relative rounding 2^-9 each), the forward's output O
-is bf16 (it enters Delta = rowsum(dO * O)), and the results are rounded once
-to bf16 (2^-9); with fp32 accumulation these independent roundings give a
-relative L2 error of a few 1e-3 and single elements within a few 2^-8 of the
-tensor's scale.  The row log-sum-exp (fp32, natural log) must be within 2e-3
-absolute."""
+Tolerance of the gradients, per tensor: the attention's own bounds, max
+|gpu - oracle| <= 2e-2 and relative L2 error <= 5e-3 (gpu_util.assert_close).
+P and dS enter the tensor cores as bf16 (relative rounding 2^-9 each), the
+forward's output O is bf16 (it enters Delta = rowsum(dO * O)), and the
+results are rounded once to bf16 (2^-9); with fp32 accumulation these
+independent roundings give a relative L2 error near 2.4e-3 and elements
+within about 1e-3 of the oracle at the gradients' scale here (|dV| <= 0.4).
+The row log-sum-exp (fp32, natural log) must be within 2e-3 absolute."""
 import numpy as np
 import pytest
 import torch
@@ -23,8 +23,6 @@ from gpu_util import assert_close, dev, host_f64
 
 pytestmark = pytest.mark.gpu
 
-GRAD_REL_L2 = 1e-2
-GRAD_MAX_REL = 2e-2
 LSE_ABS = 2e-3
 
 
@@ -34,12 +32,8 @@ def _rtr():
 
 
 def assert_grad_close(got, want, what):
-    assert np.all(np.isfinite(got)), f"{what}: non-finite"
-    diff = got - want
-    scale = float(np.max(np.abs(want)))
-    rel = float(np.linalg.norm(diff.ravel()) / max(np.linalg.norm(want.ravel()), 1e-30))
-    mx = float(np.max(np.abs(diff)))
-    assert rel <= GRAD_REL_L2 and mx <= GRAD_MAX_REL * scale, f"{what}: rel_l2={rel:.3e} max={mx:.3e} scale={scale:.3e}"
+    """A gradient against the oracle at the attention's bounds."""
+    return assert_close(got, want, what)
 
 
 def run_gpu(q, k, v, do, n, H, d, kpf):

@@ -105,3 +105,48 @@ def test_validation_before_device_work(lib):
                           None) == rtr.RTR_OK
     assert rtr.raw_status("rtr_attn_block_causal_prefill", 16, 16, 16, 10, 2, 128, 0, 0, 16, 0.0, 0,
                           None) == rtr.RTR_E_INVAL
+
+
+def test_explicit_cta_group_and_workspace_validation(lib):
+    """The MMA form is an explicit argument (1 or 2); anything else is
+    rejected before any device work, as is a negative device for the
+    scratch release."""
+    from causal_attention_rtr_b200 import rtr
+    for cg in (0, 3, -1):
+        assert rtr.raw_status("rtr_attn_block_causal_prefill_ex", 16, 16, 16, 10, 2, 128, 4, 0, 16, 0.0, cg, 0,
+                              None) == rtr.RTR_E_INVAL, cg
+        assert rtr.raw_status("rtr_attn_frame_causal_ex", None, 0, None, None, None, 1, None, 0.0, cg,
+                              None) == rtr.RTR_E_INVAL, cg
+    assert rtr.raw_status("rtr_attn_block_causal_prefill_ex", None, None, None, 0, 2, 128, 4, 0, None, 0.0, 2, 0,
+                          None) == rtr.RTR_OK
+    assert rtr.raw_status("rtr_release_workspaces", -1, None) == rtr.RTR_E_INVAL
+
+
+def test_dit_projection_validation(lib):
+    """The fused projections check shapes, epilogue and alignment on the
+    host (no GPU needed)."""
+    from causal_attention_rtr_b200 import rtr
+    p = 256
+    bad_linear = [
+        (p, p, 10, 12, 64, 0, p, None, p, 0, None),     # n not a multiple of 8
+        (p, p, 10, 64, 4, 0, p, None, p, 0, None),      # k < 8
+        (p, p, -1, 64, 64, 0, p, None, p, 0, None),     # m < 0
+        (p, p, 10, 64, 64, 7, p, None, p, 0, None),     # no such epilogue
+        (p, p, 10, 64, 64, 0, p, p, p, 0, None),        # gate with the plain bias epilogue
+        (p + 2, p, 10, 64, 64, 0, p, None, p, 0, None), # a not 16-byte aligned
+        (p, p, 10, 64, 64, 0, p, None, p, -1, None),    # device
+    ]
+    for args in bad_linear:
+        assert rtr.raw_status("rtr_dit_linear", *args) == rtr.RTR_E_INVAL, args
+    assert rtr.raw_status("rtr_dit_linear", p, p, 0, 64, 64, 2, p, p, p, 0, None) == rtr.RTR_OK
+    bad_qkv = [
+        (p, p, p, 10, 64, 2, 96, 16, 4, 0, p, p, p, 0, None),    # head_dim
+        (p, p, p, 10, 60, 2, 64, 16, 4, 0, p, p, p, 0, None),    # d_in not a multiple of 8
+        (p, p, p, 10, 64, 2, 64, 0, 4, 0, p, p, p, 0, None),     # k_per_frame
+        (p, p, p, 10, 64, 2, 64, 16, 0, 0, p, p, p, 0, None),    # grid_w
+        (p, p, p, 10, 64, 2, 64, 16, 4, -1, p, p, p, 0, None),   # t0
+        (p, p, p, 10, 64, 2, 64, 16, 4, 0, p + 8, p, p, 0, None),  # q not 16-byte aligned
+    ]
+    for args in bad_qkv:
+        assert rtr.raw_status("rtr_dit_qkv_rope", *args) == rtr.RTR_E_INVAL, args
+    assert rtr.raw_status("rtr_dit_qkv_rope", p, p, p, 0, 64, 2, 64, 16, 4, 0, p, p, p, 0, None) == rtr.RTR_OK
