@@ -65,6 +65,21 @@
 #ifndef RTR_UNIT_ORDER_RATIO
 #define RTR_UNIT_ORDER_RATIO 1.25   // head-major unit order when max/min key tiles per pair <= this
 #endif
+#ifndef RTR_PV_SPLIT
+#define RTR_PV_SPLIT 0   // 1: PV over the first 64 keys starts once their P is stored (bPh)
+#endif
+#ifndef RTR_S_SPLIT
+#define RTR_S_SPLIT 0   // 1: S(j+1) of the second 64 keys runs once the softmax has read S(j) (needs 1LD + PV split)
+#endif
+#if RTR_S_SPLIT && !(RTR_SOFTMAX_1LD && RTR_PV_SPLIT)
+#error "RTR_S_SPLIT needs RTR_SOFTMAX_1LD and RTR_PV_SPLIT"
+#endif
+#ifndef RTR_COMMIT_GLOBAL
+#define RTR_COMMIT_GLOBAL 0   // 1: the chunk write copies from the chunk's global K/V, spread over the launch
+#endif
+#ifndef RTR_SOFTMAX_1LD
+#define RTR_SOFTMAX_1LD 0   // 1: the row's 128 scores read from TMEM once, held in registers
+#endif
 #ifndef RTR_EXP2_POLY_PER8
 #define RTR_EXP2_POLY_PER8 0   // of every 8 scores, how many use exp2_poly (0 measured fastest so far)
 #endif
@@ -111,6 +126,8 @@ struct TcParams {
     long long commit_rows_per_head;
     int commit_first_slot, commit_slots, commit_row0;
     const CUtensorMap *commit_maps;   // per-slot store maps (see AttnProblem) or null
+    int commit_global;                // 1: warps 2-3 copy the chunk from its global K/V (src_k1, src_v1)
+    const __nv_bfloat16 *src_k1, *src_v1;   // the token-major run's K / V in global memory
     float *lse;         // [heads][nq] natural-log row log-sum-exp, or null
 };
 
@@ -127,7 +144,7 @@ struct Layout {
     static constexpr int kBars = kKV + kSlots * kSlotBytes; // mbarriers
     static constexpr int bQ = 0, bQfree = 1, bFull = 2, bEmpty = bFull + kSlots, bCopied = bEmpty + kSlots,
                          bGo = bCopied + kSlots, bS = bGo + kSlots, bP = bS + 2, bO = bP + 2, bEpi = bO + 2, bDrain = bEpi + 2,
-                         kNumBars = bDrain + 1;
+                         bPh = bDrain + 1, bSr = bPh + 2, kNumBars = bSr + 2;
     static constexpr int kMisc = kBars + kNumBars * 8;      // tmem holder, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1 KB alignment
@@ -270,6 +287,23 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&sr)[32], float sl
     tmem_st16(tP, pk);
 }
 
+// softmax_chunk on 32 scores held at sr[0..31] of a register-resident row.
+template <bool POLY>
+__device__ __forceinline__ void softmax_chunk_regs(const uint32_t *sr, float sl2, float neg_m, uint32_t tP,
+                                                   float2 (&acc)[4]) {
+    const float2 sl2x2 = make_float2(sl2, sl2), negm2 = make_float2(neg_m, neg_m);
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float2 x = ffma2(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2x2, negm2);
+        const bool poly = POLY && (e % 4) < (RTR_EXP2_POLY_PER8 / 2);
+        const float2 pr = poly ? exp2_poly_x2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        acc[e & 3] = fadd2(acc[e & 3], pr);
+        pk[e] = pack_bf16x2(pr.x, pr.y);
+    }
+    tmem_st16(tP, pk);
+}
+
 // Chunk write: rows [64*part, 64*part+64) of chunk key (or value) tile tt,
 // held in shared memory at `src` in the TMA layout (D/64 boxes of 128 rows x
 // 128 bytes, 128-byte swizzle), stored to their ring rows.  Lanes cover
@@ -302,6 +336,51 @@ __device__ __forceinline__ void commit_tile_rows(const TcParams &p, uint32_t src
                          : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                          : "r"(src + box * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4)));
             *reinterpret_cast<uint4 *>(dst + ((long long)head * p.commit_rows_per_head + drow) * D + piece * 8) = v;
+        }
+    }
+}
+
+// Chunk write from global memory: this CTA's 1/gridDim share of the 16-byte
+// vectors of the chunk's K and V ([nq][heads][D] each), copied to their ring
+// rows of the head-major cache by `nthr` threads, four vectors in flight per
+// thread.  Consecutive vectors are consecutive source bytes, so a warp reads
+// 512 contiguous bytes and writes whole 16-byte pieces of D-element rows.
+template <int D>
+__device__ __forceinline__ void commit_rows_global(const TcParams &p, int tid, int nthr) {
+    constexpr int VPR = D / 8;                                  // vectors per (token, head) row
+    const long long per_tensor = (long long)p.nq * p.heads * VPR;
+    const long long total = 2 * per_tensor;
+    const long long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+    for (long long base = lo + tid; base < hi; base += 4LL * nthr) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const long long i = base + (long long)u * nthr;
+            if (i < hi) {
+                const int kv = i >= per_tensor;
+                const long long j = i - kv * per_tensor;
+                const uint4 *src = reinterpret_cast<const uint4 *>(kv ? p.src_v1 : p.src_k1) + j;
+                asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(v[u].x), "=r"(v[u].y), "=r"(v[u].z), "=r"(v[u].w)
+                             : "l"(src));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const long long i = base + (long long)u * nthr;
+            if (i < hi) {
+                const int kv = i >= per_tensor;
+                const long long j = i - kv * per_tensor;
+                const long long row = j / VPR;
+                const int cv = (int)(j - row * VPR);
+                const int tok = (int)(row / p.heads), h = (int)(row - (long long)tok * p.heads);
+                const int f = tok / p.kpf, r = tok - f * p.kpf;
+                int slot = p.commit_first_slot + f;             // < 2 * commit_slots
+                if (slot >= p.commit_slots) slot -= p.commit_slots;
+                const long long drow = p.commit_row0 + (long long)slot * p.kpf + r;
+                __nv_bfloat16 *dst = (kv ? p.commit_v : p.commit_k) + ((long long)h * p.commit_rows_per_head + drow) * D;
+                reinterpret_cast<uint4 *>(dst)[cv] = v[u];
+            }
         }
     }
 }
@@ -379,6 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(L::bS + i), 1);
             mbar_init(bar(L::bP + i), 4 * CG); // one arrive per softmax warp of the cluster
+            mbar_init(bar(L::bPh + i), 4 * CG); // the same, once P of the tile's first 64 keys is stored
+            mbar_init(bar(L::bSr + i), 4 * CG); // the same, once the softmax has read all of S
             mbar_init(bar(L::bO + i), 1);
             mbar_init(bar(L::bEpi + i), kBM);  // every softmax thread
         }
@@ -452,7 +533,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     }
                     const KvSeg g = p.seg[s];
                     const int row = g.row0 + tt * kBN;
-                    const bool copied = p.commit_k != nullptr && g.src == 1 && (tt >> 1) == unit_row;
+                    const bool copied =
+                        p.commit_k != nullptr && !p.commit_global && g.src == 1 && (tt >> 1) == unit_row;
                     for (int kv = 0; kv < 2; ++kv, ++n) {
                         const int slot = n % L::kSlots, use = n / L::kSlots;
                         if (*abort_flag) { ok = false; break; }
@@ -533,10 +615,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                         mma_ss(tmem + i * 128, a0 + a_off, b0 + b_off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](int i, int slot, bool acc) {
+            // S_i of one half of the key tile (64 keys) into its half of S_i's columns
+            constexpr bool kSSplit = RTR_S_SPLIT && CG == 1;
+            constexpr uint32_t idesc_sh = idesc_bf16_f32(kBM, kBN / 2, 0, 0);
+            auto issue_s_half = [&](int i, int slot, int half) {
+                const uint64_t a0 = i ? dq1 : dq0;
+                const uint64_t b0 = dk0 + (uint64_t)((slot * L::kSlotBytes + half * (kBN / 2) * 128) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t a_off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
+                    const uint32_t b_off = ((kk / 4) * (kKRows * 128) + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem + i * 128 + half * (kBN / 2), a0 + a_off, b0 + b_off, idesc_sh, kk > 0 ? 1u : 0u);
+                }
+            };
+            // PV over key steps [kk0, kk1) of 16 keys (all of them unless split)
+            auto issue_pv = [&](int i, int slot, bool acc, int kk0 = 0, int kk1 = kBN / 16) {
                 const uint64_t b0 = dv0 + (uint64_t)((slot * L::kSlotBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
+                for (int kk = kk0; kk < kk1; ++kk) {
                     if (CG == 2)
                         mma_ts_pair(tmem + 256 + i * D, tmem + i * 128 + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4),
                                     idesc_o, (acc || kk > 0) ? 1u : 0u);
@@ -558,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 // Unit tiles from copy_lo on are the chunk's; those with chunk
                 // tile (t - copy_lo) / 2 == the unit's pair index are copied out.
                 int copy_lo = 1 << 30, copy_hi = 0, copy_pair = 0;
-                if (p.commit_k != nullptr) {
+                if (p.commit_k != nullptr && !p.commit_global) {
                     int head_m;
                     unit_coords(p, it.unit, copy_pair, head_m);
                     const int q0m = copy_pair * p.unit_rows;
@@ -594,30 +690,71 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     go(it.t0 + j, vs);
                     ++n;
                     const int vslot = vs;
-                    ok = wait(bar(L::bP + 0), jj & 1) && !*abort_flag;
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(0, vslot, j > 0);
-                    if (j == T - 1) commit(L::bO + 0);
                     int ks = -1;
-                    if (j + 1 < T) {
+                    if (kSSplit && j + 1 < T) {
+                        // next key tile's second half into S_0's free columns
                         ks = n % L::kSlots;
                         ok = wait(bar(L::bFull + ks), (n / L::kSlots) & 1);
                         if (!ok) break;
                         go(it.t0 + j + 1, ks);
+                        ok = wait(bar(L::bSr + 0), jj & 1) && !*abort_flag;
+                        if (!ok) break;
                         tc_fence_after();
+                        issue_s_half(0, ks, 1);
+                    }
+                    if (RTR_PV_SPLIT) {
+                        ok = wait(bar(L::bPh + 0), jj & 1) && !*abort_flag;
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(0, vslot, j > 0, 0, kBN / 32);
+                    }
+                    ok = wait(bar(L::bP + 0), jj & 1) && !*abort_flag;
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (RTR_PV_SPLIT)
+                        issue_pv(0, vslot, true, kBN / 32, kBN / 16);
+                    else
+                        issue_pv(0, vslot, j > 0);
+                    if (j == T - 1) commit(L::bO + 0);
+                    if (j + 1 < T) {
+                        if (kSSplit) {
+                            // the first half's columns held P_0, which PV_0 has now read
+                            issue_s_half(0, ks, 0);
+                        } else {
+                            ks = n % L::kSlots;
+                            ok = wait(bar(L::bFull + ks), (n / L::kSlots) & 1);
+                            if (!ok) break;
+                            go(it.t0 + j + 1, ks);
+                            tc_fence_after();
+                            issue_s(0, ks);
+                        }
                         kslot = ks;
-                        issue_s(0, kslot);
                         commit(L::bS + 0);
+                    }
+                    if (kSSplit && j + 1 < T) {
+                        ok = wait(bar(L::bSr + 1), jj & 1) && !*abort_flag;
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s_half(1, ks, 1);
+                    }
+                    if (RTR_PV_SPLIT) {
+                        ok = wait(bar(L::bPh + 1), jj & 1) && !*abort_flag;
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(1, vslot, j > 0, 0, kBN / 32);
                     }
                     ok = wait(bar(L::bP + 1), jj & 1) && !*abort_flag;
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(1, vslot, j > 0);
+                    if (RTR_PV_SPLIT)
+                        issue_pv(1, vslot, true, kBN / 32, kBN / 16);
+                    else
+                        issue_pv(1, vslot, j > 0);
                     commit(L::bEmpty + vs);
                     if (j == T - 1) commit(L::bO + 1);
                     if (j + 1 < T) {
-                        issue_s(1, kslot);
+                        if (kSSplit) issue_s_half(1, kslot, 0);
+                        else issue_s(1, kslot);
                         commit(L::bS + 1);
                         commit(L::bEmpty + ks);
                         ++n;
@@ -635,6 +772,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             mbar_wait(bar(L::bDrain), 0, kWaitNs);
         }
         __syncwarp();
+    } else if (warp >= 2 && p.commit_k != nullptr && p.commit_global) {
+        // ------------------------------------------------------------ chunk write from global memory
+        // CTA c copies its 1/G share of the chunk's K and V rows from the
+        // token-major source to their ring rows; it reads nothing this launch
+        // writes and writes only rows this launch never reads.
+        commit_rows_global<D>(p, (warp - 2) * 32 + lane, 64);
     } else if (warp >= 2 && p.commit_k != nullptr && (p.commit_maps == nullptr || (warp == 2 && lane == 0))) {
         // ------------------------------------------------------------ chunk write
         // Walks the producer's load sequence and waits (on bGo) only for the
@@ -728,11 +871,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 w = __all_sync(0xffffffffu, w);
                 if (!w) { ok = false; break; }
                 tc_fence_after();
-                // Pass 1: row max, 64 columns per TMEM round trip (the row is read
-                // again in pass 2 instead of being held in registers).
                 // Warp-uniform: the code below holds tcgen05 .sync.aligned
                 // instructions, which every lane of the warp must execute together.
                 const bool masked = __any_sync(0xffffffffu, lim < kBN);
+#if RTR_SOFTMAX_1LD
+                // The row's 128 scores in registers: one TMEM read, the max,
+                // then P over them in four 32-column chunks.
+                uint32_t sr[128];
+                tmem_ld128(tS, sr);
+                tmem_wait_ld();
+                if (RTR_S_SPLIT && CG == 1) {
+                    // S is in registers: the MMA may write the next tile's second half
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(L::bSr + i));
+                }
+                if (masked) {
+#pragma unroll
+                    for (int e = 0; e < 128; ++e)
+                        if (e >= lim) sr[e] = __float_as_uint(-INFINITY);
+                }
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 128; e += 8) {
+                    mx0 = max3f(mx0, __uint_as_float(sr[e + 0]), __uint_as_float(sr[e + 1]));
+                    mx1 = max3f(mx1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+                    mx2 = max3f(mx2, __uint_as_float(sr[e + 4]), __uint_as_float(sr[e + 5]));
+                    mx3 = max3f(mx3, __uint_as_float(sr[e + 6]), __uint_as_float(sr[e + 7]));
+                }
+#else
+                // Pass 1: row max, 64 columns per TMEM round trip (the row is read
+                // again in pass 2 instead of being held in registers).
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -759,6 +928,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                         mx3 = max3f(mx3, __uint_as_float(rb[e + 6]), __uint_as_float(rb[e + 7]));
                     }
                 }
+#endif
                 const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
                 const float m_new = fmaxf(m_run, mx * sl2);
                 const bool upd = m_new > m_run + 8.0f;
@@ -769,6 +939,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     l_run *= factor;
                 }
                 if (t > it.t0 && __any_sync(0xffffffffu, upd)) {
+#if RTR_SOFTMAX_1LD
+                    // 16 columns at a time: the row's scores are still live
+#pragma unroll 1
+                    for (int c = 0; c < D / 16; ++c) {
+                        uint32_t o[16];
+                        tmem_ld16(tO + 16 * c, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+                        tmem_st16(tO + 16 * c, o);
+                    }
+#else
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
@@ -778,6 +960,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
                         tmem_st32(tO + 32 * c, o);
                     }
+#endif
                 }
                 const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
                 float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -787,6 +970,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 // 64 columns, behind the scores already read.  The polynomial
                 // exp2 runs only on tiles without masked entries (every input
                 // finite); ex2 maps -inf to exactly 0.
+#if RTR_SOFTMAX_1LD
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    if (masked) softmax_chunk_regs<false>(sr + 32 * q4, sl2, neg_m, tS + 16 * q4, acc);
+                    else softmax_chunk_regs<true>(sr + 32 * q4, sl2, neg_m, tS + 16 * q4, acc);
+                    if (RTR_PV_SPLIT && q4 == 1) {
+                        // P of the first 64 keys is in TMEM: their PV may start
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (CG == 2) mbar_arrive_cluster(lead(L::bPh + i));
+                            else mbar_arrive(bar(L::bPh + i));
+                        }
+                    }
+                }
+#else
                 {
                     uint32_t buf[2][32];
                     tmem_ld32(tS, buf[0]);
@@ -803,8 +1003,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                             softmax_chunk<true>(buf[q4 & 1], sl2, neg_m, tS + 16 * q4, acc);
                         }
                         if (q4 < 3) tmem_wait_ld();
+                        if (RTR_PV_SPLIT && q4 == 1) {
+                            // P of the first 64 keys is in TMEM: their PV may start
+                            tmem_wait_st();
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) {
+                                if (CG == 2) mbar_arrive_cluster(lead(L::bPh + i));
+                                else mbar_arrive(bar(L::bPh + i));
+                            }
+                        }
                     }
                 }
+#endif
                 const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
                 const float2 a4 = fadd2(a01, a23);
                 l_run += a4.x + a4.y;
@@ -1186,6 +1397,9 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
         tp.commit_slots = p.commit_slots;
         tp.commit_row0 = p.commit_row0;
         tp.commit_maps = p.commit_maps;
+        tp.commit_global = RTR_COMMIT_GLOBAL;
+        tp.src_k1 = static_cast<const __nv_bfloat16 *>(p.k1);
+        tp.src_v1 = static_cast<const __nv_bfloat16 *>(p.v1);
     }
     if (p.head_dim == 128)
         return plan.cg == 2 ? launch_tc<128, 2>(tp, plan.has_split, s) : launch_tc<128, 1>(tp, plan.has_split, s);
