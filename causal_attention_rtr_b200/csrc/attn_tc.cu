@@ -30,11 +30,14 @@
 //               key / value tiles from the ring slots to their cache rows;
 //               idle otherwise
 //   warps 4-7   softmax for Q0, warps 8-11 softmax for Q1: one thread per
-//               query row reads its S row from TMEM, online softmax in fp32
-//               (exp2 domain; O is rescaled only when the running max grows
-//               by more than 2^8 -- exact after the final division), writes P
-//               as bf16 back over its S columns, and finally normalises O and
-//               stores it with TMA (or writes the fp32 partial).
+//               query row reads its 128 scores from TMEM once into registers,
+//               online softmax in fp32 (exp2 domain; O is rescaled only when
+//               the running max grows by more than 2^8 -- exact after the
+//               final division), writes P as bf16 back over its S columns in
+//               four 32-key chunks, and finally normalises O and stores it
+//               with TMA (or writes the fp32 partial).  Once P of the first
+//               64 keys is stored the tensor core starts their half of PV,
+//               while the softmax finishes the other half.
 // The two softmax groups ping-pong: while one works on its S tile the tensor
 // core runs the other tile's QK^T or PV.  Part of the exponentials run as a
 // polynomial on the FMA pipe (exp2_poly) so that the special-function unit
@@ -66,19 +69,19 @@
 #define RTR_UNIT_ORDER_RATIO 1.25   // head-major unit order when max/min key tiles per pair <= this
 #endif
 #ifndef RTR_PV_SPLIT
-#define RTR_PV_SPLIT 0   // 1: PV over the first 64 keys starts once their P is stored (bPh)
+#define RTR_PV_SPLIT 1   // PV over the first 64 keys starts once their P is stored (bPh); 0: after all of P
 #endif
 #ifndef RTR_S_SPLIT
 #define RTR_S_SPLIT 0   // 1: S(j+1) of the second 64 keys runs once the softmax has read S(j) (needs 1LD + PV split)
-#endif
-#if RTR_S_SPLIT && !(RTR_SOFTMAX_1LD && RTR_PV_SPLIT)
-#error "RTR_S_SPLIT needs RTR_SOFTMAX_1LD and RTR_PV_SPLIT"
 #endif
 #ifndef RTR_COMMIT_GLOBAL
 #define RTR_COMMIT_GLOBAL 0   // 1: the chunk write copies from the chunk's global K/V, spread over the launch
 #endif
 #ifndef RTR_SOFTMAX_1LD
-#define RTR_SOFTMAX_1LD 0   // 1: the row's 128 scores read from TMEM once, held in registers
+#define RTR_SOFTMAX_1LD 1   // the row's 128 scores read from TMEM once, held in registers; 0: read twice
+#endif
+#if RTR_S_SPLIT && !(RTR_SOFTMAX_1LD && RTR_PV_SPLIT)
+#error "RTR_S_SPLIT needs RTR_SOFTMAX_1LD and RTR_PV_SPLIT"
 #endif
 #ifndef RTR_EXP2_POLY_PER8
 #define RTR_EXP2_POLY_PER8 0   // of every 8 scores, how many use exp2_poly (0 measured fastest so far)

@@ -5,12 +5,24 @@ bias / GELU / gated residual / 3D rotary encoding in fp64, one rounding to
 bf16; papernotes.org note "DiT as Real-Time Rerenderer", Method > Overall
 Architecture).
 
-Tolerance: both sides round the same quantity once to bf16, the GPU from an
-fp32 accumulation and the oracle from fp64.  The two unrounded values differ
-by far less than a bf16 unit in the last place (fp32 sums over at most 8960
-exact bf16 products, fp32 sin / cos of angles below 100 rad), so the rounded
-results are equal or, where the two straddle a rounding boundary, one bf16
-ulp apart: every element must be within one ulp of the oracle."""
+Tolerance, per element: one bf16 unit in the last place of the result plus
+the error bound of the fp32 accumulation.  Both sides round the same
+quantity once to bf16, the GPU from an fp32 sum of K exact bf16 products
+and the oracle from fp64.  Whatever the order and rounding mode, an fp32
+sum of K terms is within K * 2^-23 * sum_k |a_k w_k| of the exact sum
+(the standard recursive-summation bound with truncating additions, here
+taken for any order); the bias adds |b| to the sum of magnitudes.  That
+absolute error passes through the epilogue (times at most 1.13 for GELU's
+slope, |gate| for the gated residual, and into both members of a rotary
+pair), and the epilogue's own fp32 operations add a few fp32 units of its
+result.  Where the result is far smaller than the terms that made it
+(cancellation in the sum, GELU of a strongly negative input) the bound is
+that absolute error, many bf16 ulps of the small result; elsewhere it is
+about one ulp.  As checks of the whole matrix, under 1 % of the elements
+may differ from the oracle at all (a wrong layout, tile or race changes
+nearly every element of the tiles it touches) and the relative L2 error
+must stay below 1e-3 (one-ulp differences on a small fraction of the
+elements give about 1e-4)."""
 import numpy as np
 import pytest
 import torch
@@ -34,12 +46,28 @@ def _ulp(x):
     return 2.0 ** (e - 7)
 
 
-def assert_within_one_ulp(got, want, what):
+def acc_error(A, Wt, B, k):
+    """Bound of the fp32 accumulation error of A @ Wt + B, per element."""
+    return k * 2.0 ** -23 * (np.abs(A) @ np.abs(Wt) + np.abs(B))
+
+
+def assert_parity(got, want, err_abs, what):
+    """|got - want| <= one bf16 ulp + err_abs + a few fp32 units, every
+    element; under 1 % of the elements different at all."""
     assert np.all(np.isfinite(got)), what
-    bound = _ulp(np.maximum(np.abs(got), np.abs(want)))
-    worst = float(np.max(np.abs(got - want) / bound))
+    mag = np.maximum(np.abs(got), np.abs(want))
+    bound = _ulp(mag) + err_abs + 8 * 2.0 ** -24 * mag
+    excess = np.abs(got - want) / bound
+    worst = float(np.max(excess))
     frac_diff = float(np.mean(got != want))
-    assert worst <= 1.0, f"{what}: worst |diff| / ulp = {worst:.3f}"
+    i = np.unravel_index(int(np.argmax(excess)), excess.shape)
+    detail = f"worst at {i}: got {got[i]!r} want {want[i]!r} bound {bound[i]:.3e}"
+    print(f"{what}: worst/bound={worst:.3f} differing={frac_diff:.2e} ({detail})")
+    rel = float(np.linalg.norm(got - want) / np.linalg.norm(want))
+    print(f"{what}: rel_l2={rel:.3e}")
+    assert worst <= 1.0, f"{what}: {detail}"
+    assert frac_diff < 0.01, f"{what}: {frac_diff:.2%} of the elements differ"
+    assert rel <= 1e-3, f"{what}: rel_l2={rel:.3e}"
     return worst, frac_diff
 
 
@@ -68,19 +96,24 @@ def test_dit_linear_parity(m, n, k, epi):
     a, w, b = _operands(rng, m, n, k)
     A, Wt, B = decode(a, "bf16"), decode(w, "bf16"), decode(b, "bf16")
     C = A @ Wt + B
+    E = acc_error(A, Wt, B, k)
     gate = None
     if epi.startswith("gated_residual"):
         x = synth.normal(rng, (m, n), 1.0, "bf16")
         X = decode(x, "bf16")
         if epi == "gated_residual":
             gate = synth.normal(rng, (n,), 0.5, "bf16")
-            want = db.round_bf16(X + decode(gate, "bf16") * C)
+            G = decode(gate, "bf16")
+            want = db.round_bf16(X + G * C)
+            E = E * np.abs(G) + 4 * 2.0 ** -24 * (np.abs(X) + np.abs(G * C))
         else:
             want = db.round_bf16(X + C)
+            E = E + 4 * 2.0 ** -24 * (np.abs(X) + np.abs(C))
         out = dev(x)
         code = "gated_residual"
     elif epi == "gelu":
         want = db.round_bf16(db.gelu_tanh(C))
+        E = 1.13 * E + 2.0 ** -20 * np.abs(C)
         out = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
         code = "gelu"
     else:
@@ -90,8 +123,7 @@ def test_dit_linear_parity(m, n, k, epi):
     rtr.rtr_dit_linear(dev(a), dev(w), m, n, k, code, dev(b), None if gate is None else dev(gate), out)
     torch.cuda.synchronize()
     assert rtr.rtr_get_device_status(0) == rtr.RTR_OK
-    worst, frac = assert_within_one_ulp(host_f64(out), want, f"{epi} m={m} n={n} k={k}")
-    print(f"{epi} m={m} n={n} k={k}: worst/ulp={worst:.3f} differing={frac:.2e}")
+    assert_parity(host_f64(out), want, E, f"{epi} m={m} n={n} k={k}")
 
 
 QKV_CASES = [
@@ -109,18 +141,35 @@ def test_dit_qkv_rope_parity(H, d, gh, gw, C, t0):
     m = C * k
     rng = np.random.default_rng(H * d + m)
     a, w, b = _operands(rng, m, 3 * D, D)
-    qkv = decode(a, "bf16") @ decode(w, "bf16") + decode(b, "bf16")
+    A, Wt, B = decode(a, "bf16"), decode(w, "bf16"), decode(b, "bf16")
+    qkv = A @ Wt + B
+    E = acc_error(A, Wt, B, D)
     t, yy, xx = db.token_positions(C, gh, gw, t0)
-    want = [db.round_bf16(db.rope3d(qkv[:, :D].reshape(m, H, d), t, yy, xx)),
-            db.round_bf16(db.rope3d(qkv[:, D:2 * D].reshape(m, H, d), t, yy, xx)),
-            db.round_bf16(qkv[:, 2 * D:].reshape(m, H, d))]
+
+    def pair_err(e3):
+        """A rotary pair mixes both members' errors; the fp32 angle adds a
+        few fp32 units of the pair's magnitude."""
+        e = e3.reshape(m, H, d // 2, 2).sum(axis=-1, keepdims=True)
+        return np.broadcast_to(e, (m, H, d // 2, 2)).reshape(m, H, d)
+
+    want, errs = [], []
+    for part in range(3):
+        v = qkv[:, part * D:(part + 1) * D].reshape(m, H, d)
+        e = E[:, part * D:(part + 1) * D].reshape(m, H, d)
+        if part < 2:
+            mag = np.abs(v).reshape(m, H, d // 2, 2).sum(axis=-1, keepdims=True)
+            mag = np.broadcast_to(mag, (m, H, d // 2, 2)).reshape(m, H, d)
+            want.append(db.round_bf16(db.rope3d(v, t, yy, xx)))
+            errs.append(pair_err(e) + 2.0 ** -20 * mag)
+        else:
+            want.append(db.round_bf16(v))
+            errs.append(e)
     q, kk, v = (torch.empty((m, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(3))
     rtr.rtr_dit_qkv_rope(dev(a), dev(w), dev(b), m, D, H, d, k, gw, t0, q, kk, v)
     torch.cuda.synchronize()
     assert rtr.rtr_get_device_status(0) == rtr.RTR_OK
-    for name, got, ref in zip("qkv", (q, kk, v), want):
-        worst, frac = assert_within_one_ulp(host_f64(got), ref, f"{name} H={H} d={d} m={m}")
-        print(f"qkv {name} H={H} d={d} m={m}: worst/ulp={worst:.3f} differing={frac:.2e}")
+    for name, got, ref, err in zip("qkv", (q, kk, v), want, errs):
+        assert_parity(host_f64(got), ref, err, f"{name} H={H} d={d} m={m}")
 
 
 def test_dit_linear_repeat_is_bit_identical():
