@@ -52,6 +52,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -71,17 +72,8 @@
 #ifndef RTR_PV_SPLIT
 #define RTR_PV_SPLIT 1   // PV over the first 64 keys starts once their P is stored (bPh); 0: after all of P
 #endif
-#ifndef RTR_S_SPLIT
-#define RTR_S_SPLIT 0   // 1: S(j+1) of the second 64 keys runs once the softmax has read S(j) (needs 1LD + PV split)
-#endif
-#ifndef RTR_COMMIT_GLOBAL
-#define RTR_COMMIT_GLOBAL 0   // 1: the chunk write copies from the chunk's global K/V, spread over the launch
-#endif
 #ifndef RTR_SOFTMAX_1LD
 #define RTR_SOFTMAX_1LD 1   // the row's 128 scores read from TMEM once, held in registers; 0: read twice
-#endif
-#if RTR_S_SPLIT && !(RTR_SOFTMAX_1LD && RTR_PV_SPLIT)
-#error "RTR_S_SPLIT needs RTR_SOFTMAX_1LD and RTR_PV_SPLIT"
 #endif
 #ifndef RTR_EXP2_POLY_PER8
 #define RTR_EXP2_POLY_PER8 0   // of every 8 scores, how many use exp2_poly (0 measured fastest so far)
@@ -129,8 +121,6 @@ struct TcParams {
     long long commit_rows_per_head;
     int commit_first_slot, commit_slots, commit_row0;
     const CUtensorMap *commit_maps;   // per-slot store maps (see AttnProblem) or null
-    int commit_global;                // 1: warps 2-3 copy the chunk from its global K/V (src_k1, src_v1)
-    const __nv_bfloat16 *src_k1, *src_v1;   // the token-major run's K / V in global memory
     float *lse;         // [heads][nq] natural-log row log-sum-exp, or null
 };
 
@@ -147,7 +137,7 @@ struct Layout {
     static constexpr int kBars = kKV + kSlots * kSlotBytes; // mbarriers
     static constexpr int bQ = 0, bQfree = 1, bFull = 2, bEmpty = bFull + kSlots, bCopied = bEmpty + kSlots,
                          bGo = bCopied + kSlots, bS = bGo + kSlots, bP = bS + 2, bO = bP + 2, bEpi = bO + 2, bDrain = bEpi + 2,
-                         bPh = bDrain + 1, bSr = bPh + 2, kNumBars = bSr + 2;
+                         bPh = bDrain + 1, kNumBars = bPh + 2;
     static constexpr int kMisc = kBars + kNumBars * 8;      // tmem holder, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;            // slack for 1 KB alignment
@@ -343,51 +333,6 @@ __device__ __forceinline__ void commit_tile_rows(const TcParams &p, uint32_t src
     }
 }
 
-// Chunk write from global memory: this CTA's 1/gridDim share of the 16-byte
-// vectors of the chunk's K and V ([nq][heads][D] each), copied to their ring
-// rows of the head-major cache by `nthr` threads, four vectors in flight per
-// thread.  Consecutive vectors are consecutive source bytes, so a warp reads
-// 512 contiguous bytes and writes whole 16-byte pieces of D-element rows.
-template <int D>
-__device__ __forceinline__ void commit_rows_global(const TcParams &p, int tid, int nthr) {
-    constexpr int VPR = D / 8;                                  // vectors per (token, head) row
-    const long long per_tensor = (long long)p.nq * p.heads * VPR;
-    const long long total = 2 * per_tensor;
-    const long long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
-    for (long long base = lo + tid; base < hi; base += 4LL * nthr) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const long long i = base + (long long)u * nthr;
-            if (i < hi) {
-                const int kv = i >= per_tensor;
-                const long long j = i - kv * per_tensor;
-                const uint4 *src = reinterpret_cast<const uint4 *>(kv ? p.src_v1 : p.src_k1) + j;
-                asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                             : "=r"(v[u].x), "=r"(v[u].y), "=r"(v[u].z), "=r"(v[u].w)
-                             : "l"(src));
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const long long i = base + (long long)u * nthr;
-            if (i < hi) {
-                const int kv = i >= per_tensor;
-                const long long j = i - kv * per_tensor;
-                const long long row = j / VPR;
-                const int cv = (int)(j - row * VPR);
-                const int tok = (int)(row / p.heads), h = (int)(row - (long long)tok * p.heads);
-                const int f = tok / p.kpf, r = tok - f * p.kpf;
-                int slot = p.commit_first_slot + f;             // < 2 * commit_slots
-                if (slot >= p.commit_slots) slot -= p.commit_slots;
-                const long long drow = p.commit_row0 + (long long)slot * p.kpf + r;
-                __nv_bfloat16 *dst = (kv ? p.commit_v : p.commit_k) + ((long long)h * p.commit_rows_per_head + drow) * D;
-                reinterpret_cast<uint4 *>(dst)[cv] = v[u];
-            }
-        }
-    }
-}
-
 // Chunk write by TMA: the 128 rows of chunk key (or value) tile tt, held in
 // shared memory at `src` in the TMA layout, stored to their ring slots by one
 // thread.  A tile inside one frame is one 128-row box per 64 columns; the
@@ -462,7 +407,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             mbar_init(bar(L::bS + i), 1);
             mbar_init(bar(L::bP + i), 4 * CG); // one arrive per softmax warp of the cluster
             mbar_init(bar(L::bPh + i), 4 * CG); // the same, once P of the tile's first 64 keys is stored
-            mbar_init(bar(L::bSr + i), 4 * CG); // the same, once the softmax has read all of S
             mbar_init(bar(L::bO + i), 1);
             mbar_init(bar(L::bEpi + i), kBM);  // every softmax thread
         }
@@ -536,8 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     }
                     const KvSeg g = p.seg[s];
                     const int row = g.row0 + tt * kBN;
-                    const bool copied =
-                        p.commit_k != nullptr && !p.commit_global && g.src == 1 && (tt >> 1) == unit_row;
+                    const bool copied = p.commit_k != nullptr && g.src == 1 && (tt >> 1) == unit_row;
                     for (int kv = 0; kv < 2; ++kv, ++n) {
                         const int slot = n % L::kSlots, use = n / L::kSlots;
                         if (*abort_flag) { ok = false; break; }
@@ -618,19 +561,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                         mma_ss(tmem + i * 128, a0 + a_off, b0 + b_off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            // S_i of one half of the key tile (64 keys) into its half of S_i's columns
-            constexpr bool kSSplit = RTR_S_SPLIT && CG == 1;
-            constexpr uint32_t idesc_sh = idesc_bf16_f32(kBM, kBN / 2, 0, 0);
-            auto issue_s_half = [&](int i, int slot, int half) {
-                const uint64_t a0 = i ? dq1 : dq0;
-                const uint64_t b0 = dk0 + (uint64_t)((slot * L::kSlotBytes + half * (kBN / 2) * 128) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t a_off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
-                    const uint32_t b_off = ((kk / 4) * (kKRows * 128) + (kk % 4) * 32) >> 4;
-                    mma_ss(tmem + i * 128 + half * (kBN / 2), a0 + a_off, b0 + b_off, idesc_sh, kk > 0 ? 1u : 0u);
-                }
-            };
             // PV over key steps [kk0, kk1) of 16 keys (all of them unless split)
             auto issue_pv = [&](int i, int slot, bool acc, int kk0 = 0, int kk1 = kBN / 16) {
                 const uint64_t b0 = dv0 + (uint64_t)((slot * L::kSlotBytes) >> 4);
@@ -657,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 // Unit tiles from copy_lo on are the chunk's; those with chunk
                 // tile (t - copy_lo) / 2 == the unit's pair index are copied out.
                 int copy_lo = 1 << 30, copy_hi = 0, copy_pair = 0;
-                if (p.commit_k != nullptr && !p.commit_global) {
+                if (p.commit_k != nullptr) {
                     int head_m;
                     unit_coords(p, it.unit, copy_pair, head_m);
                     const int q0m = copy_pair * p.unit_rows;
@@ -694,17 +624,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     ++n;
                     const int vslot = vs;
                     int ks = -1;
-                    if (kSSplit && j + 1 < T) {
-                        // next key tile's second half into S_0's free columns
-                        ks = n % L::kSlots;
-                        ok = wait(bar(L::bFull + ks), (n / L::kSlots) & 1);
-                        if (!ok) break;
-                        go(it.t0 + j + 1, ks);
-                        ok = wait(bar(L::bSr + 0), jj & 1) && !*abort_flag;
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_s_half(0, ks, 1);
-                    }
                     if (RTR_PV_SPLIT) {
                         ok = wait(bar(L::bPh + 0), jj & 1) && !*abort_flag;
                         if (!ok) break;
@@ -720,25 +639,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                         issue_pv(0, vslot, j > 0);
                     if (j == T - 1) commit(L::bO + 0);
                     if (j + 1 < T) {
-                        if (kSSplit) {
-                            // the first half's columns held P_0, which PV_0 has now read
-                            issue_s_half(0, ks, 0);
-                        } else {
-                            ks = n % L::kSlots;
-                            ok = wait(bar(L::bFull + ks), (n / L::kSlots) & 1);
-                            if (!ok) break;
-                            go(it.t0 + j + 1, ks);
-                            tc_fence_after();
-                            issue_s(0, ks);
-                        }
-                        kslot = ks;
-                        commit(L::bS + 0);
-                    }
-                    if (kSSplit && j + 1 < T) {
-                        ok = wait(bar(L::bSr + 1), jj & 1) && !*abort_flag;
+                        ks = n % L::kSlots;
+                        ok = wait(bar(L::bFull + ks), (n / L::kSlots) & 1);
                         if (!ok) break;
+                        go(it.t0 + j + 1, ks);
                         tc_fence_after();
-                        issue_s_half(1, ks, 1);
+                        kslot = ks;
+                        issue_s(0, kslot);
+                        commit(L::bS + 0);
                     }
                     if (RTR_PV_SPLIT) {
                         ok = wait(bar(L::bPh + 1), jj & 1) && !*abort_flag;
@@ -756,8 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                     commit(L::bEmpty + vs);
                     if (j == T - 1) commit(L::bO + 1);
                     if (j + 1 < T) {
-                        if (kSSplit) issue_s_half(1, kslot, 0);
-                        else issue_s(1, kslot);
+                        issue_s(1, kslot);
                         commit(L::bS + 1);
                         commit(L::bEmpty + ks);
                         ++n;
@@ -775,12 +682,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             mbar_wait(bar(L::bDrain), 0, kWaitNs);
         }
         __syncwarp();
-    } else if (warp >= 2 && p.commit_k != nullptr && p.commit_global) {
-        // ------------------------------------------------------------ chunk write from global memory
-        // CTA c copies its 1/G share of the chunk's K and V rows from the
-        // token-major source to their ring rows; it reads nothing this launch
-        // writes and writes only rows this launch never reads.
-        commit_rows_global<D>(p, (warp - 2) * 32 + lane, 64);
     } else if (warp >= 2 && p.commit_k != nullptr && (p.commit_maps == nullptr || (warp == 2 && lane == 0))) {
         // ------------------------------------------------------------ chunk write
         // Walks the producer's load sequence and waits (on bGo) only for the
@@ -883,12 +784,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
                 uint32_t sr[128];
                 tmem_ld128(tS, sr);
                 tmem_wait_ld();
-                if (RTR_S_SPLIT && CG == 1) {
-                    // S is in registers: the MMA may write the next tile's second half
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(L::bSr + i));
-                }
                 if (masked) {
 #pragma unroll
                     for (int e = 0; e < 128; ++e)
@@ -1181,14 +1076,16 @@ __global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcPa
 template <int D, int CG>
 cudaError_t launch_tc(const TcParams &tp, bool has_split, cudaStream_t s) {
     using L = Layout<D, CG>;
-    static int configured_mask = 0;   // per device bit (up to 32 devices)
+    static std::atomic<unsigned> configured_mask{0};   // per device bit (up to 32 devices)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!(configured_mask & (1 << dev))) {
+    const unsigned bit = 1u << (dev & 31);
+    if (!(configured_mask.load(std::memory_order_acquire) & bit)) {
+        // two threads may both set the attribute; the call is idempotent
         cudaError_t e =
             cudaFuncSetAttribute(attn_fwd_tc<D, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
         if (e != cudaSuccess) return e;
-        configured_mask |= 1 << dev;
+        configured_mask.fetch_or(bit, std::memory_order_release);
     }
     cudaError_t e;
     if (CG == 2) {
@@ -1323,11 +1220,11 @@ void plan_attn_bf16(const AttnProblem &p, int sms, int cg, AttnPlan &plan) {
 }
 
 namespace {
-int g_inject_timeouts[64] = {};   // per device: launches left that skip their loads
+std::atomic<int> g_inject_timeouts[64] = {};   // per device: launches left that skip their loads
 }
 
 void inject_wait_timeouts(int device, int launches) {
-    if (device >= 0 && device < 64) g_inject_timeouts[device] = launches > 0 ? launches : 0;
+    if (device >= 0 && device < 64) g_inject_timeouts[device].store(launches > 0 ? launches : 0);
 }
 
 cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const CUtensorMap *tm_k0,
@@ -1336,8 +1233,10 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
     TcParams tp;
     memset(&tp, 0, sizeof(tp));
     int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && g_inject_timeouts[dev] > 0) {
-        --g_inject_timeouts[dev];
+    int left = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 &&
+        (left = g_inject_timeouts[dev].load()) > 0 &&
+        g_inject_timeouts[dev].compare_exchange_strong(left, left - 1)) {
         tp.test_skip_loads = 1;
     }
     const uint64_t D = (uint64_t)p.head_dim;
@@ -1400,9 +1299,6 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
         tp.commit_slots = p.commit_slots;
         tp.commit_row0 = p.commit_row0;
         tp.commit_maps = p.commit_maps;
-        tp.commit_global = RTR_COMMIT_GLOBAL;
-        tp.src_k1 = static_cast<const __nv_bfloat16 *>(p.k1);
-        tp.src_v1 = static_cast<const __nv_bfloat16 *>(p.v1);
     }
     if (p.head_dim == 128)
         return plan.cg == 2 ? launch_tc<128, 2>(tp, plan.has_split, s) : launch_tc<128, 1>(tp, plan.has_split, s);

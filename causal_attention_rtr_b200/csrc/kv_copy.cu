@@ -6,9 +6,8 @@
 //
 // Source rows are [tokens][heads][d] (the layout a QKV projection produces);
 // the cache is head-major [heads][rows][d].  The kernel is a pure HBM-bound
-// copy: every thread keeps eight 16-byte vectors in flight (all loads before
-// the matching stores), K and V share one index space, and the grid is no
-// larger than the SMs hold at once, so a copy runs as one wave.  Index
+// copy: every thread moves four 16-byte vectors, all loads in flight before
+// the matching stores, and one grid pass covers K and V together.  Index
 // arithmetic uses multiply-high division by run-time constants (Granlund and
 // Montgomery, "Division by Invariant Integers using Multiplication", 1994).
 #include <cuda_runtime.h>
@@ -49,52 +48,43 @@ struct ScatterDev {
     uint64_t rows_per_head;
 };
 
-#ifndef RTR_SCATTER_ONE_WAVE
-#define RTR_SCATTER_ONE_WAVE 1   // 0: one block per 1024 vectors (about 1.5 waves for a 3-frame chunk)
-#endif
-
+constexpr int kUnroll = 4;
 constexpr int kBlock = 256;
-constexpr int kUnroll = RTR_SCATTER_ONE_WAVE ? 8 : 4;   // vectors in flight per thread
-constexpr int kBlocksPerSm = 4;                         // 1024 threads per SM, 128 KB in flight
 
-// K and V form one index space of 2 * per_tensor vectors.  Thread g of the
-// grid moves vectors g, g + G, g + 2G, ... (G = grid threads), kUnroll of
-// them per pass with all their loads in flight before their stores: every
-// warp access is one contiguous 512-byte run, and a grid small enough to be
-// resident at once covers the space in as few passes as its size allows.
-__global__ void __launch_bounds__(kBlock, kBlocksPerSm) kv_scatter(const ScatterDev a) {
+// K and V form one index space of 2 * per_tensor vectors; every thread moves
+// kUnroll vectors with all its loads in flight before its stores, and the
+// grid covers the space in one pass.
+__global__ void __launch_bounds__(kBlock) kv_scatter(const ScatterDev a) {
     const uint32_t vmask = (1u << a.vpr_log2) - 1u;
     const uint32_t total = 2u * a.per_tensor;
-    const uint32_t G = gridDim.x * kBlock;
-    for (uint32_t base = blockIdx.x * kBlock + threadIdx.x; base < total; base += kUnroll * G) {
-        uint4 v[kUnroll];
+    const uint32_t base = blockIdx.x * (kBlock * kUnroll) + threadIdx.x;
+    uint4 v[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t i = base + u * G;
-            if (i < total) {
-                const uint32_t t = i >= a.per_tensor;
-                const uint4 *ptr = (t ? a.src[1] : a.src[0]) + (i - t * a.per_tensor);
-                asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                             : "=r"(v[u].x), "=r"(v[u].y), "=r"(v[u].z), "=r"(v[u].w)
-                             : "l"(ptr));
-            }
+    for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t i = base + u * kBlock;
+        if (i < total) {
+            const uint32_t t = i >= a.per_tensor;
+            const uint4 *ptr = (t ? a.src[1] : a.src[0]) + (i - t * a.per_tensor);
+            asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(v[u].x), "=r"(v[u].y), "=r"(v[u].z), "=r"(v[u].w)
+                         : "l"(ptr));
         }
+    }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t i = base + u * G;
-            if (i < total) {
-                const uint32_t t = i >= a.per_tensor;
-                const uint32_t j = i - t * a.per_tensor;
-                const uint32_t row = j >> a.vpr_log2, c = j & vmask;
-                const uint32_t tok = fdiv(row, a.heads);
-                const uint32_t h = row - tok * a.heads.d;
-                const uint32_t f = fdiv(tok, a.kfr);
-                const uint32_t r = tok - f * a.kfr.d;
-                uint32_t slot = a.first_slot + f;
-                if (slot >= a.slot_mod) slot -= a.slot_mod;
-                const uint64_t drow = (uint64_t)(slot + a.slot_off) * a.kfr.d + r;
-                (t ? a.dst[1] : a.dst[0])[(((uint64_t)h * a.rows_per_head + drow) << a.vpr_log2) + c] = v[u];
-            }
+    for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t i = base + u * kBlock;
+        if (i < total) {
+            const uint32_t t = i >= a.per_tensor;
+            const uint32_t j = i - t * a.per_tensor;
+            const uint32_t row = j >> a.vpr_log2, c = j & vmask;
+            const uint32_t tok = fdiv(row, a.heads);
+            const uint32_t h = row - tok * a.heads.d;
+            const uint32_t f = fdiv(tok, a.kfr);
+            const uint32_t r = tok - f * a.kfr.d;
+            uint32_t slot = a.first_slot + f;
+            if (slot >= a.slot_mod) slot -= a.slot_mod;
+            const uint64_t drow = (uint64_t)(slot + a.slot_off) * a.kfr.d + r;
+            (t ? a.dst[1] : a.dst[0])[(((uint64_t)h * a.rows_per_head + drow) << a.vpr_log2) + c] = v[u];
         }
     }
 }
@@ -123,14 +113,7 @@ cudaError_t launch_kv_scatter(const ScatterArgs &a, cudaStream_t s) {
     d.slot_off = (uint32_t)a.slot_off;
     d.rows_per_head = (uint64_t)a.rows_per_head;
     const unsigned long long per_block = (unsigned long long)kBlock * kUnroll;
-    unsigned long long blocks = (2 * per_tensor + per_block - 1) / per_block;
-    if (RTR_SCATTER_ONE_WAVE) {
-        // no more blocks than the SMs hold at once: the grid loops instead
-        int dev = 0, sms = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess) sms = sm_count(dev);
-        const unsigned long long resident = (unsigned long long)sms * kBlocksPerSm;
-        if (blocks > resident) blocks = resident;
-    }
+    const unsigned long long blocks = (2 * per_tensor + per_block - 1) / per_block;
     kv_scatter<<<(unsigned)blocks, kBlock, 0, s>>>(d);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
