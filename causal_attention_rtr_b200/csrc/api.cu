@@ -767,19 +767,32 @@ rtr_status rtr_attn_block_causal_backward(const void *q, const void *k, const vo
     return cuda_status(launch_attn_bwd(pb, st, scratch, (cudaStream_t)stream));
 }
 
-rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer, const rtr_dit_weights *w,
-                                 const void *modulation, void *hidden, int n_cur_frames, int grid_h, int grid_w,
-                                 int t0, int commit, rtr_stream_t stream) {
-    if (!c || !x || !w || layer < 0 || layer >= c->layers || layer >= x->layers || n_cur_frames < 1 ||
-        grid_h < 1 || grid_w < 1 || t0 < 0 || (commit != 0 && commit != 1))
+}  // extern "C"
+
+namespace {
+
+// The block's weights as the projections read them: each matrix either
+// row-major [in][out] or in the packed B layout.
+struct DitW {
+    const void *wqkv, *wo, *wq2, *wo2, *w1, *w2;
+    const void *bqkv, *bo, *bq2, *bo2, *b1, *b2;
+    int d_ffn;
+    int packed;
+};
+
+rtr_status dit_block_run(rtr_kvcache *c, const rtr_xattn *x, int layer, const DitW &w, const void *modulation,
+                         void *hidden, int n_cur_frames, int grid_h, int grid_w, int t0, int commit,
+                         rtr_stream_t stream) {
+    if (!c || !x || layer < 0 || layer >= c->layers || layer >= x->layers || n_cur_frames < 1 || grid_h < 1 ||
+        grid_w < 1 || t0 < 0 || (commit != 0 && commit != 1))
         return RTR_E_INVAL;
     if (c->dt != RTR_BF16 || x->dt != RTR_BF16 || x->heads != c->heads || x->head_dim != c->head_dim ||
         x->device != c->device || (long long)grid_h * grid_w != c->k)
         return RTR_E_INVAL;
-    const int H = c->heads, d = c->head_dim, D = H * d, F = w->d_ffn;
+    const int H = c->heads, d = c->head_dim, D = H * d, F = w.d_ffn;
     if (F < 8 || F % 8 != 0 || (commit && n_cur_frames > c->W)) return RTR_E_INVAL;
-    for (const void *ptr : {modulation, (const void *)hidden, w->wqkv, w->bqkv, w->wo, w->bo, w->wq2, w->bq2,
-                            w->wo2, w->bo2, w->w1, w->b1, w->w2, w->b2})
+    for (const void *ptr : {modulation, (const void *)hidden, w.wqkv, w.bqkv, w.wo, w.bo, w.wq2, w.bq2, w.wo2, w.bo2,
+                            w.w1, w.b1, w.w2, w.b2})
         if (!aligned16(ptr)) return RTR_E_INVAL;
     const long long n = (long long)n_cur_frames * c->k;
     if (n > (1 << 24)) return RTR_E_INVAL;
@@ -789,24 +802,32 @@ rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer, 
     unsigned *status = device_status_ptr(c->device);
     if (!status) return RTR_E_CUDA;
     const int sms = sm_count(c->device);
-    // activations: h, q, k, v, o (bf16 [n][D]) and the GELU output (bf16 [n][F])
+    // Activations: q, k, v, o (bf16 [n][D]); the layer-norm output h, the
+    // projections' A operand, in the packed layout (D is a multiple of 64);
+    // the GELU output f, the last projection's A operand, packed when F is a
+    // multiple of 64, else [n][F].
+    const int f_packed = F % 64 == 0;
     auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
-    const size_t nd = up((size_t)n * D * 2), nf = up((size_t)n * F * 2);
-    char *ws = static_cast<char *>(stream_workspace(c->device, s, 5 * nd + nf, 1));
+    const size_t nd = up((size_t)n * D * 2), nh = up(packed_a_bytes(n, D));
+    const size_t nf = up(f_packed ? packed_a_bytes(n, F) : (size_t)n * F * 2);
+    char *ws = static_cast<char *>(stream_workspace(c->device, s, nh + 4 * nd + nf, 1));
     if (!ws) return RTR_E_NOMEM;
-    void *h = ws, *q = ws + nd, *k = ws + 2 * nd, *v = ws + 3 * nd, *o = ws + 4 * nd, *f = ws + 5 * nd;
+    void *h = ws, *q = ws + nh, *k = ws + nh + nd, *v = ws + nh + 2 * nd, *o = ws + nh + 3 * nd,
+         *f = ws + nh + 4 * nd;
     const char *mod = static_cast<const char *>(modulation);
     const size_t mrow = (size_t)D * 2;   // one modulation vector, bytes
     const int ni = (int)n;
     const float eps = 1e-6f;
     cudaError_t e = cudaSuccess;
     rtr_status st = RTR_OK;
-    // One projection with its epilogue: a = activations [n][in], w = [in][out].
-    auto gemm = [&](const void *a, const void *wt, int n_out, int n_in, int epi, const void *bias, const void *gate,
-                    void *out) {
+    // One projection with its epilogue: a = activations [n][in] (packed when
+    // a_packed), wt = [in][out] weights (packed when w.packed).
+    auto gemm = [&](const void *a, int a_packed, const void *wt, int n_out, int n_in, int epi, const void *bias,
+                    const void *gate, void *out, int out_packed) {
         GemmArgs g;
         memset(&g, 0, sizeof(g));
         g.a = a; g.w = wt; g.m = ni; g.n = n_out; g.k = n_in; g.epi = epi;
+        g.a_packed = a_packed; g.w_packed = w.packed; g.out_packed = out_packed;
         g.bias = bias; g.gate = gate; g.out = out;
         if (epi == kEpiQkvRope) {
             g.q = q; g.k_out = k; g.v = v;
@@ -823,27 +844,117 @@ rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer, 
         if ((st = (call)) != RTR_OK) return st;         \
     } while (0)
     // self attention branch
-    RTR_TRY(launch_ln_modulate(hidden, mod, mod + mrow, h, ni, D, eps, s));
-    RTR_TRY(gemm(h, w->wqkv, 3 * D, D, kEpiQkvRope, w->bqkv, nullptr, nullptr));
+    RTR_TRY(launch_ln_modulate(hidden, mod, mod + mrow, h, ni, D, eps, s, 1));
+    RTR_TRY(gemm(h, 1, w.wqkv, 3 * D, D, kEpiQkvRope, w.bqkv, nullptr, nullptr, 0));
     if (commit && c->S - c->W >= n_cur_frames) {
         RTR_TRY_ST(rtr_attn_frame_causal_commit(c, layer, q, k, v, n_cur_frames, o, 0.f, stream));
     } else {
         RTR_TRY_ST(rtr_attn_frame_causal(c, layer, q, k, v, n_cur_frames, o, 0.f, stream));
         if (commit) RTR_TRY_ST(rtr_kvcache_append_frame(c, layer, k, v, n_cur_frames, stream));
     }
-    RTR_TRY(gemm(o, w->wo, D, D, kEpiGatedResidual, w->bo, mod + 2 * mrow, hidden));
+    RTR_TRY(gemm(o, 0, w.wo, D, D, kEpiGatedResidual, w.bo, mod + 2 * mrow, hidden, 0));
     // cross attention branch
-    RTR_TRY(launch_ln_modulate(hidden, nullptr, nullptr, h, ni, D, eps, s));
-    RTR_TRY(gemm(h, w->wq2, D, D, kEpiBias, w->bq2, nullptr, q));
+    RTR_TRY(launch_ln_modulate(hidden, nullptr, nullptr, h, ni, D, eps, s, 1));
+    RTR_TRY(gemm(h, 1, w.wq2, D, D, kEpiBias, w.bq2, nullptr, q, 0));
     RTR_TRY_ST(rtr_attn_cross(x, layer, q, ni, o, 0.f, stream));
-    RTR_TRY(gemm(o, w->wo2, D, D, kEpiGatedResidual, w->bo2, nullptr, hidden));
+    RTR_TRY(gemm(o, 0, w.wo2, D, D, kEpiGatedResidual, w.bo2, nullptr, hidden, 0));
     // feed-forward branch
-    RTR_TRY(launch_ln_modulate(hidden, mod + 3 * mrow, mod + 4 * mrow, h, ni, D, eps, s));
-    RTR_TRY(gemm(h, w->w1, F, D, kEpiBiasGelu, w->b1, nullptr, f));
-    RTR_TRY(gemm(f, w->w2, D, F, kEpiGatedResidual, w->b2, mod + 5 * mrow, hidden));
+    RTR_TRY(launch_ln_modulate(hidden, mod + 3 * mrow, mod + 4 * mrow, h, ni, D, eps, s, 1));
+    RTR_TRY(gemm(h, 1, w.w1, F, D, kEpiBiasGelu, w.b1, nullptr, f, f_packed));
+    RTR_TRY(gemm(f, f_packed, w.w2, D, F, kEpiGatedResidual, w.b2, mod + 5 * mrow, hidden, 0));
 #undef RTR_TRY
 #undef RTR_TRY_ST
     return RTR_OK;
+}
+
+}  // namespace
+
+struct rtr_dit_packed {
+    int device, d_model, d_ffn;
+    char *buf = nullptr;   // the six packed matrices, then copies of the six biases
+    DitW w;
+};
+
+extern "C" {
+
+rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer, const rtr_dit_weights *w,
+                                 const void *modulation, void *hidden, int n_cur_frames, int grid_h, int grid_w,
+                                 int t0, int commit, rtr_stream_t stream) {
+    if (!w) return RTR_E_INVAL;
+    DitW dw = {w->wqkv, w->wo, w->wq2, w->wo2, w->w1, w->w2, w->bqkv, w->bo, w->bq2, w->bo2, w->b1, w->b2,
+               w->d_ffn, 0};
+    return dit_block_run(c, x, layer, dw, modulation, hidden, n_cur_frames, grid_h, grid_w, t0, commit, stream);
+}
+
+rtr_status rtr_dit_block_forward_packed(rtr_kvcache *c, const rtr_xattn *x, int layer, const rtr_dit_packed *pw,
+                                        const void *modulation, void *hidden, int n_cur_frames, int grid_h,
+                                        int grid_w, int t0, int commit, rtr_stream_t stream) {
+    if (!pw || !c || pw->device != c->device || pw->d_model != c->heads * c->head_dim) return RTR_E_INVAL;
+    return dit_block_run(c, x, layer, pw->w, modulation, hidden, n_cur_frames, grid_h, grid_w, t0, commit, stream);
+}
+
+rtr_status rtr_dit_pack_weights(const rtr_dit_weights *w, int d_model, int device, rtr_stream_t stream,
+                                rtr_dit_packed **out) {
+    if (!out) return RTR_E_INVAL;
+    *out = nullptr;
+    if (!w || device < 0 || d_model < 64 || d_model % 64 != 0 || w->d_ffn < 64 || w->d_ffn % 64 != 0)
+        return RTR_E_INVAL;
+    for (const void *ptr : {w->wqkv, w->bqkv, w->wo, w->bo, w->wq2, w->bq2, w->wo2, w->bo2, w->w1, w->b1, w->w2,
+                            w->b2})
+        if (!aligned16(ptr)) return RTR_E_INVAL;
+    const int D = d_model, F = w->d_ffn;
+    DeviceGuard dg(device);
+    if (!dg.ok) return RTR_E_INVAL;
+    const cudaStream_t s = (cudaStream_t)stream;
+    // matrices (k, n) and biases (length) in buffer order
+    const int mk[6] = {D, D, D, D, D, F}, mn[6] = {3 * D, D, D, D, F, D};
+    const void *msrc[6] = {w->wqkv, w->wo, w->wq2, w->wo2, w->w1, w->w2};
+    const void *bsrc[6] = {w->bqkv, w->bo, w->bq2, w->bo2, w->b1, w->b2};
+    size_t off[12], total = 0;
+    for (int i = 0; i < 6; ++i) {
+        off[i] = total;
+        total += (packed_b_bytes(mk[i], mn[i]) + 255) & ~size_t(255);
+    }
+    for (int i = 0; i < 6; ++i) {
+        off[6 + i] = total;
+        total += ((size_t)mn[i] * 2 + 255) & ~size_t(255);
+    }
+    rtr_dit_packed *pw = new (std::nothrow) rtr_dit_packed();
+    if (!pw) return RTR_E_NOMEM;
+    void *raw = nullptr;
+    if (lib_malloc(&raw, total) != cudaSuccess) {
+        cudaGetLastError();
+        delete pw;
+        return RTR_E_NOMEM;
+    }
+    pw->buf = static_cast<char *>(raw);
+    pw->device = device;
+    pw->d_model = D;
+    pw->d_ffn = F;
+    cudaError_t e = cudaSuccess;
+    for (int i = 0; i < 6 && e == cudaSuccess; ++i) e = launch_pack_b(msrc[i], pw->buf + off[i], mk[i], mn[i], s);
+    for (int i = 0; i < 6 && e == cudaSuccess; ++i)
+        e = cudaMemcpyAsync(pw->buf + off[6 + i], bsrc[i], (size_t)mn[i] * 2, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(pw->buf);
+        delete pw;
+        return RTR_E_CUDA;
+    }
+    const char *b = pw->buf;
+    pw->w = DitW{b + off[0], b + off[1], b + off[2], b + off[3], b + off[4], b + off[5],
+                 b + off[6], b + off[7], b + off[8], b + off[9], b + off[10], b + off[11], F, 1};
+    *out = pw;
+    return RTR_OK;
+}
+
+void rtr_dit_packed_destroy(rtr_dit_packed *pw) {
+    if (!pw) return;
+    DeviceGuard dg(pw->device);
+    cudaDeviceSynchronize();
+    cudaFree(pw->buf);
+    delete pw;
 }
 
 rtr_status rtr_dit_linear(const void *a, const void *w, int m, int n, int k, rtr_epilogue epilogue, const void *bias,

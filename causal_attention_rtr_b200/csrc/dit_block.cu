@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256) ln_modulate(const __nv_bfloat16 *x, const
 // sums; the normalised, modulated row in one rounding.
 __global__ void __launch_bounds__(1024) ln_modulate_reg(const __nv_bfloat16 *x, const __nv_bfloat16 *shift,
                                                         const __nv_bfloat16 *scale, __nv_bfloat16 *out, int D,
-                                                        float eps) {
+                                                        float eps, int out_packed) {
     __shared__ float red[32];
     const size_t row = blockIdx.x;
     const int nv = D / 8, i = threadIdx.x;
@@ -121,8 +121,23 @@ __global__ void __launch_bounds__(1024) ln_modulate_reg(const __nv_bfloat16 *x, 
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = (f[e] - mean) * rstd;
     }
-    reinterpret_cast<uint4 *>(out + row * D)[i] =
-        make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+    const uint4 v = make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+    if (out_packed)
+        *reinterpret_cast<uint4 *>(reinterpret_cast<char *>(out) + packed_a_offset((long long)row, 8 * i, D)) = v;
+    else
+        reinterpret_cast<uint4 *>(out + row * D)[i] = v;
+}
+
+// One thread per 16-byte piece of w: its 8 n-consecutive elements move to
+// their place in the packed layout.
+__global__ void __launch_bounds__(256) pack_b(const uint4 *w, char *out, int k, int n8) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long long)k * n8) return;
+    const int kr = (int)(idx / n8), c8 = (int)(idx - (long long)kr * n8);
+    const int n = n8 * 8, nc = c8 * 8;
+    const size_t off = ((size_t)(kr / 64) * (size_t)(n / 64) + (size_t)(nc / 64)) * 8192 + (size_t)(kr % 64) * 128 +
+                       (size_t)((((nc % 64) / 8) ^ (kr % 8)) * 16);
+    *reinterpret_cast<uint4 *>(out + off) = w[idx];
 }
 
 cudaError_t launched() {
@@ -134,19 +149,29 @@ cudaError_t launched() {
 }  // namespace
 
 cudaError_t launch_ln_modulate(const void *x, const void *shift, const void *scale, void *out, int n, int D,
-                               float eps, cudaStream_t s) {
+                               float eps, cudaStream_t s, int out_packed) {
     if (n <= 0) return cudaSuccess;
     if (D % 8 != 0 || (scale == nullptr) != (shift == nullptr)) return cudaErrorInvalidValue;
+    if (out_packed && (D % 64 != 0 || D / 8 > 1024)) return cudaErrorInvalidValue;
     if (D / 8 <= 1024) {
         const int threads = (D / 8 + 31) / 32 * 32;
         ln_modulate_reg<<<n, threads, 0, s>>>(
             static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(shift),
-            static_cast<const __nv_bfloat16 *>(scale), static_cast<__nv_bfloat16 *>(out), D, eps);
+            static_cast<const __nv_bfloat16 *>(scale), static_cast<__nv_bfloat16 *>(out), D, eps, out_packed);
         return launched();
     }
     ln_modulate<<<n, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(shift),
                                   static_cast<const __nv_bfloat16 *>(scale), static_cast<__nv_bfloat16 *>(out), D,
                                   eps);
+    return launched();
+}
+
+cudaError_t launch_pack_b(const void *w, void *packed, int k, int n, cudaStream_t s) {
+    if (k <= 0 || n <= 0) return cudaSuccess;
+    if (k % 64 != 0 || n % 64 != 0) return cudaErrorInvalidValue;
+    const long long total = (long long)k * (n / 8);
+    pack_b<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(static_cast<const uint4 *>(w), static_cast<char *>(packed), k,
+                                                            n / 8);
     return launched();
 }
 

@@ -4,12 +4,42 @@
 #pragma once
 #include <cuda_runtime.h>
 
+#include <cstddef>
+
 namespace rtr {
 
+// Tile-packed operand layouts of the tensor-core projection.  Each holds,
+// contiguously, the exact shared-memory image that a 128-byte-swizzled TMA
+// box would produce, so one 1-D bulk copy fills a pipeline stage (a tiled
+// TMA box moves one 128-byte row per request and reaches about half the
+// bulk copy's bytes per clock).
+//
+// Packed A (activations, K contiguous): element (row, col) of an [m][k]
+// matrix, k a multiple of 64, at byte
+//     ((row / 128 * (k / 64) + col / 64) * 128 + row % 128) * 128
+//     + (((col % 64) / 8) ^ (row % 8)) * 16 + (col % 8) * 2,
+// i.e. 16 KB per (128-row tile, 64-column block); ceil(m / 128) row tiles.
+// Packed B (weights [k][n], n contiguous): element (kr, nc) at byte
+//     ((kr / 64 * (n / 64) + nc / 64) * 64 + kr % 64) * 128
+//     + (((nc % 64) / 8) ^ (kr % 8)) * 16 + (nc % 8) * 2,
+// 8 KB per (64-row block of k, 64-column block of n); k and n multiples of 64.
+__host__ __device__ inline size_t packed_a_offset(long long row, int col, int k) {
+    return ((size_t)(row / 128) * (size_t)(k / 64) + (size_t)(col / 64)) * 16384 +
+           (size_t)(row % 128) * 128 + (size_t)((((col % 64) / 8) ^ (int)(row % 8)) * 16) + (size_t)(col % 8) * 2;
+}
+__host__ __device__ inline size_t packed_a_bytes(long long m, int k) {
+    return (size_t)((m + 127) / 128) * (size_t)(k / 64) * 16384;
+}
+__host__ __device__ inline size_t packed_b_bytes(int k, int n) { return (size_t)(k / 64) * (size_t)(n / 64) * 8192; }
+
 // out[i] = LN(x[i]) * (1 + scale) + shift over D channels (eps, no affine);
-// scale / shift null: LN(x[i]) alone.  x, out: [n][D]; scale, shift: [D].
+// scale / shift null: LN(x[i]) alone.  x: [n][D]; scale, shift: [D]; out:
+// [n][D], or packed A (D a multiple of 64) when out_packed != 0.
 cudaError_t launch_ln_modulate(const void *x, const void *shift, const void *scale, void *out, int n, int D,
-                               float eps, cudaStream_t s);
+                               float eps, cudaStream_t s, int out_packed = 0);
+
+// w [k][n] row-major -> packed B (k, n multiples of 64).
+cudaError_t launch_pack_b(const void *w, void *packed, int k, int n, cudaStream_t s);
 
 
 // Epilogues of the tensor-core projection (gemm_tc.cu), applied to the fp32
@@ -25,8 +55,10 @@ cudaError_t launch_ln_modulate(const void *x, const void *shift, const void *sca
 enum { kEpiBias = 0, kEpiBiasGelu = 1, kEpiGatedResidual = 2, kEpiQkvRope = 3 };
 
 struct GemmArgs {
-    const void *a;        // bf16 [m][k], 16-byte aligned
-    const void *w;        // bf16 [k][n] ([in][out]), 16-byte aligned
+    const void *a;        // bf16 [m][k], 16-byte aligned (packed A when a_packed)
+    const void *w;        // bf16 [k][n] ([in][out]), 16-byte aligned (packed B when w_packed)
+    int a_packed, w_packed;   // operand in the tile-packed layout (k, and n for B, multiples of 64)
+    int out_packed;       // kEpiBias / kEpiBiasGelu: out in packed A layout of [m][n] (n a multiple of 64)
     int m, n, k;          // n and k multiples of 8
     int epi;
     const void *bias;     // bf16 [n]

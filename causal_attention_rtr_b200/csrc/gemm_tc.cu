@@ -59,6 +59,10 @@ constexpr float kLog2RopeBase = 13.287712379549449f;   // log2(10000)
 struct GemmParams {
     CUtensorMap tm_a;   // A [m][k]: dims (k, m, 1), box (64, 128, 1)
     CUtensorMap tm_w;   // W [k][n]: dims (n, k, 1), box (64, 64, 1)
+    const char *a_pk;   // packed A (a_packed) or null
+    const char *w_pk;   // packed B (w_packed) or null
+    int kb_total, nb_total;   // k / 64, n / 64 of the packed layouts
+    int out_packed;     // bias / GELU output written in the packed A layout of [m][n]
     int m, n, k;
     int bn, n_tiles_n, n_tiles, k_blocks, stages;
     const __nv_bfloat16 *bias, *gate;
@@ -175,7 +179,11 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
                 r[e] = __uint_as_float(acc[8 * g + e]) + b[e];
                 if (EPI == kEpiBiasGelu) r[e] = gelu_tanh(r[e]);
             }
-            *reinterpret_cast<uint4 *>(o + 8 * g) = pack8(r);
+            if (p.out_packed)
+                *reinterpret_cast<uint4 *>(reinterpret_cast<char *>(p.out) + packed_a_offset(row, col + 8 * g, p.n)) =
+                    pack8(r);
+            else
+                *reinterpret_cast<uint4 *>(o + 8 * g) = pack8(r);
         }
     }
 }
@@ -213,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         mbar_fence_init();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tmap(&p.tm_a);
-        prefetch_tmap(&p.tm_w);
+        if (!p.a_pk) prefetch_tmap(&p.tm_a);
+        if (!p.w_pk) prefetch_tmap(&p.tm_w);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), 512);
@@ -230,9 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         if (lane == 0) {
             int it = 0;                                  // stage loads issued
             bool ok = true;
-            const uint32_t tx = (uint32_t)stage_bytes;
             for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
                 const int m0 = (t / p.n_tiles_n) * kBM, n0 = (t % p.n_tiles_n) * p.bn;
+                // packed B: the tile's 64-column boxes that exist (the rest of
+                // the stage keeps stale data, which reaches only discarded columns)
+                const int w_boxes = p.w_pk ? min(p.bn / 64, p.nb_total - n0 / 64) : p.bn / 64;
+                const uint32_t tx = (uint32_t)(kATileBytes + w_boxes * kBBoxBytes);
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % S, use = it / S;
                     if (use > 0 && !wait_bar(empty(s), (use - 1) & 1, abort_flag)) {
@@ -242,9 +253,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                     }
                     const uint32_t sa = s_base + (uint32_t)(s * stage_bytes);
                     mbar_arrive_tx(full(s), tx);
-                    tma_load_3d(sa, &p.tm_a, full(s), kb * kBK, m0, 0);
-                    for (int j = 0; j < p.bn / 64; ++j)
-                        tma_load_3d(sa + kATileBytes + j * kBBoxBytes, &p.tm_w, full(s), n0 + 64 * j, kb * kBK, 0);
+                    if (p.a_pk)
+                        bulk_load_1d(sa, p.a_pk + ((size_t)(m0 / kBM) * p.kb_total + kb) * kATileBytes, kATileBytes,
+                                     full(s));
+                    else
+                        tma_load_3d(sa, &p.tm_a, full(s), kb * kBK, m0, 0);
+                    if (p.w_pk) {
+                        bulk_load_1d(sa + kATileBytes, p.w_pk + ((size_t)kb * p.nb_total + n0 / 64) * kBBoxBytes,
+                                     (uint32_t)(w_boxes * kBBoxBytes), full(s));
+                    } else {
+                        for (int j = 0; j < p.bn / 64; ++j)
+                            tma_load_3d(sa + kATileBytes + j * kBBoxBytes, &p.tm_w, full(s), n0 + 64 * j, kb * kBK, 0);
+                    }
                 }
             }
             // Loads still in flight land before the CTA can exit: wait for
@@ -388,11 +408,19 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
                                  g.kpf < 1 || g.grid_w < 1))
         return cudaErrorInvalidValue;
     if (!status || sms < 1) return cudaErrorInvalidValue;
+    if ((g.a_packed || g.w_packed) && g.k % 64 != 0) return cudaErrorInvalidValue;
+    if ((g.w_packed || g.out_packed) && g.n % 64 != 0) return cudaErrorInvalidValue;
+    if (g.out_packed && g.epi != kEpiBias && g.epi != kEpiBiasGelu) return cudaErrorInvalidValue;
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    if (!make_tmap_bf16(&p.tm_a, g.a, (uint64_t)g.k, (uint64_t)g.m, 1, kBM, 1) ||
-        !make_tmap_bf16(&p.tm_w, g.w, (uint64_t)g.n, (uint64_t)g.k, 1, kBK, 1))
+    if ((!g.a_packed && !make_tmap_bf16(&p.tm_a, g.a, (uint64_t)g.k, (uint64_t)g.m, 1, kBM, 1)) ||
+        (!g.w_packed && !make_tmap_bf16(&p.tm_w, g.w, (uint64_t)g.n, (uint64_t)g.k, 1, kBK, 1)))
         return cudaErrorInvalidValue;
+    p.a_pk = g.a_packed ? static_cast<const char *>(g.a) : nullptr;
+    p.w_pk = g.w_packed ? static_cast<const char *>(g.w) : nullptr;
+    p.kb_total = g.k / 64;
+    p.nb_total = g.n / 64;
+    p.out_packed = g.out_packed;
     p.m = g.m; p.n = g.n; p.k = g.k;
     p.bn = pick_bn(g.m, g.n, sms);
     p.n_tiles_n = (g.n + p.bn - 1) / p.bn;

@@ -67,6 +67,9 @@ _SIGNATURES = [
     ("rtr_attn_block_causal_prefill_lse", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _i, _vp]),
     ("rtr_dit_block_forward", _i, [_vp, _vp, _i, ctypes.POINTER(DitWeights), _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     ("rtr_attn_block_causal_prefill_cache", _i, [_vp, _i, _vp, _vp, _vp, _i, _i, _vp, _f, _vp]),
+    ("rtr_dit_pack_weights", _i, [ctypes.POINTER(DitWeights), _i, _i, _vp, ctypes.POINTER(_vp)]),
+    ("rtr_dit_packed_destroy", None, [_vp]),
+    ("rtr_dit_block_forward_packed", _i, [_vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     ("rtr_dit_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
     ("rtr_dit_qkv_rope", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
     ("rtr_attn_block_causal_backward", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f,
@@ -258,6 +261,26 @@ def rtr_dit_block_forward(c, x, layer, weights, modulation, hidden, n_cur_frames
                                              n_cur_frames, grid_h, grid_w, t0, 1 if commit else 0,
                                              _stream(stream)),
                   "rtr_dit_block_forward")
+
+
+def rtr_dit_pack_weights(weights, d_model, device=0, stream=None):
+    """Pack a block's weights once (see include/rtr.h); returns the handle."""
+    w = weights if isinstance(weights, DitWeights) else dit_weights(weights, weights["d_ffn"])
+    h = _vp()
+    _check(_lib.rtr_dit_pack_weights(ctypes.byref(w), d_model, device, _stream(stream), ctypes.byref(h)),
+           "rtr_dit_pack_weights")
+    return h.value
+
+
+def rtr_dit_packed_destroy(pw):
+    _lib.rtr_dit_packed_destroy(pw)
+
+
+def rtr_dit_block_forward_packed(c, x, layer, pw, modulation, hidden, n_cur_frames, grid_h, grid_w, t0, commit=False,
+                                 stream=None):
+    return _check(_lib.rtr_dit_block_forward_packed(c, x, layer, pw, _ptr(modulation), _ptr(hidden), n_cur_frames,
+                                                    grid_h, grid_w, t0, int(bool(commit)), _stream(stream)),
+                  "rtr_dit_block_forward_packed")
 
 
 def rtr_dit_linear(a, w, m, n, k, epilogue, bias, gate, out, device=0, stream=None):

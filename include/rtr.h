@@ -358,6 +358,35 @@ rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer,
                                  int n_cur_frames, int grid_h, int grid_w,
                                  int t0, int commit, rtr_stream_t stream);
 
+/* The block's weights packed once for its projections.  Each matrix is
+ * stored as the tensor core's shared-memory tiles, contiguously, so that a
+ * projection moves a stage of weights with one bulk copy instead of one
+ * transfer per 128-byte row (measured on B200: about 81 against 44-49 bytes
+ * per clock per SM).  Weights are fixed during inference, so a caller packs
+ * a block's weights once and passes the handle to every
+ * rtr_dit_block_forward_packed call.  d_model = heads * head_dim and
+ * w->d_ffn must be multiples of 64; pointers as for rtr_dit_block_forward.
+ * The library allocates the packed copy (the six matrices and their biases,
+ * about the size of the weights) on `device`; the call returns once packing
+ * is done, after which the source weights may be freed or changed (the
+ * handle keeps its own copy).  Release with rtr_dit_packed_destroy. */
+typedef struct rtr_dit_packed rtr_dit_packed;
+rtr_status rtr_dit_pack_weights(const rtr_dit_weights *w, int d_model,
+                                int device, rtr_stream_t stream,
+                                rtr_dit_packed **out);
+void rtr_dit_packed_destroy(rtr_dit_packed *pw);
+
+/* rtr_dit_block_forward with weights packed by rtr_dit_pack_weights: the
+ * same block, bit for bit (the projections read identical tiles, only
+ * their transfer differs).  pw must be packed for d_model = heads *
+ * head_dim of c on c's device (else RTR_E_INVAL). */
+rtr_status rtr_dit_block_forward_packed(rtr_kvcache *c, const rtr_xattn *x,
+                                        int layer, const rtr_dit_packed *pw,
+                                        const void *modulation, void *hidden,
+                                        int n_cur_frames, int grid_h,
+                                        int grid_w, int t0, int commit,
+                                        rtr_stream_t stream);
+
 /* The projections of the DiT block, for callers that assemble their own
  * blocks: out = epilogue(a w + bias) on the tensor cores, with the epilogue
  * applied to the fp32 product before anything is stored and each output

@@ -135,6 +135,40 @@ def test_dit_block_parity(case, commit):
         rtr.rtr_crossattn_destroy(x)
 
 
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"H{c[0]}-d{c[1]}-k{c[2] * c[3]}-C{c[9]}")
+def test_dit_block_packed_weights_bit_identical(case):
+    """The block with weights packed once (rtr_dit_pack_weights) gives the
+    same bits as with the row-major weights: the projections read the same
+    tiles, only their transfer differs.  Both match the oracle."""
+    H, d, gh, gw, R, W, appends, T, F, C, t0 = case
+    rtr = _rtr()
+    runs = []
+    for packed in (False, True):
+        c, o, x, ox, w, mod, hidden = _setup(H, d, gh, gw, R, W, appends, T, F, C, seed=H * 100 + d + C + 7)
+        try:
+            tw = {n: dev(a) for n, a in w.items()}
+            tw["d_ffn"] = F
+            th = dev(hidden)
+            if packed:
+                pw = rtr.rtr_dit_pack_weights(tw, H * d, 0)
+                try:
+                    rtr.rtr_dit_block_forward_packed(c, x, 0, pw, dev(mod), th, C, gh, gw, t0, False)
+                    torch.cuda.synchronize()
+                finally:
+                    rtr.rtr_dit_packed_destroy(pw)
+            else:
+                rtr.rtr_dit_block_forward(c, x, 0, tw, dev(mod), th, C, gh, gw, t0, False)
+                torch.cuda.synchronize()
+            runs.append(th)
+            want = db.dit_block(hidden, mod, w, o, ox, C, gh, gw, t0)
+            _check(host_f64(th).reshape(want["out"].shape), want["out"], f"{case} packed={packed}")
+            assert rtr.rtr_get_device_status(0) == rtr.RTR_OK
+        finally:
+            rtr.rtr_kvcache_destroy(c)
+            rtr.rtr_crossattn_destroy(x)
+    assert torch.equal(runs[0].view(torch.int16), runs[1].view(torch.int16))
+
+
 def test_dit_block_fused_commit_equals_append():
     """A cache with commit room writes the chunk from the attention launch;
     the block's output and the committed bytes equal the append path's."""
@@ -199,6 +233,17 @@ def test_full_wan13_block_sampled():
                                | set(np.random.default_rng(9).integers(0, C * gh * gw, 9).tolist())))
         want = db.dit_block(hidden, mod, w, o, ox, C, gh, gw, 22, rows=rows)
         _check(host_f64(th).reshape(C * gh * gw, H * d)[rows], want["out"], "sampled rows")
+        # the same block with packed weights: bit-identical
+        tw = {n: dev(a) for n, a in w.items()}
+        tw["d_ffn"] = F
+        pw = rtr.rtr_dit_pack_weights(tw, H * d, 0)
+        try:
+            th2 = dev(hidden)
+            rtr.rtr_dit_block_forward_packed(c, x, 0, pw, dev(mod), th2, C, gh, gw, 22, False)
+            torch.cuda.synchronize()
+        finally:
+            rtr.rtr_dit_packed_destroy(pw)
+        assert torch.equal(th.view(torch.int16), th2.view(torch.int16))
         assert rtr.rtr_get_device_status(0) == rtr.RTR_OK
     finally:
         rtr.rtr_kvcache_destroy(c)

@@ -150,3 +150,24 @@ def test_dit_projection_validation(lib):
     for args in bad_qkv:
         assert rtr.raw_status("rtr_dit_qkv_rope", *args) == rtr.RTR_E_INVAL, args
     assert rtr.raw_status("rtr_dit_qkv_rope", p, p, p, 0, 64, 2, 64, 16, 4, 0, p, p, p, 0, None) == rtr.RTR_OK
+
+
+def test_dit_packed_validation(lib):
+    """Packing checks its shape and pointers on the host (no GPU needed)."""
+    import ctypes as ct
+    from causal_attention_rtr_b200 import rtr
+    w = rtr.DitWeights(*([256] * 12), 512)
+    h = ct.c_void_p()
+    for d_model in (0, 96, 100):
+        assert rtr.raw_status("rtr_dit_pack_weights", ct.byref(w), d_model, 0, None, ct.byref(h)) == rtr.RTR_E_INVAL
+        assert h.value is None
+    w_bad_ffn = rtr.DitWeights(*([256] * 12), 200)            # d_ffn not a multiple of 64
+    assert rtr.raw_status("rtr_dit_pack_weights", ct.byref(w_bad_ffn), 128, 0, None, ct.byref(h)) == rtr.RTR_E_INVAL
+    w_misaligned = rtr.DitWeights(*([256] * 11 + [258]), 512)
+    assert rtr.raw_status("rtr_dit_pack_weights", ct.byref(w_misaligned), 128, 0, None,
+                          ct.byref(h)) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_dit_pack_weights", ct.byref(w), 128, -1, None, ct.byref(h)) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_dit_pack_weights", ct.byref(w), 128, 0, None, None) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_dit_block_forward_packed", None, None, 0, None, None, None, 1, 1, 1, 0, 0,
+                          None) == rtr.RTR_E_INVAL
+    rtr.rtr_dit_packed_destroy(None)                          # no-op
