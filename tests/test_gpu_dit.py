@@ -7,12 +7,16 @@ Tolerance: the block's output passes through about ten bf16 storage points
 and two attentions; both sides store at the same points, so they differ by
 fp32-versus-fp64 accumulation and the attention's bf16 P.  The bar is the
 attention's relative L2 of 5e-3 and, elementwise, the attention's 2e-2
-absolute or two bf16 units in the last place of the oracle's value,
-whichever is larger.  The residual stream holds values up to about 5, where
-one bf16 ulp is 2^-5 = 0.031: both sides round their fp32 / fp64 sums to
-bf16 at the same point, and where those sums straddle a rounding boundary
-they land one ulp apart, which an absolute 2e-2 would reject although
-neither side is wrong."""
+absolute or four bf16 units in the last place of the oracle's value,
+whichever is larger.  The output is the residual stream after three
+residual additions (gated self attention, cross attention, gated
+feed-forward), each rounded to bf16 on both sides: where the fp32 and fp64
+sums straddle a rounding boundary the stored values land one ulp apart, so
+three additions can leave them three ulps apart, and a flip upstream (the
+layer norms, the projections) can add one more through the branch that
+reads it.  The residual stream holds values up to about 5, where one ulp is
+2^-5 = 0.031, so an absolute 2e-2 would reject results that are right on
+both sides.
 import math
 
 import numpy as np
@@ -45,7 +49,7 @@ def _bf16_ulp(x):
 def _check(got, want, what):
     assert np.all(np.isfinite(got)), what
     rel = float(np.linalg.norm(got - want) / np.linalg.norm(want))
-    bound = np.maximum(2e-2, 2.0 * _bf16_ulp(want))
+    bound = np.maximum(2e-2, 4.0 * _bf16_ulp(want))
     worst = float(np.max(np.abs(got - want) / bound))
     print(f"{what}: rel_l2={rel:.3e} max_abs={float(np.max(np.abs(got - want))):.3e} worst/bound={worst:.3f}")
     assert rel <= 5e-3 and worst <= 1.0, f"{what}: rel_l2={rel:.3e} worst/bound={worst:.3f}"
