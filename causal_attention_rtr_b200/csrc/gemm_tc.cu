@@ -25,16 +25,20 @@
 //               MN-major from 128-byte-swizzled shared memory
 //   warps 2-9   epilogue: two warps per TMEM lane quarter (one thread per
 //               row), each taking alternate 32-column chunks of the tile
-// Two accumulators of up to 256 columns live in TMEM, so the epilogue of
-// one tile overlaps the MMAs of the next.  Tiles are numbered with N
-// fastest and dealt round-robin; the host picks BN in {128, 192, 256} so
-// that the tile count fills the SMs in as few, evenly loaded rounds as it
-// can.  Every wait is bounded (1 s); a timeout latches RTR_E_TIMEOUT in the
+// A tile is 128 rows by BN = 128, 192 or 256 columns, or 256 by 256 (two
+// 128-row sub-tiles whose MMAs share each stage of W).  When a tile's
+// accumulators take at most 256 TMEM columns there are two buffers, so the
+// epilogue of one tile overlaps the MMAs of the next; a 256 x 256 tile fills
+// TMEM and waits for its epilogue.  Tiles are numbered with N fastest and
+// dealt round-robin; the host picks the shape with a cost model (pick_tile).
+// Operands come by TMA boxes from row-major memory, or as whole stages by
+// one bulk copy from the packed layouts (dit_internal.h).  Every wait is bounded (1 s); a timeout latches RTR_E_TIMEOUT in the
 // device status word and every role stops.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -65,6 +69,8 @@ struct GemmParams {
     int out_packed;     // bias / GELU output written in the packed A layout of [m][n]
     int m, n, k;
     int bn, n_tiles_n, n_tiles, k_blocks, stages;
+    int msub;           // 128-row sub-tiles per tile (1 or 2): tiles of 128 * msub rows share each W stage
+    int nbuf;           // accumulator buffers in TMEM (2 when msub * bn <= 256, else 1)
     const __nv_bfloat16 *bias, *gate;
     __nv_bfloat16 *out;                 // bias / GELU: [m][n]; gated residual: [m][n] in place
     __nv_bfloat16 *q, *kk, *v;          // QKV: [m][D] each, D = n / 3
@@ -194,7 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_u32(smem);
     const int S = p.stages;
-    const int stage_bytes = kATileBytes + (p.bn / 64) * kBBoxBytes;
+    const int a_bytes = p.msub * kATileBytes;               // A sub-tiles, then W boxes
+    const int stage_bytes = a_bytes + (p.bn / 64) * kBBoxBytes;
+    const int BMt = kBM * p.msub;                              // rows per tile
     const uint32_t bars = s_base + (uint32_t)(S * stage_bytes);
     // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
     auto full = [&](int s) { return bars + 8u * (uint32_t)s; };
@@ -239,11 +247,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
             int it = 0;                                  // stage loads issued
             bool ok = true;
             for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
-                const int m0 = (t / p.n_tiles_n) * kBM, n0 = (t % p.n_tiles_n) * p.bn;
+                const int m0 = (t / p.n_tiles_n) * BMt, n0 = (t % p.n_tiles_n) * p.bn;
                 // packed B: the tile's 64-column boxes that exist (the rest of
                 // the stage keeps stale data, which reaches only discarded columns)
                 const int w_boxes = p.w_pk ? min(p.bn / 64, p.nb_total - n0 / 64) : p.bn / 64;
-                const uint32_t tx = (uint32_t)(kATileBytes + w_boxes * kBBoxBytes);
+                // A sub-tiles holding rows below m (a sub-tile wholly past m is neither loaded nor multiplied)
+                const int a_subs = min(p.msub, (p.m - m0 + kBM - 1) / kBM);
+                const uint32_t tx = (uint32_t)(a_subs * kATileBytes + w_boxes * kBBoxBytes);
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % S, use = it / S;
                     if (use > 0 && !wait_bar(empty(s), (use - 1) & 1, abort_flag)) {
@@ -253,17 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                     }
                     const uint32_t sa = s_base + (uint32_t)(s * stage_bytes);
                     mbar_arrive_tx(full(s), tx);
-                    if (p.a_pk)
-                        bulk_load_1d(sa, p.a_pk + ((size_t)(m0 / kBM) * p.kb_total + kb) * kATileBytes, kATileBytes,
-                                     full(s));
-                    else
-                        tma_load_3d(sa, &p.tm_a, full(s), kb * kBK, m0, 0);
+                    for (int u = 0; u < a_subs; ++u) {
+                        if (p.a_pk)
+                            bulk_load_1d(sa + u * kATileBytes,
+                                         p.a_pk + ((size_t)(m0 / kBM + u) * p.kb_total + kb) * kATileBytes,
+                                         kATileBytes, full(s));
+                        else
+                            tma_load_3d(sa + u * kATileBytes, &p.tm_a, full(s), kb * kBK, m0 + u * kBM, 0);
+                    }
                     if (p.w_pk) {
-                        bulk_load_1d(sa + kATileBytes, p.w_pk + ((size_t)kb * p.nb_total + n0 / 64) * kBBoxBytes,
+                        bulk_load_1d(sa + a_bytes, p.w_pk + ((size_t)kb * p.nb_total + n0 / 64) * kBBoxBytes,
                                      (uint32_t)(w_boxes * kBBoxBytes), full(s));
                     } else {
                         for (int j = 0; j < p.bn / 64; ++j)
-                            tma_load_3d(sa + kATileBytes + j * kBBoxBytes, &p.tm_w, full(s), n0 + 64 * j, kb * kBK, 0);
+                            tma_load_3d(sa + a_bytes + j * kBBoxBytes, &p.tm_w, full(s), n0 + 64 * j, kb * kBK, 0);
                     }
                 }
             }
@@ -282,13 +295,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
             int it = 0, tc = 0;                          // stages consumed, tiles done
             bool ok = true;
             for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++tc) {
-                const int b = tc & 1, use_b = tc >> 1;
+                const int b = tc % p.nbuf, use_b = tc / p.nbuf;
+                const int m0 = (t / p.n_tiles_n) * BMt;
+                const int a_subs = min(p.msub, (p.m - m0 + kBM - 1) / kBM);
                 if (use_b > 0 && !wait_bar(acce(b), (use_b - 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(b * 256);
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % S;
                     if (!wait_bar(full(s), (it / S) & 1, abort_flag)) {
@@ -297,12 +311,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                     }
                     tc_fence_after();
                     const uint32_t sa = s_base + (uint32_t)(s * stage_bytes);
-                    const uint64_t da = smem_desc_sw128(sa, 16, 1024);
-                    const uint64_t dw = smem_desc_sw128(sa + kATileBytes, kBBoxBytes, 1024);
+                    const uint64_t dw = smem_desc_sw128(sa + a_bytes, kBBoxBytes, 1024);
+                    // sub-tile u accumulates at TMEM column b * 256 + u * bn
+                    for (int u = 0; u < a_subs; ++u) {
+                        const uint64_t da = smem_desc_sw128(sa + u * kATileBytes, 16, 1024);
+                        const uint32_t d_tmem = tmem + (uint32_t)(b * 256 + u * p.bn);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        mma_ss(d_tmem, da + (uint64_t)((kk * 32) >> 4), dw + (uint64_t)((kk * 2048) >> 4), idesc,
-                               (kb > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            mma_ss(d_tmem, da + (uint64_t)((kk * 32) >> 4), dw + (uint64_t)((kk * 2048) >> 4), idesc,
+                                   (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
                     tc_commit(empty(s));
                 }
                 if (!ok) break;
@@ -320,9 +338,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
         int tc = 0;
         bool ok = true;
+        // one sub-tile: the two warps of a lane quarter take alternate 32-column
+        // chunks; two sub-tiles: warp half u takes all chunks of sub-tile u
+        const int sub = p.msub == 2 ? half : 0;
+        const int c_first = p.msub == 2 ? 0 : half, c_step = p.msub == 2 ? 1 : 2;
         for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++tc) {
-            const int b = tc & 1, use_b = tc >> 1;
-            const int m0 = (t / p.n_tiles_n) * kBM, n0 = (t % p.n_tiles_n) * p.bn;
+            const int b = tc % p.nbuf, use_b = tc / p.nbuf;
+            const int m0 = (t / p.n_tiles_n) * BMt, n0 = (t % p.n_tiles_n) * p.bn;
             bool w = wait_bar(accf(b), use_b & 1, abort_flag);
             w = __all_sync(0xffffffffu, w);
             if (!w) {
@@ -330,7 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                 break;
             }
             tc_fence_after();
-            const long long row = (long long)m0 + quarter * 32 + lane;
+            const long long row = (long long)m0 + sub * kBM + quarter * 32 + lane;
+            const bool sub_live = m0 + sub * kBM < p.m;           // warp-uniform
             const bool row_ok = row < p.m;
             int f_pos = 0, y_pos = 0, x_pos = 0;
             if (EPI == kEpiQkvRope) {
@@ -339,11 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                 y_pos = r / p.grid_w;
                 x_pos = r - y_pos * p.grid_w;
             }
-            for (int c = half; c < p.bn / 32; c += 2) {
+            for (int c = c_first; sub_live && c < p.bn / 32; c += c_step) {
                 const int col = n0 + 32 * c;
                 if (col >= p.n) break;                   // warp-uniform
                 uint32_t acc[32];
-                tmem_ld32(tmem + lane_bits + (uint32_t)(b * 256 + 32 * c), acc);
+                tmem_ld32(tmem + lane_bits + (uint32_t)(b * 256 + sub * p.bn + 32 * c), acc);
                 tmem_wait_ld();
                 if (row_ok) epi_chunk<EPI>(p, acc, row, col, min(32, p.n - col), f_pos, y_pos, x_pos);
             }
@@ -369,22 +392,44 @@ cudaError_t set_smem_attr_once() {
     return err;
 }
 
-// Tile width: the candidate whose rounds of `grid` tiles take the least
-// time, counting a tile's time as proportional to BN plus a fixed 32-column
-// cost of its prologue and epilogue hand-off; ties go to the wider tile.
-int pick_bn(int m, int n, int sms) {
-    const int m_tiles = (m + kBM - 1) / kBM;
-    int best = 256;
-    long long best_cost = -1;
-    for (int bn : {256, 192, 128}) {
-        const long long tiles = (long long)m_tiles * ((n + bn - 1) / bn);
-        const long long rounds = (tiles + sms - 1) / sms;
-        const long long cost = rounds * (bn + 32);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best = bn;
+// Tile shape (128 rows by 128, 192 or 256 columns, or 256 by 256): the candidate
+// whose rounds of `sms` tiles take the least time under a model measured on
+// B200.  Per 64-deep K block a tile takes the longer of
+//   its MMAs: 128 x N x 16 costs 85, 106 or 128 cycles for N = 128, 192,
+//     256 (one per k16 step and 128-row sub-tile), and
+//   its loads: stages in flight over a loaded round trip of about 4,400
+//     cycles (the latency times the bandwidth of the memory system reaching
+//     one SM is the shared memory that holds the stages, so a stage's bytes
+//     arrive every latency / stages cycles, whatever their size).
+// A tile whose two accumulators fill TMEM (256 x 256) cannot overlap its
+// epilogue with the next tile's MMAs: it pays about 2,000 more cycles.
+struct TileShape {
+    int msub, bn, stages;
+};
+
+int stage_bytes_of(int msub, int bn) { return msub * kATileBytes + (bn / 64) * kBBoxBytes; }
+
+TileShape pick_tile(int m, int n, int k, int sms) {
+    const int k_blocks = (k + kBK - 1) / kBK;
+    TileShape best = {1, 256, 4};
+    double best_cost = -1.0;
+    // 256-row tiles only with 256 columns: narrower ones load the same A
+    // per K block for less MMA work and never win under this model
+    for (int msub : {2, 1})
+        for (int bn : {256, 192, 128}) {
+            if (msub == 2 && bn != 256) continue;
+            const int stages = std::min(8, kMaxSmem / stage_bytes_of(msub, bn));
+            const double mma = msub * 4.0 * (bn == 256 ? 128.0 : bn == 192 ? 106.0 : 85.0);
+            const double load = 4400.0 / stages;
+            const double epi = msub * bn > 256 ? 2000.0 : 0.0;
+            const long long tiles = (long long)((m + kBM * msub - 1) / (kBM * msub)) * ((n + bn - 1) / bn);
+            const long long rounds = (tiles + sms - 1) / sms;
+            const double cost = rounds * (k_blocks * std::max(mma, load) + epi);
+            if (best_cost < 0 || cost < best_cost * 0.999) {
+                best_cost = cost;
+                best = {msub, bn, stages};
+            }
         }
-    }
     return best;
 }
 
@@ -422,13 +467,15 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
     p.nb_total = g.n / 64;
     p.out_packed = g.out_packed;
     p.m = g.m; p.n = g.n; p.k = g.k;
-    p.bn = pick_bn(g.m, g.n, sms);
+    const TileShape ts = pick_tile(g.m, g.n, g.k, sms);
+    p.msub = ts.msub;
+    p.bn = ts.bn;
+    p.stages = ts.stages;
+    p.nbuf = p.msub * p.bn <= 256 ? 2 : 1;
     p.n_tiles_n = (g.n + p.bn - 1) / p.bn;
-    p.n_tiles = ((g.m + kBM - 1) / kBM) * p.n_tiles_n;
+    p.n_tiles = ((g.m + kBM * p.msub - 1) / (kBM * p.msub)) * p.n_tiles_n;
     p.k_blocks = (g.k + kBK - 1) / kBK;
-    const int stage_bytes = kATileBytes + (p.bn / 64) * kBBoxBytes;
-    p.stages = kMaxSmem / stage_bytes;
-    if (p.stages > 8) p.stages = 8;
+    const int stage_bytes = stage_bytes_of(p.msub, p.bn);
     p.bias = static_cast<const __nv_bfloat16 *>(g.bias);
     p.gate = static_cast<const __nv_bfloat16 *>(g.gate);
     p.out = static_cast<__nv_bfloat16 *>(g.out);
