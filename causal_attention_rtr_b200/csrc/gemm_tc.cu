@@ -402,14 +402,18 @@ cudaError_t set_smem_attr_once() {
 //     one SM is the shared memory that holds the stages, so a stage's bytes
 //     arrive every latency / stages cycles, whatever their size).
 // A tile whose two accumulators fill TMEM (256 x 256) cannot overlap its
-// epilogue with the next tile's MMAs: it pays about 2,000 more cycles.
+// epilogue with the next tile's MMAs: it pays about 2,000 more cycles for a
+// light epilogue (bias, gated residual).  Heavy epilogues (GELU's tanh, the
+// rotary sine and cosine) take longer than that per 256 x 256 tile (the
+// GELU projection measured 184 against 144 us), so they keep 128-row tiles,
+// whose two buffers hide the epilogue behind the next tile's MMAs.
 struct TileShape {
     int msub, bn, stages;
 };
 
 int stage_bytes_of(int msub, int bn) { return msub * kATileBytes + (bn / 64) * kBBoxBytes; }
 
-TileShape pick_tile(int m, int n, int k, int sms) {
+TileShape pick_tile(int m, int n, int k, int sms, bool heavy_epilogue) {
     const int k_blocks = (k + kBK - 1) / kBK;
     TileShape best = {1, 256, 4};
     double best_cost = -1.0;
@@ -417,7 +421,7 @@ TileShape pick_tile(int m, int n, int k, int sms) {
     // per K block for less MMA work and never win under this model
     for (int msub : {2, 1})
         for (int bn : {256, 192, 128}) {
-            if (msub == 2 && bn != 256) continue;
+            if (msub == 2 && (bn != 256 || heavy_epilogue)) continue;
             const int stages = std::min(8, kMaxSmem / stage_bytes_of(msub, bn));
             const double mma = msub * 4.0 * (bn == 256 ? 128.0 : bn == 192 ? 106.0 : 85.0);
             const double load = 4400.0 / stages;
@@ -467,7 +471,7 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
     p.nb_total = g.n / 64;
     p.out_packed = g.out_packed;
     p.m = g.m; p.n = g.n; p.k = g.k;
-    const TileShape ts = pick_tile(g.m, g.n, g.k, sms);
+    const TileShape ts = pick_tile(g.m, g.n, g.k, sms, g.epi == kEpiBiasGelu || g.epi == kEpiQkvRope);
     p.msub = ts.msub;
     p.bn = ts.bn;
     p.stages = ts.stages;

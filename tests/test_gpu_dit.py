@@ -16,7 +16,7 @@ three additions can leave them three ulps apart, and a flip upstream (the
 layer norms, the projections) can add one more through the branch that
 reads it.  The residual stream holds values up to about 5, where one ulp is
 2^-5 = 0.031, so an absolute 2e-2 would reject results that are right on
-both sides.
+both sides."""
 import math
 
 import numpy as np

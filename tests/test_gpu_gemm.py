@@ -86,7 +86,7 @@ LINEAR_CASES = [
     (1000, 1536, 8960, "gated_residual"),   # long K: the feed-forward output projection
     (777, 1536, 1536, "gated_residual_nogate"),
     (4680, 1536, 1536, "bias"),          # the cross-attention query projection
-    (4800, 3072, 512, "gelu"),           # 256-row tiles whose last has a partial second sub-tile
+    (4800, 3072, 512, "bias"),           # 256-row tiles whose last has a partial second sub-tile
 ]
 
 
