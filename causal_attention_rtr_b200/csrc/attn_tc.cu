@@ -91,6 +91,7 @@ constexpr int kPairRows = 2 * kBM;   // query rows per CTA (two tiles)
 constexpr int kThreads = 384;     // 12 warps
 constexpr int kMaxGrid = 160;     // persistent CTAs at most (B200: 148 SMs)
 constexpr uint64_t kWaitNs = 1000000000ull;   // bounded waits: 1 s
+constexpr long long kSplitPenaltyTiles = 15;   // a split unit's extra cost, in key-tile steps (planner)
 
 struct TcParams {
     CUtensorMap tm_q;   // token-major [nq][H][D], box (64, 1, 128)
@@ -1190,10 +1191,30 @@ void plan_attn_bf16(const AttnProblem &p, int sms, int cg, AttnPlan &plan) {
     // A split part costs a Q load and an epilogue: with no full rounds, give
     // each CTA at least 8 key tiles.
     if (plan.full_rounds == 0) budget = std::max<long long>(budget, 8);
+    // The alternative: the remaining units whole, unit i to CTA i (when they
+    // are no more than the CTAs).  Splitting evens the CTAs' totals out, but
+    // every split part pays a work item's fixed cost (its Q load, the first
+    // S before any softmax, its epilogue: measured at roughly 8 key-tile
+    // steps) and the partial results need the combine kernel (about 7 more).
+    // For short units (cross attention over 4 key tiles, single-frame chunks)
+    // whole units finish first.
+    const int R = plan.n_units - plan.full_rounds * G;
+    bool whole = false;
+    if (R > 0 && R <= G) {
+        long long make_whole = 0;
+        for (int c = 0; c < G; ++c)
+            make_whole = std::max(make_whole, load[c] + (c < R ? unit_T(plan.full_rounds * G + c) : 0));
+        whole = make_whole <= budget + kSplitPenaltyTiles;
+    }
     plan.rem_lo.assign(G + 1, 0);
-    for (int c = 0; c < G; ++c) {
-        const long long share = std::max<long long>(0, budget - load[c]);
-        plan.rem_lo[c + 1] = (int)std::min(rem_total, plan.rem_lo[c] + share);
+    if (whole) {
+        for (int c = 0; c < G; ++c)
+            plan.rem_lo[c + 1] = plan.rem_lo[c] + (c < R ? unit_T(plan.full_rounds * G + c) : 0);
+    } else {
+        for (int c = 0; c < G; ++c) {
+            const long long share = std::max<long long>(0, budget - load[c]);
+            plan.rem_lo[c + 1] = (int)std::min(rem_total, plan.rem_lo[c] + share);
+        }
     }
     plan.grid = G;
     if (plan.full_rounds == 0) {

@@ -36,7 +36,7 @@ def _rtr():
 CASES = [
     # n, H, d, k, dtype, oracle rows (None: all)
     (3000, 4, 128, 300, "bf16", None),       # fewer units than SMs: every unit split
-    (10000, 8, 128, 1560, "bf16", 48),       # full rounds plus a split remainder; sampled rows
+    (10000, 8, 128, 1560, "bf16", 48),       # two full rounds, then whole remainder units; sampled rows
     (2000, 3, 64, 250, "bf16", None),        # head_dim 64
     (600, 2, 64, 100, "f32", None),          # fp32 storage: the CUDA-core kernel, no scratch
 ]
