@@ -7,9 +7,9 @@ against the fp64 oracle at the attention tolerance, and bit for bit against
 rtr_attn_block_causal_prefill on the same inputs: both entry points plan and
 launch the same kernels, so a stale partial result left in the shared array
 by the first call, or a merge that reads the wrong part, shows as a
-difference.  The bf16 shapes split attention units across SMs, so the static
-scratch is written and read; head_dim 64 and the fp32 path (which needs no
-scratch) are covered too.  A separate test checks that a call allocates
+difference.  The first shape splits attention units across SMs, so the
+static scratch is written and read; head_dim 64 and the fp32 path (which
+needs no scratch) are covered too.  A separate test checks that a call allocates
 nothing (device free memory is unchanged across it) and that bad arguments
 are rejected.
 
@@ -35,7 +35,7 @@ def _rtr():
 
 CASES = [
     # n, H, d, k, dtype, oracle rows (None: all)
-    (3000, 4, 128, 300, "bf16", None),       # fewer units than SMs: every unit split
+    (3000, 4, 128, 300, "bf16", None),       # fewer units than SMs: the long ones split over CTAs
     (10000, 8, 128, 1560, "bf16", 48),       # two full rounds, then whole remainder units; sampled rows
     (2000, 3, 64, 250, "bf16", None),        # head_dim 64
     (600, 2, 64, 100, "f32", None),          # fp32 storage: the CUDA-core kernel, no scratch
