@@ -192,6 +192,7 @@ struct Sched {
     int r = 0, ru = 0;
     long long U = 0;
     bool first_rem = true;
+    bool placed = false;   // remainder walk moved to this CTA's first unit
 };
 
 template <int CG>
@@ -211,6 +212,23 @@ __device__ bool sched_next(const TcParams &p, Sched &s, Item &it) {
     }
     const long long lo = p.rem_lo[c];
     const long long hi = p.rem_lo[c + 1];
+    if (!s.placed) {
+        // Jump to the last remainder unit that starts at or before this CTA's
+        // first tile (binary search of the tile prefix): the units before it
+        // end at or before `lo`.  Walking them one by one cost a few hundred
+        // cycles each, tens of microseconds for the last CTAs of a launch.
+        s.placed = true;
+        const int base = s.ru;
+        int a = 0, b = p.n_units - base;   // rem_U[a] <= lo; answer in [a, b)
+        if (b > 0) {
+            while (b - a > 1) {
+                const int m = (a + b) >> 1;
+                if (p.rem_U[m] <= lo) a = m; else b = m;
+            }
+            s.ru = base + a;
+            s.U = p.rem_U[a];
+        }
+    }
     while (s.ru < p.n_units && s.U < hi) {
         int pair, head;
         unit_coords(p, s.ru, pair, head);
