@@ -16,20 +16,22 @@
 //               L +inf, so padded query rows carry exactly zero probability).
 //   bwd_dkdv    key-stationary: one CTA per (head, 128-key tile); streams the
 //               query tiles that see it (frame-causal: query frames >= the
-//               key tile's first frame), each as two halves of 64 queries.
-//               Per half: S^T = K Q^T and dP^T = V dO^T into one of two TMEM
-//               buffers, the softmax warps turn them into P^T and dS^T (bf16,
-//               back into TMEM), then dV += P^T dO and dK += dS^T Q with the
-//               "A in tensor memory" form; the tensor core runs the other
-//               buffer's MMAs meanwhile.
+//               key tile's first frame).  Per query tile: S^T = K Q^T and
+//               dP^T = V dO^T into TMEM (N = 128: the 64-wide forms of an
+//               earlier half-tile version ran at a third of the tensor
+//               core's rate); the softmax warps read the S^T row into
+//               registers at once, which frees its columns for the next
+//               tile's S^T, then write P^T and dS^T (bf16) over the dP^T
+//               columns they have read; dV += P^T dO and dK += dS^T Q with
+//               the "A in tensor memory" form, the first 64 queries' part
+//               while the softmax does the other 64.
 //   bwd_dq      query-stationary: one CTA per (head, 128-query tile); streams
-//               the key tiles it sees.  S = Q K^T and dP = dO V^T into TMEM,
-//               dS (bf16) back into TMEM, dQ += dS K.  S has two TMEM
-//               buffers, so S of the next key tile runs during this tile's
-//               softmax; dP has one (dS lives in it until dQ has read it).
-//               (bwd_dkdv's half-tile scheme measured 14 % slower here: its
-//               64-wide S and dP MMAs re-read Q and dO per half, and each
-//               half pays the softmax hand-off again.)
+//               the key tiles it sees (K through 3 shared-memory slots, V
+//               through 2).  S = Q K^T into one of two TMEM buffers and
+//               dP = dO V^T into one; the softmax reads the dP row into
+//               registers at once, which frees dP's columns for the next
+//               tile's dP, and writes dS (bf16) over S's columns; dQ += dS K,
+//               the first 64 keys' part while the softmax does the rest.
 // Splitting dQ from dK/dV recomputes S and dP once more (7 tile MMAs per
 // (query tile, key tile) instead of 5) but needs no atomic accumulation of
 // dQ across CTAs: every output tile is written once, in bf16, by TMA.
@@ -54,6 +56,7 @@ namespace rtr {
 namespace {
 
 constexpr int kBT = 128;                  // rows of every tile
+constexpr int kHalf = 64;                 // query columns after which bwd_dkdv starts dV / dK
 constexpr int kBwdThreads = 256;
 constexpr uint64_t kBwdWaitNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -74,22 +77,45 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
                  : "memory");
 }
 
-// Shared-memory layout of both main kernels: two stationary tiles A0, A1
-// (dkdv: K, V; dq: Q, dO), two stages of two streamed tiles B0, B1 (dkdv: Q,
-// dO; dq: K, V) plus, per stage, 128 floats each of L*log2e and Delta
-// (dkdv only), then the barriers.
+// Shared memory of bwd_dkdv: the stationary K and V tiles, then two stages
+// of one streamed query tile each (Q and dO, 128 rows, plus 128 floats each
+// of L*log2e and Delta), then the barriers.
 template <int D>
-struct BwdLayout {
-    static constexpr int kTile = kBT * D * 2;
-    static constexpr int kA = 0;                         // A0, A1
-    static constexpr int kStage = 2 * kTile + 1024;      // B0, B1, row stats
-    static constexpr int kB = 2 * kTile;                 // stage s at kB + s * kStage
+struct DkdvLayout {
+    static constexpr int kTile = kBT * D * 2;             // K, V, Q or dO
+    static constexpr int kA = 0;                          // K, V
+    static constexpr int kStage = 2 * kTile + 1024;       // Q, dO, L2[128], Delta[128]
+    static constexpr int kB = 2 * kTile;                  // stage s at kB + s * kStage
     static constexpr int kBars = kB + 2 * kStage;
-    static constexpr int bA = 0, bFull = 1, bEmpty = 3, bS = 5, bP = 7, bO = 9, bEpi = 10, kNumBars = 11;
+    static constexpr int bA = 0, bFull = 1, bEmpty = 3, bS = 5, bSread = 6, bPh = 7, bP = 8, bO = 9, bEpi = 10,
+                         kNumBars = 11;
     static constexpr int kMisc = kBars + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
 };
+static_assert(DkdvLayout<128>::kAlloc <= 232448, "bwd_dkdv shared memory");
+
+// Shared memory of bwd_dq: the stationary Q and dO tiles, then separate
+// rings for K (3 slots) and V (2 slots).  K(t) is read by S(t) and by
+// dQ(t), the last MMA of step t, so its slot frees late; a third K slot
+// lets the load of K(t+3) start a full step before S(t+3) wants it.  V(t)
+// is read by dP(t) alone and frees a step earlier, so two slots suffice.
+template <int D>
+struct DqLayout {
+    static constexpr int kTile = kBT * D * 2;
+    static constexpr int kKSlots = 3, kVSlots = 2;
+    static constexpr int kA = 0;                          // Q, dO
+    static constexpr int kK = 2 * kTile;                  // K slot s at kK + s * kTile
+    static constexpr int kV = kK + kKSlots * kTile;       // V slot s at kV + s * kTile
+    static constexpr int kBars = kV + kVSlots * kTile;
+    static constexpr int bA = 0, bKFull = 1, bKEmpty = bKFull + kKSlots, bVFull = bKEmpty + kKSlots,
+                         bVEmpty = bVFull + kVSlots, bS = bVEmpty + kVSlots, bDPread = bS + 1, bPh = bDPread + 1,
+                         bP = bPh + 1, bO = bP + 1, bEpi = bO + 1, kNumBars = bEpi + 1;
+    static constexpr int kMisc = kBars + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+static_assert(DqLayout<128>::kAlloc <= 232448, "bwd_dq shared memory");
 
 __device__ __forceinline__ void bwd_timeout(const BwdParams &p, volatile int *abort_flag) {
     *abort_flag = 1;
@@ -114,18 +140,7 @@ __device__ __forceinline__ void mma_tile_ss(uint32_t d_tmem, uint64_t a0, uint64
     }
 }
 
-// TS MMA chain over KR rows of B: C[128 x D] (+)= A[128 x KR] B[KR x D] with
-// A packed bf16 pairs in TMEM at a_tmem (8 columns per 16 rows of B) and B
-// read as MN-major from the TMA layout (16 rows = 2048 bytes per step).
-template <int D, int KR>
-__device__ __forceinline__ void mma_tile_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
-                                            bool acc) {
-#pragma unroll
-    for (int kk = 0; kk < KR / 16; ++kk)
-        mma_ts(d_tmem, a_tmem + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc, (acc || kk > 0) ? 1u : 0u);
-}
 
-constexpr int kHalf = 64;     // rows of the streamed half tile (MMA N of S / dP)
 
 // Epilogue: 128 x D fp32 accumulator rows (this thread's TMEM lane) times
 // `mul`, to bf16 in the swizzled TMA layout at `dst`.
@@ -182,32 +197,42 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16 *o, const __
     }
 }
 
-// Packed P / dS for 32 columns of one row: p = exp2(s * sl2 - l2) (0 where
-// masked), ds = p * (dp - delta).  `l2`, `dl` are per column (dkdv) or
-// broadcast scalars (dq), chosen by the caller through the arrays.
-__device__ __forceinline__ void p_ds_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float (&l2)[32],
-                                           const float (&dl)[32], float sl2, int lo, int hi, uint32_t (&pk)[16],
-                                           uint32_t (&dk)[16]) {
+
+// ---------------------------------------------------------------- dK, dV
+// P^T and dS^T for 32 query columns [32c, 32c+32) of one key row, written
+// packed as bf16 pairs: p = exp2(s * sl2 - l2) (0 for columns below `lo`),
+// ds = p * (dp - delta), with L*log2e and Delta of each column read from
+// shared memory (broadcast: every thread reads the same column).
+__device__ __forceinline__ void pt_dst_chunk(const uint32_t (&s)[128], int c, const uint32_t (&dp)[32],
+                                             const float *l2s, const float *dls, float sl2, int lo,
+                                             uint32_t (&pk)[16], uint32_t (&dk)[16]) {
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        float p0 = fast_exp2(fmaf(__uint_as_float(s[e]), sl2, -l2[e]));
-        float p1 = fast_exp2(fmaf(__uint_as_float(s[e + 1]), sl2, -l2[e + 1]));
-        p0 = (e >= lo && e < hi) ? p0 : 0.f;
-        p1 = (e + 1 >= lo && e + 1 < hi) ? p1 : 0.f;
-        pk[e / 2] = pack_bf16x2(p0, p1);
-        dk[e / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[e]) - dl[e]), p1 * (__uint_as_float(dp[e + 1]) - dl[e + 1]));
+    for (int e = 0; e < 32; e += 4) {
+        const float4 l = *reinterpret_cast<const float4 *>(l2s + 32 * c + e);
+        const float4 d = *reinterpret_cast<const float4 *>(dls + 32 * c + e);
+        const float le[4] = {l.x, l.y, l.z, l.w}, de[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int u = 0; u < 4; u += 2) {
+            const int col = e + u;
+            float p0 = fast_exp2(fmaf(__uint_as_float(s[32 * c + col]), sl2, -le[u]));
+            float p1 = fast_exp2(fmaf(__uint_as_float(s[32 * c + col + 1]), sl2, -le[u + 1]));
+            p0 = col >= lo ? p0 : 0.f;
+            p1 = col + 1 >= lo ? p1 : 0.f;
+            pk[col / 2] = pack_bf16x2(p0, p1);
+            dk[col / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[col]) - de[u]),
+                                      p1 * (__uint_as_float(dp[col + 1]) - de[u + 1]));
+        }
     }
 }
 
-// ---------------------------------------------------------------- dK, dV
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant__ BwdParams p) {
-    using L = BwdLayout<D>;
+    using L = DkdvLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_u32(smem);
     const uint32_t sK = s_base + L::kA, sV = sK + L::kTile;
-    auto stage_b = [&](int st) { return s_base + L::kB + st * L::kStage; };   // Q, dO, L2[128], Delta[128]
+    auto stage_b = [&](int t) { return s_base + L::kB + (t & 1) * L::kStage; };   // Q, dO, L2[128], Delta[128]
     const uint32_t bars = s_base + L::kBars;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L::kMisc);
@@ -226,10 +251,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
             mbar_init(bar(L::bFull + s), 1);
             mbar_init(bar(L::bEmpty + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar(L::bS + b), 1);
-            mbar_init(bar(L::bP + b), 4);
-        }
+        mbar_init(bar(L::bS), 1);
+        mbar_init(bar(L::bSread), 4);
+        mbar_init(bar(L::bPh), 4);
+        mbar_init(bar(L::bP), 4);
         mbar_init(bar(L::bO), 1);
         mbar_init(bar(L::bEpi), kBT);
         *abort_flag = 0;
@@ -243,11 +268,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    // TMEM: S^T / P^T buffers [0,64), [64,128); dP^T / dS^T buffers [128,192),
-    // [192,256); dV [256,256+D); dK [256+D,256+2D).  Each streamed query tile
-    // is taken as two halves of 64 queries (step t: tile t/2, half t%2,
-    // buffer t%2): while the softmax works on step t the tensor core runs
-    // dV/dK of step t-1 and S^T/dP^T of step t+1.
+    // TMEM: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D).
+    // Step t (query tile i_first + t): the softmax reads the whole S^T row
+    // into registers first, so S^T(t+1) can be computed into [0,128) while
+    // it works; P^T and dS^T of each 32-column group c go, packed, into the
+    // dP^T columns [128+32c, 128+32c+32) the group has just read (P^T in
+    // the first 16, dS^T in the last 16).  dV and dK of the first 64 query
+    // columns start while the softmax does the other 64; dP^T(t+1) follows
+    // the last of them.
 
     if (warp == 0) {
         if (lane == 0) {
@@ -262,7 +290,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
                 }
                 if (*abort_flag) break;
                 const int i = i_first + t;
-                const uint32_t sb = stage_b(st);
+                const uint32_t sb = stage_b(t);
                 mbar_arrive_tx(bar(L::bFull + st), 2 * L::kTile + 1024);
                 load_tile<D>(sb, &p.tm_q, bar(L::bFull + st), head, i * kBT);
                 load_tile<D>(sb + L::kTile, &p.tm_do, bar(L::bFull + st), head, i * kBT);
@@ -274,37 +302,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, 0, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBT, D, 0, 1);
             const uint64_t descK = smem_desc_sw128(sK, 16, 1024), descV = smem_desc_sw128(sV, 16, 1024);
-            constexpr uint32_t idesc_h = idesc_bf16_f32(kBT, kHalf, 0, 0);
-            bool ok = mbar_wait(bar(L::bA), 0, kBwdWaitNs);
-            for (int t = 0; ok && t <= 2 * T; ++t) {
-                if (t < 2 * T) {
-                    const int ti = t >> 1, h = t & 1, b = t & 1;
-                    const uint32_t sb = stage_b(ti & 1);
-                    if (h == 0) {
-                        ok = mbar_wait(bar(L::bFull + (ti & 1)), (ti >> 1) & 1, kBwdWaitNs) && !*abort_flag;
-                        if (!ok) break;
-                    }
-                    tc_fence_after();
-                    const uint32_t hoff = (uint32_t)(h * kHalf * 128);
-                    mma_tile_ss<D>(tmem + 64 * b, descK, smem_desc_sw128(sb + hoff, 16, 1024), idesc_h);   // S^T
-                    mma_tile_ss<D>(tmem + 128 + 64 * b, descV, smem_desc_sw128(sb + L::kTile + hoff, 16, 1024),
-                                   idesc_h);                                                           // dP^T
-                    tc_commit(bar(L::bS + b));
+            auto full = [&](int t) {
+                return mbar_wait(bar(L::bFull + (t & 1)), (t >> 1) & 1, kBwdWaitNs) && !*abort_flag;
+            };
+            // dV += P^T dO and dK += dS^T Q over query rows [64h, 64h+64) of step t
+            auto dvdk_half = [&](int t, int h) {
+                const uint32_t sb = stage_b(t);
+#pragma unroll
+                for (int kk = 0; kk < kHalf / 16; ++kk) {
+                    const int q16 = h * (kHalf / 16) + kk;                       // 16-row group of queries
+                    const uint32_t col = 128 + 32 * (q16 >> 1) + 8 * (q16 & 1);  // its packed P^T columns
+                    const uint32_t acc = (t > 0 || q16 > 0) ? 1u : 0u;
+                    const uint64_t rows = (uint64_t)((q16 * 2048) >> 4);
+                    mma_ts(tmem + 256, tmem + col, smem_desc_sw128(sb + L::kTile, 16384, 1024) + rows, idesc_o, acc);
+                    mma_ts(tmem + 256 + D, tmem + col + 16, smem_desc_sw128(sb, 16384, 1024) + rows, idesc_o, acc);
                 }
-                if (t >= 1) {
-                    const int tp = t - 1, ti = tp >> 1, h = tp & 1, b = tp & 1;
-                    const uint32_t sb = stage_b(ti & 1);
-                    ok = mbar_wait(bar(L::bP + b), (tp >> 1) & 1, kBwdWaitNs) && !*abort_flag;
+            };
+            bool ok = mbar_wait(bar(L::bA), 0, kBwdWaitNs) && full(0);
+            if (ok) {
+                tc_fence_after();
+                mma_tile_ss<D>(tmem + 0, descK, smem_desc_sw128(stage_b(0), 16, 1024), idesc_s);              // S^T(0)
+                mma_tile_ss<D>(tmem + 128, descV, smem_desc_sw128(stage_b(0) + L::kTile, 16, 1024), idesc_s); // dP^T(0)
+                tc_commit(bar(L::bS));
+            }
+            for (int t = 0; ok && t < T; ++t) {
+                ok = mbar_wait(bar(L::bSread), t & 1, kBwdWaitNs) && !*abort_flag;
+                if (!ok) break;
+                if (t + 1 < T) {
+                    ok = full(t + 1);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t hoff = (uint32_t)(h * kHalf * 128);
-                    mma_tile_ts<D, kHalf>(tmem + 256, tmem + 64 * b, smem_desc_sw128(sb + L::kTile + hoff, 16384, 1024),
-                                          idesc_o, tp > 0);                                    // dV += P^T dO
-                    mma_tile_ts<D, kHalf>(tmem + 256 + D, tmem + 128 + 64 * b, smem_desc_sw128(sb + hoff, 16384, 1024),
-                                          idesc_o, tp > 0);                                    // dK += dS^T Q
-                    if (h == 1) tc_commit(bar(L::bEmpty + (ti & 1)));
+                    mma_tile_ss<D>(tmem + 0, descK, smem_desc_sw128(stage_b(t + 1), 16, 1024), idesc_s);      // S^T(t+1)
+                }
+                ok = mbar_wait(bar(L::bPh), t & 1, kBwdWaitNs) && !*abort_flag;
+                if (!ok) break;
+                tc_fence_after();
+                dvdk_half(t, 0);
+                ok = mbar_wait(bar(L::bP), t & 1, kBwdWaitNs) && !*abort_flag;
+                if (!ok) break;
+                tc_fence_after();
+                dvdk_half(t, 1);
+                tc_commit(bar(L::bEmpty + (t & 1)));   // Q(t), dO(t) read by their last MMAs
+                if (t + 1 < T) {
+                    mma_tile_ss<D>(tmem + 128, descV, smem_desc_sw128(stage_b(t + 1) + L::kTile, 16, 1024),
+                                   idesc_s);                                                               // dP^T(t+1)
+                    tc_commit(bar(L::bS));
                 }
             }
             if (!ok) bwd_timeout(p, abort_flag);
@@ -315,43 +360,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
         const uint32_t lane_bits = (uint32_t)(sub * 32) << 16;
+        const uint32_t tS = tmem + lane_bits, tdP = tS + 128;
         const int kr = kt * kBT + row;                     // key row
         const int q_lo = (kr / p.kpf) * p.kpf;             // first query row that sees it
         bool ok = true;
-        for (int t = 0; t < 2 * T; ++t) {
-            const int ti = t >> 1, h = t & 1, b = t & 1;
-            const int i = i_first + ti;
-            const float *l2s =
-                reinterpret_cast<const float *>(smem + L::kB + (ti & 1) * L::kStage + 2 * L::kTile) + h * kHalf;
-            const float *dls = l2s + 128;
-            const uint32_t tS = tmem + lane_bits + 64 * b, tdP = tS + 128;
-            bool w = !*abort_flag && mbar_wait(bar(L::bS + b), (t >> 1) & 1, kBwdWaitNs);
+        for (int t = 0; t < T; ++t) {
+            const int i = i_first + t;
+            const float *l2s = reinterpret_cast<const float *>(smem + L::kB + (t & 1) * L::kStage + 2 * L::kTile);
+            const float *dls = l2s + kBT;
+            bool w = !*abort_flag && mbar_wait(bar(L::bS), t & 1, kBwdWaitNs);
             w = __all_sync(0xffffffffu, w);
             if (!w) { ok = false; break; }
             tc_fence_after();
-            const int lo = q_lo - i * kBT - h * kHalf;     // columns below lo are hidden from this key
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-                uint32_t s[32], dp[32], pk[16], dk[16];
-                float l2[32], dl[32];
-                tmem_ld32(tS + 32 * c, s);
-                tmem_ld32(tdP + 32 * c, dp);
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    const float4 a = *reinterpret_cast<const float4 *>(l2s + 32 * c + e);
-                    const float4 bq = *reinterpret_cast<const float4 *>(dls + 32 * c + e);
-                    l2[e] = a.x; l2[e + 1] = a.y; l2[e + 2] = a.z; l2[e + 3] = a.w;
-                    dl[e] = bq.x; dl[e + 1] = bq.y; dl[e + 2] = bq.z; dl[e + 3] = bq.w;
-                }
-                tmem_wait_ld();
-                p_ds_chunk(s, dp, l2, dl, p.scale_log2, lo - 32 * c, 32, pk, dk);
-                tmem_st16(tS + 16 * c, pk);
-                tmem_st16(tdP + 16 * c, dk);
-            }
-            tmem_wait_st();
+            uint32_t sr[128];
+            tmem_ld128(tS, sr);
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::bP + b));
+            if (lane == 0) mbar_arrive(bar(L::bSread));   // S^T's columns are free for S^T(t+1)
+            const int lo = q_lo - i * kBT;                 // columns below lo are hidden from this key
+#pragma unroll   // constant c: the row stays in registers
+            for (int c = 0; c < 4; ++c) {
+                uint32_t dp[32], pk[16], dk[16];
+                tmem_ld32(tdP + 32 * c, dp);
+                tmem_wait_ld();
+                pt_dst_chunk(sr, c, dp, l2s, dls, p.scale_log2, lo - 32 * c, pk, dk);
+                tmem_st16(tdP + 32 * c, pk);
+                tmem_st16(tdP + 32 * c + 16, dk);
+                if (c == 1 || c == 3) {
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(c == 1 ? L::bPh : L::bP));
+                }
+            }
         }
         // epilogue: dV -> V's tile, dK * scale -> K's tile, then TMA stores
         bool w = ok && !*abort_flag && mbar_wait(bar(L::bO), 0, kBwdWaitNs);
@@ -386,14 +428,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
 }
 
 // ---------------------------------------------------------------- dQ
+// dS for 32 key columns [32c, 32c+32) of one query row, packed as bf16
+// pairs: p = exp2(s * sl2 - l2) (0 for columns at or past `hi`),
+// ds = p * (dp - delta), dp from the row's registers.
+__device__ __forceinline__ void ds_chunk(const uint32_t (&s)[32], const uint32_t (&dpr)[128], int c, float l2,
+                                         float dl, float sl2, int hi, uint32_t (&dk)[16]) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float p0 = fast_exp2(fmaf(__uint_as_float(s[e]), sl2, -l2));
+        float p1 = fast_exp2(fmaf(__uint_as_float(s[e + 1]), sl2, -l2));
+        p0 = e < hi ? p0 : 0.f;
+        p1 = e + 1 < hi ? p1 : 0.f;
+        dk[e / 2] = pack_bf16x2(p0 * (__uint_as_float(dpr[32 * c + e]) - dl),
+                                p1 * (__uint_as_float(dpr[32 * c + e + 1]) - dl));
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__ BwdParams p) {
-    using L = BwdLayout<D>;
+    using L = DqLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_u32(smem);
     const uint32_t sQ = s_base + L::kA, sdO = sQ + L::kTile;
-    auto stage_b = [&](int st) { return s_base + L::kB + st * L::kStage; };   // K, V
+    auto k_slot = [&](int t) { return s_base + L::kK + (t % L::kKSlots) * L::kTile; };
+    auto v_slot = [&](int t) { return s_base + L::kV + (t % L::kVSlots) * L::kTile; };
     const uint32_t bars = s_base + L::kBars;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L::kMisc);
@@ -408,11 +467,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
 
     if (threadIdx.x == 0) {
         mbar_init(bar(L::bA), 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(L::bFull + s), 1);
-            mbar_init(bar(L::bEmpty + s), 1);
+        for (int s = 0; s < L::kKSlots; ++s) {
+            mbar_init(bar(L::bKFull + s), 1);
+            mbar_init(bar(L::bKEmpty + s), 1);
         }
-        mbar_init(bar(L::bS), 1);   // one S / dP buffer: bS + 0, bP + 0
+        for (int s = 0; s < L::kVSlots; ++s) {
+            mbar_init(bar(L::bVFull + s), 1);
+            mbar_init(bar(L::bVEmpty + s), 1);
+        }
+        mbar_init(bar(L::bS), 1);
+        mbar_init(bar(L::bDPread), 4);
+        mbar_init(bar(L::bPh), 4);
         mbar_init(bar(L::bP), 4);
         mbar_init(bar(L::bO), 1);
         mbar_init(bar(L::bEpi), kBT);
@@ -427,8 +492,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    // TMEM: S buffers [0,128), [128,256) (tile t in buffer t % 2); dP / dS
-    // [256,384); dQ [384,384+D).
+    // TMEM: S buffers [0,128), [128,256) (key tile t in buffer t % 2; its dS
+    // is written, packed, over the first 16 of each 32-column group of S it
+    // came from); dP [256,384); dQ [384,384+D).  The softmax reads the whole
+    // dP row into registers first, so dP(t+1) is computed while it works;
+    // S(t+1) runs earlier still.  dQ of the first 64 keys starts while the
+    // softmax does the other 64.
 
     if (warp == 0) {
         if (lane == 0) {
@@ -436,16 +505,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
             load_tile<D>(sQ, &p.tm_q, bar(L::bA), head, qt * kBT);
             load_tile<D>(sdO, &p.tm_do, bar(L::bA), head, qt * kBT);
             for (int t = 0; t < T; ++t) {
-                const int st = t & 1, use = t >> 1;
-                if (use > 0 && !mbar_wait(bar(L::bEmpty + st), (use - 1) & 1, kBwdWaitNs)) {
+                const int ks = t % L::kKSlots, ku = t / L::kKSlots;
+                if (ku > 0 && !mbar_wait(bar(L::bKEmpty + ks), (ku - 1) & 1, kBwdWaitNs)) {
                     bwd_timeout(p, abort_flag);
                     break;
                 }
                 if (*abort_flag) break;
-                const uint32_t sb = stage_b(st);
-                mbar_arrive_tx(bar(L::bFull + st), 2 * L::kTile);
-                load_tile<D>(sb, &p.tm_k, bar(L::bFull + st), head, t * kBT);
-                load_tile<D>(sb + L::kTile, &p.tm_v, bar(L::bFull + st), head, t * kBT);
+                mbar_arrive_tx(bar(L::bKFull + ks), L::kTile);
+                load_tile<D>(k_slot(t), &p.tm_k, bar(L::bKFull + ks), head, t * kBT);
+                const int vs = t % L::kVSlots, vu = t / L::kVSlots;
+                if (vu > 0 && !mbar_wait(bar(L::bVEmpty + vs), (vu - 1) & 1, kBwdWaitNs)) {
+                    bwd_timeout(p, abort_flag);
+                    break;
+                }
+                if (*abort_flag) break;
+                mbar_arrive_tx(bar(L::bVFull + vs), L::kTile);
+                load_tile<D>(v_slot(t), &p.tm_v, bar(L::bVFull + vs), head, t * kBT);
             }
         }
         __syncwarp();
@@ -454,34 +529,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, 0, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBT, D, 0, 1);
             const uint64_t descQ = smem_desc_sw128(sQ, 16, 1024), descdO = smem_desc_sw128(sdO, 16, 1024);
-            // S(t+1) goes into the other S buffer while the softmax works on
-            // tile t; dP(t+1) follows dQ(t), which reads dS(t) from dP's columns.
-            bool ok = mbar_wait(bar(L::bA), 0, kBwdWaitNs) &&
-                      mbar_wait(bar(L::bFull + 0), 0, kBwdWaitNs) && !*abort_flag;
+            auto k_full = [&](int t) {
+                return mbar_wait(bar(L::bKFull + t % L::kKSlots), (t / L::kKSlots) & 1, kBwdWaitNs) && !*abort_flag;
+            };
+            auto v_full = [&](int t) {
+                return mbar_wait(bar(L::bVFull + t % L::kVSlots), (t / L::kVSlots) & 1, kBwdWaitNs) && !*abort_flag;
+            };
+            // dQ += dS K over keys [64h, 64h+64) of tile t
+            auto dq_half = [&](int t, int h) {
+                const uint32_t buf = 128 * (t & 1);
+#pragma unroll
+                for (int kk = 0; kk < kHalf / 16; ++kk) {
+                    const int k16 = h * (kHalf / 16) + kk;                       // 16-key group
+                    const uint32_t col = buf + 32 * (k16 >> 1) + 8 * (k16 & 1);  // its packed dS columns
+                    mma_ts(tmem + 384, tmem + col,
+                           smem_desc_sw128(k_slot(t), 16384, 1024) + (uint64_t)((k16 * 2048) >> 4), idesc_o,
+                           (t > 0 || k16 > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(bar(L::bA), 0, kBwdWaitNs) && k_full(0) && v_full(0);
             if (ok) {
                 tc_fence_after();
-                mma_tile_ss<D>(tmem + 0, descQ, smem_desc_sw128(stage_b(0), 16, 1024), idesc_s);                  // S(0)
-                mma_tile_ss<D>(tmem + 256, descdO, smem_desc_sw128(stage_b(0) + L::kTile, 16, 1024), idesc_s);   // dP(0)
+                mma_tile_ss<D>(tmem + 0, descQ, smem_desc_sw128(k_slot(0), 16, 1024), idesc_s);     // S(0)
+                mma_tile_ss<D>(tmem + 256, descdO, smem_desc_sw128(v_slot(0), 16, 1024), idesc_s);  // dP(0)
                 tc_commit(bar(L::bS));
+                tc_commit(bar(L::bVEmpty + 0));
             }
             for (int t = 0; ok && t < T; ++t) {
-                const int st = t & 1, stn = st ^ 1;
-                const uint32_t sb = stage_b(st), sbn = stage_b(stn);
                 if (t + 1 < T) {
-                    ok = mbar_wait(bar(L::bFull + stn), ((t + 1) >> 1) & 1, kBwdWaitNs) && !*abort_flag;
+                    ok = k_full(t + 1);
                     if (!ok) break;
                     tc_fence_after();
-                    mma_tile_ss<D>(tmem + 128 * ((t + 1) & 1), descQ, smem_desc_sw128(sbn, 16, 1024), idesc_s);  // S(t+1)
+                    mma_tile_ss<D>(tmem + 128 * ((t + 1) & 1), descQ, smem_desc_sw128(k_slot(t + 1), 16, 1024),
+                                   idesc_s);                                                          // S(t+1)
                 }
+                ok = mbar_wait(bar(L::bDPread), t & 1, kBwdWaitNs) && !*abort_flag;
+                if (!ok) break;
+                if (t + 1 < T) {
+                    ok = v_full(t + 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    mma_tile_ss<D>(tmem + 256, descdO, smem_desc_sw128(v_slot(t + 1), 16, 1024), idesc_s);  // dP(t+1)
+                    tc_commit(bar(L::bS));
+                    tc_commit(bar(L::bVEmpty + (t + 1) % L::kVSlots));
+                }
+                ok = mbar_wait(bar(L::bPh), t & 1, kBwdWaitNs) && !*abort_flag;
+                if (!ok) break;
+                tc_fence_after();
+                dq_half(t, 0);
                 ok = mbar_wait(bar(L::bP), t & 1, kBwdWaitNs) && !*abort_flag;
                 if (!ok) break;
                 tc_fence_after();
-                mma_tile_ts<D, kBT>(tmem + 384, tmem + 256, smem_desc_sw128(sb, 16384, 1024), idesc_o, t > 0);  // dQ += dS K
-                tc_commit(bar(L::bEmpty + st));
-                if (t + 1 < T) {
-                    mma_tile_ss<D>(tmem + 256, descdO, smem_desc_sw128(sbn + L::kTile, 16, 1024), idesc_s);      // dP(t+1)
-                    tc_commit(bar(L::bS));
-                }
+                dq_half(t, 1);
+                tc_commit(bar(L::bKEmpty + t % L::kKSlots));
             }
             if (!ok) bwd_timeout(p, abort_flag);
             tc_commit(bar(L::bO));
@@ -496,33 +596,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
         const int row_end = min(p.n, (qr / p.kpf + 1) * p.kpf);        // keys it sees: [0, row_end)
         const float l2v = p.lse2[(size_t)head * p.n_pad + qr];          // +inf past n: P = 0
         const float dlv = p.delta[(size_t)head * p.n_pad + qr];
-        float l2[32], dl[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            l2[e] = l2v;
-            dl[e] = dlv;
-        }
         bool ok = true;
         for (int t = 0; t < T; ++t) {
             bool w = !*abort_flag && mbar_wait(bar(L::bS), t & 1, kBwdWaitNs);
             w = __all_sync(0xffffffffu, w);
             if (!w) { ok = false; break; }
             tc_fence_after();
-            const uint32_t tS = tmem + lane_bits + 128 * (t & 1);
-            const int hi = row_end - t * kBT;                           // columns at and past hi are hidden
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t s[32], dp[32], pk[16], dk[16];
-                tmem_ld32(tS + 32 * c, s);
-                tmem_ld32(tdP + 32 * c, dp);
-                tmem_wait_ld();
-                p_ds_chunk(s, dp, l2, dl, p.scale_log2, 0, hi - 32 * c, pk, dk);
-                tmem_st16(tdP + 16 * c, dk);
-            }
-            tmem_wait_st();
+            uint32_t dpr[128];
+            tmem_ld128(tdP, dpr);
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::bP));
+            if (lane == 0) mbar_arrive(bar(L::bDPread));   // dP's columns are free for dP(t+1)
+            const uint32_t tS = tmem + lane_bits + 128 * (t & 1);
+            const int hi = row_end - t * kBT;                           // columns at and past hi are hidden
+#pragma unroll   // constant c: the dP row stays in registers
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32], dk[16];
+                tmem_ld32(tS + 32 * c, sv);
+                tmem_wait_ld();
+                ds_chunk(sv, dpr, c, l2v, dlv, p.scale_log2, hi - 32 * c, dk);
+                tmem_st16(tS + 32 * c, dk);
+                if (c == 1 || c == 3) {
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(c == 1 ? L::bPh : L::bP));
+                }
+            }
         }
         bool w = ok && !*abort_flag && mbar_wait(bar(L::bO), 0, kBwdWaitNs);
         w = __all_sync(0xffffffffu, w);
@@ -553,7 +654,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
 
 template <int D>
 cudaError_t launch_bwd_t(const BwdParams &bp, const BwdProblem &pb, cudaStream_t s) {
-    using L = BwdLayout<D>;
+    using L = DkdvLayout<D>;
     static std::atomic<unsigned long long> configured{0};   // one bit per device (0..63)
     int dev = 0;
     cudaGetDevice(&dev);
@@ -561,7 +662,7 @@ cudaError_t launch_bwd_t(const BwdParams &bp, const BwdProblem &pb, cudaStream_t
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         cudaError_t e = cudaFuncSetAttribute(bwd_dkdv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(bwd_dq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+            e = cudaFuncSetAttribute(bwd_dq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqLayout<D>::kAlloc);
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_release);
     }
@@ -577,7 +678,7 @@ cudaError_t launch_bwd_t(const BwdParams &bp, const BwdProblem &pb, cudaStream_t
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();
-    bwd_dq<D><<<tiles, kBwdThreads, L::kAlloc, s>>>(bp);
+    bwd_dq<D><<<tiles, kBwdThreads, DqLayout<D>::kAlloc, s>>>(bp);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
