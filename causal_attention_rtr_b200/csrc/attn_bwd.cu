@@ -57,7 +57,8 @@ namespace {
 
 constexpr int kBT = 128;                  // rows of every tile
 constexpr int kHalf = 64;                 // query columns after which bwd_dkdv starts dV / dK
-constexpr int kBwdThreads = 256;
+constexpr int kDkdvThreads = 384;           // bwd_dkdv: producer, MMA, 2 idle, 8 softmax warps
+constexpr int kDqThreads = 256;             // bwd_dq: producer, MMA, 2 idle, 4 softmax warps
 constexpr uint64_t kBwdWaitNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -199,23 +200,23 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16 *o, const __
 
 
 // ---------------------------------------------------------------- dK, dV
-// P^T and dS^T for 32 query columns [32c, 32c+32) of one key row, written
-// packed as bf16 pairs: p = exp2(s * sl2 - l2) (0 for columns below `lo`),
-// ds = p * (dp - delta), with L*log2e and Delta of each column read from
-// shared memory (broadcast: every thread reads the same column).
-__device__ __forceinline__ void pt_dst_chunk(const uint32_t (&s)[128], int c, const uint32_t (&dp)[32],
-                                             const float *l2s, const float *dls, float sl2, int lo,
-                                             uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+// P^T and dS^T for 32 query columns of one key row, written packed as bf16
+// pairs: p = exp2(s * sl2 - l2) (0 for columns below `lo`), ds = p * (dp -
+// delta), with L*log2e and Delta of each column read from shared memory
+// (broadcast: every thread reads the same column).
+__device__ __forceinline__ void pt_dst_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float *l2s,
+                                             const float *dls, float sl2, int lo, uint32_t (&pk)[16],
+                                             uint32_t (&dk)[16]) {
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
-        const float4 l = *reinterpret_cast<const float4 *>(l2s + 32 * c + e);
-        const float4 d = *reinterpret_cast<const float4 *>(dls + 32 * c + e);
+        const float4 l = *reinterpret_cast<const float4 *>(l2s + e);
+        const float4 d = *reinterpret_cast<const float4 *>(dls + e);
         const float le[4] = {l.x, l.y, l.z, l.w}, de[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
         for (int u = 0; u < 4; u += 2) {
             const int col = e + u;
-            float p0 = fast_exp2(fmaf(__uint_as_float(s[32 * c + col]), sl2, -le[u]));
-            float p1 = fast_exp2(fmaf(__uint_as_float(s[32 * c + col + 1]), sl2, -le[u + 1]));
+            float p0 = fast_exp2(fmaf(__uint_as_float(s[col]), sl2, -le[u]));
+            float p1 = fast_exp2(fmaf(__uint_as_float(s[col + 1]), sl2, -le[u + 1]));
             p0 = col >= lo ? p0 : 0.f;
             p1 = col + 1 >= lo ? p1 : 0.f;
             pk[col / 2] = pack_bf16x2(p0, p1);
@@ -226,7 +227,7 @@ __device__ __forceinline__ void pt_dst_chunk(const uint32_t (&s)[128], int c, co
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kDkdvThreads, 1) bwd_dkdv(const __grid_constant__ BwdParams p) {
     using L = DkdvLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -252,11 +253,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
             mbar_init(bar(L::bEmpty + s), 1);
         }
         mbar_init(bar(L::bS), 1);
-        mbar_init(bar(L::bSread), 4);
-        mbar_init(bar(L::bPh), 4);
-        mbar_init(bar(L::bP), 4);
+        mbar_init(bar(L::bSread), 8);
+        mbar_init(bar(L::bPh), 4);   // the softmax group of query columns 0-63
+        mbar_init(bar(L::bP), 4);    // the group of columns 64-127
         mbar_init(bar(L::bO), 1);
-        mbar_init(bar(L::bEpi), kBT);
+        mbar_init(bar(L::bEpi), 2 * kBT);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -357,55 +358,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv(const __grid_constant
         }
         __syncwarp();
     } else if (warp >= 4) {
-        const int sub = warp & 3;
+        const int sub = warp & 3;                          // TMEM lane quarter (warp id mod 4)
+        const int grp = (warp - 4) >> 2;                   // query columns [64 grp, 64 grp + 64)
         const int row = sub * 32 + lane;
         const uint32_t lane_bits = (uint32_t)(sub * 32) << 16;
-        const uint32_t tS = tmem + lane_bits, tdP = tS + 128;
+        const uint32_t tS = tmem + lane_bits + 64 * grp, tdP = tmem + lane_bits + 128 + 64 * grp;
         const int kr = kt * kBT + row;                     // key row
         const int q_lo = (kr / p.kpf) * p.kpf;             // first query row that sees it
         bool ok = true;
         for (int t = 0; t < T; ++t) {
             const int i = i_first + t;
-            const float *l2s = reinterpret_cast<const float *>(smem + L::kB + (t & 1) * L::kStage + 2 * L::kTile);
+            const float *l2s =
+                reinterpret_cast<const float *>(smem + L::kB + (t & 1) * L::kStage + 2 * L::kTile) + 64 * grp;
             const float *dls = l2s + kBT;
             bool w = !*abort_flag && mbar_wait(bar(L::bS), t & 1, kBwdWaitNs);
             w = __all_sync(0xffffffffu, w);
             if (!w) { ok = false; break; }
             tc_fence_after();
-            uint32_t sr[128];
-            tmem_ld128(tS, sr);
+            uint32_t s0[32], s1[32];
+            tmem_ld32(tS, s0);
+            tmem_ld32(tS + 32, s1);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::bSread));   // S^T's columns are free for S^T(t+1)
-            const int lo = q_lo - i * kBT;                 // columns below lo are hidden from this key
-#pragma unroll   // constant c: the row stays in registers
-            for (int c = 0; c < 4; ++c) {
+            const int lo = q_lo - i * kBT - 64 * grp;      // columns below lo are hidden from this key
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
                 uint32_t dp[32], pk[16], dk[16];
-                tmem_ld32(tdP + 32 * c, dp);
+                tmem_ld32(tdP + 32 * h, dp);
                 tmem_wait_ld();
-                pt_dst_chunk(sr, c, dp, l2s, dls, p.scale_log2, lo - 32 * c, pk, dk);
-                tmem_st16(tdP + 32 * c, pk);
-                tmem_st16(tdP + 32 * c + 16, dk);
-                if (c == 1 || c == 3) {
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(c == 1 ? L::bPh : L::bP));
-                }
+                pt_dst_chunk(h ? s1 : s0, dp, l2s + 32 * h, dls + 32 * h, p.scale_log2, lo - 32 * h, pk, dk);
+                tmem_st16(tdP + 32 * h, pk);
+                tmem_st16(tdP + 32 * h + 16, dk);
             }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(grp == 0 ? L::bPh : L::bP));
         }
         // epilogue: dV -> V's tile, dK * scale -> K's tile, then TMA stores
         bool w = ok && !*abort_flag && mbar_wait(bar(L::bO), 0, kBwdWaitNs);
         w = __all_sync(0xffffffffu, w);
         if (w) {
             tc_fence_after();
-            acc_to_smem<D>(tmem + lane_bits + 256, 1.f, sV, row);
-            acc_to_smem<D>(tmem + lane_bits + 256 + D, p.scale, sK, row);
+            if (grp == 0) acc_to_smem<D>(tmem + lane_bits + 256, 1.f, sV, row);
+            else acc_to_smem<D>(tmem + lane_bits + 256 + D, p.scale, sK, row);
             fence_proxy_async_smem();
         }
         mbar_arrive(bar(L::bEpi));
-        if (row == 0) {
+        if (grp == 0 && row == 0) {
             const bool all = w && mbar_wait(bar(L::bEpi), 0, kBwdWaitNs);
             if (all) {
                 for (int b = 0; b < D / 64; ++b) {
@@ -445,7 +447,7 @@ __device__ __forceinline__ void ds_chunk(const uint32_t (&s)[32], const uint32_t
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kDqThreads, 1) bwd_dq(const __grid_constant__ BwdParams p) {
     using L = DqLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -495,9 +497,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
     // TMEM: S buffers [0,128), [128,256) (key tile t in buffer t % 2; its dS
     // is written, packed, over the first 16 of each 32-column group of S it
     // came from); dP [256,384); dQ [384,384+D).  The softmax reads the whole
-    // dP row into registers first, so dP(t+1) is computed while it works;
-    // S(t+1) runs earlier still.  dQ of the first 64 keys starts while the
-    // softmax does the other 64.
+    // dP row into registers first, so dP(t+1) is computed while it works.
+    // dQ of the first 64 keys starts while the softmax does the other 64.
 
     if (warp == 0) {
         if (lane == 0) {
@@ -555,14 +556,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
                 tc_commit(bar(L::bS));
                 tc_commit(bar(L::bVEmpty + 0));
             }
+            // Per step: dP(t+1) once the softmax holds dP(t), dQ of the first
+            // 64 keys, then S(t+1): K(t+1) reuses the slot of K(t-2), freed
+            // by the last dQ MMA two steps back, and issuing S(t+1) this late
+            // gives its load time to land.
             for (int t = 0; ok && t < T; ++t) {
-                if (t + 1 < T) {
-                    ok = k_full(t + 1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    mma_tile_ss<D>(tmem + 128 * ((t + 1) & 1), descQ, smem_desc_sw128(k_slot(t + 1), 16, 1024),
-                                   idesc_s);                                                          // S(t+1)
-                }
                 ok = mbar_wait(bar(L::bDPread), t & 1, kBwdWaitNs) && !*abort_flag;
                 if (!ok) break;
                 if (t + 1 < T) {
@@ -570,13 +568,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
                     if (!ok) break;
                     tc_fence_after();
                     mma_tile_ss<D>(tmem + 256, descdO, smem_desc_sw128(v_slot(t + 1), 16, 1024), idesc_s);  // dP(t+1)
-                    tc_commit(bar(L::bS));
                     tc_commit(bar(L::bVEmpty + (t + 1) % L::kVSlots));
                 }
                 ok = mbar_wait(bar(L::bPh), t & 1, kBwdWaitNs) && !*abort_flag;
                 if (!ok) break;
                 tc_fence_after();
                 dq_half(t, 0);
+                if (t + 1 < T) {
+                    ok = k_full(t + 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    mma_tile_ss<D>(tmem + 128 * ((t + 1) & 1), descQ, smem_desc_sw128(k_slot(t + 1), 16, 1024),
+                                   idesc_s);                                                          // S(t+1)
+                    tc_commit(bar(L::bS));   // S(t+1) and dP(t+1) done
+                }
                 ok = mbar_wait(bar(L::bP), t & 1, kBwdWaitNs) && !*abort_flag;
                 if (!ok) break;
                 tc_fence_after();
@@ -602,20 +607,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
             w = __all_sync(0xffffffffu, w);
             if (!w) { ok = false; break; }
             tc_fence_after();
-            uint32_t dpr[128];
+            const uint32_t tS = tmem + lane_bits + 128 * (t & 1);
+            uint32_t dpr[128], sv0[32], sv1[32];
             tmem_ld128(tdP, dpr);
+            tmem_ld32(tS, sv0);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::bDPread));   // dP's columns are free for dP(t+1)
-            const uint32_t tS = tmem + lane_bits + 128 * (t & 1);
             const int hi = row_end - t * kBT;                           // columns at and past hi are hidden
+            // S group c+1 loads while group c is computed
 #pragma unroll   // constant c: the dP row stays in registers
             for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], dk[16];
-                tmem_ld32(tS + 32 * c, sv);
-                tmem_wait_ld();
-                ds_chunk(sv, dpr, c, l2v, dlv, p.scale_log2, hi - 32 * c, dk);
+                uint32_t(&cur)[32] = (c & 1) ? sv1 : sv0;
+                uint32_t(&nxt)[32] = (c & 1) ? sv0 : sv1;
+                if (c + 1 < 4) tmem_ld32(tS + 32 * (c + 1), nxt);
+                uint32_t dk[16];
+                ds_chunk(cur, dpr, c, l2v, dlv, p.scale_log2, hi - 32 * c, dk);
                 tmem_st16(tS + 32 * c, dk);
                 if (c == 1 || c == 3) {
                     tmem_wait_st();
@@ -623,6 +631,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq(const __grid_constant__
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(c == 1 ? L::bPh : L::bP));
                 }
+                if (c + 1 < 4) tmem_wait_ld_regs(nxt);
             }
         }
         bool w = ok && !*abort_flag && mbar_wait(bar(L::bO), 0, kBwdWaitNs);
@@ -674,11 +683,11 @@ cudaError_t launch_bwd_t(const BwdParams &bp, const BwdProblem &pb, cudaStream_t
     if (e != cudaSuccess) return e;
     count_launch();
     const unsigned tiles = (unsigned)((bp.n + kBT - 1) / kBT) * (unsigned)bp.heads;
-    bwd_dkdv<D><<<tiles, kBwdThreads, L::kAlloc, s>>>(bp);
+    bwd_dkdv<D><<<tiles, kDkdvThreads, L::kAlloc, s>>>(bp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch();
-    bwd_dq<D><<<tiles, kBwdThreads, DqLayout<D>::kAlloc, s>>>(bp);
+    bwd_dq<D><<<tiles, kDqThreads, DqLayout<D>::kAlloc, s>>>(bp);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
