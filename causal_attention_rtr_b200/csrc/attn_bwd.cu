@@ -203,25 +203,34 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16 *o, const __
 // P^T and dS^T for 32 query columns of one key row, written packed as bf16
 // pairs: p = exp2(s * sl2 - l2) (0 for columns below `lo`), ds = p * (dp -
 // delta), with L*log2e and Delta of each column read from shared memory
-// (broadcast: every thread reads the same column).
+// (broadcast: every thread reads the same column).  The arithmetic is in
+// f32x2 pairs: scalar fp32 FMA, add and multiply instructions slow the
+// tensor core of the SM down (by almost half, in a probe where one warp
+// issues them beside an MMA loop), the paired forms hardly at all.
+template <bool MASK>
 __device__ __forceinline__ void pt_dst_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float *l2s,
                                              const float *dls, float sl2, int lo, uint32_t (&pk)[16],
                                              uint32_t (&dk)[16]) {
+    const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
         const float4 l = *reinterpret_cast<const float4 *>(l2s + e);
         const float4 d = *reinterpret_cast<const float4 *>(dls + e);
-        const float le[4] = {l.x, l.y, l.z, l.w}, de[4] = {d.x, d.y, d.z, d.w};
+        const float2 nl[2] = {make_float2(-l.x, -l.y), make_float2(-l.z, -l.w)};
+        const float2 nd[2] = {make_float2(-d.x, -d.y), make_float2(-d.z, -d.w)};
 #pragma unroll
-        for (int u = 0; u < 4; u += 2) {
-            const int col = e + u;
-            float p0 = fast_exp2(fmaf(__uint_as_float(s[col]), sl2, -le[u]));
-            float p1 = fast_exp2(fmaf(__uint_as_float(s[col + 1]), sl2, -le[u + 1]));
-            p0 = col >= lo ? p0 : 0.f;
-            p1 = col + 1 >= lo ? p1 : 0.f;
-            pk[col / 2] = pack_bf16x2(p0, p1);
-            dk[col / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[col]) - de[u]),
-                                      p1 * (__uint_as_float(dp[col + 1]) - de[u + 1]));
+        for (int u = 0; u < 2; ++u) {
+            const int col = e + 2 * u;
+            const float2 x = ffma2(make_float2(__uint_as_float(s[col]), __uint_as_float(s[col + 1])), sl2x2, nl[u]);
+            float2 pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            if (MASK) {
+                pr.x = col >= lo ? pr.x : 0.f;
+                pr.y = col + 1 >= lo ? pr.y : 0.f;
+            }
+            const float2 g = fadd2(make_float2(__uint_as_float(dp[col]), __uint_as_float(dp[col + 1])), nd[u]);
+            const float2 ds = fmul2(pr, g);
+            pk[col / 2] = pack_bf16x2(pr.x, pr.y);
+            dk[col / 2] = pack_bf16x2(ds.x, ds.y);
         }
     }
 }
@@ -388,7 +397,10 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) bwd_dkdv(const __grid_constan
                 uint32_t dp[32], pk[16], dk[16];
                 tmem_ld32(tdP + 32 * h, dp);
                 tmem_wait_ld();
-                pt_dst_chunk(h ? s1 : s0, dp, l2s + 32 * h, dls + 32 * h, p.scale_log2, lo - 32 * h, pk, dk);
+                if (__any_sync(0xffffffffu, lo - 32 * h > 0))   // warp-uniform: some column hidden
+                    pt_dst_chunk<true>(h ? s1 : s0, dp, l2s + 32 * h, dls + 32 * h, p.scale_log2, lo - 32 * h, pk, dk);
+                else
+                    pt_dst_chunk<false>(h ? s1 : s0, dp, l2s + 32 * h, dls + 32 * h, p.scale_log2, 0, pk, dk);
                 tmem_st16(tdP + 32 * h, pk);
                 tmem_st16(tdP + 32 * h + 16, dk);
             }
@@ -432,17 +444,24 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) bwd_dkdv(const __grid_constan
 // ---------------------------------------------------------------- dQ
 // dS for 32 key columns [32c, 32c+32) of one query row, packed as bf16
 // pairs: p = exp2(s * sl2 - l2) (0 for columns at or past `hi`),
-// ds = p * (dp - delta), dp from the row's registers.
+// ds = p * (dp - delta), dp from the row's registers; f32x2 arithmetic (see
+// pt_dst_chunk).
+template <bool MASK>
 __device__ __forceinline__ void ds_chunk(const uint32_t (&s)[32], const uint32_t (&dpr)[128], int c, float l2,
                                          float dl, float sl2, int hi, uint32_t (&dk)[16]) {
+    const float2 sl2x2 = make_float2(sl2, sl2), nl2 = make_float2(-l2, -l2), ndl = make_float2(-dl, -dl);
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-        float p0 = fast_exp2(fmaf(__uint_as_float(s[e]), sl2, -l2));
-        float p1 = fast_exp2(fmaf(__uint_as_float(s[e + 1]), sl2, -l2));
-        p0 = e < hi ? p0 : 0.f;
-        p1 = e + 1 < hi ? p1 : 0.f;
-        dk[e / 2] = pack_bf16x2(p0 * (__uint_as_float(dpr[32 * c + e]) - dl),
-                                p1 * (__uint_as_float(dpr[32 * c + e + 1]) - dl));
+        const float2 x = ffma2(make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2x2, nl2);
+        float2 pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        if (MASK) {
+            pr.x = e < hi ? pr.x : 0.f;
+            pr.y = e + 1 < hi ? pr.y : 0.f;
+        }
+        const float2 g =
+            fadd2(make_float2(__uint_as_float(dpr[32 * c + e]), __uint_as_float(dpr[32 * c + e + 1])), ndl);
+        const float2 ds = fmul2(pr, g);
+        dk[e / 2] = pack_bf16x2(ds.x, ds.y);
     }
 }
 
@@ -623,7 +642,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq(const __grid_constant__ 
                 uint32_t(&nxt)[32] = (c & 1) ? sv0 : sv1;
                 if (c + 1 < 4) tmem_ld32(tS + 32 * (c + 1), nxt);
                 uint32_t dk[16];
-                ds_chunk(cur, dpr, c, l2v, dlv, p.scale_log2, hi - 32 * c, dk);
+                if (__any_sync(0xffffffffu, hi - 32 * c < 32))   // warp-uniform: some column hidden
+                    ds_chunk<true>(cur, dpr, c, l2v, dlv, p.scale_log2, hi - 32 * c, dk);
+                else
+                    ds_chunk<false>(cur, dpr, c, l2v, dlv, p.scale_log2, 32, dk);
                 tmem_st16(tS + 32 * c, dk);
                 if (c == 1 || c == 3) {
                     tmem_wait_st();
