@@ -24,7 +24,10 @@
 //               D[128 x BN] += A[128 x 16] W[16 x BN], A K-major and W
 //               MN-major from 128-byte-swizzled shared memory
 //   warps 2-9   epilogue: two warps per TMEM lane quarter (one thread per
-//               row), each taking alternate 32-column chunks of the tile
+//               row), each taking alternate 32-column chunks of the tile;
+//               its arithmetic is in f32x2 pairs and the special-function
+//               unit (scalar fp32 instructions slow the next tile's MMAs),
+//               the rotary angles come from a table each CTA fills once
 // A tile is 128 rows by BN = 128, 192 or 256 columns, or 256 by 256 (two
 // 128-row sub-tiles whose MMAs share each stage of W).  When a tile's
 // accumulators take at most 256 TMEM columns there are two buffers, so the
@@ -59,6 +62,7 @@ constexpr int kBBoxBytes = kBK * 64 * 2;            // 8 KB: 64 K rows x 64 N co
 constexpr int kMaxSmem = 200 * 1024;                // stages share this
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr float kLog2RopeBase = 13.287712379549449f;   // log2(10000)
+constexpr int kRopeTabMax = 2048;                       // table entries (float2) at most: 16 KB
 
 struct GemmParams {
     CUtensorMap tm_a;   // A [m][k]: dims (k, m, 1), box (64, 128, 1)
@@ -75,6 +79,10 @@ struct GemmParams {
     __nv_bfloat16 *out;                 // bias / GELU: [m][n]; gated residual: [m][n] in place
     __nv_bfloat16 *q, *kk, *v;          // QKV: [m][D] each, D = n / 3
     int D, head_dim, kpf, grid_w, t0, rope_dt, rope_dp;
+    // rotary table in shared memory: (cos, sin) per (frame, time pair), then
+    // per (row, row pair) and per (column, column pair); 0 entries: the
+    // epilogue computes each angle itself
+    int rope_entries, rope_frames, rope_rows;
     unsigned *status;
 };
 
@@ -96,9 +104,32 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
 }
 
-__device__ __forceinline__ float gelu_tanh(float x) {
-    const float kS = 0.7978845608028654f;   // sqrt(2 / pi)
-    return 0.5f * x * (1.0f + tanhf(kS * (x + 0.044715f * x * x * x)));
+// GELU, tanh form, for a pair: 0.5 x (1 + tanh(y)) = x sigmoid(2y) =
+// x / (1 + 2^(-2 y log2 e)), y = sqrt(2/pi) (x + 0.044715 x^3).  The pair
+// arithmetic is f32x2 and the exponential and reciprocal are the special
+// function unit's: scalar fp32 instructions in the epilogue would slow the
+// next tile's MMAs down.  The sigmoid form has no cancellation; relative
+// error about 1e-6, far below a bf16 step.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float2 gelu_tanh2(float2 x) {
+    const float kC = -2.0f * 0.7978845608028654f * 1.4426950408889634f;   // -2 sqrt(2/pi) log2(e)
+    const float2 v = ffma2(fmul2(x, x), make_float2(0.044715f, 0.044715f), make_float2(1.f, 1.f));
+    const float2 z = fmul2(fmul2(x, v), make_float2(kC, kC));
+    const float2 d = fadd2(make_float2(fast_exp2(z.x), fast_exp2(z.y)), make_float2(1.f, 1.f));
+    return fmul2(x, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
+// Angle of rotary channel pair j of a section with `size` channels at
+// position pos, as (cos, sin).
+__device__ __forceinline__ float2 rope_angle(int j, int size, int pos) {
+    const float theta = exp2f(-(float)(2 * j) / (float)size * kLog2RopeBase);
+    float sn, cs;
+    sincosf((float)pos * theta, &sn, &cs);
+    return make_float2(cs, sn);
 }
 
 // Bounded wait that also gives up as soon as another role has aborted.
@@ -118,40 +149,43 @@ __device__ __forceinline__ void raise_timeout(const GemmParams &p, volatile int 
 }
 
 // The epilogue of 32 consecutive accumulator columns [col, col + 32) of one
-// row (nvalid of them inside the matrix, a multiple of 8).
+// row (nvalid of them inside the matrix, a multiple of 8), in f32x2 pairs.
+// `rope` is the shared-memory rotary table (null: angles computed here).
 template <int EPI>
 __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&acc)[32], long long row, int col,
-                                          int nvalid, int f_pos, int y_pos, int x_pos) {
+                                          int nvalid, int f_pos, int y_pos, int x_pos, const float2 *rope) {
     if (EPI == kEpiQkvRope) {
         const int part = col / p.D, cc = col - part * p.D;
         __nv_bfloat16 *dst = (part == 0 ? p.q : part == 1 ? p.kk : p.v) + row * p.D + cc;
         const int c0 = cc % p.head_dim;                 // channel of the first column within its head
+        const int nt = p.rope_dt / 2, nd = p.rope_dp / 2;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             if (8 * g >= nvalid) break;
             float b[8], r[8];
             unpack8(*reinterpret_cast<const uint4 *>(p.bias + col + 8 * g), b);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) r[e] = __uint_as_float(acc[8 * g + e]) + b[e];
-            if (part < 2) {
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
+            for (int e = 0; e < 8; e += 2) {
+                float2 v = fadd2(make_float2(__uint_as_float(acc[8 * g + e]), __uint_as_float(acc[8 * g + e + 1])),
+                                 make_float2(b[e], b[e + 1]));
+                if (part < 2) {
                     const int c = c0 + 8 * g + e;       // even channel of the pair
-                    int j, size, pos;
+                    float2 cs;
                     if (c < p.rope_dt) {
-                        j = c / 2; size = p.rope_dt; pos = f_pos;
+                        cs = rope ? rope[(f_pos - p.t0) * nt + c / 2] : rope_angle(c / 2, p.rope_dt, f_pos);
                     } else if (c < p.rope_dt + p.rope_dp) {
-                        j = (c - p.rope_dt) / 2; size = p.rope_dp; pos = y_pos;
+                        const int j = (c - p.rope_dt) / 2;
+                        cs = rope ? rope[p.rope_frames * nt + y_pos * nd + j] : rope_angle(j, p.rope_dp, y_pos);
                     } else {
-                        j = (c - p.rope_dt - p.rope_dp) / 2; size = p.rope_dp; pos = x_pos;
+                        const int j = (c - p.rope_dt - p.rope_dp) / 2;
+                        cs = rope ? rope[p.rope_frames * nt + (p.rope_rows + x_pos) * nd + j]
+                                  : rope_angle(j, p.rope_dp, x_pos);
                     }
-                    const float theta = exp2f(-(float)(2 * j) / (float)size * kLog2RopeBase);
-                    float sn, cs;
-                    sincosf((float)pos * theta, &sn, &cs);
-                    const float a0 = r[e], a1 = r[e + 1];
-                    r[e] = a0 * cs - a1 * sn;
-                    r[e + 1] = a0 * sn + a1 * cs;
+                    // (a0 cos - a1 sin, a1 cos + a0 sin)
+                    v = ffma2(v, make_float2(cs.x, cs.x), fmul2(make_float2(v.y, v.x), make_float2(-cs.y, cs.y)));
                 }
+                r[e] = v.x;
+                r[e + 1] = v.y;
             }
             *reinterpret_cast<uint4 *>(dst + 8 * g) = pack8(r);
         }
@@ -170,7 +204,13 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
                 for (int e = 0; e < 8; ++e) gt[e] = 1.f;
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) r[e] = xv[e] + gt[e] * (__uint_as_float(acc[8 * g + e]) + b[e]);
+            for (int e = 0; e < 8; e += 2) {
+                const float2 t = fadd2(make_float2(__uint_as_float(acc[8 * g + e]), __uint_as_float(acc[8 * g + e + 1])),
+                                       make_float2(b[e], b[e + 1]));
+                const float2 v = ffma2(make_float2(gt[e], gt[e + 1]), t, make_float2(xv[e], xv[e + 1]));
+                r[e] = v.x;
+                r[e + 1] = v.y;
+            }
             *reinterpret_cast<uint4 *>(x + 8 * g) = pack8(r);
         }
     } else {
@@ -181,9 +221,12 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
             float b[8], r[8];
             unpack8(*reinterpret_cast<const uint4 *>(p.bias + col + 8 * g), b);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                r[e] = __uint_as_float(acc[8 * g + e]) + b[e];
-                if (EPI == kEpiBiasGelu) r[e] = gelu_tanh(r[e]);
+            for (int e = 0; e < 8; e += 2) {
+                float2 v = fadd2(make_float2(__uint_as_float(acc[8 * g + e]), __uint_as_float(acc[8 * g + e + 1])),
+                                 make_float2(b[e], b[e + 1]));
+                if (EPI == kEpiBiasGelu) v = gelu_tanh2(v);
+                r[e] = v.x;
+                r[e + 1] = v.y;
             }
             if (p.out_packed)
                 *reinterpret_cast<uint4 *>(reinterpret_cast<char *>(p.out) + packed_a_offset(row, col + 8 * g, p.n)) =
@@ -204,15 +247,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
     const int stage_bytes = a_bytes + (p.bn / 64) * kBBoxBytes;
     const int BMt = kBM * p.msub;                              // rows per tile
     const uint32_t bars = s_base + (uint32_t)(S * stage_bytes);
-    // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
+    // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain, rope table ready
     auto full = [&](int s) { return bars + 8u * (uint32_t)s; };
     auto empty = [&](int s) { return bars + 8u * (uint32_t)(S + s); };
     auto accf = [&](int b) { return bars + 8u * (uint32_t)(2 * S + b); };
     auto acce = [&](int b) { return bars + 8u * (uint32_t)(2 * S + 2 + b); };
     const uint32_t drain = bars + 8u * (uint32_t)(2 * S + 4);
-    uint8_t *misc = smem + S * stage_bytes + 8 * (2 * S + 5);
+    const uint32_t rope_ready = bars + 8u * (uint32_t)(2 * S + 5);
+    uint8_t *misc = smem + S * stage_bytes + 8 * (2 * S + 6);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 4);
+    float2 *rope_tab = reinterpret_cast<float2 *>(misc + 16);   // p.rope_entries of them
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -225,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
             mbar_init(acce(b), kEpiWarps);
         }
         mbar_init(drain, 1);
+        mbar_init(rope_ready, kEpiWarps * 32);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -338,11 +384,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
         int tc = 0;
         bool ok = true;
+        const float2 *rope = nullptr;
+        if (EPI == kEpiQkvRope && p.rope_entries > 0) {
+            // the chunk's rotary angles, once per CTA while the first tile's
+            // MMAs run: time pairs per frame, row pairs per row, column
+            // pairs per column
+            const int nt = p.rope_dt / 2, nd = p.rope_dp / 2;
+            const int e_t = p.rope_frames * nt, e_y = p.rope_rows * nd;
+            for (int e = threadIdx.x - 64; e < p.rope_entries; e += kEpiWarps * 32) {
+                float2 v;
+                if (e < e_t) v = rope_angle(e % nt, p.rope_dt, p.t0 + e / nt);
+                else if (e < e_t + e_y) v = rope_angle((e - e_t) % nd, p.rope_dp, (e - e_t) / nd);
+                else v = rope_angle((e - e_t - e_y) % nd, p.rope_dp, (e - e_t - e_y) / nd);
+                rope_tab[e] = v;
+            }
+            mbar_arrive(rope_ready);
+            ok = wait_bar(rope_ready, 0, abort_flag);
+            rope = rope_tab;
+        }
         // one sub-tile: the two warps of a lane quarter take alternate 32-column
         // chunks; two sub-tiles: warp half u takes all chunks of sub-tile u
         const int sub = p.msub == 2 ? half : 0;
         const int c_first = p.msub == 2 ? 0 : half, c_step = p.msub == 2 ? 1 : 2;
-        for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++tc) {
+        for (int t = blockIdx.x; ok && t < p.n_tiles; t += gridDim.x, ++tc) {
             const int b = tc % p.nbuf, use_b = tc / p.nbuf;
             const int m0 = (t / p.n_tiles_n) * BMt, n0 = (t % p.n_tiles_n) * p.bn;
             bool w = wait_bar(accf(b), use_b & 1, abort_flag);
@@ -368,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                 uint32_t acc[32];
                 tmem_ld32(tmem + lane_bits + (uint32_t)(b * 256 + sub * p.bn + 32 * c), acc);
                 tmem_wait_ld();
-                if (row_ok) epi_chunk<EPI>(p, acc, row, col, min(32, p.n - col), f_pos, y_pos, x_pos);
+                if (row_ok) epi_chunk<EPI>(p, acc, row, col, min(32, p.n - col), f_pos, y_pos, x_pos, rope);
             }
             tc_fence_before();
             __syncwarp();
@@ -387,7 +451,8 @@ cudaError_t set_smem_attr_once() {
     static std::once_flag once;
     static cudaError_t err = cudaSuccess;
     std::call_once(once, [] {
-        err = cudaFuncSetAttribute(gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem + 2048);
+        err = cudaFuncSetAttribute(gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   kMaxSmem + 2048 + kRopeTabMax * 8);
     });
     return err;
 }
@@ -493,11 +558,20 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
     p.t0 = g.t0;
     p.rope_dp = g.head_dim > 0 ? 2 * (g.head_dim / 6) : 0;
     p.rope_dt = g.head_dim - 2 * p.rope_dp;
+    if (g.epi == kEpiQkvRope) {
+        // rows [0, m) cover frames t0 .. t0 + rope_frames - 1; a frame's rows
+        // are rope_rows rows of grid_w columns
+        p.rope_frames = (g.m - 1) / g.kpf + 1;
+        p.rope_rows = (g.kpf + g.grid_w - 1) / g.grid_w;
+        const long long entries = (long long)p.rope_frames * (p.rope_dt / 2) +
+                                  (long long)(p.rope_rows + g.grid_w) * (p.rope_dp / 2);
+        p.rope_entries = entries <= kRopeTabMax ? (int)entries : 0;
+    }
     p.status = status;
     const int grid = p.n_tiles < sms ? p.n_tiles : sms;
-    // stages, barriers (2S + 5), the TMEM holder and the abort flag, plus
-    // slack for the 1 KB alignment of the stage ring
-    const int smem = p.stages * stage_bytes + 8 * (2 * p.stages + 5) + 16 + 1024;
+    // stages, barriers (2S + 6), the TMEM holder and the abort flag, the
+    // rotary table, plus slack for the 1 KB alignment of the stage ring
+    const int smem = p.stages * stage_bytes + 8 * (2 * p.stages + 6) + 16 + p.rope_entries * 8 + 1024;
     switch (g.epi) {
         case kEpiBias: return launch_epi<kEpiBias>(p, grid, smem, s);
         case kEpiBiasGelu: return launch_epi<kEpiBiasGelu>(p, grid, smem, s);
