@@ -240,10 +240,11 @@ def oracle_rows(w, ops, rows, nthreads=0):
     return oracle.attention(Q[rows], pos[rows], K, V, w.k, True, None, nthreads)
 
 
-def time_oracle(w, ops, seconds_target, nthreads=0):
+def time_oracle(w, ops, seconds_target, nthreads=0, keep=None):
     """Time the oracle on sampled query rows (all heads) of the chunk,
     growing the sample until it takes about ``seconds_target``, on
-    ``nthreads`` threads (0: all).  Returns (flops, seconds, rows)."""
+    ``nthreads`` threads (0: all).  Returns (flops, seconds, rows); with a
+    ``keep`` list, the last sample's outputs are appended to it."""
     import numpy as np
     nq = w.chunk_frames * w.k
     rng = np.random.default_rng(123)
@@ -251,11 +252,45 @@ def time_oracle(w, ops, seconds_target, nthreads=0):
     while True:
         rows = np.sort(rng.choice(nq, size=min(n, nq), replace=False))
         t0 = time.perf_counter()
-        oracle_rows(w, ops, rows, nthreads)
+        got = oracle_rows(w, ops, rows, nthreads)
         dt = time.perf_counter() - t0
         if dt >= 0.5 * seconds_target or n >= nq:
+            if keep is not None:
+                keep.append(got)
             return oracle_sample_flops(w, rows), dt, rows
         n = min(nq, max(n * 2, int(n * seconds_target / max(dt, 1e-3) * 0.9)))
+
+
+def output_accuracy(rtr, torch, w, x, dev, rows, want, dev_id):
+    """The layer's attention on a fresh cache (the same history the oracle
+    holds) through rtr_attn_frame_causal (bf16 output) and
+    rtr_attn_frame_causal_f32out (fp32 output), against the oracle's rows."""
+    import numpy as np
+    c = rtr.rtr_kvcache_create(1, w.heads, w.head_dim, w.k, w.ref_frames, w.window_frames, "bf16", dev_id)
+    try:
+        rtr.rtr_kvcache_set_reference(c, 0, dev(x.ref_k), dev(x.ref_v))
+        for fk, fv in zip(x.window_k, x.window_v):
+            rtr.rtr_kvcache_append_frame(c, 0, dev(fk), dev(fv), 1)
+        q, kc, vc = dev(x.q), dev(x.k_cur), dev(x.v_cur)
+        o16 = torch.empty_like(q)
+        o32 = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+        rtr.rtr_attn_frame_causal(c, 0, q, kc, vc, w.chunk_frames, o16)
+        rtr.rtr_attn_frame_causal_f32out(c, 0, q, kc, vc, w.chunk_frames, o32)
+        torch.cuda.synchronize()
+    finally:
+        rtr.rtr_kvcache_destroy(c)
+    idx = torch.from_numpy(np.asarray(rows, dtype=np.int64)).cuda()
+    res = {}
+    for name, o in (("bf16_out", o16), ("f32_out", o32)):
+        got = o.index_select(0, idx).double().cpu().numpy()
+        diff = got - want
+        res[name] = {"max_abs": float(np.max(np.abs(diff))),
+                     "rel_l2": float(np.linalg.norm(diff.ravel()) / np.linalg.norm(want.ravel()))}
+    res["rows"] = int(len(rows))
+    res["bound"] = {"max_abs": 2e-2, "rel_l2": 5e-3}
+    res["how"] = ("the cpu_baseline sample's query rows (all heads) against the fp64 oracle; f32_out is "
+                  "rtr_attn_frame_causal_f32out, the same rows before the bf16 rounding")
+    return res
 
 
 def cpu_baseline_entry(flops, seconds, rows, w):
@@ -544,8 +579,10 @@ def run_ours(args, rank, world, local_rank):
         del cx
     if world == 1 and not args.no_cpu_baseline:
         ops = oracle_operands(w, x)
-        fl, dt, rows = time_oracle(w, ops, 12.0)
+        kept = []
+        fl, dt, rows = time_oracle(w, ops, 12.0, keep=kept)
         line["cpu_baseline"] = cpu_baseline_entry(fl, dt, rows, w)
+        line["accuracy"] = output_accuracy(rtr, torch, w, x, dev, rows, kept[0], dev_id)
         fl1, dt1, rows1 = time_oracle(w, ops, 4.0, nthreads=1)
         line["cpu_baseline"]["single_core"] = {
             "value": fl1 / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1,

@@ -595,6 +595,21 @@ rtr_status rtr_attn_frame_causal_ex(const rtr_kvcache *c, int layer, const void 
     return run_attention(pb, c->dt, tk, tkh, tv, c->device, (cudaStream_t)stream, cta_group);
 }
 
+rtr_status rtr_attn_frame_causal_f32out(const rtr_kvcache *c, int layer, const void *q, const void *k_cur,
+                                        const void *v_cur, int n_cur_frames, float *out, float scale,
+                                        rtr_stream_t stream) {
+    if (c && c->dt == RTR_F32)   // the fp32 path's output is fp32 already
+        return rtr_attn_frame_causal_ex(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale, 1, stream);
+    AttnProblem pb;
+    const rtr_status st = stream_problem(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale, pb);
+    if (st != RTR_OK) return st;
+    pb.o_f32 = out;
+    pb.o = nullptr;
+    DeviceGuard dg(c->device);
+    return run_attention(pb, c->dt, &c->tmk[layer], &c->tmk64[layer], &c->tmv[layer], c->device,
+                         (cudaStream_t)stream, 1);
+}
+
 rtr_status rtr_attn_frame_causal_commit(rtr_kvcache *c, int layer, const void *q, const void *k_cur,
                                         const void *v_cur, int n_cur_frames, void *out, float scale,
                                         rtr_stream_t stream) {

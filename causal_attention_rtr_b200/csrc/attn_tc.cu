@@ -123,6 +123,7 @@ struct TcParams {
     int commit_first_slot, commit_slots, commit_row0;
     const CUtensorMap *commit_maps;   // per-slot store maps (see AttnProblem) or null
     float *lse;         // [heads][nq] natural-log row log-sum-exp, or null
+    float *out_f32;     // token-major fp32 output instead of bf16 (whole rows stored directly), or null
 };
 
 // CG = CTAs per cluster working one MMA: 1, or 2 for the CTA-pair MMA
@@ -951,7 +952,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             if (!w) { ok = false; break; }
             tc_fence_after();
             const int prow = i * kBM + row_local;       // row within the pair
-            if (it.slot < 0) {
+            if (it.slot < 0 && p.out_f32 != nullptr) {
+                // fp32 output: the normalised row straight to global memory
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                if (p.lse != nullptr && q_row < p.nq)
+                    p.lse[(size_t)head * p.nq + q_row] =
+                        l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+                float4 *dst = reinterpret_cast<float4 *>(p.out_f32 + ((size_t)q_row * p.heads + head) * D);
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
+                    if (q_row < p.nq) {
+#pragma unroll
+                        for (int t4 = 0; t4 < 8; ++t4)
+                            dst[8 * c + t4] = make_float4(
+                                __uint_as_float(o[4 * t4 + 0]) * inv, __uint_as_float(o[4 * t4 + 1]) * inv,
+                                __uint_as_float(o[4 * t4 + 2]) * inv, __uint_as_float(o[4 * t4 + 3]) * inv);
+                    }
+                }
+            } else if (it.slot < 0) {
                 const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
                 if (p.lse != nullptr && q_row < p.nq)
                     p.lse[(size_t)head * p.nq + q_row] =
@@ -1000,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc(const __grid_constant
             if (row_local == 0) {
                 const bool all = mbar_wait(bar(L::bEpi + i), k & 1, kWaitNs);
                 if (!all) raise_timeout(p, abort_flag);
-                if (all && it.slot < 0 && my_q0 + i * kBM < p.nq) {
+                if (all && it.slot < 0 && p.out_f32 == nullptr && my_q0 + i * kBM < p.nq) {
                     for (int b = 0; b < NBOX; ++b)
                         tma_store_3d(&p.tm_o, sOut + b * 16384, b * 64, head, my_q0 + i * kBM);
                     bulk_commit();
@@ -1080,6 +1101,13 @@ __global__ void __launch_bounds__(256) attn_combine(const __grid_constant__ TcPa
     const float inv = l > 0.f ? 1.f / l : 0.f;
     if (p.lse != nullptr && quarter == 0)
         p.lse[(size_t)head * p.nq + q] = l > 0.f ? (M + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (p.out_f32 != nullptr) {
+        float4 *df = reinterpret_cast<float4 *>(p.out_f32 + ((size_t)q * p.heads + head) * D + quarter * (D / 4));
+#pragma unroll
+        for (int e = 0; e < NV; ++e)
+            df[e] = make_float4(acc[e].x * inv, acc[e].y * inv, acc[e].z * inv, acc[e].w * inv);
+        return;
+    }
     uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)q * p.heads + head) * D + quarter * (D / 4));
 #pragma unroll
     for (int e = 0; e < NV / 2; ++e) {
@@ -1280,7 +1308,8 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
     }
     const uint64_t D = (uint64_t)p.head_dim;
     if (!make_tmap_bf16(&tp.tm_q, p.q, D, p.heads, p.nq, 1, kBM)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16(&tp.tm_o, p.o, D, p.heads, p.nq, 1, kBM)) return cudaErrorInvalidValue;
+    // with an fp32 output the bf16 output map is never used: any valid map
+    if (!make_tmap_bf16(&tp.tm_o, p.o_f32 ? p.q : p.o, D, p.heads, p.nq, 1, kBM)) return cudaErrorInvalidValue;
     bool have0 = false, have1 = false;
     for (int i = 0; i < p.nseg; ++i) (p.seg[i].src == 0 ? have0 : have1) = true;
     if (have1) {
@@ -1324,6 +1353,8 @@ cudaError_t launch_attn_bf16(const AttnProblem &p, const AttnPlan &plan, const C
     tp.part_o = static_cast<float4 *>(scratch);
     tp.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(scratch) + part_o_bytes);
     tp.out = static_cast<__nv_bfloat16 *>(p.o);
+    tp.out_f32 = p.o_f32;
+    if (p.o_f32 && (plan.cg != 1 || p.commit_k)) return cudaErrorInvalidValue;
     tp.lse = p.lse;
     if (p.commit_k) {
         // the chunk write is implemented for one CTA per MMA and needs the

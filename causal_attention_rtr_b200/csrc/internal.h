@@ -58,6 +58,9 @@ struct AttnProblem {
     // Optional row statistics: lse[h * nq + i] = log sum_j exp(scale q_i.k_j)
     // over the keys row i sees (natural log, fp32).  Null: not written.
     float *lse;
+    // Optional fp32 output (bf16 path, one CTA per MMA, no chunk write):
+    // token-major [nq][heads][d] written instead of the bf16 `o`.
+    float *o_f32;
 };
 
 // Schedule of the persistent tensor-core kernel for one problem: units are

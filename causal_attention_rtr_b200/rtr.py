@@ -60,6 +60,7 @@ _SIGNATURES = [
     ("rtr_test_fail_allocs", _i, [_i, _i]),
     ("rtr_attn_frame_causal", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
     ("rtr_attn_frame_causal_ex", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _i, _vp]),
+    ("rtr_attn_frame_causal_f32out", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
     ("rtr_attn_frame_causal_commit", _i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _f, _vp]),
     ("rtr_attn_block_causal_prefill", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     ("rtr_attn_block_causal_prefill_ex", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _i, _i, _vp]),
@@ -224,6 +225,14 @@ def rtr_attn_frame_causal_ex(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale
     return _check(_lib.rtr_attn_frame_causal_ex(c, layer, _ptr(q), _ptr(k_cur), _ptr(v_cur), n_cur_frames,
                                                 _ptr(out), float(scale), cta_group, _stream(stream)),
                   "rtr_attn_frame_causal_ex")
+
+
+def rtr_attn_frame_causal_f32out(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale=0.0, stream=None):
+    """rtr_attn_frame_causal with an fp32 output tensor (the rows before the
+    bf16 rounding)."""
+    return _check(_lib.rtr_attn_frame_causal_f32out(c, layer, _ptr(q), _ptr(k_cur), _ptr(v_cur), n_cur_frames,
+                                                    _ptr(out), float(scale), _stream(stream)),
+                  "rtr_attn_frame_causal_f32out")
 
 
 def rtr_attn_frame_causal_commit(c, layer, q, k_cur, v_cur, n_cur_frames, out, scale=0.0, stream=None):

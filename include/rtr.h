@@ -205,6 +205,20 @@ rtr_status rtr_attn_frame_causal_ex(const rtr_kvcache *c, int layer,
                                     void *out, float scale, int cta_group,
                                     rtr_stream_t stream);
 
+/* rtr_attn_frame_causal with an fp32 output: out receives
+ * [n_cur_frames*k][heads][head_dim] fp32, the normalised rows before the
+ * bf16 rounding that rtr_attn_frame_causal applies (its bf16 output is
+ * exactly these values rounded to nearest even).  The pages fix no output
+ * precision; this entry point measures the bf16 path's error without its
+ * final rounding.  out must be 16-byte aligned; ownership stays with the
+ * caller.  On
+ * an fp32 cache this is rtr_attn_frame_causal.  Errors as for
+ * rtr_attn_frame_causal. */
+rtr_status rtr_attn_frame_causal_f32out(const rtr_kvcache *c, int layer,
+                                        const void *q, const void *k_cur,
+                                        const void *v_cur, int n_cur_frames,
+                                        float *out, float scale, rtr_stream_t stream);
+
 /* rtr_attn_frame_causal followed by the commit of the chunk, as in
  * rtr_kvcache_append_frame(c, layer, k_cur, v_cur, n_cur_frames), with the
  * chunk written by the attention launch itself (Key Designs 4: the chunk's
