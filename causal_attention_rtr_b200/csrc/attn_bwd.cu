@@ -200,20 +200,21 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16 *o, const __
 
 
 // ---------------------------------------------------------------- dK, dV
-// P^T and dS^T for 32 query columns of one key row, written packed as bf16
-// pairs: p = exp2(s * sl2 - l2) (0 for columns below `lo`), ds = p * (dp -
-// delta), with L*log2e and Delta of each column read from shared memory
+// P^T and dS^T for 16 query columns of one key row (scores s[s0 .. s0+15]),
+// written packed as bf16 pairs: p = exp2(s * sl2 - l2) (0 for columns below
+// `lo`), ds = p * (dp - delta), with L*log2e and Delta of each column read
+// from shared memory
 // (broadcast: every thread reads the same column).  The arithmetic is in
 // f32x2 pairs: scalar fp32 FMA, add and multiply instructions slow the
 // tensor core of the SM down (by almost half, in a probe where one warp
 // issues them beside an MMA loop), the paired forms hardly at all.
 template <bool MASK>
-__device__ __forceinline__ void pt_dst_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], const float *l2s,
-                                             const float *dls, float sl2, int lo, uint32_t (&pk)[16],
-                                             uint32_t (&dk)[16]) {
+__device__ __forceinline__ void pt_dst_piece(const uint32_t (&s)[32], int s0, const uint32_t (&dp)[16],
+                                             const float *l2s, const float *dls, float sl2, int lo,
+                                             uint32_t (&pk)[8], uint32_t (&dk)[8]) {
     const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) {
+    for (int e = 0; e < 16; e += 4) {
         const float4 l = *reinterpret_cast<const float4 *>(l2s + e);
         const float4 d = *reinterpret_cast<const float4 *>(dls + e);
         const float2 nl[2] = {make_float2(-l.x, -l.y), make_float2(-l.z, -l.w)};
@@ -221,7 +222,8 @@ __device__ __forceinline__ void pt_dst_chunk(const uint32_t (&s)[32], const uint
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int col = e + 2 * u;
-            const float2 x = ffma2(make_float2(__uint_as_float(s[col]), __uint_as_float(s[col + 1])), sl2x2, nl[u]);
+            const float2 x =
+                ffma2(make_float2(__uint_as_float(s[s0 + col]), __uint_as_float(s[s0 + col + 1])), sl2x2, nl[u]);
             float2 pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
             if (MASK) {
                 pr.x = col >= lo ? pr.x : 0.f;
@@ -281,9 +283,9 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) bwd_dkdv(const __grid_constan
     // TMEM: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D).
     // Step t (query tile i_first + t): the softmax reads the whole S^T row
     // into registers first, so S^T(t+1) can be computed into [0,128) while
-    // it works; P^T and dS^T of each 32-column group c go, packed, into the
-    // dP^T columns [128+32c, 128+32c+32) the group has just read (P^T in
-    // the first 16, dS^T in the last 16).  dV and dK of the first 64 query
+    // it works; P^T and dS^T of each 16-column group g go, packed, into the
+    // dP^T columns [128+16g, 128+16g+16) the group has just read (P^T in
+    // the first 8, dS^T in the last 8).  dV and dK of the first 64 query
     // columns start while the softmax does the other 64; dP^T(t+1) follows
     // the last of them.
 
@@ -324,11 +326,11 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) bwd_dkdv(const __grid_constan
 #pragma unroll
                 for (int kk = 0; kk < kHalf / 16; ++kk) {
                     const int q16 = h * (kHalf / 16) + kk;                       // 16-row group of queries
-                    const uint32_t col = 128 + 32 * (q16 >> 1) + 8 * (q16 & 1);  // its packed P^T columns
+                    const uint32_t col = 128 + 16 * q16;                         // its packed P^T, then dS^T
                     const uint32_t acc = (t > 0 || q16 > 0) ? 1u : 0u;
                     const uint64_t rows = (uint64_t)((q16 * 2048) >> 4);
                     mma_ts(tmem + 256, tmem + col, smem_desc_sw128(sb + L::kTile, 16384, 1024) + rows, idesc_o, acc);
-                    mma_ts(tmem + 256 + D, tmem + col + 16, smem_desc_sw128(sb, 16384, 1024) + rows, idesc_o, acc);
+                    mma_ts(tmem + 256 + D, tmem + col + 8, smem_desc_sw128(sb, 16384, 1024) + rows, idesc_o, acc);
                 }
             };
             bool ok = mbar_wait(bar(L::bA), 0, kBwdWaitNs) && full(0);
@@ -384,25 +386,33 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) bwd_dkdv(const __grid_constan
             w = __all_sync(0xffffffffu, w);
             if (!w) { ok = false; break; }
             tc_fence_after();
-            uint32_t s0[32], s1[32];
+            uint32_t s0[32], s1[32], dpa[16], dpb[16];
             tmem_ld32(tS, s0);
             tmem_ld32(tS + 32, s1);
+            tmem_ld16(tdP, dpa);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::bSread));   // S^T's columns are free for S^T(t+1)
             const int lo = q_lo - i * kBT - 64 * grp;      // columns below lo are hidden from this key
+            // 16-column pieces of this warp's 64: piece h's dP^T loads while
+            // piece h-1 is computed, and its P^T and dS^T (8 packed columns
+            // each) go over its own 16 dP^T columns
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t dp[32], pk[16], dk[16];
-                tmem_ld32(tdP + 32 * h, dp);
-                tmem_wait_ld();
-                if (__any_sync(0xffffffffu, lo - 32 * h > 0))   // warp-uniform: some column hidden
-                    pt_dst_chunk<true>(h ? s1 : s0, dp, l2s + 32 * h, dls + 32 * h, p.scale_log2, lo - 32 * h, pk, dk);
+            for (int h = 0; h < 4; ++h) {
+                uint32_t(&cur)[16] = (h & 1) ? dpb : dpa;
+                uint32_t(&nxt)[16] = (h & 1) ? dpa : dpb;
+                if (h + 1 < 4) tmem_ld16(tdP + 16 * (h + 1), nxt);
+                uint32_t pk[8], dk[8];
+                if (__any_sync(0xffffffffu, lo - 16 * h > 0))   // warp-uniform: some column hidden
+                    pt_dst_piece<true>(h < 2 ? s0 : s1, 16 * (h & 1), cur, l2s + 16 * h, dls + 16 * h,
+                                       p.scale_log2, lo - 16 * h, pk, dk);
                 else
-                    pt_dst_chunk<false>(h ? s1 : s0, dp, l2s + 32 * h, dls + 32 * h, p.scale_log2, 0, pk, dk);
-                tmem_st16(tdP + 32 * h, pk);
-                tmem_st16(tdP + 32 * h + 16, dk);
+                    pt_dst_piece<false>(h < 2 ? s0 : s1, 16 * (h & 1), cur, l2s + 16 * h, dls + 16 * h,
+                                        p.scale_log2, 0, pk, dk);
+                tmem_st8(tdP + 16 * h, pk);
+                tmem_st8(tdP + 16 * h + 8, dk);
+                if (h + 1 < 4) tmem_wait_ld_regs16(nxt);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -445,7 +455,7 @@ __global__ void __launch_bounds__(kDkdvThreads, 1) bwd_dkdv(const __grid_constan
 // dS for 32 key columns [32c, 32c+32) of one query row, packed as bf16
 // pairs: p = exp2(s * sl2 - l2) (0 for columns at or past `hi`),
 // ds = p * (dp - delta), dp from the row's registers; f32x2 arithmetic (see
-// pt_dst_chunk).
+// pt_dst_piece).
 template <bool MASK>
 __device__ __forceinline__ void ds_chunk(const uint32_t (&s)[32], const uint32_t (&dpr)[128], int c, float l2,
                                          float dl, float sl2, int hi, uint32_t (&dk)[16]) {
