@@ -97,6 +97,19 @@ bool make_tmap_bf16_strided(CUtensorMap *m, const void *base, uint64_t d, uint64
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_rows256(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || !aligned16(base) || rows < box_rows) return false;
+    cuuint64_t dims[3] = {128, rows, 1};
+    cuuint64_t strides[2] = {256, rows * 256};
+    cuuint32_t box[3] = {128, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 std::atomic<unsigned long long> g_launches{0};
 }
@@ -1012,6 +1025,19 @@ rtr_status rtr_dit_qkv_rope(const void *a, const void *wqkv, const void *bqkv, i
     g.bias = bqkv; g.q = q; g.k_out = k; g.v = v;
     g.head_dim = head_dim; g.kpf = k_per_frame; g.grid_w = grid_w; g.t0 = t0;
     return cuda_status(launch_gemm_bf16(g, status, sm_count(device), (cudaStream_t)stream));
+}
+
+rtr_status rtr_dit_linear_tile(int m, int n, int k, rtr_epilogue epilogue, int qkv_rope, int device, int *rows,
+                               int *cols, int *cta_pair, int *ctas) {
+    if (m < 1 || n < 1 || k < 1 || device < 0 || !rows || !cols || !cta_pair || !ctas ||
+        (epilogue != RTR_EPI_BIAS && epilogue != RTR_EPI_BIAS_GELU && epilogue != RTR_EPI_GATED_RESIDUAL))
+        return RTR_E_INVAL;
+    const int epi = qkv_rope ? kEpiQkvRope
+                    : epilogue == RTR_EPI_BIAS ? kEpiBias
+                    : epilogue == RTR_EPI_BIAS_GELU ? kEpiBiasGelu : kEpiGatedResidual;
+    DeviceGuard dg(device);
+    gemm_tile_shape(m, n, k, epi, device, sm_count(device), rows, cols, cta_pair, ctas);
+    return RTR_OK;
 }
 
 rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_text, rtr_dtype dt, int device,

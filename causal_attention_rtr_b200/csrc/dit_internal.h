@@ -72,4 +72,9 @@ struct GemmArgs {
 // `sms` CTAs); a bounded wait that expires latches RTR_E_TIMEOUT in *status.
 cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaStream_t s);
 
+// The tile launch_gemm_bf16 picks for an m x n x k product on `device`
+// (rows, columns, whether a CTA pair shares it) and the CTAs it launches.
+void gemm_tile_shape(int m, int n, int k, int epi, int device, int sms, int *rows, int *cols, int *pair,
+                     int *ctas);
+
 }  // namespace rtr

@@ -42,6 +42,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -143,17 +144,59 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     }
 }
 
+// The same with cluster-scope acquire, for barriers the peer CTA of a pair
+// signals (its commits and its epilogue's releases).
+__device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitNs) return false;
+    }
+}
+
 __device__ __forceinline__ void raise_timeout(const GemmParams &p, volatile int *abort_flag) {
     *abort_flag = 1;
     atomicExch(p.status, (unsigned)RTR_E_TIMEOUT);
 }
 
-// The epilogue of 32 consecutive accumulator columns [col, col + 32) of one
-// row (nvalid of them inside the matrix, a multiple of 8), in f32x2 pairs.
-// `rope` is the shared-memory rotary table (null: angles computed here).
+// The global inputs of one 32-column chunk of a row: bias (all epilogues),
+// and for the gated residual the residual x and the gate.  They are loaded
+// together, before the chunk's accumulators arrive from TMEM and before any
+// of the chunk's stores, so their latencies overlap (loads issued one
+// 8-column group at a time, each after the previous group's store, paid a
+// DRAM round trip per group and made the epilogue, not the MMAs, bound the
+// projection).
+struct EpiIn {
+    uint4 b[4], x[4], g[4];
+};
+
+__device__ __forceinline__ uint4 ld_nc(const __nv_bfloat16 *ptr) {
+    return __ldg(reinterpret_cast<const uint4 *>(ptr));
+}
+
 template <int EPI>
-__device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&acc)[32], long long row, int col,
-                                          int nvalid, int f_pos, int y_pos, int x_pos, const float2 *rope) {
+__device__ __forceinline__ void epi_load(const GemmParams &p, long long row, int col, int nvalid, EpiIn &in) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        if (8 * g >= nvalid) break;
+        in.b[g] = ld_nc(p.bias + col + 8 * g);
+        if (EPI == kEpiGatedResidual) {
+            in.x[g] = *reinterpret_cast<const uint4 *>(p.out + row * p.n + col + 8 * g);
+            if (p.gate != nullptr) in.g[g] = ld_nc(p.gate + col + 8 * g);
+        }
+    }
+}
+
+// The epilogue of 32 consecutive accumulator columns [col, col + 32) of one
+// row (nvalid of them inside the matrix, a multiple of 8), in f32x2 pairs,
+// from the chunk's inputs `in`.  `rope` is the shared-memory rotary table
+// (null: angles computed here).
+template <int EPI>
+__device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&acc)[32], const EpiIn &in,
+                                          long long row, int col, int nvalid, int f_pos, int y_pos, int x_pos,
+                                          const float2 *rope) {
     if (EPI == kEpiQkvRope) {
         const int part = col / p.D, cc = col - part * p.D;
         __nv_bfloat16 *dst = (part == 0 ? p.q : part == 1 ? p.kk : p.v) + row * p.D + cc;
@@ -163,7 +206,7 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
         for (int g = 0; g < 4; ++g) {
             if (8 * g >= nvalid) break;
             float b[8], r[8];
-            unpack8(*reinterpret_cast<const uint4 *>(p.bias + col + 8 * g), b);
+            unpack8(in.b[g], b);
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
                 float2 v = fadd2(make_float2(__uint_as_float(acc[8 * g + e]), __uint_as_float(acc[8 * g + e + 1])),
@@ -195,10 +238,10 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
         for (int g = 0; g < 4; ++g) {
             if (8 * g >= nvalid) break;
             float b[8], xv[8], gt[8], r[8];
-            unpack8(*reinterpret_cast<const uint4 *>(p.bias + col + 8 * g), b);
-            unpack8(*reinterpret_cast<const uint4 *>(x + 8 * g), xv);
+            unpack8(in.b[g], b);
+            unpack8(in.x[g], xv);
             if (p.gate != nullptr) {
-                unpack8(*reinterpret_cast<const uint4 *>(p.gate + col + 8 * g), gt);
+                unpack8(in.g[g], gt);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) gt[e] = 1.f;
@@ -219,7 +262,7 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
         for (int g = 0; g < 4; ++g) {
             if (8 * g >= nvalid) break;
             float b[8], r[8];
-            unpack8(*reinterpret_cast<const uint4 *>(p.bias + col + 8 * g), b);
+            unpack8(in.b[g], b);
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
                 float2 v = fadd2(make_float2(__uint_as_float(acc[8 * g + e]), __uint_as_float(acc[8 * g + e + 1])),
@@ -237,15 +280,23 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
     }
 }
 
-template <int EPI>
+// PAIR: a cluster of two CTAs works each 256 x 256 tile with cta_group::2
+// MMAs issued by its first CTA (rank 0).  Rank r loads A rows [128 r, 128 r +
+// 128) and W columns [128 r, 128 r + 128) of the tile into its own shared
+// memory, counted on rank 0's stage barrier; each CTA's TMEM holds the fp32
+// accumulator of its own 128 rows (all 256 columns), which its own epilogue
+// warps drain.  Per SM and K block that is 32 KB of operands for 128 x 256
+// x 64 of MMA work, two thirds of what a 128 x 256 tile of one CTA loads.
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t s_base = smem_u32(smem);
     const int S = p.stages;
     const int a_bytes = p.msub * kATileBytes;               // A sub-tiles, then W boxes
-    const int stage_bytes = a_bytes + (p.bn / 64) * kBBoxBytes;
-    const int BMt = kBM * p.msub;                              // rows per tile
+    const int w_cols = PAIR ? p.bn / 2 : p.bn;                 // W columns held by this CTA
+    const int stage_bytes = a_bytes + (w_cols / 64) * kBBoxBytes;
+    const int BMt = kBM * p.msub * (PAIR ? 2 : 1);             // rows per tile
     const uint32_t bars = s_base + (uint32_t)(S * stage_bytes);
     // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain, rope table ready
     auto full = [&](int s) { return bars + 8u * (uint32_t)s; };
@@ -260,6 +311,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
     float2 *rope_tab = reinterpret_cast<float2 *>(misc + 16);   // p.rope_entries of them
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // pair: rank 0 issues the MMAs; both CTAs' loads and epilogue releases
+    // count on rank 0's barriers (`lead`)
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    auto lead = [&](uint32_t b) -> uint32_t { return PAIR ? mapa_shared(b, 0) : b; };
+    auto wait_lead = [&](uint32_t b, uint32_t parity) -> bool {
+        return PAIR ? wait_bar_cluster(b, parity, abort_flag) : wait_bar(b, parity, abort_flag);
+    };
+    const int cl = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;     // cluster (or CTA)
+    const int n_cl = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full(s), 1);
@@ -267,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf(b), 1);
-            mbar_init(acce(b), kEpiWarps);
+            mbar_init(acce(b), PAIR ? 2 * kEpiWarps : kEpiWarps);
         }
         mbar_init(drain, 1);
         mbar_init(rope_ready, kEpiWarps * 32);
@@ -275,15 +335,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         mbar_fence_init();
     }
     if (warp == 0 && lane == 0) {
-        if (!p.a_pk) prefetch_tmap(&p.tm_a);
-        if (!p.w_pk) prefetch_tmap(&p.tm_w);
+        if (PAIR || !p.a_pk) prefetch_tmap(&p.tm_a);
+        if (PAIR || !p.w_pk) prefetch_tmap(&p.tm_w);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_holder), 512);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(smem_u32(tmem_holder), 512);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_holder), 512);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();                  // the peer's barriers exist before anything signals them
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
@@ -292,8 +358,53 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         if (lane == 0) {
             int it = 0;                                  // stage loads issued
             bool ok = true;
-            for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+            for (int t = cl; t < p.n_tiles && ok; t += n_cl) {
                 const int m0 = (t / p.n_tiles_n) * BMt, n0 = (t % p.n_tiles_n) * p.bn;
+                if (PAIR) {
+                    // rank r: A rows from m0 + 128 r (loaded if they start below
+                    // m) and the 64-column W boxes from n0 + 128 r that start
+                    // inside the matrix; what is not loaded keeps stale data,
+                    // which reaches only discarded rows and columns
+                    auto a_in = [&](int r) { return m0 + r * kBM < p.m ? 1 : 0; };
+                    auto w_in = [&](int r) {
+                        const int c0 = n0 + r * 128;
+                        return max(0, min(2, (p.n - c0 + 63) / 64));
+                    };
+                    const uint32_t tx = (uint32_t)((a_in(0) + a_in(1)) * kATileBytes +
+                                                   (w_in(0) + w_in(1)) * kBBoxBytes);
+                    const int my_m0 = m0 + (int)rank * kBM, my_n0 = n0 + (int)rank * 128;
+                    const int my_a = a_in((int)rank), my_w = w_in((int)rank);
+                    for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                        const int s = it % S, use = it / S;
+                        if (use > 0 && !wait_lead(empty(s), (use - 1) & 1)) {
+                            raise_timeout(p, abort_flag);
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t sa = s_base + (uint32_t)(s * stage_bytes);
+                        const uint32_t fb = lead(full(s));
+                        if (rank == 0) mbar_arrive_tx(full(s), tx);
+                        if (my_a) {
+                            if (p.a_pk) {
+                                // packed A as rows of 256 bytes: a 16 KB tile image is 64 of them
+                                const int r0 = ((my_m0 / kBM) * p.kb_total + kb) * 64;
+                                tma_load_3d_pair(sa, &p.tm_a, fb, 0, r0, 0);
+                                tma_load_3d_pair(sa + kATileBytes / 2, &p.tm_a, fb, 0, r0 + 32, 0);
+                            } else {
+                                tma_load_3d_pair(sa, &p.tm_a, fb, kb * kBK, my_m0, 0);
+                            }
+                        }
+                        for (int j = 0; j < my_w; ++j) {
+                            if (p.w_pk)   // an 8 KB box image is 32 rows of 256 bytes
+                                tma_load_3d_pair(sa + a_bytes + j * kBBoxBytes, &p.tm_w, fb, 0,
+                                                 (kb * p.nb_total + my_n0 / 64 + j) * 32, 0);
+                            else
+                                tma_load_3d_pair(sa + a_bytes + j * kBBoxBytes, &p.tm_w, fb, my_n0 + 64 * j,
+                                                 kb * kBK, 0);
+                        }
+                    }
+                    continue;
+                }
                 // packed B: the tile's 64-column boxes that exist (the rest of
                 // the stage keeps stale data, which reaches only discarded columns)
                 const int w_boxes = p.w_pk ? min(p.bn / 64, p.nb_total - n0 / 64) : p.bn / 64;
@@ -327,8 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                 }
             }
             // Loads still in flight land before the CTA can exit: wait for
-            // the last load of every stage (bounded).
-            for (int s = 0; s < S && s < it; ++s) {
+            // the last load of every stage (bounded).  Pair: both CTAs' loads
+            // count on rank 0's barriers, and neither CTA leaves before the
+            // other (the cluster barrier at the end).
+            for (int s = 0; rank == 0 && s < S && s < it; ++s) {
                 const int last = ((it - 1 - s) / S) * S + s;   // last load index that used stage s
                 mbar_wait(full(s), (last / S) & 1, kWaitNs);
             }
@@ -336,22 +449,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(kBM, p.bn, 0, 1);
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kBM : kBM, p.bn, 0, 1);
             int it = 0, tc = 0;                          // stages consumed, tiles done
             bool ok = true;
-            for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++tc) {
+            for (int t = cl; t < p.n_tiles && ok; t += n_cl, ++tc) {
                 const int b = tc % p.nbuf, use_b = tc / p.nbuf;
                 const int m0 = (t / p.n_tiles_n) * BMt;
-                const int a_subs = min(p.msub, (p.m - m0 + kBM - 1) / kBM);
-                if (use_b > 0 && !wait_bar(acce(b), (use_b - 1) & 1, abort_flag)) {
+                const int a_subs = PAIR ? 1 : min(p.msub, (p.m - m0 + kBM - 1) / kBM);
+                if (use_b > 0 && !wait_lead(acce(b), (use_b - 1) & 1)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % S;
-                    if (!wait_bar(full(s), (it / S) & 1, abort_flag)) {
+                    if (!wait_lead(full(s), (it / S) & 1)) {
                         ok = false;
                         break;
                     }
@@ -363,18 +476,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                         const uint64_t da = smem_desc_sw128(sa + u * kATileBytes, 16, 1024);
                         const uint32_t d_tmem = tmem + (uint32_t)(b * 256 + u * p.bn);
 #pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk)
-                            mma_ss(d_tmem, da + (uint64_t)((kk * 32) >> 4), dw + (uint64_t)((kk * 2048) >> 4), idesc,
-                                   (kb > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            const uint64_t a_k = da + (uint64_t)((kk * 32) >> 4);
+                            const uint64_t w_k = dw + (uint64_t)((kk * 2048) >> 4);
+                            if (PAIR) mma_ss_pair(d_tmem, a_k, w_k, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                            else mma_ss(d_tmem, a_k, w_k, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
-                    tc_commit(empty(s));
+                    if (PAIR) tc_commit_pair(empty(s));
+                    else tc_commit(empty(s));
                 }
                 if (!ok) break;
-                tc_commit(accf(b));
+                if (PAIR) tc_commit_pair(accf(b));
+                else tc_commit(accf(b));
             }
             if (!ok) raise_timeout(p, abort_flag);
             // every MMA issued above completes before TMEM is freed
-            tc_commit(drain);
+            if (PAIR) tc_commit_pair(drain);
+            else tc_commit(drain);
             mbar_wait(drain, 0, kWaitNs);
         }
         __syncwarp();
@@ -406,10 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
         // chunks; two sub-tiles: warp half u takes all chunks of sub-tile u
         const int sub = p.msub == 2 ? half : 0;
         const int c_first = p.msub == 2 ? 0 : half, c_step = p.msub == 2 ? 1 : 2;
-        for (int t = blockIdx.x; ok && t < p.n_tiles; t += gridDim.x, ++tc) {
+        for (int t = cl; ok && t < p.n_tiles; t += n_cl, ++tc) {
             const int b = tc % p.nbuf, use_b = tc / p.nbuf;
-            const int m0 = (t / p.n_tiles_n) * BMt, n0 = (t % p.n_tiles_n) * p.bn;
-            bool w = wait_bar(accf(b), use_b & 1, abort_flag);
+            const int m0 = (t / p.n_tiles_n) * BMt + (int)rank * kBM, n0 = (t % p.n_tiles_n) * p.bn;
+            bool w = wait_lead(accf(b), use_b & 1);
             w = __all_sync(0xffffffffu, w);
             if (!w) {
                 ok = false;
@@ -426,90 +545,174 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                 y_pos = r / p.grid_w;
                 x_pos = r - y_pos * p.grid_w;
             }
+            // chunk c's inputs are loaded while chunk c - c_step is computed
+            EpiIn in;
+            if (sub_live && row_ok && n0 + 32 * c_first < p.n)
+                epi_load<EPI>(p, row, n0 + 32 * c_first, min(32, p.n - (n0 + 32 * c_first)), in);
             for (int c = c_first; sub_live && c < p.bn / 32; c += c_step) {
                 const int col = n0 + 32 * c;
                 if (col >= p.n) break;                   // warp-uniform
                 uint32_t acc[32];
                 tmem_ld32(tmem + lane_bits + (uint32_t)(b * 256 + sub * p.bn + 32 * c), acc);
+                EpiIn next;
+                const int col_n = col + 32 * c_step;
+                if (row_ok && c + c_step < p.bn / 32 && col_n < p.n)
+                    epi_load<EPI>(p, row, col_n, min(32, p.n - col_n), next);
                 tmem_wait_ld();
-                if (row_ok) epi_chunk<EPI>(p, acc, row, col, min(32, p.n - col), f_pos, y_pos, x_pos, rope);
+                if (row_ok) epi_chunk<EPI>(p, acc, in, row, col, min(32, p.n - col), f_pos, y_pos, x_pos, rope);
+                in = next;
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acce(b));
+            if (lane == 0) {
+                if (PAIR) mbar_arrive_cluster(lead(acce(b)));
+                else mbar_arrive(acce(b));
+            }
         }
         if (!ok) raise_timeout(p, abort_flag);
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();                  // neither CTA leaves while the pair's MMAs may touch it
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == 1) {
+        if (PAIR) tmem_dealloc_pair(tmem, 512);
+        else tmem_dealloc(tmem, 512);
+    }
 }
 
-template <int EPI>
+template <int EPI, bool PAIR>
 cudaError_t set_smem_attr_once() {
     static std::once_flag once;
     static cudaError_t err = cudaSuccess;
     std::call_once(once, [] {
-        err = cudaFuncSetAttribute(gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        err = cudaFuncSetAttribute(gemm_tc<EPI, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    kMaxSmem + 2048 + kRopeTabMax * 8);
     });
     return err;
 }
 
-// Tile shape (128 rows by 128, 192 or 256 columns, or 256 by 256): the candidate
-// whose rounds of `sms` tiles take the least time under a model measured on
-// B200.  Per 64-deep K block a tile takes the longer of
+// Tile shape (128 rows by 128, 192 or 256 columns, 256 by 256 on one CTA,
+// or 256 by 256 on a CTA pair): the candidate whose rounds of tiles take the
+// least time under a model measured on B200.  Per 64-deep K block a tile
+// takes the longer of
 //   its MMAs: 128 x N x 16 costs 85, 106 or 128 cycles for N = 128, 192,
-//     256 (one per k16 step and 128-row sub-tile), and
+//     256 (one per k16 step and 128-row sub-tile); the pair's 256 x 256 x 16
+//     runs at 128 per SM alone but takes about 232 in this kernel, with the
+//     stage loads in flight (clock stamps of its K blocks), and
 //   its loads: stages in flight over a loaded round trip of about 4,400
 //     cycles (the latency times the bandwidth of the memory system reaching
 //     one SM is the shared memory that holds the stages, so a stage's bytes
 //     arrive every latency / stages cycles, whatever their size).
-// A tile whose two accumulators fill TMEM (256 x 256) cannot overlap its
-// epilogue with the next tile's MMAs: it pays about 2,000 more cycles for a
-// light epilogue (bias, gated residual).  Heavy epilogues (GELU's tanh, the
-// rotary sine and cosine) take longer than that per 256 x 256 tile (the
-// GELU projection measured 184 against 144 us), so they keep 128-row tiles,
-// whose two buffers hide the epilogue behind the next tile's MMAs.
+// A 256 x 256 tile on one CTA fills TMEM with its two accumulators and
+// cannot overlap its epilogue with the next tile's MMAs: it pays about 2,000
+// more cycles for a light epilogue (bias, gated residual).  Heavy epilogues
+// (GELU's tanh, the rotary sine and cosine) take longer than that per 256 x
+// 256 tile (the GELU projection measured 184 against 144 us), so there they
+// are not candidates.  A pair's tile holds 128 x 256 per SM, so it keeps two
+// accumulator buffers; its rounds are of sms / 2 tiles.
 struct TileShape {
-    int msub, bn, stages;
+    int msub, bn, stages, pair;
 };
 
-int stage_bytes_of(int msub, int bn) { return msub * kATileBytes + (bn / 64) * kBBoxBytes; }
+int stage_bytes_of(int msub, int bn, int pair) { return msub * kATileBytes + (bn / (pair ? 128 : 64)) * kBBoxBytes; }
 
-TileShape pick_tile(int m, int n, int k, int sms, bool heavy_epilogue) {
+TileShape pick_tile(int m, int n, int k, int sms, int pair_slots, bool heavy_epilogue) {
     const int k_blocks = (k + kBK - 1) / kBK;
-    TileShape best = {1, 256, 4};
+    TileShape best = {1, 256, 4, 0};
     double best_cost = -1.0;
-    // 256-row tiles only with 256 columns: narrower ones load the same A
-    // per K block for less MMA work and never win under this model
-    for (int msub : {2, 1})
-        for (int bn : {256, 192, 128}) {
-            if (msub == 2 && (bn != 256 || heavy_epilogue)) continue;
-            const int stages = std::min(8, kMaxSmem / stage_bytes_of(msub, bn));
-            const double mma = msub * 4.0 * (bn == 256 ? 128.0 : bn == 192 ? 106.0 : 85.0);
-            const double load = 4400.0 / stages;
-            const double epi = msub * bn > 256 ? 2000.0 : 0.0;
-            const long long tiles = (long long)((m + kBM * msub - 1) / (kBM * msub)) * ((n + bn - 1) / bn);
-            const long long rounds = (tiles + sms - 1) / sms;
-            const double cost = rounds * (k_blocks * std::max(mma, load) + epi);
-            if (best_cost < 0 || cost < best_cost * 0.999) {
-                best_cost = cost;
-                best = {msub, bn, stages};
-            }
+    struct Cand { int msub, bn, pair; };
+    for (const Cand c : {Cand{1, 256, 1}, Cand{2, 256, 0}, Cand{1, 256, 0}, Cand{1, 192, 0}, Cand{1, 128, 0}}) {
+        if (c.msub == 2 && heavy_epilogue) continue;
+        if (c.pair && pair_slots < 1) continue;
+        const int stages = std::min(8, kMaxSmem / stage_bytes_of(c.msub, c.bn, c.pair));
+        const double mma = c.pair ? 4.0 * 232.0 : c.msub * 4.0 * (c.bn == 256 ? 128.0 : c.bn == 192 ? 106.0 : 85.0);
+        const double load = 4400.0 / stages;
+        const double epi = !c.pair && c.msub * c.bn > 256 ? 2000.0 : 0.0;
+        const int rows = kBM * c.msub * (c.pair ? 2 : 1);
+        const long long tiles = (long long)((m + rows - 1) / rows) * ((n + c.bn - 1) / c.bn);
+        const int slots = c.pair ? pair_slots : sms;
+        const long long rounds = (tiles + slots - 1) / slots;
+        const double cost = rounds * (k_blocks * std::max(mma, load) + epi);
+        if (best_cost < 0 || cost < best_cost * 0.999) {
+            best_cost = cost;
+            best = {c.msub, c.bn, stages, c.pair};
         }
+    }
     return best;
 }
 
-template <int EPI>
+template <int EPI, bool PAIR>
 cudaError_t launch_epi(const GemmParams &p, int grid, int smem, cudaStream_t s) {
-    const cudaError_t e = set_smem_attr_once<EPI>();
+    const cudaError_t e = set_smem_attr_once<EPI, PAIR>();
     if (e != cudaSuccess) return e;
-    gemm_tc<EPI><<<grid, kThreads, smem, s>>>(p);
-    const cudaError_t le = cudaGetLastError();
+    cudaError_t le;
+    if (PAIR) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        le = cudaLaunchKernelEx(&cfg, gemm_tc<EPI, PAIR>, p);
+    } else {
+        gemm_tc<EPI, PAIR><<<grid, kThreads, smem, s>>>(p);
+        le = cudaGetLastError();
+    }
     if (le == cudaSuccess) count_launch();
     return le;
+}
+
+// Clusters of two CTAs of gemm_tc<EPI, true> that can be resident at once
+// on `device` (at most sms / 2): the two CTAs of a cluster take two SMs of
+// one GPC, so a GPC with an odd number of SMs leaves one of them out.  0 if
+// the query fails (no pair launches then).
+template <int EPI>
+int pair_slots_of(int device, int sms) {
+    static std::atomic<int> cache[64] = {};
+    if (device < 0 || device >= 64) return 0;
+    int n = cache[device].load(std::memory_order_relaxed);
+    if (n) return n > 0 ? n : 0;
+    n = -1;
+    if (set_smem_attr_once<EPI, true>() == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (sms / 2 > 0 ? sms / 2 : 1));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kMaxSmem + 2048 + kRopeTabMax * 8;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int c = 0;
+        if (cudaOccupancyMaxActiveClusters(&c, gemm_tc<EPI, true>, &cfg) == cudaSuccess && c > 0)
+            n = std::min(c, sms / 2);
+    }
+    cudaGetLastError();
+    cache[device].store(n, std::memory_order_relaxed);
+    return n > 0 ? n : 0;
+}
+
+int pair_slots(int epi, int device, int sms) {
+    switch (epi) {
+        case kEpiBias: return pair_slots_of<kEpiBias>(device, sms);
+        case kEpiBiasGelu: return pair_slots_of<kEpiBiasGelu>(device, sms);
+        case kEpiGatedResidual: return pair_slots_of<kEpiGatedResidual>(device, sms);
+        default: return pair_slots_of<kEpiQkvRope>(device, sms);
+    }
+}
+
+template <int EPI>
+cudaError_t launch_epi(const GemmParams &p, int grid, int smem, bool pair, cudaStream_t s) {
+    return pair ? launch_epi<EPI, true>(p, grid, smem, s) : launch_epi<EPI, false>(p, grid, smem, s);
 }
 
 }  // namespace
@@ -527,24 +730,39 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
     if (g.out_packed && g.epi != kEpiBias && g.epi != kEpiBiasGelu) return cudaErrorInvalidValue;
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    if ((!g.a_packed && !make_tmap_bf16(&p.tm_a, g.a, (uint64_t)g.k, (uint64_t)g.m, 1, kBM, 1)) ||
-        (!g.w_packed && !make_tmap_bf16(&p.tm_w, g.w, (uint64_t)g.n, (uint64_t)g.k, 1, kBK, 1)))
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess) return cudaErrorInvalidValue;
+    const int slots2 = pair_slots(g.epi, device, sms);
+    const TileShape ts = pick_tile(g.m, g.n, g.k, sms, slots2, g.epi == kEpiBiasGelu || g.epi == kEpiQkvRope);
+    // Row-major operands load by 128-byte-swizzled TMA boxes.  Packed ones
+    // load by 1-D bulk copies, or, on a CTA pair (whose loads must count on
+    // the first CTA's barrier), by unswizzled boxes of 256-byte rows, which
+    // land byte for byte as they lie in memory.
+    if (g.a_packed && ts.pair) {
+        if (!make_tmap_rows256(&p.tm_a, g.a, packed_a_bytes(g.m, g.k) / 256, 32)) return cudaErrorInvalidValue;
+    } else if (!g.a_packed && !make_tmap_bf16(&p.tm_a, g.a, (uint64_t)g.k, (uint64_t)g.m, 1, kBM, 1)) {
         return cudaErrorInvalidValue;
+    }
+    if (g.w_packed && ts.pair) {
+        if (!make_tmap_rows256(&p.tm_w, g.w, packed_b_bytes(g.k, g.n) / 256, 32)) return cudaErrorInvalidValue;
+    } else if (!g.w_packed && !make_tmap_bf16(&p.tm_w, g.w, (uint64_t)g.n, (uint64_t)g.k, 1, kBK, 1)) {
+        return cudaErrorInvalidValue;
+    }
     p.a_pk = g.a_packed ? static_cast<const char *>(g.a) : nullptr;
     p.w_pk = g.w_packed ? static_cast<const char *>(g.w) : nullptr;
     p.kb_total = g.k / 64;
     p.nb_total = g.n / 64;
     p.out_packed = g.out_packed;
     p.m = g.m; p.n = g.n; p.k = g.k;
-    const TileShape ts = pick_tile(g.m, g.n, g.k, sms, g.epi == kEpiBiasGelu || g.epi == kEpiQkvRope);
     p.msub = ts.msub;
     p.bn = ts.bn;
     p.stages = ts.stages;
     p.nbuf = p.msub * p.bn <= 256 ? 2 : 1;
     p.n_tiles_n = (g.n + p.bn - 1) / p.bn;
-    p.n_tiles = ((g.m + kBM * p.msub - 1) / (kBM * p.msub)) * p.n_tiles_n;
+    const int tile_rows = kBM * p.msub * (ts.pair ? 2 : 1);
+    p.n_tiles = ((g.m + tile_rows - 1) / tile_rows) * p.n_tiles_n;
     p.k_blocks = (g.k + kBK - 1) / kBK;
-    const int stage_bytes = stage_bytes_of(p.msub, p.bn);
+    const int stage_bytes = stage_bytes_of(p.msub, p.bn, ts.pair);
     p.bias = static_cast<const __nv_bfloat16 *>(g.bias);
     p.gate = static_cast<const __nv_bfloat16 *>(g.gate);
     p.out = static_cast<__nv_bfloat16 *>(g.out);
@@ -568,16 +786,32 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
         p.rope_entries = entries <= kRopeTabMax ? (int)entries : 0;
     }
     p.status = status;
-    const int grid = p.n_tiles < sms ? p.n_tiles : sms;
+    // one CTA (pair: one cluster of two) per SM (pair of SMs) at most
+    const int slots = ts.pair ? slots2 : sms;
+    const int grid = (p.n_tiles < slots ? p.n_tiles : slots) * (ts.pair ? 2 : 1);
     // stages, barriers (2S + 6), the TMEM holder and the abort flag, the
     // rotary table, plus slack for the 1 KB alignment of the stage ring
     const int smem = p.stages * stage_bytes + 8 * (2 * p.stages + 6) + 16 + p.rope_entries * 8 + 1024;
+    const bool pair = ts.pair != 0;
     switch (g.epi) {
-        case kEpiBias: return launch_epi<kEpiBias>(p, grid, smem, s);
-        case kEpiBiasGelu: return launch_epi<kEpiBiasGelu>(p, grid, smem, s);
-        case kEpiGatedResidual: return launch_epi<kEpiGatedResidual>(p, grid, smem, s);
-        default: return launch_epi<kEpiQkvRope>(p, grid, smem, s);
+        case kEpiBias: return launch_epi<kEpiBias>(p, grid, smem, pair, s);
+        case kEpiBiasGelu: return launch_epi<kEpiBiasGelu>(p, grid, smem, pair, s);
+        case kEpiGatedResidual: return launch_epi<kEpiGatedResidual>(p, grid, smem, pair, s);
+        default: return launch_epi<kEpiQkvRope>(p, grid, smem, pair, s);
     }
+}
+
+void gemm_tile_shape(int m, int n, int k, int epi, int device, int sms, int *rows, int *cols, int *pair,
+                     int *ctas) {
+    const int slots2 = pair_slots(epi, device, sms);
+    const TileShape ts = pick_tile(m, n, k, sms, slots2, epi == kEpiBiasGelu || epi == kEpiQkvRope);
+    const int tile_rows = kBM * ts.msub * (ts.pair ? 2 : 1);
+    const long long tiles = (long long)((m + tile_rows - 1) / tile_rows) * ((n + ts.bn - 1) / ts.bn);
+    const int slots = ts.pair ? slots2 : sms;
+    *rows = tile_rows;
+    *cols = ts.bn;
+    *pair = ts.pair;
+    *ctas = (int)std::min<long long>(tiles, slots) * (ts.pair ? 2 : 1);
 }
 
 }  // namespace rtr

@@ -73,6 +73,8 @@ _SIGNATURES = [
     ("rtr_dit_block_forward_packed", _i, [_vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     ("rtr_dit_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
     ("rtr_dit_qkv_rope", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
+    ("rtr_dit_linear_tile", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
+                                 ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     ("rtr_attn_block_causal_backward", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f,
                                             _i, _vp]),
     ("rtr_crossattn_create", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
@@ -292,12 +294,15 @@ def rtr_dit_block_forward_packed(c, x, layer, pw, modulation, hidden, n_cur_fram
                   "rtr_dit_block_forward_packed")
 
 
+def _epilogue(epilogue):
+    return int({"bias": RTR_EPI_BIAS, "gelu": RTR_EPI_BIAS_GELU,
+                "gated_residual": RTR_EPI_GATED_RESIDUAL}.get(epilogue, epilogue))
+
+
 def rtr_dit_linear(a, w, m, n, k, epilogue, bias, gate, out, device=0, stream=None):
     """out = epilogue(a w + bias) on the tensor cores (see include/rtr.h)."""
-    epi = {"bias": RTR_EPI_BIAS, "gelu": RTR_EPI_BIAS_GELU, "gated_residual": RTR_EPI_GATED_RESIDUAL}.get(epilogue,
-                                                                                                       epilogue)
-    return _check(_lib.rtr_dit_linear(_ptr(a), _ptr(w), m, n, k, int(epi), _ptr(bias), _ptr(gate), _ptr(out),
-                                      device, _stream(stream)), "rtr_dit_linear")
+    return _check(_lib.rtr_dit_linear(_ptr(a), _ptr(w), m, n, k, _epilogue(epilogue), _ptr(bias), _ptr(gate),
+                                      _ptr(out), device, _stream(stream)), "rtr_dit_linear")
 
 
 def rtr_dit_qkv_rope(a, wqkv, bqkv, m, d_in, heads, head_dim, k_per_frame, grid_w, t0, q, k, v, device=0,
@@ -306,6 +311,16 @@ def rtr_dit_qkv_rope(a, wqkv, bqkv, m, d_in, heads, head_dim, k_per_frame, grid_
     return _check(_lib.rtr_dit_qkv_rope(_ptr(a), _ptr(wqkv), _ptr(bqkv), m, d_in, heads, head_dim, k_per_frame,
                                         grid_w, t0, _ptr(q), _ptr(k), _ptr(v), device, _stream(stream)),
                   "rtr_dit_qkv_rope")
+
+
+def rtr_dit_linear_tile(m, n, k, epilogue, qkv_rope=False, device=0):
+    """(rows, cols, cta_pair, ctas) of the tile the projection picks and its
+    launch's CTAs (see include/rtr.h)."""
+    rows, cols, pair, ctas = _i(), _i(), _i(), _i()
+    _check(_lib.rtr_dit_linear_tile(m, n, k, _epilogue(epilogue), int(bool(qkv_rope)), device, ctypes.byref(rows),
+                                    ctypes.byref(cols), ctypes.byref(pair), ctypes.byref(ctas)),
+           "rtr_dit_linear_tile")
+    return rows.value, cols.value, pair.value, ctas.value
 
 
 def rtr_attn_block_causal_backward(q, k, v, out, dout, lse, n_tokens, heads, head_dim, k_per_frame, dt, dq, dk, dv,

@@ -437,6 +437,18 @@ rtr_status rtr_dit_qkv_rope(const void *a, const void *wqkv, const void *bqkv,
                             int k_per_frame, int grid_w, int t0, void *q,
                             void *k, void *v, int device, rtr_stream_t stream);
 
+/* The output tile rtr_dit_linear (epilogue as there) or, with qkv_rope = 1,
+ * rtr_dit_qkv_rope picks for an m x n x k product on `device`: *rows x
+ * *cols outputs per tile, *cta_pair = 1 when two CTAs of a cluster share
+ * each tile (tcgen05 cta_group::2 MMAs, each CTA holding half the rows and
+ * loading half the weight columns), and *ctas, the CTAs of the persistent
+ * launch.  A planning query: it launches nothing (without a usable device
+ * it plans for 148 SMs and no CTA pairs).  m, n, k >= 1; RTR_E_INVAL for
+ * bad sizes or null outputs. */
+rtr_status rtr_dit_linear_tile(int m, int n, int k, rtr_epilogue epilogue,
+                               int qkv_rope, int device, int *rows, int *cols,
+                               int *cta_pair, int *ctas);
+
 /* Backward pass of the block-causal attention (Key Designs 2 and 3: the
  * causal student is trained with Self Forcing and DMD, whose gradients flow
  * through this attention).  Given the forward's inputs q, k, v, its output

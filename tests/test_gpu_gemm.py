@@ -87,6 +87,8 @@ LINEAR_CASES = [
     (777, 1536, 1536, "gated_residual_nogate"),
     (4680, 1536, 1536, "bias"),          # the cross-attention query projection
     (4800, 3072, 512, "bias"),           # 256-row tiles whose last has a partial second sub-tile
+    (4800, 4600, 1024, "bias"),          # CTA-pair tiles: the last row tile's second CTA holds 64 rows,
+                                         # the last column tile's second CTA a partial weight box
 ]
 
 
@@ -171,6 +173,29 @@ def test_dit_qkv_rope_parity(H, d, gh, gw, C, t0):
     assert rtr.rtr_get_device_status(0) == rtr.RTR_OK
     for name, got, ref, err in zip("qkv", (q, kk, v), want, errs):
         assert_parity(host_f64(got), ref, err, f"{name} H={H} d={d} m={m}")
+
+
+def test_cases_cover_both_tilings():
+    """The cases above reach both kernels: tiles of one CTA, and 256 x 256
+    tiles shared by a CTA pair (as the Wan-1.3B feed-forward input and QKV
+    projections are)."""
+    rtr = _rtr()
+    plans = {}
+    for m, n, k, epi in LINEAR_CASES:
+        code = "gated_residual" if epi.startswith("gated_residual") else epi
+        plans[(m, n, k, epi)] = rtr.rtr_dit_linear_tile(m, n, k, code)
+    for H, d, gh, gw, C, t0 in QKV_CASES:
+        D = H * d
+        plans[("qkv", H, d, C * gh * gw)] = rtr.rtr_dit_linear_tile(C * gh * gw, 3 * D, D, "bias", qkv_rope=True)
+    for key, plan in plans.items():
+        print(key, plan)
+    pairs = [key for key, plan in plans.items() if plan[2] == 1]
+    singles = [key for key, plan in plans.items() if plan[2] == 0]
+    assert (4680, 8960, 1536, "gelu") in pairs and ("qkv", 12, 128, 4680) in pairs
+    assert (4800, 4600, 1024, "bias") in pairs
+    assert len(singles) >= 4
+    for key in pairs:
+        assert plans[key][:2] == (256, 256) and plans[key][3] % 2 == 0
 
 
 def test_dit_linear_repeat_is_bit_identical():
