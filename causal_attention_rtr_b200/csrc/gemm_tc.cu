@@ -370,8 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                         const int c0 = n0 + r * 128;
                         return max(0, min(2, (p.n - c0 + 63) / 64));
                     };
+                    // packed W moves whole 16 KB boxes (two images) per CTA that has columns
+                    auto w_bytes = [&](int r) { return p.w_pk ? (w_in(r) > 0 ? 2 : 0) : w_in(r); };
                     const uint32_t tx = (uint32_t)((a_in(0) + a_in(1)) * kATileBytes +
-                                                   (w_in(0) + w_in(1)) * kBBoxBytes);
+                                                   (w_bytes(0) + w_bytes(1)) * kBBoxBytes);
                     const int my_m0 = m0 + (int)rank * kBM, my_n0 = n0 + (int)rank * 128;
                     const int my_a = a_in((int)rank), my_w = w_in((int)rank);
                     for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
@@ -385,20 +387,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                         const uint32_t fb = lead(full(s));
                         if (rank == 0) mbar_arrive_tx(full(s), tx);
                         if (my_a) {
-                            if (p.a_pk) {
-                                // packed A as rows of 256 bytes: a 16 KB tile image is 64 of them
-                                const int r0 = ((my_m0 / kBM) * p.kb_total + kb) * 64;
-                                tma_load_3d_pair(sa, &p.tm_a, fb, 0, r0, 0);
-                                tma_load_3d_pair(sa + kATileBytes / 2, &p.tm_a, fb, 0, r0 + 32, 0);
-                            } else {
-                                tma_load_3d_pair(sa, &p.tm_a, fb, kb * kBK, my_m0, 0);
-                            }
-                        }
-                        for (int j = 0; j < my_w; ++j) {
-                            if (p.w_pk)   // an 8 KB box image is 32 rows of 256 bytes
-                                tma_load_3d_pair(sa + a_bytes + j * kBBoxBytes, &p.tm_w, fb, 0,
-                                                 (kb * p.nb_total + my_n0 / 64 + j) * 32, 0);
+                            if (p.a_pk)   // packed A as rows of 256 bytes: a 16 KB tile image is 64 of them
+                                tma_load_3d_pair(sa, &p.tm_a, fb, 0, ((my_m0 / kBM) * p.kb_total + kb) * 64, 0);
                             else
+                                tma_load_3d_pair(sa, &p.tm_a, fb, kb * kBK, my_m0, 0);
+                        }
+                        if (p.w_pk) {
+                            // this CTA's two 8 KB W images are adjacent: one box of 64 rows of 256
+                            // bytes.  With one image left (n / 64 odd) the box's second half is the
+                            // next K block's first image, or past the end (zero fill): either way
+                            // it reaches only discarded columns.
+                            if (my_w > 0)
+                                tma_load_3d_pair(sa + a_bytes, &p.tm_w, fb, 0, (kb * p.nb_total + my_n0 / 64) * 32, 0);
+                        } else {
+                            for (int j = 0; j < my_w; ++j)
                                 tma_load_3d_pair(sa + a_bytes + j * kBBoxBytes, &p.tm_w, fb, my_n0 + 64 * j,
                                                  kb * kBK, 0);
                         }
@@ -732,19 +734,21 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
     memset(&p, 0, sizeof(p));
     int device = 0;
     if (cudaGetDevice(&device) != cudaSuccess) return cudaErrorInvalidValue;
-    const int slots2 = pair_slots(g.epi, device, sms);
+    // a pair moves packed W two images at a time, so it needs at least two
+    const int slots2 = g.w_packed && packed_b_bytes(g.k, g.n) < 2 * (size_t)kBBoxBytes ? 0
+                                                                                    : pair_slots(g.epi, device, sms);
     const TileShape ts = pick_tile(g.m, g.n, g.k, sms, slots2, g.epi == kEpiBiasGelu || g.epi == kEpiQkvRope);
     // Row-major operands load by 128-byte-swizzled TMA boxes.  Packed ones
     // load by 1-D bulk copies, or, on a CTA pair (whose loads must count on
     // the first CTA's barrier), by unswizzled boxes of 256-byte rows, which
     // land byte for byte as they lie in memory.
     if (g.a_packed && ts.pair) {
-        if (!make_tmap_rows256(&p.tm_a, g.a, packed_a_bytes(g.m, g.k) / 256, 32)) return cudaErrorInvalidValue;
+        if (!make_tmap_rows256(&p.tm_a, g.a, packed_a_bytes(g.m, g.k) / 256, 64)) return cudaErrorInvalidValue;
     } else if (!g.a_packed && !make_tmap_bf16(&p.tm_a, g.a, (uint64_t)g.k, (uint64_t)g.m, 1, kBM, 1)) {
         return cudaErrorInvalidValue;
     }
     if (g.w_packed && ts.pair) {
-        if (!make_tmap_rows256(&p.tm_w, g.w, packed_b_bytes(g.k, g.n) / 256, 32)) return cudaErrorInvalidValue;
+        if (!make_tmap_rows256(&p.tm_w, g.w, packed_b_bytes(g.k, g.n) / 256, 64)) return cudaErrorInvalidValue;
     } else if (!g.w_packed && !make_tmap_bf16(&p.tm_w, g.w, (uint64_t)g.n, (uint64_t)g.k, 1, kBK, 1)) {
         return cudaErrorInvalidValue;
     }
