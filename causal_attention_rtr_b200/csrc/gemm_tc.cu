@@ -294,8 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
     const uint32_t s_base = smem_u32(smem);
     const int S = p.stages;
     const int a_bytes = p.msub * kATileBytes;               // A sub-tiles, then W boxes
-    const int w_cols = PAIR ? p.bn / 2 : p.bn;                 // W columns held by this CTA
-    const int stage_bytes = a_bytes + (w_cols / 64) * kBBoxBytes;
+    // pair: two K blocks of this CTA's 128 rows of A and 128 columns of W
+    const int stage_bytes = PAIR ? 2 * (kATileBytes + 2 * kBBoxBytes) : a_bytes + (p.bn / 64) * kBBoxBytes;
     const int BMt = kBM * p.msub * (PAIR ? 2 : 1);             // rows per tile
     const uint32_t bars = s_base + (uint32_t)(S * stage_bytes);
     // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain, rope table ready
@@ -361,22 +361,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
             for (int t = cl; t < p.n_tiles && ok; t += n_cl) {
                 const int m0 = (t / p.n_tiles_n) * BMt, n0 = (t % p.n_tiles_n) * p.bn;
                 if (PAIR) {
-                    // rank r: A rows from m0 + 128 r (loaded if they start below
-                    // m) and the 64-column W boxes from n0 + 128 r that start
-                    // inside the matrix; what is not loaded keeps stale data,
-                    // which reaches only discarded rows and columns
+                    // A stage holds two 64-deep K blocks: [A kb][A kb+1][W kb][W kb+1],
+                    // 16 KB each.  Rank r: A rows from m0 + 128 r (loaded if they start
+                    // below m) and the W columns from n0 + 128 r that start inside the
+                    // matrix; what is not loaded keeps stale data, which reaches only
+                    // discarded rows and columns.
                     auto a_in = [&](int r) { return m0 + r * kBM < p.m ? 1 : 0; };
                     auto w_in = [&](int r) {
                         const int c0 = n0 + r * 128;
                         return max(0, min(2, (p.n - c0 + 63) / 64));
                     };
-                    // packed W moves whole 16 KB boxes (two images) per CTA that has columns
-                    auto w_bytes = [&](int r) { return p.w_pk ? (w_in(r) > 0 ? 2 : 0) : w_in(r); };
-                    const uint32_t tx = (uint32_t)((a_in(0) + a_in(1)) * kATileBytes +
-                                                   (w_bytes(0) + w_bytes(1)) * kBBoxBytes);
                     const int my_m0 = m0 + (int)rank * kBM, my_n0 = n0 + (int)rank * 128;
                     const int my_a = a_in((int)rank), my_w = w_in((int)rank);
-                    for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    for (int kb = 0; kb < p.k_blocks; kb += 2, ++it) {
+                        const int nk = min(2, p.k_blocks - kb);
                         const int s = it % S, use = it / S;
                         if (use > 0 && !wait_lead(empty(s), (use - 1) & 1)) {
                             raise_timeout(p, abort_flag);
@@ -385,24 +383,41 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                         }
                         const uint32_t sa = s_base + (uint32_t)(s * stage_bytes);
                         const uint32_t fb = lead(full(s));
-                        if (rank == 0) mbar_arrive_tx(full(s), tx);
-                        if (my_a) {
-                            if (p.a_pk)   // packed A as rows of 256 bytes: a 16 KB tile image is 64 of them
-                                tma_load_3d_pair(sa, &p.tm_a, fb, 0, ((my_m0 / kBM) * p.kb_total + kb) * 64, 0);
-                            else
-                                tma_load_3d_pair(sa, &p.tm_a, fb, kb * kBK, my_m0, 0);
+                        if (rank == 0) {
+                            // bytes both CTAs move into this stage: packed A as one 32 KB box
+                            // (two adjacent images), packed W as one 16 KB box per K block,
+                            // row-major operands as 16 KB A and 8 KB W boxes per K block
+                            uint32_t tx = 0;
+                            for (int r = 0; r < 2; ++r) {
+                                if (a_in(r)) tx += p.a_pk ? 2u * kATileBytes : (uint32_t)(nk * kATileBytes);
+                                if (w_in(r) > 0)
+                                    tx += (uint32_t)(nk * (p.w_pk ? 2 : w_in(r)) * kBBoxBytes);
+                            }
+                            mbar_arrive_tx(full(s), tx);
                         }
-                        if (p.w_pk) {
-                            // this CTA's two 8 KB W images are adjacent: one box of 64 rows of 256
-                            // bytes.  With one image left (n / 64 odd) the box's second half is the
-                            // next K block's first image, or past the end (zero fill): either way
-                            // it reaches only discarded columns.
-                            if (my_w > 0)
-                                tma_load_3d_pair(sa + a_bytes, &p.tm_w, fb, 0, (kb * p.nb_total + my_n0 / 64) * 32, 0);
-                        } else {
-                            for (int j = 0; j < my_w; ++j)
-                                tma_load_3d_pair(sa + a_bytes + j * kBBoxBytes, &p.tm_w, fb, my_n0 + 64 * j,
-                                                 kb * kBK, 0);
+                        if (my_a) {
+                            if (p.a_pk) {
+                                // packed A as rows of 256 bytes: the tile's images for K blocks kb
+                                // and kb + 1 are adjacent, 64 rows each (with one K block left
+                                // the second is the next image or past the end, unused)
+                                tma_load_3d_pair(sa, &p.tm_a, fb, 0, ((my_m0 / kBM) * p.kb_total + kb) * 64, 0);
+                            } else {
+                                for (int j = 0; j < nk; ++j)
+                                    tma_load_3d_pair(sa + j * kATileBytes, &p.tm_a, fb, (kb + j) * kBK, my_m0, 0);
+                            }
+                        }
+                        for (int j = 0; j < nk && my_w > 0; ++j) {
+                            const uint32_t sw = sa + 2 * kATileBytes + j * 2 * kBBoxBytes;
+                            if (p.w_pk) {
+                                // this CTA's two 8 KB W images are adjacent: one box of 64 rows of
+                                // 256 bytes.  With one image left (n / 64 odd) the box's second
+                                // half is the next K block's first image, or past the end (zero
+                                // fill): either way it reaches only discarded columns.
+                                tma_load_3d_pair(sw, &p.tm_w, fb, 0, ((kb + j) * p.nb_total + my_n0 / 64) * 32, 0);
+                            } else {
+                                for (int q = 0; q < my_w; ++q)
+                                    tma_load_3d_pair(sw + q * kBBoxBytes, &p.tm_w, fb, my_n0 + 64 * q, (kb + j) * kBK, 0);
+                            }
                         }
                     }
                     continue;
@@ -464,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                for (int kb = 0; kb < p.k_blocks; kb += PAIR ? 2 : 1, ++it) {
                     const int s = it % S;
                     if (!wait_lead(full(s), (it / S) & 1)) {
                         ok = false;
@@ -472,18 +487,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc(const __grid_constant__ G
                     }
                     tc_fence_after();
                     const uint32_t sa = s_base + (uint32_t)(s * stage_bytes);
+                    if (PAIR) {
+                        // the stage's K blocks: A at sa + 16 KB j, W at sa + 32 KB + 16 KB j
+                        const int nk = min(2, p.k_blocks - kb);
+                        for (int j = 0; j < nk; ++j) {
+                            const uint64_t da = smem_desc_sw128(sa + j * kATileBytes, 16, 1024);
+                            const uint64_t dw = smem_desc_sw128(sa + 2 * kATileBytes + j * 2 * kBBoxBytes, kBBoxBytes, 1024);
+                            const uint32_t d_tmem = tmem + (uint32_t)(b * 256);
+#pragma unroll
+                            for (int kk = 0; kk < kBK / 16; ++kk)
+                                mma_ss_pair(d_tmem, da + (uint64_t)((kk * 32) >> 4), dw + (uint64_t)((kk * 2048) >> 4),
+                                            idesc, (kb + j > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
                     const uint64_t dw = smem_desc_sw128(sa + a_bytes, kBBoxBytes, 1024);
                     // sub-tile u accumulates at TMEM column b * 256 + u * bn
-                    for (int u = 0; u < a_subs; ++u) {
+                    for (int u = 0; !PAIR && u < a_subs; ++u) {
                         const uint64_t da = smem_desc_sw128(sa + u * kATileBytes, 16, 1024);
                         const uint32_t d_tmem = tmem + (uint32_t)(b * 256 + u * p.bn);
 #pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk) {
-                            const uint64_t a_k = da + (uint64_t)((kk * 32) >> 4);
-                            const uint64_t w_k = dw + (uint64_t)((kk * 2048) >> 4);
-                            if (PAIR) mma_ss_pair(d_tmem, a_k, w_k, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                            else mma_ss(d_tmem, a_k, w_k, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                        }
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            mma_ss(d_tmem, da + (uint64_t)((kk * 32) >> 4), dw + (uint64_t)((kk * 2048) >> 4), idesc,
+                                   (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     if (PAIR) tc_commit_pair(empty(s));
                     else tc_commit(empty(s));
@@ -617,7 +642,10 @@ struct TileShape {
     int msub, bn, stages, pair;
 };
 
-int stage_bytes_of(int msub, int bn, int pair) { return msub * kATileBytes + (bn / (pair ? 128 : 64)) * kBBoxBytes; }
+// A pair's stage holds two K blocks of its 128 rows of A and 128 columns of W.
+int stage_bytes_of(int msub, int bn, int pair) {
+    return pair ? 2 * (kATileBytes + 2 * kBBoxBytes) : msub * kATileBytes + (bn / 64) * kBBoxBytes;
+}
 
 TileShape pick_tile(int m, int n, int k, int sms, int pair_slots, bool heavy_epilogue) {
     const int k_blocks = (k + kBK - 1) / kBK;
@@ -629,7 +657,7 @@ TileShape pick_tile(int m, int n, int k, int sms, int pair_slots, bool heavy_epi
         if (c.pair && pair_slots < 1) continue;
         const int stages = std::min(8, kMaxSmem / stage_bytes_of(c.msub, c.bn, c.pair));
         const double mma = c.pair ? 4.0 * 232.0 : c.msub * 4.0 * (c.bn == 256 ? 128.0 : c.bn == 192 ? 106.0 : 85.0);
-        const double load = 4400.0 / stages;
+        const double load = 4400.0 / (c.pair ? 2 * stages : stages);   // per K block
         const double epi = !c.pair && c.msub * c.bn > 256 ? 2000.0 : 0.0;
         const int rows = kBM * c.msub * (c.pair ? 2 : 1);
         const long long tiles = (long long)((m + rows - 1) / rows) * ((n + c.bn - 1) / c.bn);
@@ -734,16 +762,19 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
     memset(&p, 0, sizeof(p));
     int device = 0;
     if (cudaGetDevice(&device) != cudaSuccess) return cudaErrorInvalidValue;
-    // a pair moves packed W two images at a time, so it needs at least two
-    const int slots2 = g.w_packed && packed_b_bytes(g.k, g.n) < 2 * (size_t)kBBoxBytes ? 0
-                                                                                    : pair_slots(g.epi, device, sms);
+    // a pair moves packed W two images and packed A two tile images at a time,
+    // so it needs at least that many
+    const int slots2 = (g.w_packed && packed_b_bytes(g.k, g.n) < 2 * (size_t)kBBoxBytes) ||
+                               (g.a_packed && packed_a_bytes(g.m, g.k) < 2 * (size_t)kATileBytes)
+                           ? 0
+                           : pair_slots(g.epi, device, sms);
     const TileShape ts = pick_tile(g.m, g.n, g.k, sms, slots2, g.epi == kEpiBiasGelu || g.epi == kEpiQkvRope);
     // Row-major operands load by 128-byte-swizzled TMA boxes.  Packed ones
     // load by 1-D bulk copies, or, on a CTA pair (whose loads must count on
     // the first CTA's barrier), by unswizzled boxes of 256-byte rows, which
     // land byte for byte as they lie in memory.
     if (g.a_packed && ts.pair) {
-        if (!make_tmap_rows256(&p.tm_a, g.a, packed_a_bytes(g.m, g.k) / 256, 64)) return cudaErrorInvalidValue;
+        if (!make_tmap_rows256(&p.tm_a, g.a, packed_a_bytes(g.m, g.k) / 256, 128)) return cudaErrorInvalidValue;
     } else if (!g.a_packed && !make_tmap_bf16(&p.tm_a, g.a, (uint64_t)g.k, (uint64_t)g.m, 1, kBM, 1)) {
         return cudaErrorInvalidValue;
     }
