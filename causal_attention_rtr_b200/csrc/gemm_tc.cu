@@ -625,8 +625,10 @@ cudaError_t set_smem_attr_once() {
 // takes the longer of
 //   its MMAs: 128 x N x 16 costs 85, 106 or 128 cycles for N = 128, 192,
 //     256 (one per k16 step and 128-row sub-tile); the pair's 256 x 256 x 16
-//     runs at 128 per SM alone but takes about 232 in this kernel, with the
-//     stage loads in flight (clock stamps of its K blocks), and
+//     runs at 128 per SM alone but, with the stage loads in flight, about
+//     170 with packed weights and 232 with row-major ones, whose 8 KB boxes
+//     take more TMA instructions to issue (measured on the Wan-1.3B
+//     projections), and
 //   its loads: stages in flight over a loaded round trip of about 4,400
 //     cycles (the latency times the bandwidth of the memory system reaching
 //     one SM is the shared memory that holds the stages, so a stage's bytes
@@ -647,7 +649,7 @@ int stage_bytes_of(int msub, int bn, int pair) {
     return pair ? 2 * (kATileBytes + 2 * kBBoxBytes) : msub * kATileBytes + (bn / 64) * kBBoxBytes;
 }
 
-TileShape pick_tile(int m, int n, int k, int sms, int pair_slots, bool heavy_epilogue) {
+TileShape pick_tile(int m, int n, int k, int sms, int pair_slots, bool heavy_epilogue, bool w_packed) {
     const int k_blocks = (k + kBK - 1) / kBK;
     TileShape best = {1, 256, 4, 0};
     double best_cost = -1.0;
@@ -656,7 +658,8 @@ TileShape pick_tile(int m, int n, int k, int sms, int pair_slots, bool heavy_epi
         if (c.msub == 2 && heavy_epilogue) continue;
         if (c.pair && pair_slots < 1) continue;
         const int stages = std::min(8, kMaxSmem / stage_bytes_of(c.msub, c.bn, c.pair));
-        const double mma = c.pair ? 4.0 * 232.0 : c.msub * 4.0 * (c.bn == 256 ? 128.0 : c.bn == 192 ? 106.0 : 85.0);
+        const double mma = c.pair ? 4.0 * (w_packed ? 170.0 : 232.0)
+                                  : c.msub * 4.0 * (c.bn == 256 ? 128.0 : c.bn == 192 ? 106.0 : 85.0);
         const double load = 4400.0 / (c.pair ? 2 * stages : stages);   // per K block
         const double epi = !c.pair && c.msub * c.bn > 256 ? 2000.0 : 0.0;
         const int rows = kBM * c.msub * (c.pair ? 2 : 1);
@@ -768,7 +771,8 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
                                (g.a_packed && packed_a_bytes(g.m, g.k) < 2 * (size_t)kATileBytes)
                            ? 0
                            : pair_slots(g.epi, device, sms);
-    const TileShape ts = pick_tile(g.m, g.n, g.k, sms, slots2, g.epi == kEpiBiasGelu || g.epi == kEpiQkvRope);
+    const TileShape ts =
+        pick_tile(g.m, g.n, g.k, sms, slots2, g.epi == kEpiBiasGelu || g.epi == kEpiQkvRope, g.w_packed != 0);
     // Row-major operands load by 128-byte-swizzled TMA boxes.  Packed ones
     // load by 1-D bulk copies, or, on a CTA pair (whose loads must count on
     // the first CTA's barrier), by unswizzled boxes of 256-byte rows, which
@@ -839,7 +843,7 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
 void gemm_tile_shape(int m, int n, int k, int epi, int device, int sms, int *rows, int *cols, int *pair,
                      int *ctas) {
     const int slots2 = pair_slots(epi, device, sms);
-    const TileShape ts = pick_tile(m, n, k, sms, slots2, epi == kEpiBiasGelu || epi == kEpiQkvRope);
+    const TileShape ts = pick_tile(m, n, k, sms, slots2, epi == kEpiBiasGelu || epi == kEpiQkvRope, false);
     const int tile_rows = kBM * ts.msub * (ts.pair ? 2 : 1);
     const long long tiles = (long long)((m + tile_rows - 1) / tile_rows) * ((n + ts.bn - 1) / ts.bn);
     const int slots = ts.pair ? slots2 : sms;
