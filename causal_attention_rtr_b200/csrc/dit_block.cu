@@ -128,6 +128,72 @@ __global__ void __launch_bounds__(1024) ln_modulate_reg(const __nv_bfloat16 *x, 
         reinterpret_cast<uint4 *>(out + row * D)[i] = v;
 }
 
+// One warp per row, the row in registers (VPL 8-channel vectors a lane, D <=
+// 256 VPL): mean and variance by warp shuffles, no shared memory and no
+// block barrier, eight rows a CTA, so every row of a chunk is in flight at
+// once (the one-CTA-per-row kernel above ran about three waves of small CTAs
+// with two block barriers each).  Same arithmetic as ln_modulate_reg; only
+// the order of the fp32 sums differs.
+template <int VPL>
+__global__ void __launch_bounds__(256) ln_modulate_warp(const __nv_bfloat16 *x, const __nv_bfloat16 *shift,
+                                                       const __nv_bfloat16 *scale, __nv_bfloat16 *out, int n, int D,
+                                                       float eps, int out_packed) {
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= n) return;
+    const int nv = D / 8;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * D);
+    float f[VPL][8];
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int i = lane + 32 * j;
+        if (i < nv) {
+            unpack8(xr[i], f[j]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[j][e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += f[j][e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / (float)D;
+    float q = 0.f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        if (lane + 32 * j < nv) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) q += (f[j][e] - mean) * (f[j][e] - mean);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float rstd = 1.0f / sqrtf(q / (float)D + eps);
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int i = lane + 32 * j;
+        if (i >= nv) break;
+        if (scale != nullptr) {
+            float sc[8], sh[8];
+            unpack8(reinterpret_cast<const uint4 *>(scale)[i], sc);
+            unpack8(reinterpret_cast<const uint4 *>(shift)[i], sh);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[j][e] = (f[j][e] - mean) * rstd * (1.0f + sc[e]) + sh[e];
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[j][e] = (f[j][e] - mean) * rstd;
+        }
+        const uint4 v = make_uint4(pack2(f[j][0], f[j][1]), pack2(f[j][2], f[j][3]), pack2(f[j][4], f[j][5]),
+                                   pack2(f[j][6], f[j][7]));
+        if (out_packed)
+            *reinterpret_cast<uint4 *>(reinterpret_cast<char *>(out) + packed_a_offset(row, 8 * i, D)) = v;
+        else
+            reinterpret_cast<uint4 *>(out + row * D)[i] = v;
+    }
+}
+
 // One thread per 16-byte piece of w: its 8 n-consecutive elements move to
 // their place in the packed layout.
 __global__ void __launch_bounds__(256) pack_b(const uint4 *w, char *out, int k, int n8) {
@@ -153,6 +219,25 @@ cudaError_t launch_ln_modulate(const void *x, const void *shift, const void *sca
     if (n <= 0) return cudaSuccess;
     if (D % 8 != 0 || (scale == nullptr) != (shift == nullptr)) return cudaErrorInvalidValue;
     if (out_packed && (D % 64 != 0 || D / 8 > 1024)) return cudaErrorInvalidValue;
+    const int vpl = (D / 8 + 31) / 32;          // 8-channel vectors a lane, one warp per row
+    if (vpl <= 8) {
+        const auto *xx = static_cast<const __nv_bfloat16 *>(x);
+        const auto *sh = static_cast<const __nv_bfloat16 *>(shift);
+        const auto *sc = static_cast<const __nv_bfloat16 *>(scale);
+        auto *o = static_cast<__nv_bfloat16 *>(out);
+        const unsigned grid = (unsigned)((n + 7) / 8);
+        switch (vpl) {
+            case 1: ln_modulate_warp<1><<<grid, 256, 0, s>>>(xx, sh, sc, o, n, D, eps, out_packed); break;
+            case 2: ln_modulate_warp<2><<<grid, 256, 0, s>>>(xx, sh, sc, o, n, D, eps, out_packed); break;
+            case 3: ln_modulate_warp<3><<<grid, 256, 0, s>>>(xx, sh, sc, o, n, D, eps, out_packed); break;
+            case 4: ln_modulate_warp<4><<<grid, 256, 0, s>>>(xx, sh, sc, o, n, D, eps, out_packed); break;
+            case 5: ln_modulate_warp<5><<<grid, 256, 0, s>>>(xx, sh, sc, o, n, D, eps, out_packed); break;
+            case 6: ln_modulate_warp<6><<<grid, 256, 0, s>>>(xx, sh, sc, o, n, D, eps, out_packed); break;
+            case 7: ln_modulate_warp<7><<<grid, 256, 0, s>>>(xx, sh, sc, o, n, D, eps, out_packed); break;
+            default: ln_modulate_warp<8><<<grid, 256, 0, s>>>(xx, sh, sc, o, n, D, eps, out_packed); break;
+        }
+        return launched();
+    }
     if (D / 8 <= 1024) {
         const int threads = (D / 8 + 31) / 32 * 32;
         ln_modulate_reg<<<n, threads, 0, s>>>(
