@@ -171,3 +171,23 @@ def test_dit_packed_validation(lib):
     assert rtr.raw_status("rtr_dit_block_forward_packed", None, None, 0, None, None, None, 1, 1, 1, 0, 0,
                           None) == rtr.RTR_E_INVAL
     rtr.rtr_dit_packed_destroy(None)                          # no-op
+
+
+def test_dit_linear_tile_plan_on_host(lib):
+    """The projection's tile planner answers without a GPU: without a device
+    it plans for 148 SMs and single-CTA tiles (no CTA pairs, whose residency
+    it cannot query); shapes and pointers are checked first."""
+    import ctypes as ct
+    from causal_attention_rtr_b200 import rtr
+    for m, n, k, epi, qkv in [(4680, 8960, 1536, "gelu", False), (4680, 1536, 8960, "gated_residual", False),
+                              (4680, 4608, 1536, "bias", True), (7, 64, 8, "bias", False)]:
+        rows, cols, pair, ctas = rtr.rtr_dit_linear_tile(m, n, k, epi, qkv)
+        assert pair == 0 and rows in (128, 256) and cols in (128, 192, 256)
+        tiles = -(-m // rows) * -(-n // cols)
+        assert ctas == min(tiles, 148), (m, n, k, rows, cols, ctas)
+    r = [ct.c_int() for _ in range(4)]
+    refs = [ct.byref(x) for x in r]
+    assert rtr.raw_status("rtr_dit_linear_tile", 0, 64, 64, 0, 0, 0, *refs) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_dit_linear_tile", 64, 64, 64, 7, 0, 0, *refs) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_dit_linear_tile", 64, 64, 64, 0, 0, -1, *refs) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_dit_linear_tile", 64, 64, 64, 0, 0, 0, refs[0], refs[1], None, refs[3]) == rtr.RTR_E_INVAL
