@@ -202,6 +202,29 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
         __nv_bfloat16 *dst = (part == 0 ? p.q : part == 1 ? p.kk : p.v) + row * p.D + cc;
         const int c0 = cc % p.head_dim;                 // channel of the first column within its head
         const int nt = p.rope_dt / 2, nd = p.rope_dp / 2;
+        // the chunk's 16 (cos, sin) pairs first, all table reads issued before
+        // any is used: channel pair c / 2 lies in the time, row or column
+        // section, each indexed by the token's frame, row or column
+        float2 cs[16];
+        if (part < 2) {
+            const int t_base = (f_pos - p.t0) * nt, y_base = p.rope_frames * nt + y_pos * nd - p.rope_dt / 2,
+                      x_base = p.rope_frames * nt + (p.rope_rows + x_pos) * nd - (p.rope_dt + p.rope_dp) / 2;
+#pragma unroll
+            for (int pr = 0; pr < 16; ++pr) {
+                if (2 * pr >= nvalid) break;
+                const int c = c0 + 2 * pr, h = c / 2;
+                if (rope != nullptr) {
+                    const int idx = c < p.rope_dt ? t_base + h : c < p.rope_dt + p.rope_dp ? y_base + h : x_base + h;
+                    cs[pr] = rope[idx];
+                } else if (c < p.rope_dt) {
+                    cs[pr] = rope_angle(h, p.rope_dt, f_pos);
+                } else if (c < p.rope_dt + p.rope_dp) {
+                    cs[pr] = rope_angle(h - p.rope_dt / 2, p.rope_dp, y_pos);
+                } else {
+                    cs[pr] = rope_angle(h - (p.rope_dt + p.rope_dp) / 2, p.rope_dp, x_pos);
+                }
+            }
+        }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             if (8 * g >= nvalid) break;
@@ -212,20 +235,9 @@ __device__ __forceinline__ void epi_chunk(const GemmParams &p, const uint32_t (&
                 float2 v = fadd2(make_float2(__uint_as_float(acc[8 * g + e]), __uint_as_float(acc[8 * g + e + 1])),
                                  make_float2(b[e], b[e + 1]));
                 if (part < 2) {
-                    const int c = c0 + 8 * g + e;       // even channel of the pair
-                    float2 cs;
-                    if (c < p.rope_dt) {
-                        cs = rope ? rope[(f_pos - p.t0) * nt + c / 2] : rope_angle(c / 2, p.rope_dt, f_pos);
-                    } else if (c < p.rope_dt + p.rope_dp) {
-                        const int j = (c - p.rope_dt) / 2;
-                        cs = rope ? rope[p.rope_frames * nt + y_pos * nd + j] : rope_angle(j, p.rope_dp, y_pos);
-                    } else {
-                        const int j = (c - p.rope_dt - p.rope_dp) / 2;
-                        cs = rope ? rope[p.rope_frames * nt + (p.rope_rows + x_pos) * nd + j]
-                                  : rope_angle(j, p.rope_dp, x_pos);
-                    }
+                    const float2 t = cs[4 * g + e / 2];
                     // (a0 cos - a1 sin, a1 cos + a0 sin)
-                    v = ffma2(v, make_float2(cs.x, cs.x), fmul2(make_float2(v.y, v.x), make_float2(-cs.y, cs.y)));
+                    v = ffma2(v, make_float2(t.x, t.x), fmul2(make_float2(v.y, v.x), make_float2(-t.y, t.y)));
                 }
                 r[e] = v.x;
                 r[e + 1] = v.y;
