@@ -142,8 +142,10 @@ def test_dit_block_parity(case, commit):
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"H{c[0]}-d{c[1]}-k{c[2] * c[3]}-C{c[9]}")
 def test_dit_block_packed_weights_bit_identical(case):
     """The block with weights packed once (rtr_dit_pack_weights) gives the
-    same bits as with the row-major weights: the projections read the same
-    tiles, only their transfer differs.  Both match the oracle."""
+    same bits as with the row-major weights: each output element is the same
+    K-ordered fp32 accumulation of the same products, whether one CTA or a
+    CTA pair computes its tile and however the operands travel.  Both match
+    the oracle."""
     H, d, gh, gw, R, W, appends, T, F, C, t0 = case
     rtr = _rtr()
     runs = []
