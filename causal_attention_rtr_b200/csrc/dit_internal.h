@@ -2,6 +2,7 @@
 // the host side of the C ABI (api.cu).  All tensors are row-major, bf16
 // unless stated; every launcher returns the CUDA error of its launch.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -71,6 +72,11 @@ struct GemmArgs {
 // C = A W on the tensor cores with the epilogue fused (persistent, up to
 // `sms` CTAs); a bounded wait that expires latches RTR_E_TIMEOUT in *status.
 cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaStream_t s);
+
+// A byte buffer seen as `rows` rows of 256 bytes (128 bf16), boxes of
+// box_rows rows, no swizzle: a box lands in shared memory byte for byte as
+// it lies in global memory (api.cu).
+bool make_tmap_rows256(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows);
 
 // The tile launch_gemm_bf16 picks for an m x n x k product on `device`
 // (rows, columns, whether a CTA pair shares it) and the CTAs it launches.

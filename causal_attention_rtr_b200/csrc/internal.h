@@ -124,11 +124,6 @@ bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, 
 bool make_tmap_bf16_strided(CUtensorMap *m, const void *base, uint64_t d, uint64_t mid, uint64_t outer,
                             uint64_t stride_outer, uint32_t box_mid, uint32_t box_outer);
 
-// A byte buffer seen as `rows` rows of 256 bytes (128 bf16), boxes of
-// box_rows rows, no swizzle: a box lands in shared memory byte for byte as
-// it lies in global memory.
-bool make_tmap_rows256(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows);
-
 unsigned *device_status_ptr(int device);
 
 // Count of kernels this library has launched (all devices, since load).
