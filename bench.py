@@ -576,6 +576,13 @@ def run_ours(args, rank, world, local_rank):
         line["prefill_22"] = clocked(cx, bus, leg_prefill_22, 100, False)
         line["prefill_22_bwd"] = clocked(cx, bus, leg_prefill_22_bwd, 40)
         line["switch_14b"] = clocked(cx, bus, leg_switch_14b, 8)
+        # one Wan-1.3B-shaped DiT block around the attention (projections,
+        # layer norms, cross attention); a failure here is reported in its
+        # own entry and leaves the rest of the line intact
+        try:
+            line["dit_block_13b"] = clocked(cx, bus, leg_dit_block_13b, 20)
+        except Exception as exc:                # noqa: BLE001 (reported, not hidden)
+            line["dit_block_13b"] = {"error": f"{type(exc).__name__}: {exc}"}
         del cx
     if world == 1 and not args.no_cpu_baseline:
         ops = oracle_operands(w, x)
@@ -1004,8 +1011,11 @@ def clocked(cx, bus, fn, *args):
     per-clock tensor peak where the leg reports TFLOP/s."""
     sampler = ClockSampler(bus)
     sampler.start()
-    res = fn(cx, *args)
-    res["clocks"] = sampler.stop()
+    try:
+        res = fn(cx, *args)
+    finally:
+        clk = sampler.stop()
+    res["clocks"] = clk
     pc = per_clock_peak_tflops(cx.sms, res["clocks"].get("sm_mhz"))
     if pc and "tflops" in res:
         res["frac_per_clock"] = res["tflops"] / pc
