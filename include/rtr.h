@@ -374,9 +374,10 @@ rtr_status rtr_dit_block_forward(rtr_kvcache *c, const rtr_xattn *x, int layer,
 
 /* The block's weights packed once for its projections.  Each matrix is
  * stored as the tensor core's shared-memory tiles, contiguously, so that a
- * projection moves a stage of weights with one bulk copy instead of one
- * transfer per 128-byte row (measured on B200: about 81 against 44-49 bytes
- * per clock per SM).  Weights are fixed during inference, so a caller packs
+ * projection moves a stage of weights with one bulk copy (or, on CTA-pair
+ * tiles, one 16 KB box per CTA and K block) instead of one transfer per
+ * 128-byte row (measured on B200: about 81 against 44-49 bytes per clock
+ * per SM).  Weights are fixed during inference, so a caller packs
  * a block's weights once and passes the handle to every
  * rtr_dit_block_forward_packed call.  d_model = heads * head_dim and
  * w->d_ffn must be multiples of 64; pointers as for rtr_dit_block_forward.
@@ -391,9 +392,10 @@ rtr_status rtr_dit_pack_weights(const rtr_dit_weights *w, int d_model,
 void rtr_dit_packed_destroy(rtr_dit_packed *pw);
 
 /* rtr_dit_block_forward with weights packed by rtr_dit_pack_weights: the
- * same block, bit for bit (the projections read identical tiles, only
- * their transfer differs).  pw must be packed for d_model = heads *
- * head_dim of c on c's device (else RTR_E_INVAL). */
+ * same block, bit for bit (each output element is the same K-ordered fp32
+ * accumulation of the same products, whichever tile shape the projection
+ * picks; only the operands' transfer differs).  pw must be packed for
+ * d_model = heads * head_dim of c on c's device (else RTR_E_INVAL). */
 rtr_status rtr_dit_block_forward_packed(rtr_kvcache *c, const rtr_xattn *x,
                                         int layer, const rtr_dit_packed *pw,
                                         const void *modulation, void *hidden,
