@@ -1040,6 +1040,19 @@ rtr_status rtr_dit_linear_tile(int m, int n, int k, rtr_epilogue epilogue, int q
     return RTR_OK;
 }
 
+rtr_status rtr_dit_plan_tile(int m, int n, int k, rtr_epilogue epilogue, int qkv_rope, int w_packed, int sms,
+                             int pair_clusters, int *rows, int *cols, int *cta_pair, int *ctas) {
+    if (m < 1 || n < 1 || k < 1 || sms < 1 || pair_clusters < 0 || pair_clusters > sms / 2 || !rows || !cols ||
+        !cta_pair || !ctas ||
+        (epilogue != RTR_EPI_BIAS && epilogue != RTR_EPI_BIAS_GELU && epilogue != RTR_EPI_GATED_RESIDUAL))
+        return RTR_E_INVAL;
+    const int epi = qkv_rope ? kEpiQkvRope
+                    : epilogue == RTR_EPI_BIAS ? kEpiBias
+                    : epilogue == RTR_EPI_BIAS_GELU ? kEpiBiasGelu : kEpiGatedResidual;
+    gemm_plan_tile(m, n, k, epi, w_packed != 0, sms, pair_clusters, rows, cols, cta_pair, ctas);
+    return RTR_OK;
+}
+
 rtr_status rtr_crossattn_create(int layers, int heads, int head_dim, int max_text, rtr_dtype dt, int device,
                                 rtr_xattn **out) {
     if (!out) return RTR_E_INVAL;

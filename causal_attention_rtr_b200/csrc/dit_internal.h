@@ -78,6 +78,11 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
 // it lies in global memory (api.cu).
 bool make_tmap_rows256(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows);
 
+// The planner alone, for `sms` SMs of which `pair_slots` CTA pairs can be
+// resident at once (0: no pairs), weights packed or row-major.
+void gemm_plan_tile(int m, int n, int k, int epi, bool w_packed, int sms, int pair_slots, int *rows, int *cols,
+                    int *pair, int *ctas);
+
 // The tile launch_gemm_bf16 picks for an m x n x k product on `device`
 // (rows, columns, whether a CTA pair shares it) and the CTAs it launches.
 void gemm_tile_shape(int m, int n, int k, int epi, int device, int sms, int *rows, int *cols, int *pair,

@@ -852,10 +852,9 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, unsigned *status, int sms, cudaS
     }
 }
 
-void gemm_tile_shape(int m, int n, int k, int epi, int device, int sms, int *rows, int *cols, int *pair,
-                     int *ctas) {
-    const int slots2 = pair_slots(epi, device, sms);
-    const TileShape ts = pick_tile(m, n, k, sms, slots2, epi == kEpiBiasGelu || epi == kEpiQkvRope, false);
+void gemm_plan_tile(int m, int n, int k, int epi, bool w_packed, int sms, int slots2, int *rows, int *cols,
+                    int *pair, int *ctas) {
+    const TileShape ts = pick_tile(m, n, k, sms, slots2, epi == kEpiBiasGelu || epi == kEpiQkvRope, w_packed);
     const int tile_rows = kBM * ts.msub * (ts.pair ? 2 : 1);
     const long long tiles = (long long)((m + tile_rows - 1) / tile_rows) * ((n + ts.bn - 1) / ts.bn);
     const int slots = ts.pair ? slots2 : sms;
@@ -863,6 +862,11 @@ void gemm_tile_shape(int m, int n, int k, int epi, int device, int sms, int *row
     *cols = ts.bn;
     *pair = ts.pair;
     *ctas = (int)std::min<long long>(tiles, slots) * (ts.pair ? 2 : 1);
+}
+
+void gemm_tile_shape(int m, int n, int k, int epi, int device, int sms, int *rows, int *cols, int *pair,
+                     int *ctas) {
+    gemm_plan_tile(m, n, k, epi, false, sms, pair_slots(epi, device, sms), rows, cols, pair, ctas);
 }
 
 }  // namespace rtr

@@ -75,6 +75,8 @@ _SIGNATURES = [
     ("rtr_dit_qkv_rope", _i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp]),
     ("rtr_dit_linear_tile", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
                                  ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    ("rtr_dit_plan_tile", _i, [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
+                               ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     ("rtr_attn_block_causal_backward", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f,
                                             _i, _vp]),
     ("rtr_crossattn_create", _i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
@@ -320,6 +322,16 @@ def rtr_dit_linear_tile(m, n, k, epilogue, qkv_rope=False, device=0):
     _check(_lib.rtr_dit_linear_tile(m, n, k, _epilogue(epilogue), int(bool(qkv_rope)), device, ctypes.byref(rows),
                                     ctypes.byref(cols), ctypes.byref(pair), ctypes.byref(ctas)),
            "rtr_dit_linear_tile")
+    return rows.value, cols.value, pair.value, ctas.value
+
+
+def rtr_dit_plan_tile(m, n, k, epilogue, qkv_rope=False, w_packed=False, sms=148, pair_clusters=74):
+    """(rows, cols, cta_pair, ctas) the projection planner picks for a
+    hypothetical device (host arithmetic only; see include/rtr.h)."""
+    rows, cols, pair, ctas = _i(), _i(), _i(), _i()
+    _check(_lib.rtr_dit_plan_tile(m, n, k, _epilogue(epilogue), int(bool(qkv_rope)), int(bool(w_packed)), sms,
+                                  pair_clusters, ctypes.byref(rows), ctypes.byref(cols), ctypes.byref(pair),
+                                  ctypes.byref(ctas)), "rtr_dit_plan_tile")
     return rows.value, cols.value, pair.value, ctas.value
 
 

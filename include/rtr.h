@@ -451,6 +451,18 @@ rtr_status rtr_dit_linear_tile(int m, int n, int k, rtr_epilogue epilogue,
                                int qkv_rope, int device, int *rows, int *cols,
                                int *cta_pair, int *ctas);
 
+/* The same planner for a hypothetical device, host arithmetic only: `sms`
+ * SMs of which `pair_clusters` CTA pairs (clusters of two) can be resident
+ * at once (0: pairs not available; at most sms / 2), weights packed by
+ * rtr_dit_pack_weights (w_packed = 1, as rtr_dit_block_forward_packed
+ * uses them) or row-major (0, as rtr_dit_linear and rtr_dit_block_forward
+ * pass them).  Outputs as for rtr_dit_linear_tile; RTR_E_INVAL for bad
+ * sizes or null outputs. */
+rtr_status rtr_dit_plan_tile(int m, int n, int k, rtr_epilogue epilogue,
+                             int qkv_rope, int w_packed, int sms,
+                             int pair_clusters, int *rows, int *cols,
+                             int *cta_pair, int *ctas);
+
 /* Backward pass of the block-causal attention (Key Designs 2 and 3: the
  * causal student is trained with Self Forcing and DMD, whose gradients flow
  * through this attention).  Given the forward's inputs q, k, v, its output

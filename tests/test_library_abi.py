@@ -191,3 +191,50 @@ def test_dit_linear_tile_plan_on_host(lib):
     assert rtr.raw_status("rtr_dit_linear_tile", 64, 64, 64, 7, 0, 0, *refs) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_dit_linear_tile", 64, 64, 64, 0, 0, -1, *refs) == rtr.RTR_E_INVAL
     assert rtr.raw_status("rtr_dit_linear_tile", 64, 64, 64, 0, 0, 0, refs[0], refs[1], None, refs[3]) == rtr.RTR_E_INVAL
+
+
+# The six projections of a Wan-1.3B-shaped block on its 3-frame chunk
+# (4680 tokens, D = 1536, FFN 8960): name, m, n, k, epilogue, qkv_rope.
+WAN13_PROJECTIONS = [("qkv", 4680, 4608, 1536, "bias", True), ("out", 4680, 1536, 1536, "gated_residual", False),
+                     ("cross_q", 4680, 1536, 1536, "bias", False),
+                     ("cross_out", 4680, 1536, 1536, "gated_residual", False),
+                     ("ffn_in", 4680, 8960, 1536, "gelu", False), ("ffn_out", 4680, 1536, 8960, "gated_residual", False)]
+
+
+def test_projection_planner_for_a_b200(lib):
+    """The planner's choices for a B200 (148 SMs, 74 resident CTA pairs), as
+    measured on the Wan-1.3B block: with packed weights every projection
+    takes 256 x 256 CTA-pair tiles; with row-major weights (8 KB boxes, more
+    TMA instructions) the 1,536-wide ones keep 256 x 256 tiles of one CTA.
+    Without pairs the planner never picks one; a pair launch takes an even
+    number of CTAs, never more than the SMs."""
+    from causal_attention_rtr_b200 import rtr
+    for name, m, n, k, epi, qkv in WAN13_PROJECTIONS:
+        assert rtr.rtr_dit_plan_tile(m, n, k, epi, qkv, True) == (256, 256, 1, 148), name
+        plan = rtr.rtr_dit_plan_tile(m, n, k, epi, qkv, False)
+        want_pair = name in ("qkv", "ffn_in")
+        assert plan[2] == int(want_pair), (name, plan)
+        if not want_pair:
+            assert plan == (256, 256, 0, 114), (name, plan)
+        for packed in (True, False):
+            rows, cols, pair, ctas = rtr.rtr_dit_plan_tile(m, n, k, epi, qkv, packed, 148, 0)
+            assert pair == 0 and ctas <= 148, (name, packed)
+    for m, n, k in [(7, 64, 8), (300, 200, 72), (20000, 8960, 1536), (1560, 5120, 5120)]:
+        for packed in (True, False):
+            rows, cols, pair, ctas = rtr.rtr_dit_plan_tile(m, n, k, "bias", False, packed, 148, 74)
+            tiles = -(-m // rows) * -(-n // cols)
+            assert ctas <= 148 and (not pair or (ctas % 2 == 0 and rows == 256 and cols == 256))
+            assert ctas == min(tiles, 74 if pair else 148) * (2 if pair else 1)
+
+
+def test_projection_planner_validation(lib):
+    import ctypes as ct
+    from causal_attention_rtr_b200 import rtr
+    r = [ct.c_int() for _ in range(4)]
+    refs = [ct.byref(x) for x in r]
+    for args in [(0, 64, 64, 0, 0, 0, 148, 74), (64, 64, 64, 0, 0, 0, 0, 0), (64, 64, 64, 0, 0, 0, 148, 75),
+                 (64, 64, 64, 0, 0, 0, 148, -1), (64, 64, 64, 3, 0, 0, 148, 74)]:
+        assert rtr.raw_status("rtr_dit_plan_tile", *args, *refs) == rtr.RTR_E_INVAL, args
+    assert rtr.raw_status("rtr_dit_plan_tile", 64, 64, 64, 0, 0, 0, 148, 74, refs[0], None, refs[2],
+                          refs[3]) == rtr.RTR_E_INVAL
+    assert rtr.raw_status("rtr_dit_plan_tile", 64, 64, 64, 0, 0, 0, 148, 74, *refs) == rtr.RTR_OK
